@@ -1,0 +1,410 @@
+"""Throughput of the routed-expert MoE layer on B200.
+
+Workload (default): the BF16 decode layer -- E=128 experts, top-8, d=2048,
+SwiGLU intermediate 768, weights ~N(0, 0.02^2) in bf16, router logits N(0,1)
+plus a per-expert bias N(0, 0.5^2), T=64 tokens per step, every expert
+resident in HBM.  One step = route -> permute -> expert FFN -> combine over
+one batch, captured in a CUDA graph.  R independent replicas of the layer
+(weights, routing, activations) are cycled so that the bytes read between two
+uses of a replica exceed the 126 MB L2 several times.
+
+Output: one JSON line on rank 0 (see the keys below).  `--impl reference`
+times the CPU oracle instead, on a bounded sample of the same workload.
+Multi-GPU: launch with torchrun; every rank runs its own replica set
+(independent batches, no data-path collective), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOPS vs B200 peak"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- workload
+def build_replicas(cfg, T, R, seed0=0):
+    """R independent resident layers with their inputs on the device."""
+    from expert_offload_serving_b200.layer import MoeLayer, pack_pool
+    reps = []
+    for r in range(R):
+        seed = seed0 + r
+        logits, x = synth.make_routing(cfg, T, seed)
+        w = synth.make_experts(cfg, range(cfg.E), seed, device="cuda")
+        pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()},
+                         range(cfg.E), pin=False).cuda()
+        del w
+        layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=pool)
+        reps.append(dict(layer=layer, logits=logits.cuda(), x=x.cuda(), logits_h=logits.pin_memory(),
+                         x_h=x.pin_memory()))
+    return reps
+
+
+def experts_touched(layer):
+    """Distinct experts of the last step (non-empty groups of the layer's
+    offsets): the algorithmic weight bytes are this count x blob bytes."""
+    off = layer.offsets.cpu()
+    return int(((off[1:] - off[:-1]) > 0).sum())
+
+
+def run_gpu(args, rank, world, local):
+    import expert_offload_serving_b200 as moe
+    moe.lib()
+    cfg = synth.CONFIGS["decode_bf16"]
+    T = args.tokens
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    blob = moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
+    # replicas: the bytes between two uses of one replica >= 4 x L2
+    per_step = None
+    R = args.replicas
+    reps = build_replicas(cfg, T, R, seed0=1000 * rank)
+    U = []
+    for r in reps:
+        r["layer"].forward(r["logits"], r["x"])
+        torch.cuda.synchronize()
+        U.append(experts_touched(r["layer"]))
+    per_step = [u * blob for u in U]
+    if R > 1 and min(sum(per_step) - p for p in per_step) < 4 * L2_BYTES:
+        print(f"warning: replicas stream only {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
+              "between reuses", file=sys.stderr)
+    stream = torch.cuda.Stream(device=dev)
+    launches_per_step = 5   # route, permute, ffn gate/up, ffn down, combine
+
+    def step_fn(r):
+        L = r["layer"]
+        L.forward(r["logits"], r["x"])
+
+    # CUDA graph per replica
+    graphs = []
+    with torch.cuda.stream(stream):
+        for r in reps:                      # warm the code paths once before capture
+            step_fn(r)
+        stream.synchronize()
+        for r in reps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step_fn(r)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    # ---- device-timed steps
+    for i in range(args.warmup):
+        graphs[i % R].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(dev.index)
+    with ClockSampler(smi_id) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(args.steps):
+                graphs[i % R].replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    barrier(world)
+    ms_max = max_over_ranks(ms, world)
+    value = world * args.steps * T / (ms_max / 1e3)
+
+    # ---- dominant kernel: moe_expert_ffn (gate/up + down launches), timed alone
+    ffn_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            reps[i % R]["layer"].ffn(reps[i % R]["x"])
+        n_ffn = max(20, args.steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_ffn):
+            reps[i % R]["layer"].ffn(reps[i % R]["x"])
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ffn_avg_ms = e0.elapsed_time(e1) / n_ffn
+    alg_bytes = sum(per_step[i % R] for i in range(n_ffn)) / n_ffn
+    hbm_peak, peak_src = peaks()
+    achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(3, min(args.steps, 50))
+    outs_h = [torch.empty((T, cfg.d), dtype=torch.float32, pin_memory=True) for _ in range(R)]
+    with torch.cuda.stream(stream):
+        def e2e_step(i):
+            r = reps[i % R]
+            r["logits"].copy_(r["logits_h"], non_blocking=True)
+            r["x"].copy_(r["x_h"], non_blocking=True)
+            out = r["layer"].forward(r["logits"], r["x"])
+            outs_h[i % R].copy_(out, non_blocking=True)
+        for i in range(max(3, args.warmup)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * e2e_steps * T / (e2e_ms / 1e3)
+    h2d = T * cfg.E * 4 + T * cfg.d * 2
+    d2h = T * cfg.d * 4
+
+    st = reps[0]["layer"].status
+    moe.moe_check_status(st)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, T, args.cpu_tokens)
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"decode_bf16: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, all experts resident",
+            "global_batch": T * world,
+            "replicas": R,
+            "l2": f"inputs larger than L2: {R} replicas, >= {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
+                  "read between reuses" if R > 1 else "single replica",
+            "experts_touched_per_step": U,
+            "parallelism": f"dp{world} (independent batches)",
+            "cuda_graph": True,
+        },
+        "roofline": {
+            "kernel": "moe_expert_ffn (ffn_decode gate/up + down)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": None,
+            "algorithmic_bytes_per_launch": int(alg_bytes),
+            "avg_launch_ms": round(ffn_avg_ms, 5),
+        },
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        result["cpu_baseline"] = cpu
+    return result
+
+
+# ---------------------------------------------------------------- CPU oracle arms
+def _cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_step(cfg, T_sample, seed, weights_cache):
+    from oracle import moe as M
+    logits, x = synth.make_routing(cfg, T_sample, seed)
+
+    def w(e):
+        if e not in weights_cache:
+            ww = synth.make_experts(cfg, [e], 0, device="cpu")
+            weights_cache[e] = M.dequant_expert(cfg.fmt, ww, 0)
+        return weights_cache[e]
+    return M.moe_layer(x.double().numpy(), logits.numpy(), cfg.k, w)
+
+
+def cpu_baseline(cfg, T, T_sample):
+    """The oracle as it stands on the host cores: one layer pass over T_sample
+    tokens of the same workload (expert weights generated and dequantised
+    beforehand, outside the timed region)."""
+    from oracle import moe as M
+    cache = {}
+    logits, x = synth.make_routing(cfg, T_sample, 99)
+    idx, _ = M.route_topk(logits.numpy(), cfg.k)
+    for e in sorted(set(idx.ravel().tolist())):
+        ww = synth.make_experts(cfg, [e], 0, device="cpu")
+        cache[e] = M.dequant_expert(cfg.fmt, ww, 0)
+    t0 = time.perf_counter()
+    M.moe_layer(x.double().numpy(), logits.numpy(), cfg.k, lambda e: cache[e])
+    dt = time.perf_counter() - t0
+    return {"value": round(T_sample / dt, 2), "unit": "tokens/s", "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"one layer pass over {T_sample} tokens of the decode_bf16 workload (float64 oracle, "
+                      f"{len(cache)} experts, weights dequantised before timing)",
+            "seconds": round(dt, 3)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS["decode_bf16"]
+    T_s = args.cpu_tokens
+    from oracle import moe as M
+    cache = {}
+    for i in range(args.warmup):
+        oracle_step(cfg, T_s, 5000 + i, cache)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(cfg, T_s, 6000 + i, cache)
+    dt = time.perf_counter() - t0
+    v = args.steps * T_s / dt
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"decode_bf16: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I}; each step a sample "
+                               f"of {T_s} tokens", "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": _cpu_cores(), "kind": "oracle",
+                         "sample": f"{T_s} tokens per step; expert weights generated and dequantised "
+                                   "on first use (inside the warm-up where possible)"},
+        "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--tokens", type=int, default=64, help="tokens per step (1, 16 or 64)")
+    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--cpu-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_gpu(args, rank, world, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

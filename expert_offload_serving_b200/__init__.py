@@ -1,0 +1,204 @@
+"""B200 routed-expert MoE layer: Python binding of libmoe.so.
+
+The functions here carry the C ABI's names (include/moe.h) and only marshal
+arguments: torch tensors give device pointers, torch streams give
+cudaStream_t.  Every step of the layer runs in libmoe's CUDA kernels; there is
+no Python or CPU fallback, and loading fails loudly if the library is absent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_CAPACITY, \
+    MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = range(7)
+STATUS_NAMES = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA",
+                "MOE_ERR_CAPACITY", "MOE_ERR_TIMEOUT", "MOE_ERR_DEVICE"]
+MOE_W_BF16, MOE_W_MXFP4, MOE_W_NVFP4 = 0, 1, 2
+FORMATS = {"bf16": MOE_W_BF16, "mxfp4": MOE_W_MXFP4, "nvfp4": MOE_W_NVFP4}
+MOE_FFN_ACT_NVFP4 = 1
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else str(status)
+        super().__init__(f"{name}: {msg}")
+        self.status = status
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int32), ("d", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("fmt", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "moe_abi_version": (_I, []),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_expert_blob_bytes": (_SZ, [moe_shape]),
+    "moe_pack_expert": (_I, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_permute_scratch_bytes": (_SZ, [_I, _I, _I]),
+    "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_expert_ffn_workspace_bytes": (_SZ, [moe_shape, _I, _I, _I]),
+    "moe_expert_ffn": (_I, [moe_shape, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P, _P]),
+    "moe_combine_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "moe_cache_create": (_I, [moe_shape, _I, _P, _P, _P, ctypes.POINTER(_P)]),
+    "moe_cache_fill": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "moe_cache_query": (_I, [_P, _P, _P, _P]),
+    "moe_cache_destroy": (_I, [_P]),
+    "moe_check_status": (_I, [_P, _P]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded libmoe.so (ctypes.CDLL); raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m expert_offload_serving_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def declared_symbols():
+    return list(_SIGS)
+
+
+def _check(status: int):
+    if status != MOE_OK:
+        raise MoeError(status, lib().moe_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def shape(E: int, d: int, I: int, fmt) -> moe_shape:
+    return moe_shape(E, d, I, FORMATS[fmt] if isinstance(fmt, str) else int(fmt))
+
+
+# ------------------------------------------------------------------ the ABI
+def moe_abi_version() -> int:
+    return lib().moe_abi_version()
+
+
+def moe_expert_blob_bytes(s: moe_shape) -> int:
+    return lib().moe_expert_blob_bytes(s)
+
+
+def moe_pack_expert(s: moe_shape, wg, wu, wd, sg=None, su=None, sd=None, tensor_scales=None, blob_out=None):
+    """Canonical CPU tensors -> blob_out (CPU uint8 tensor of moe_expert_blob_bytes)."""
+    _check(lib().moe_pack_expert(s, _ptr(wg), _ptr(wu), _ptr(wd), _ptr(sg), _ptr(su), _ptr(sd),
+                                 _ptr(tensor_scales), _ptr(blob_out)))
+
+
+def moe_route_topk(logits, k: int, idx, gate, stream=None):
+    T, E = logits.shape
+    _check(lib().moe_route_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(gate), _stream(stream)))
+
+
+def moe_permute_scratch_bytes(T: int, k: int, E: int) -> int:
+    return lib().moe_permute_scratch_bytes(T, k, E)
+
+
+def moe_permute(idx, E: int, offsets, perm, inv_perm, scratch=None, dev_status=None, stream=None):
+    T, k = idx.shape
+    nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+                             _ptr(scratch), nbytes, _ptr(dev_status), _stream(stream)))
+
+
+def moe_expert_ffn_workspace_bytes(s: moe_shape, T: int, k: int, flags: int = 0) -> int:
+    return lib().moe_expert_ffn_workspace_bytes(s, T, k, flags)
+
+
+def moe_expert_ffn(s: moe_shape, x, k: int, offsets, perm, slot_of_expert, slot_pool, n_slots: int,
+                   gate=None, y_perm=None, out=None, flags: int = 0, workspace=None,
+                   dev_status=None, stream=None):
+    T = x.shape[0]
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().moe_expert_ffn(s, _ptr(x), T, k, _ptr(offsets), _ptr(perm), _ptr(slot_of_expert),
+                                _ptr(slot_pool), n_slots, _ptr(gate), _ptr(y_perm), _ptr(out), flags,
+                                _ptr(workspace), nbytes, _ptr(dev_status), _stream(stream)))
+
+
+def moe_combine_merge(y_perm, idx, gate, inv_perm, slot_of_expert, host_partial, E: int, out, stream=None):
+    T, k = idx.shape
+    d = out.shape[1]
+    _check(lib().moe_combine_merge(_ptr(y_perm), _ptr(idx), _ptr(gate), _ptr(inv_perm),
+                                   _ptr(slot_of_expert), _ptr(host_partial), T, k, d, E, _ptr(out),
+                                   _stream(stream)))
+
+
+def moe_check_status(dev_status, stream=None):
+    _check(lib().moe_check_status(_ptr(dev_status), _stream(stream)))
+
+
+class MoeCache:
+    """Handle of the host-side LRU bookkeeping (moe_cache_*)."""
+
+    def __init__(self, s: moe_shape, n_slots: int, slot_pool=None, host_pool=None, slot_of_expert_dev=None):
+        h = ctypes.c_void_p()
+        _check(lib().moe_cache_create(s, n_slots, _ptr(slot_pool), _ptr(host_pool),
+                                      _ptr(slot_of_expert_dev), ctypes.byref(h)))
+        self.h = h
+        self.E, self.n_slots = s.E, n_slots
+
+    def fill(self, experts, step: int, protect=(), side=None, reads_done=None, fill_done=None):
+        """moe_cache_fill; returns the list of (expert, slot, evicted) fills."""
+        ex = (ctypes.c_int32 * max(1, len(experts)))(*[int(e) for e in experts])
+        pr = (ctypes.c_int32 * max(1, len(protect)))(*[int(e) for e in protect])
+        fills = (ctypes.c_int32 * (3 * max(1, len(experts))))()
+        nf = ctypes.c_int32(0)
+        side_h = None if side is None else _stream(side)
+        _check(lib().moe_cache_fill(self.h, ex, len(experts), step, pr, len(protect), side_h,
+                                    None if reads_done is None else reads_done.cuda_event,
+                                    None if fill_done is None else fill_done.cuda_event,
+                                    fills, ctypes.byref(nf)))
+        return [(fills[3 * i], fills[3 * i + 1], fills[3 * i + 2]) for i in range(nf.value)]
+
+    def query(self):
+        soe = (ctypes.c_int32 * self.E)()
+        eos = (ctypes.c_int32 * self.n_slots)()
+        lu = (ctypes.c_int32 * self.n_slots)()
+        _check(lib().moe_cache_query(self.h, soe, eos, lu))
+        return list(soe), list(eos), list(lu)
+
+    def close(self):
+        if self.h:
+            lib().moe_cache_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

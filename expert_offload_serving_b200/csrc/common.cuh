@@ -1,0 +1,98 @@
+// Shared definitions of libmoe: error reporting, argument checks, the expert
+// blob layout, and small device helpers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- errors
+moe_status fail(moe_status st, const char* fmt, ...);
+void clear_error();
+
+#define MOE_REQUIRE(cond, ...)                                   \
+  do {                                                           \
+    if (!(cond)) return ::moe::fail(MOE_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define MOE_CUDA_TRY(call)                                                        \
+  do {                                                                            \
+    cudaError_t e_ = (call);                                                      \
+    if (e_ != cudaSuccess)                                                        \
+      return ::moe::fail(MOE_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define MOE_LAUNCH_CHECK(what)                                                    \
+  do {                                                                            \
+    cudaError_t e_ = cudaGetLastError();                                          \
+    if (e_ != cudaSuccess)                                                        \
+      return ::moe::fail(MOE_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Device attributes of the current device (cached per device id).
+struct DeviceInfo { int id, sm_count, cc_major, cc_minor; size_t smem_optin; };
+moe_status current_device(DeviceInfo* out);
+
+// ---------------------------------------------------------------- blob layout
+// One expert = one blob; every region starts on a 256-byte boundary.
+//   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16, row-major).
+//   MXFP4: codes wg [I][d/2], wu [I][d/2], wd [d][I/2] (low nibble = even
+//          element), then E8M0 scales sg [I][d/32], su [I][d/32], sd [d][I/32].
+//   NVFP4: codes as MXFP4; E4M3 scales in tensor-core atoms (see sf_atom_offset)
+//          for each matrix; then 3 fp32 tensor scales (gate, up, down).
+struct BlobLayout {
+  size_t wg, wu, wd, sg, su, sd, ts, bytes;
+};
+
+__host__ __device__ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+__host__ __device__ inline BlobLayout blob_layout(int fmt, int d, int I) {
+  BlobLayout L{};
+  size_t m = static_cast<size_t>(I) * d;   // elements of one matrix
+  size_t o = 0;
+  if (fmt == MOE_W_BF16) {
+    L.wg = o; o = round_up(o + m * 2, 256);
+    L.wu = o; o = round_up(o + m * 2, 256);
+    L.wd = o; o = round_up(o + m * 2, 256);
+    L.sg = L.su = L.sd = L.ts = o;
+  } else {
+    L.wg = o; o = round_up(o + m / 2, 256);
+    L.wu = o; o = round_up(o + m / 2, 256);
+    L.wd = o; o = round_up(o + m / 2, 256);
+    size_t per_blk = (fmt == MOE_W_MXFP4) ? 32 : 16;
+    L.sg = o; o = round_up(o + m / per_blk, 256);
+    L.su = o; o = round_up(o + m / per_blk, 256);
+    L.sd = o; o = round_up(o + m / per_blk, 256);
+    L.ts = o;
+    if (fmt == MOE_W_NVFP4) o = round_up(o + 3 * sizeof(float), 256);
+  }
+  L.bytes = o;
+  return L;
+}
+
+// Byte offset of the E4M3 scale of (row r, 16-element block b) of an NVFP4
+// matrix with K columns, in the scale-factor atom layout the FP4 tensor-core
+// MMA reads: atoms of 128 rows x 4 blocks (512 bytes), atoms ordered
+// [row/128][block/4]; inside an atom row r sits at (r%32)*16 + ((r/32)%4)*4
+// and block b at b%4.
+__host__ __device__ inline size_t sf_atom_offset(int r, int b, int K) {
+  return (static_cast<size_t>(r >> 7) * (K >> 6) + (b >> 2)) * 512 +
+         (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
+}
+
+moe_status check_shape(moe_shape s);
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ void report(int32_t* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+constexpr unsigned kFull = 0xffffffffu;
+
+}  // namespace moe

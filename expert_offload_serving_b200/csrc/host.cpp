@@ -1,0 +1,119 @@
+// Host-only parts of libmoe: error strings, shape checks, device attributes,
+// and moe_pack_expert (canonical tensors -> device-final expert blob).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+
+static thread_local char g_err[512] = "";
+
+moe_status fail(moe_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+moe_status check_shape(moe_shape s) {
+  MOE_REQUIRE(s.E >= 1 && s.E <= 1024, "E=%d outside [1, 1024]", s.E);
+  MOE_REQUIRE(s.d >= 1 && s.I >= 1 && s.d <= 16384 && s.I <= 16384,
+              "d=%d, I=%d outside [1, 16384]", s.d, s.I);
+  if (s.fmt == MOE_W_BF16) {
+    MOE_REQUIRE(s.d % 8 == 0 && s.I % 8 == 0, "BF16 needs d, I multiples of 8 (d=%d, I=%d)", s.d, s.I);
+  } else if (s.fmt == MOE_W_MXFP4) {
+    MOE_REQUIRE(s.d % 32 == 0 && s.I % 32 == 0, "MXFP4 needs d, I multiples of 32 (d=%d, I=%d)", s.d, s.I);
+  } else if (s.fmt == MOE_W_NVFP4) {
+    MOE_REQUIRE(s.d % 128 == 0 && s.I % 128 == 0, "NVFP4 needs d, I multiples of 128 (d=%d, I=%d)", s.d, s.I);
+  } else {
+    return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", s.fmt);
+  }
+  return MOE_OK;
+}
+
+moe_status current_device(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device id %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    DeviceInfo d{};
+    d.id = dev;
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev));
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev));
+    int optin = 0;
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    d.smem_optin = static_cast<size_t>(optin);
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  if (out->cc_major != 10)
+    return fail(MOE_ERR_UNSUPPORTED, "libmoe is built for sm_100a; device %d is sm_%d%d",
+                dev, out->cc_major, out->cc_minor);
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int moe_abi_version(void) { return 1; }
+
+extern "C" const char* moe_last_error(void) { return g_err; }
+
+extern "C" size_t moe_expert_blob_bytes(moe_shape s) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return blob_layout(s.fmt, s.d, s.I).bytes;
+}
+
+extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* wu, const void* wd,
+                                      const uint8_t* sg, const uint8_t* su, const uint8_t* sd,
+                                      const float* tensor_scales, void* blob_out) {
+  clear_error();
+  moe_status st = check_shape(s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(wg && wu && wd && blob_out, "null weight or output pointer");
+  const BlobLayout L = blob_layout(s.fmt, s.d, s.I);
+  uint8_t* b = static_cast<uint8_t*>(blob_out);
+  std::memset(b, 0, L.bytes);
+  const size_t m = static_cast<size_t>(s.I) * s.d;
+  if (s.fmt == MOE_W_BF16) {
+    std::memcpy(b + L.wg, wg, m * 2);
+    std::memcpy(b + L.wu, wu, m * 2);
+    std::memcpy(b + L.wd, wd, m * 2);
+    return MOE_OK;
+  }
+  MOE_REQUIRE(sg && su && sd, "null scale pointer for an FP4 format");
+  std::memcpy(b + L.wg, wg, m / 2);
+  std::memcpy(b + L.wu, wu, m / 2);
+  std::memcpy(b + L.wd, wd, m / 2);
+  if (s.fmt == MOE_W_MXFP4) {
+    std::memcpy(b + L.sg, sg, m / 32);
+    std::memcpy(b + L.su, su, m / 32);
+    std::memcpy(b + L.sd, sd, m / 32);
+    return MOE_OK;
+  }
+  MOE_REQUIRE(tensor_scales != nullptr, "NVFP4 needs 3 tensor scales");
+  // scale bytes move from row-major [R][K/16] into the MMA atom layout
+  struct M { const uint8_t* src; size_t off; int R, K; } mats[3] = {
+      {sg, L.sg, s.I, s.d}, {su, L.su, s.I, s.d}, {sd, L.sd, s.d, s.I}};
+  for (const M& mt : mats) {
+    const int nb = mt.K / 16;
+    for (int r = 0; r < mt.R; ++r)
+      for (int blk = 0; blk < nb; ++blk)
+        b[mt.off + sf_atom_offset(r, blk, mt.K)] = mt.src[static_cast<size_t>(r) * nb + blk];
+  }
+  std::memcpy(b + L.ts, tensor_scales, 3 * sizeof(float));
+  return MOE_OK;
+}

@@ -1,0 +1,234 @@
+/*
+ * moe.h -- C ABI of the B200 routed-expert MoE layer (libmoe.so).
+ *
+ * The layer is the routed-expert MoE forward described in the FreeToken
+ * write-ups: each token picks k of E experts (freetoken.wiki, "FreeToken 753b
+ * model", section "FreeToken 753b Model Explained"), the experts live in a
+ * GPU expert cache that follows router demand with LRU eviction (same page,
+ * mechanism table, "Global LRU expert cache"), missed experts are either
+ * filled over PCIe or computed on the CPU, and the two shares of partial sums
+ * are added without approximation (explainx.ai hardware guide, section
+ * "Decode: decide whether to move an expert or compute where it lives";
+ * ainewsfeed.tech, third paragraph).
+ *
+ * Conventions for every call
+ *   - Ownership: the caller allocates every device buffer, the pinned host
+ *     pool and every output; no call allocates device memory.  The only
+ *     library-owned object is the host-side cache handle (moe_cache).
+ *   - Asynchrony: calls that take a cudaStream_t validate their arguments
+ *     synchronously, enqueue kernels or copies on that stream and return.
+ *     Results are ready when the stream reaches that point.
+ *   - Errors: every call returns moe_status.  MOE_OK = success.  On failure
+ *     nothing was enqueued, and moe_last_error() (per thread) describes it.
+ *     Kernels that detect a bad index at run time (an expert id or slot out of
+ *     range) skip the access and record MOE_ERR_DEVICE in the caller's
+ *     dev_status word (first error wins); moe_check_status() reads it.
+ *     No kernel traps, and no call throws across the ABI.
+ *   - Pointers marked "device" must be device memory of the current device;
+ *     float/bf16 tensors and byte pools must be 16-byte aligned; int32 arrays
+ *     4-byte aligned.
+ *   - Index conventions: T tokens, E experts, k experts per token, d hidden
+ *     size, I SwiGLU intermediate size; pair p = t*k + j is the j-th choice
+ *     of token t; "sorted position" q is the index of a pair after grouping
+ *     pairs by expert.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* bad size, null or misaligned pointer, bad id */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_CAPACITY = 4,     /* not enough cache slots, workspace or scratch */
+  MOE_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+  MOE_ERR_DEVICE = 6        /* a kernel reported an out-of-range index */
+} moe_status;
+
+/* Expert weight formats (explainx.ai hardware guide: NVFP4 routed experts;
+ * freetoken.wiki: NVFP4 or MXFP4 builds; fervorai.dev, "What to know before
+ * you commit": NVFP4, MXFP4, FP8 and BF16).  Bit layouts: BF16; MXFP4 = E2M1
+ * values with one E8M0 scale per 32 elements (OCP MX v1.0); NVFP4 = E2M1
+ * values with one E4M3 scale per 16 elements and one fp32 scale per matrix. */
+typedef enum moe_wfmt { MOE_W_BF16 = 0, MOE_W_MXFP4 = 1, MOE_W_NVFP4 = 2 } moe_wfmt;
+
+/* Layer shape.  Limits: 1 <= E <= 1024; d and I multiples of 8 (BF16),
+ * 32 (MXFP4) or 128 (NVFP4); d, I <= 16384. */
+typedef struct moe_shape { int32_t E, d, I, fmt; } moe_shape;
+
+/* moe_expert_ffn flags. */
+enum {
+  /* Quantise x and the SwiGLU output to NVFP4 (unit tensor scale, one E4M3
+   * scale per 16 elements, round-to-nearest-even) before the two products and
+   * run them on the FP4 tensor cores.  Requires MOE_W_NVFP4.  Without this
+   * flag activations stay in bf16/fp32 and the CUDA-core path runs. */
+  MOE_FFN_ACT_NVFP4 = 1
+};
+
+/* Version of this ABI (bumped on any signature change). */
+int moe_abi_version(void);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Expert blobs.  An expert's weights are stored as one contiguous blob in a
+ * device-final layout, identical in the pinned host pool and in a GPU cache
+ * slot, so a cache fill is a single copy (futuresignalnews.com, mechanism 3:
+ * experts are read into their final host layout and pinned; explainx.ai
+ * hardware guide: the FTW layout).  The layout is private to the library. */
+
+/* Bytes of one expert blob (a multiple of 256), or 0 if the shape is invalid.
+ * Slot s of a pool starts at pool + s * moe_expert_blob_bytes(shape). */
+size_t moe_expert_blob_bytes(moe_shape s);
+
+/* Host-only: build the blob of one expert from canonical row-major tensors.
+ *   BF16 : wg, wu = bf16 [I][d]; wd = bf16 [d][I]; sg/su/sd/tensor_scales NULL.
+ *   MXFP4: wg, wu = [I][d/2] bytes, wd = [d][I/2] bytes (element 2i in the low
+ *          nibble); sg, su = [I][d/32], sd = [d][I/32] E8M0 bytes.
+ *   NVFP4: codes as MXFP4; sg, su = [I][d/16], sd = [d][I/16] E4M3 bytes;
+ *          tensor_scales = 3 floats (gate, up, down).
+ * blob_out: host buffer of moe_expert_blob_bytes(s) bytes.  No CUDA call. */
+moe_status moe_pack_expert(moe_shape s, const void* wg, const void* wu, const void* wd,
+                           const uint8_t* sg, const uint8_t* su, const uint8_t* sd,
+                           const float* tensor_scales, void* blob_out);
+
+/* ------------------------------------------------------------------------ */
+/* Step 1 -- top-k expert selection (freetoken.wiki, "FreeToken 753b Model
+ * Explained": a token routes through 6 of 256 experts; explainx.ai, "Decode":
+ * expert choice per token).  The router is not modified (ainewsfeed.tech,
+ * third paragraph): gates are the softmax of the k selected logits.
+ *   logits: device fp32 [T][E], finite.
+ *   idx:    device int32 [T][k]: the k largest logits of each row, ordered by
+ *           logit descending then expert index ascending (ties, including
+ *           -0.0 vs +0.0, go to the lower index).
+ *   gate:   device fp32 [T][k]: exp(l_j - l_0) / sum_i exp(l_i - l_0).
+ * Limits: 1 <= k <= min(E, 32), E <= 1024, T >= 0 (T = 0 enqueues nothing). */
+moe_status moe_route_topk(const float* logits, int T, int E, int k,
+                          int32_t* idx, float* gate, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 2 -- permutation of token-expert pairs by expert, so each expert's
+ * FFN runs once per step on all the tokens routed to it (ainewsfeed.tech,
+ * second paragraph: many tokens of a layer route to nearly the whole expert
+ * set).  A stable counting sort of the pairs p = t*k + j by idx[t][j]:
+ *   offsets:  device int32 [E+1], offsets[e] = number of pairs with expert < e.
+ *   perm:     device int32 [T*k], perm[q] = pair at sorted position q; pairs of
+ *             one expert appear in ascending p.
+ *   inv_perm: device int32 [T*k], inv_perm[perm[q]] = q.
+ *   scratch:  device buffer of at least moe_permute_scratch_bytes(T, k, E)
+ *             bytes (may be NULL when that is 0); contents need no setup.
+ *   dev_status: device int32 word or NULL; an idx value outside [0, E) is
+ *             recorded there as MOE_ERR_DEVICE and its pair is dropped. */
+size_t moe_permute_scratch_bytes(int T, int k, int E);
+moe_status moe_permute(const int32_t* idx, int T, int k, int E,
+                       int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                       void* scratch, size_t scratch_bytes, int32_t* dev_status,
+                       cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 3 -- grouped SwiGLU expert FFN over the expert cache.  For every
+ * expert e with slot_of_expert[e] >= 0 and every pair at sorted position q in
+ * [offsets[e], offsets[e+1]) with token t = perm[q] / k:
+ *     h = W_g x_t,  u = W_u x_t,  a = silu(h) * u,  y_q = W_d a
+ * with the weights read from the blob at slot_pool + slot * blob_bytes.
+ * Experts with slot -1 are not evaluated here: their pairs are computed
+ * elsewhere (the host share of the misses; explainx.ai, "Decode").
+ *   x:      device bf16 [T][d].
+ *   offsets, perm: from moe_permute.  slot_of_expert: device int32 [E].
+ *   slot_pool: device, n_slots blobs.
+ *   Output, one of:
+ *     y_perm != NULL: y_perm[q][:] = y_q (fp32 [T*k][d], unweighted); rows of
+ *                     skipped experts are left untouched.  Not available with
+ *                     MOE_FFN_ACT_NVFP4.
+ *     y_perm == NULL: out[t][:] += gate[t][j] * y_q (fp32 [T][d]) for p = t*k+j,
+ *                     accumulated with atomic adds; the caller initialises out
+ *                     (zeros, or the host partial).
+ *   flags: 0 or MOE_FFN_ACT_NVFP4.
+ *   workspace: device, >= moe_expert_ffn_workspace_bytes(s, T, k, flags).
+ *   dev_status: device int32 word or NULL (slot or expert out of range).
+ * Limits: T*k <= 1<<24. */
+size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int flags);
+moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k,
+                          const int32_t* offsets, const int32_t* perm,
+                          const int32_t* slot_of_expert, const void* slot_pool, int n_slots,
+                          const float* gate, float* y_perm, float* out, int flags,
+                          void* workspace, size_t ws_bytes, int32_t* dev_status,
+                          cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 4 -- gate-weighted combine with the exact merge of partial sums
+ * computed elsewhere (explainx.ai hardware guide, "Decode": CPU and GPU
+ * partial results are merged exactly; ainewsfeed.tech, third paragraph).
+ *   out[t][c] = sum_{j=0..k-1, slot_of_expert[idx[t][j]] >= 0}
+ *                   gate[t][j] * y_perm[inv_perm[t*k+j]][c]
+ *               + host_partial[t][c]            (if host_partial != NULL)
+ * summed in that order in fp32.  y_perm fp32 [T*k][d]; idx, gate [T][k];
+ * inv_perm [T*k]; slot_of_expert [E] (NULL: every expert counts);
+ * host_partial fp32 [T][d] or NULL; out fp32 [T][d] (may alias host_partial).
+ * E bounds the expert ids looked up in slot_of_expert (an id outside [0, E)
+ * or an inv_perm entry outside [0, T*k) drops that term).
+ * All device pointers.  d must be a multiple of 4. */
+moe_status moe_combine_merge(const float* y_perm, const int32_t* idx, const float* gate,
+                             const int32_t* inv_perm, const int32_t* slot_of_expert,
+                             const float* host_partial, int T, int k, int d, int E, float* out,
+                             cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 5 -- the GPU expert cache: LRU residency of expert blobs in device
+ * slots, filled from a pinned host pool (freetoken.wiki mechanism table:
+ * "Global LRU expert cache"; explainx.ai hardware guide: experts are copied
+ * over PCIe into the GPU cache and kept; the host pool is the source of
+ * truth; futuresignalnews.com mechanism 3: a cold cache serves the first
+ * request).  The handle keeps the bookkeeping on the host:
+ * expert_of_slot[S], last_used[S], slot_of_expert[E].
+ *
+ * moe_cache_create: slot_pool (device, n_slots blobs), host_pool (pinned host,
+ *   E blobs in expert order), slot_of_expert_dev (device int32 [E]; this call
+ *   does not write it -- the caller sets it to -1 before the first fill).  A
+ *   handle made with slot_pool, host_pool and slot_of_expert_dev all NULL only
+ *   plans (no CUDA call is ever made by it).
+ * moe_cache_fill: makes the experts of `experts` (n ids, any order, duplicates
+ *   ignored) resident for step `step`.  Distinct ids are handled in ascending
+ *   order: a resident expert has its last_used set to `step` (a hit); a
+ *   missing one takes the lowest free slot, else the slot with the smallest
+ *   last_used (ties: lowest slot) whose expert is neither in `experts` nor in
+ *   `protect` (the other experts of this step, e.g. the host-computed ones).
+ *   For each fill it enqueues on `side`: a wait on `reads_done` (if non-NULL;
+ *   the last kernel that read the pool), the blob copy host -> slot with
+ *   cudaMemcpyAsync, and one kernel that writes the slot-table changes
+ *   (evicted expert -> -1, new expert -> slot); then records `fill_done` (if
+ *   non-NULL).  fills (host int32 [n][3] or NULL) receives
+ *   (expert, slot, evicted expert or -1) per fill; *n_fills their count.
+ *   If there are not enough evictable slots, MOE_ERR_CAPACITY is returned
+ *   and the cache state is unchanged. */
+typedef struct moe_cache moe_cache;
+moe_status moe_cache_create(moe_shape s, int n_slots, void* slot_pool, const void* host_pool,
+                            int32_t* slot_of_expert_dev, moe_cache** out);
+moe_status moe_cache_fill(moe_cache* c, const int32_t* experts, int n, int step,
+                          const int32_t* protect, int n_protect,
+                          cudaStream_t side, cudaEvent_t reads_done, cudaEvent_t fill_done,
+                          int32_t* fills, int32_t* n_fills);
+/* Copies of the host bookkeeping: slot_of_expert [E], expert_of_slot [S],
+ * last_used [S] (any may be NULL). */
+moe_status moe_cache_query(const moe_cache* c, int32_t* slot_of_expert,
+                           int32_t* expert_of_slot, int32_t* last_used);
+moe_status moe_cache_destroy(moe_cache* c);
+
+/* ------------------------------------------------------------------------ */
+/* Synchronises `stream`, reads the device status word written by kernels,
+ * resets it to 0 and returns it as a moe_status (MOE_OK if it was 0). */
+moe_status moe_check_status(int32_t* dev_status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

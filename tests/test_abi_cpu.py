@@ -1,0 +1,173 @@
+"""The C ABI on the CPU: the library loads and exports every declared symbol,
+host-only calls work, arguments are rejected before any CUDA call, and the
+cache's host bookkeeping makes the oracle's LRU decisions (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import formats as F
+from oracle import lru as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    from expert_offload_serving_b200 import build
+    build.build()
+    import expert_offload_serving_b200 as m
+    m.lib()
+    return m
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound(moe):
+    names = header_functions()
+    assert len(names) >= 15
+    L_ = moe.lib()
+    for n in names:
+        assert hasattr(L_, n), n
+    assert sorted(moe.declared_symbols()) == names
+
+
+def test_abi_version(moe):
+    assert moe.moe_abi_version() == 1
+
+
+@pytest.mark.parametrize("name,expect", [
+    ("decode_bf16", 3 * 2048 * 768 * 2),
+    ("decode_mxfp4", 3 * 4096 * 2048 // 2 + 3 * 4096 * 2048 // 32),
+    ("prefill_nvfp4", 3 * 4096 * 2048 // 2 + 3 * 4096 * 2048 // 16 + 256),
+])
+def test_blob_bytes(moe, name, expect):
+    c = synth.CONFIGS[name]
+    assert moe.moe_expert_blob_bytes(moe.shape(c.E, c.d, c.I, c.fmt)) == expect
+
+
+@pytest.mark.parametrize("E,d,I,fmt", [(0, 64, 64, "bf16"), (2000, 64, 64, "bf16"), (4, 60, 64, "bf16"),
+                                       (4, 48, 64, "mxfp4"), (4, 64, 64, "nvfp4"), (4, 64, 64, 7)])
+def test_invalid_shapes_have_no_blob(moe, E, d, I, fmt):
+    assert moe.moe_expert_blob_bytes(moe.shape(E, d, I, fmt)) == 0
+
+
+def _host_ptr(a):
+    return a.ctypes.data
+
+
+def test_argument_errors_before_any_cuda_call(moe):
+    L_ = moe.lib()
+    buf = np.zeros(1024, dtype=np.float32)
+    p = _host_ptr(buf)
+    assert L_.moe_route_topk(p, 4, 8, 9, p, p, None) == moe.MOE_ERR_INVALID_ARG      # k > E
+    assert L_.moe_route_topk(p, 4, 2000, 2, p, p, None) == moe.MOE_ERR_INVALID_ARG   # E > 1024
+    assert L_.moe_route_topk(p, 4, 64, 33, p, p, None) == moe.MOE_ERR_INVALID_ARG    # k > 32
+    assert L_.moe_route_topk(None, 4, 8, 2, p, p, None) == moe.MOE_ERR_INVALID_ARG   # null
+    assert b"k=" in L_.moe_last_error() or b"null" in L_.moe_last_error()
+    assert L_.moe_permute(p, 4, 2, 0, p, p, p, None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
+    s_bad = moe.shape(8, 60, 64, "bf16")
+    assert L_.moe_expert_ffn(s_bad, p, 4, 2, p, p, p, p, 8, p, p, None, 0, p, 1 << 20, None,
+                             None) == moe.MOE_ERR_INVALID_ARG
+    s = moe.shape(8, 64, 64, "bf16")
+    assert L_.moe_expert_ffn(s, p, 4, 2, p, p, p, p, 8, p, None, None, 0, p, 1 << 20, None,
+                             None) == moe.MOE_ERR_INVALID_ARG                          # no output
+    assert L_.moe_expert_ffn(s, p + 4, 4, 2, p, p, p, p, 8, p, p, None, 0, p, 1 << 20, None,
+                             None) == moe.MOE_ERR_INVALID_ARG                          # misaligned x
+    assert L_.moe_expert_ffn(s, p, 4, 2, p, p, p, p, 8, p, p, None, 1, p, 1 << 20, None,
+                             None) == moe.MOE_ERR_INVALID_ARG                          # act flag, bf16
+    assert L_.moe_combine_merge(p, p, p, p, None, None, 4, 2, 6, 8, p, None) == moe.MOE_ERR_INVALID_ARG
+    assert L_.moe_cache_fill(None, None, 0, 0, None, 0, None, None, None, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_and_scratch_sizes(moe):
+    s = moe.shape(128, 2048, 768, "bf16")
+    assert moe.moe_expert_ffn_workspace_bytes(s, 64, 8) >= 64 * 8 * 768 * 4
+    assert moe.moe_permute_scratch_bytes(64, 8, 128) == 0           # one tile
+    assert moe.moe_permute_scratch_bytes(4096, 6, 256) == 24 * 256 * 4
+
+
+def _canonical(name, E=3):
+    base = synth.CONFIGS[name]
+    cfg = synth.LayerConfig(name, E=E, k=2, d=256, I=128, fmt=base.fmt)
+    return cfg, synth.make_experts(cfg, range(E), seed=3)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_mxfp4", "prefill_nvfp4"])
+def test_pack_expert_layout(moe, name):
+    """Blob regions hold the canonical tensors (scales of NVFP4 in the MMA
+    atom layout: row r, block b at ((r/128)*(K/64) + b/4)*512 + (r%32)*16 +
+    ((r/32)%4)*4 + b%4)."""
+    from expert_offload_serving_b200.layer import pack_pool
+    cfg, w = _canonical(name)
+    pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w, range(cfg.E), pin=False).numpy()
+    m = cfg.I * cfg.d
+    for e in range(cfg.E):
+        b = pool[e]
+        if cfg.fmt == "bf16":
+            for n, key in enumerate(("wg", "wu", "wd")):
+                ref = w[key][e].contiguous().view(torch.uint8).numpy().ravel()
+                assert np.array_equal(b[n * 2 * m:(n + 1) * 2 * m], ref)
+            continue
+        for n, key in enumerate(("wg", "wu", "wd")):
+            assert np.array_equal(b[n * m // 2:(n + 1) * m // 2], w[key][e].numpy().ravel())
+        base = 3 * m // 2
+        if cfg.fmt == "mxfp4":
+            for n, key in enumerate(("sg", "su", "sd")):
+                assert np.array_equal(b[base + n * m // 32: base + (n + 1) * m // 32], w[key][e].numpy().ravel())
+        else:
+            for n, key in enumerate(("sg", "su", "sd")):
+                sc = w[key][e].numpy()
+                R, nb = sc.shape
+                K = nb * 16
+                reg = b[base + n * m // 16: base + (n + 1) * m // 16]
+                rr, bb = np.meshgrid(np.arange(R), np.arange(nb), indexing="ij")
+                off = ((rr // 128) * (K // 64) + bb // 4) * 512 + (rr % 32) * 16 + ((rr // 32) % 4) * 4 + bb % 4
+                assert np.array_equal(reg[off], sc)
+            ts = b[base + 3 * m // 16: base + 3 * m // 16 + 12].view(np.float32)
+            assert np.array_equal(ts, w["ts"][e].numpy())
+
+
+def test_cache_planner_matches_oracle_lru(moe):
+    """A plan-only cache handle makes exactly the oracle's LRU decisions on a
+    drifting-bias routing trace, including protected host-computed experts."""
+    cfg = synth.CONFIGS["decode_mxfp4"]
+    trace = synth.make_trace(cfg, 8, steps=60, seed=1)
+    s = moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt)
+    c = moe.MoeCache(s, cfg.n_slots)
+    ref = L.LRUCache(cfg.n_slots, cfg.E)
+    from oracle import moe as M
+    rng = np.random.default_rng(0)
+    total_fills = 0
+    for t, (logits, _) in enumerate(trace):
+        idx, _ = M.route_topk(logits.numpy(), cfg.k)
+        U = sorted(set(idx.ravel().tolist()))
+        host = set(rng.choice(U, len(U) // 4, replace=False).tolist())
+        gpu = [e for e in U if e not in host or ref.resident(e)]
+        got = c.fill(gpu, t, protect=U)
+        hits, fills = ref.step(t, gpu, protect=U)
+        assert got == fills
+        total_fills += len(fills)
+        soe, eos, lu = c.query()
+        assert soe == ref.slot_of_expert and eos == ref.expert_of_slot and lu == ref.last_used
+    assert total_fills > cfg.n_slots            # the trace evicts
+
+
+def test_cache_capacity_error_leaves_state(moe):
+    s = moe.shape(16, 64, 64, "bf16")
+    c = moe.MoeCache(s, 2)
+    c.fill([1, 2], 0)
+    before = c.query()
+    with pytest.raises(moe.MoeError) as ei:
+        c.fill([3, 4, 5], 1)
+    assert ei.value.status == moe.MOE_ERR_CAPACITY
+    assert c.query() == before
