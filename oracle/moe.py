@@ -5,14 +5,14 @@ What the pages fix (titles and sections):
     model", "FreeToken 753b Model Explained": 6 of 256 experts per layer) and
     expert choice is per token (explainx.ai hardware guide, "Decode: decide
     whether to move an expert or compute where it lives").
-  * Misses are split between GPU cache fills and CPU execution, and "the
-    partial CPU and GPU results are merged exactly; this is a scheduling
-    change, not approximate expert skipping" (explainx.ai, same section;
-    ainewsfeed.tech third paragraph: no router modification).  So the layer's
-    result does not depend on where an expert runs, and this oracle is the
-    plain MoE definition, independent of cache state and of the split.
+  * Misses are split between GPU cache fills and CPU execution, and the
+    CPU-side and GPU-side partial sums are added exactly: the split changes
+    the schedule, it skips or approximates no expert (explainx.ai, same
+    section; ainewsfeed.tech third paragraph: the router is left unchanged).
+    So the layer's result does not depend on where an expert runs, and this
+    oracle is the plain MoE definition, independent of cache state and split.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
   * gates = softmax over the k selected logits (equal to the full softmax
     renormalised over the selected experts);
   * order of selected experts: logit descending, ties to the lower index;
@@ -26,7 +26,7 @@ Readings where the pages are silent (each listed in the design doc):
     scale) before the two products, the decision taken in fp32
     (formats.nvfp4_quantize_rows).
 
-Pins (tests/test_oracle_layer.py, test_oracle_route.py): brute force on tiny
+Pins (tests/test_oracle_layer.py): brute force on tiny
 inputs in pure-Python loops; E=1, k=1 equals a dense SwiGLU from torch's silu
 and matmul; token-order invariance; subset A plus complement B equals the
 whole layer; top-k against a sorted() brute force with constructed ties.
