@@ -44,8 +44,12 @@ moe_status current_device(DeviceInfo* out);
 //   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16, row-major).
 //   MXFP4: codes wg [I][d/2], wu [I][d/2], wd [d][I/2] (low nibble = even
 //          element), then E8M0 scales sg [I][d/32], su [I][d/32], sd [d][I/32].
-//   NVFP4: codes as MXFP4; E4M3 scales in tensor-core atoms (see sf_atom_offset)
-//          for each matrix; then 3 fp32 tensor scales (gate, up, down).
+//   NVFP4: codes of W_gu [2I][d/2] -- gate and up rows interleaved in blocks
+//          of 64 (rows 128b..128b+63 = gate rows 64b.., rows 128b+64.. = up
+//          rows 64b..), so one 128-row tensor-core tile holds the gate and up
+//          rows of the same 64 intermediate indices -- then W_d [d][I/2];
+//          E4M3 scales of W_gu and W_d in tensor-core atoms (sf_atom_offset);
+//          then 3 fp32 tensor scales (gate, up, down).  wu/su alias wg/sg.
 struct BlobLayout {
   size_t wg, wu, wd, sg, su, sd, ts, bytes;
 };
@@ -61,20 +65,27 @@ __host__ __device__ inline BlobLayout blob_layout(int fmt, int d, int I) {
     L.wu = o; o = round_up(o + m * 2, 256);
     L.wd = o; o = round_up(o + m * 2, 256);
     L.sg = L.su = L.sd = L.ts = o;
-  } else {
+  } else if (fmt == MOE_W_MXFP4) {
     L.wg = o; o = round_up(o + m / 2, 256);
     L.wu = o; o = round_up(o + m / 2, 256);
     L.wd = o; o = round_up(o + m / 2, 256);
-    size_t per_blk = (fmt == MOE_W_MXFP4) ? 32 : 16;
-    L.sg = o; o = round_up(o + m / per_blk, 256);
-    L.su = o; o = round_up(o + m / per_blk, 256);
-    L.sd = o; o = round_up(o + m / per_blk, 256);
+    L.sg = o; o = round_up(o + m / 32, 256);
+    L.su = o; o = round_up(o + m / 32, 256);
+    L.sd = o; o = round_up(o + m / 32, 256);
     L.ts = o;
-    if (fmt == MOE_W_NVFP4) o = round_up(o + 3 * sizeof(float), 256);
+  } else {
+    L.wg = L.wu = o; o = round_up(o + m, 256);         // W_gu codes
+    L.wd = o; o = round_up(o + m / 2, 256);
+    L.sg = L.su = o; o = round_up(o + m / 8, 256);     // W_gu scales
+    L.sd = o; o = round_up(o + m / 16, 256);
+    L.ts = o; o = round_up(o + 3 * sizeof(float), 256);
   }
   L.bytes = o;
   return L;
 }
+
+// Row of W_gu holding gate row i (up = false) or up row i (up = true).
+__host__ __device__ inline int gu_row(int i, bool up) { return (i >> 6) * 128 + (up ? 64 : 0) + (i & 63); }
 
 // Byte offset of the E4M3 scale of (row r, 16-element block b) of an NVFP4
 // matrix with K columns, in the scale-factor atom layout the FP4 tensor-core

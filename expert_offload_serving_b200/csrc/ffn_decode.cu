@@ -10,17 +10,20 @@
 // Two launches:
 //   phase 1  rows of W_g and W_u -> a[q][i] (fp32 workspace, q = sorted pair)
 //   phase 2  rows of W_d         -> y_perm[q][c]  or  out[t][c] += gate * y
-// A warp tile is 4 weight rows (phase 1: gate rows i, i+1 and up rows i, i+1,
-// so the SwiGLU is formed in registers; phase 2: 4 rows of W_d) against up to
-// 8 token rows at a time.  Lanes split K in 16-byte chunks (8 bf16 or 32 FP4
-// weights): chunk c of a row is read by lane c % 32 with one 128-bit
-// streaming load, dequantised in registers (E2M1 -> f16x2 by cvt, times the
-// E8M0 or E4M3 block scale), and multiplied with the token's activations by
-// packed fp32 FMAs (fma.rn.f32x2).  A reduce-scatter over the warp (31
-// shuffles for 32 values) leaves each lane one finished dot product.
-// Work: every (active expert, warp tile) pair, split into contiguous ranges
-// over all warps of a persistent grid; each CTA first compacts the list of
-// active experts (tokens > 0 and slot >= 0) from the offsets and slot table.
+// Work unit = (active expert, warp tile of 8 weight rows, pass of <= 4 token
+// rows).  Phase 1 tiles hold gate rows i..i+3 and up rows i..i+3, so the
+// SwiGLU is formed in registers; phase 2 tiles hold 8 rows of W_d.
+// Weights are streamed HBM -> shared memory by cp.async.bulk into a 3-stage
+// ring per warp (8 rows x 1 KB per stage, mbarrier-completed), so the number
+// of bytes in flight (up to 128 KB per SM) does not depend on registers.
+// Lanes split each 1 KB row slice in 16-byte chunks (8 bf16 or 32 FP4
+// weights): conflict-free 128-bit shared loads, dequantisation in registers
+// (E2M1 -> f16x2 by cvt, times the E8M0 or E4M3 block scale), packed fp32
+// FMAs (fma.rn.f32x2) against the token activations (read through L1), and a
+// warp reduce-scatter (V-1 shuffles for V partial sums) at the end of a tile.
+// Units are split into contiguous ranges over all warps of a persistent grid;
+// each CTA first builds the list of active experts (tokens > 0, slot >= 0)
+// and their unit counts from the offsets and the slot table.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -28,9 +31,13 @@
 namespace moe {
 namespace {
 
-constexpr int kWarps = 4;    // warps per CTA
-constexpr int kRW = 4;       // weight rows per warp tile
-constexpr int kNTMax = 8;    // token rows per pass
+constexpr int kWarps = 8;                  // warps per CTA (each its own pipeline)
+constexpr int kRW = 8;                     // weight rows per warp tile
+constexpr int kNTMax = 4;                  // token rows per pass
+constexpr int kSlice = 1024;               // bytes of one row per stage
+constexpr int kStages = 3;                 // ring depth per warp
+constexpr int kStageBytes = kRW * kSlice;  // 8 KB
+constexpr size_t kSmemBytes = static_cast<size_t>(kWarps) * kStages * kStageBytes + 1024;
 
 struct FfnParams {
   int E, d, I, T, k, n_slots, fmt;
@@ -49,14 +56,6 @@ struct FfnParams {
 };
 
 // ------------------------------------------------------------ small helpers
-__device__ __forceinline__ uint4 ld_stream(const uint8_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
 __device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
   unsigned long long A, B, C;
   asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
@@ -129,12 +128,13 @@ __device__ int block_scan(int v, int* ws, int* total) {
   return r;
 }
 
-// Reduce-scatter of V partial sums across the warp: afterwards the lane
-// returns the full sum of value index (lane >> (5 - log2 V)).
+// Reduce-scatter of V partial sums across the warp.  After it, the lane holds
+// R = max(1, V/32) full sums in v[0..R-1], for value indices
+// (lane >> (5 - S)) * R + i, S = min(log2 V, 5).
 template <int V>
-__device__ __forceinline__ float warp_reduce_scatter(float (&v)[V], int lane) {
-  constexpr int LOGV = (V >= 32) ? 5 : (V >= 16) ? 4 : (V >= 8) ? 3 : (V >= 4) ? 2 : (V >= 2) ? 1 : 0;
-  static_assert((1 << LOGV) == V && V <= 32, "V must be a power of two <= 32");
+__device__ __forceinline__ void warp_reduce_scatter(float (&v)[V], int lane) {
+  constexpr int LOGV = (V >= 64) ? 6 : (V >= 32) ? 5 : (V >= 16) ? 4 : (V >= 8) ? 3 : (V >= 4) ? 2 : (V >= 2) ? 1 : 0;
+  static_assert((1 << LOGV) == V && V <= 64, "V must be a power of two <= 64");
 #pragma unroll
   for (int st = 0; st < 5; ++st) {
     const int s = 16 >> st;
@@ -153,7 +153,47 @@ __device__ __forceinline__ float warp_reduce_scatter(float (&v)[V], int lane) {
       v[0] += __shfl_xor_sync(kFull, v[0], s);
     }
   }
-  return v[0];
+}
+
+// ------------------------------------------------------------ bulk copies
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+constexpr uint64_t kWaitNs = 2000000000ull;   // a stage that has not landed in 2 s is an error
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255u) == 255u && now_ns() - t0 > kWaitNs) return false;
+  }
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------ weight decode
@@ -243,85 +283,113 @@ struct XF32 {
 // Dot products of kRW weight rows with NT token rows over K.
 //   wrow[r]: byte address of row r's codes; srow/rg: scale region and global
 //   row index of row r (FP4); xrows[t]: row index into xs.
-template <int FMT, int NT, class XS>
-__device__ __forceinline__ void tile_dot(const uint8_t* const (&wrow)[kRW], const uint8_t* const (&sreg)[kRW],
-                                         const int (&rg)[kRW], int K, const XS& xs,
-                                         const int (&xrows)[NT], int lane, float (&res)[kRW * NT]) {
-  using W = Weights<FMT>;
-  float2 acc[kRW][NT];
+// ------------------------------------------------------------ work decomposition
+struct Unit {
+  int e, tile, q0, tb, nt;   // expert, warp tile, first sorted row, first token row of the pass, rows
+};
+
+template <int PHASE>
+__device__ __forceinline__ Unit decode_unit(const FfnParams& P, const int16_t* act, const int32_t* ustart,
+                                            int n_act, long long u) {
+  int lo = 0, hi = n_act;   // last a with ustart[a] <= u
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ustart[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit U;
+  U.e = act[lo];
+  U.q0 = __ldg(P.offsets + U.e);
+  const int ne = __ldg(P.offsets + U.e + 1) - U.q0;
+  const int passes = (ne + kNTMax - 1) / kNTMax;
+  const int local = static_cast<int>(u - ustart[lo]);
+  U.tile = local / passes;
+  const int pass = local % passes;
+  U.tb = pass * kNTMax;
+  U.nt = min(kNTMax, ne - U.tb);
+  return U;
+}
+
+// Byte address of weight row r (0..7) of a unit's tile.
+template <int FMT, int PHASE>
+__device__ __forceinline__ const uint8_t* tile_row(const FfnParams& P, const uint8_t* blob, int tile, int r,
+                                                   size_t row_bytes, int* grow, int* mat) {
+  if (PHASE == 1) {
+    const bool up = r >= 4;
+    const int i = 4 * tile + (r & 3);
+    const int row = (FMT == MOE_W_NVFP4) ? gu_row(i, up) : i;
+    *grow = row;
+    *mat = up ? 1 : 0;
+    return blob + (up ? P.L.wu : P.L.wg) + static_cast<size_t>(row) * row_bytes;
+  }
+  const int row = 8 * tile + r;
+  *grow = row;
+  *mat = 2;
+  return blob + P.L.wd + static_cast<size_t>(row) * row_bytes;
+}
+
+// The warp's pipeline state: items are (unit, slice) in order; item j lives
+// in stage j % kStages and completes phase (j / kStages) & 1 of its barrier.
+struct Pipe {
+  uint8_t* ring;       // kStages * kStageBytes
+  uint64_t* bar;       // kStages
+  long long beg, n_units, next_issue, n_items;
+  int slices;
+  bool ok;
+};
+
+template <int FMT, int PHASE>
+__device__ __forceinline__ void issue_item(const FfnParams& P, const int16_t* act, const int32_t* ustart,
+                                           int n_act, Pipe& pp, size_t row_bytes, int lane) {
+  const long long j = pp.next_issue++;
+  const long long u = pp.beg + j / pp.slices;
+  const int sl = static_cast<int>(j % pp.slices);
+  const int st = static_cast<int>(j % kStages);
+  __syncwarp();
+  if (lane == 0) {
+    const Unit U = decode_unit<PHASE>(P, act, ustart, n_act, u);
+    const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
+    const size_t off = static_cast<size_t>(sl) * kSlice;
+    const uint32_t bytes = static_cast<uint32_t>(min(static_cast<size_t>(kSlice), row_bytes - off));
+    // the stage was last read by this warp's generic loads; order them before the async writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_expect_tx(&pp.bar[st], bytes * kRW);
+    uint8_t* dst = pp.ring + st * kStageBytes;
 #pragma unroll
-  for (int r = 0; r < kRW; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[r][t] = make_float2(0.f, 0.f);
-  const int nc = K / W::EPC;
-#pragma unroll 2
-  for (int c = lane; c < nc; c += 32) {
-    uint4 raw[kRW];
-    typename W::Scale sc[kRW];
-#pragma unroll
-    for (int r = 0; r < kRW; ++r) raw[r] = ld_stream(wrow[r] + static_cast<size_t>(c) * 16);
-#pragma unroll
-    for (int r = 0; r < kRW; ++r) sc[r] = W::scale(sreg[r], rg[r], c, K);
-#pragma unroll
-    for (int m = 0; m < W::SUB; ++m) {
-      float2 w[kRW][4];
-#pragma unroll
-      for (int r = 0; r < kRW; ++r) W::decode(raw[r], m, sc[r], w[r]);
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        float2 xf[4];
-        xs.load(xrows[t], c * W::EPC + 8 * m, xf);
-#pragma unroll
-        for (int r = 0; r < kRW; ++r)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) ffma2(acc[r][t], w[r][j], xf[j]);
-      }
+    for (int r = 0; r < kRW; ++r) {
+      int g, m;
+      const uint8_t* src = tile_row<FMT, PHASE>(P, blob, U.tile, r, row_bytes, &g, &m);
+      bulk_load(dst + r * kSlice, src + off, bytes, &pp.bar[st]);
     }
   }
-#pragma unroll
-  for (int r = 0; r < kRW; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t) res[r * NT + t] = acc[r][t].x + acc[r][t].y;
+  __syncwarp();
 }
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
-// One warp tile of phase 1 (gate/up rows i0, i0+1) or phase 2 (W_d rows
-// 4*tile .. 4*tile+3) for the token rows [tb, tb + nt) of expert e.
+// All slices of one unit with NT token rows per pass.
 template <int FMT, int PHASE, int NT>
-__device__ void run_tile(const FfnParams& P, const uint8_t* blob, int tile, int q0, int tb, int nt,
-                         int lane) {
+__device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* ustart, int n_act, Pipe& pp,
+                         const Unit& U, size_t row_bytes, long long& j, int lane) {
+  using W = Weights<FMT>;
   const int K = (PHASE == 1) ? P.d : P.I;
-  const size_t row_bytes = (FMT == MOE_W_BF16) ? static_cast<size_t>(K) * 2 : static_cast<size_t>(K) / 2;
-  const uint8_t* wrow[kRW];
+  const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
   const uint8_t* sreg[kRW];
-  int rg[kRW];
+  int grow[kRW];
   float tscale[kRW];
   const float* ts = reinterpret_cast<const float*>(blob + P.L.ts);
 #pragma unroll
   for (int r = 0; r < kRW; ++r) {
-    size_t moff, soff;
-    int row, mat;
-    if (PHASE == 1) {
-      mat = (r < 2) ? 0 : 1;            // gate rows first, then up rows
-      row = 2 * tile + (r & 1);
-      moff = mat == 0 ? P.L.wg : P.L.wu;
-      soff = mat == 0 ? P.L.sg : P.L.su;
-    } else {
-      mat = 2;
-      row = 4 * tile + r;
-      moff = P.L.wd;
-      soff = P.L.sd;
-    }
-    wrow[r] = blob + moff + static_cast<size_t>(row) * row_bytes;
-    sreg[r] = blob + soff;
-    rg[r] = row;
+    int g, mat;
+    tile_row<FMT, PHASE>(P, blob, U.tile, r, row_bytes, &g, &mat);
+    grow[r] = g;
+    sreg[r] = blob + (mat == 0 ? P.L.sg : mat == 1 ? P.L.su : P.L.sd);
     tscale[r] = (FMT == MOE_W_NVFP4) ? __ldg(ts + mat) : 1.0f;
   }
   int xrows[NT];
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    const int q = q0 + tb + min(t, nt - 1);   // padding rows repeat the last real one
+    const int q = U.q0 + U.tb + min(t, U.nt - 1);   // padding rows repeat the last real one
     if (PHASE == 1) {
       int p = __ldg(P.perm + q);
       if (p < 0 || p >= P.T * P.k) {
@@ -333,57 +401,108 @@ __device__ void run_tile(const FfnParams& P, const uint8_t* blob, int tile, int 
       xrows[t] = q;
     }
   }
-  float res[kRW * NT];
-  if (PHASE == 1) {
-    XBf16 xs{P.x, P.d};
-    tile_dot<FMT, NT>(wrow, sreg, rg, K, xs, xrows, lane, res);
-  } else {
-    XF32 xs{P.a_ws, P.I};
-    tile_dot<FMT, NT>(wrow, sreg, rg, K, xs, xrows, lane, res);
-  }
-  constexpr int V = kRW * NT;
-  constexpr int LOGV = (V >= 32) ? 5 : (V >= 16) ? 4 : (V >= 8) ? 3 : 2;
-  const float val = warp_reduce_scatter<V>(res, lane);
-  const int vi = lane >> (5 - LOGV);
-  const int r = vi / NT, t = vi % NT;
-  const bool writer = (lane & ((1 << (5 - LOGV)) - 1)) == 0;
-  if (PHASE == 1) {
-    // lanes < 16 hold gate rows, lane ^ 16 the up row of the same (i, token)
-    const float other = __shfl_xor_sync(kFull, val, 16);
-    if (writer && lane < 16 && t < nt) {
-      const float h = val * tscale[0];
-      const float u = other * tscale[2];
-      const int q = q0 + tb + t;
-      P.a_ws[static_cast<size_t>(q) * P.I + 2 * tile + r] = silu(h) * u;
+  float2 acc[kRW][NT];
+#pragma unroll
+  for (int r = 0; r < kRW; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[r][t] = make_float2(0.f, 0.f);
+
+  for (int sl = 0; sl < pp.slices; ++sl, ++j) {
+    if (pp.next_issue < pp.n_items) issue_item<FMT, PHASE>(P, act, ustart, n_act, pp, row_bytes, lane);
+    const int st = static_cast<int>(j % kStages);
+    if (!mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1))) {
+      pp.ok = false;
+      return;
     }
-  } else if (writer && t < nt) {
-    const int q = q0 + tb + t;
-    const int row = 4 * tile + r;
-    const float y = val * tscale[0];
-    if (P.y_perm != nullptr) {
-      P.y_perm[static_cast<size_t>(q) * P.d + row] = y;
-    } else {
-      const int p = __ldg(P.perm + q);
-      if (p >= 0 && p < P.T * P.k)
-        atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * y);
+    const uint8_t* stage = pp.ring + st * kStageBytes;
+    const int valid = static_cast<int>(min(static_cast<size_t>(kSlice), row_bytes - static_cast<size_t>(sl) * kSlice));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = lane + 32 * h;                 // 16-byte chunk inside the 1 KB slice
+      if (c * 16 >= valid) break;
+      const int k0 = (sl * kSlice + c * 16) * W::EPC / 16;   // first K element of the chunk
+      uint4 raw[kRW];
+      typename W::Scale sc[kRW];
+#pragma unroll
+      for (int r = 0; r < kRW; ++r) {
+        raw[r] = *reinterpret_cast<const uint4*>(stage + r * kSlice + c * 16);
+        sc[r] = W::scale(sreg[r], grow[r], k0 / W::EPC, K);
+      }
+#pragma unroll
+      for (int m = 0; m < W::SUB; ++m) {
+        float2 w[kRW][4];
+#pragma unroll
+        for (int r = 0; r < kRW; ++r) W::decode(raw[r], m, sc[r], w[r]);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          float2 xf[4];
+          if (PHASE == 1) XBf16{P.x, P.d}.load(xrows[t], k0 + 8 * m, xf);
+          else XF32{P.a_ws, P.I}.load(xrows[t], k0 + 8 * m, xf);
+#pragma unroll
+          for (int r = 0; r < kRW; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ffma2(acc[r][t], w[r][q], xf[q]);
+        }
+      }
+    }
+  }
+  // reduce over the warp: value index v = r * NT + t
+  constexpr int V = kRW * NT;
+  constexpr int LOGV = (V >= 64) ? 6 : (V >= 32) ? 5 : (V >= 16) ? 4 : (V >= 8) ? 3 : 2;
+  constexpr int S = LOGV < 5 ? LOGV : 5;
+  constexpr int R = (V >> S);
+  float v[V];
+#pragma unroll
+  for (int r = 0; r < kRW; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) v[r * NT + t] = acc[r][t].x + acc[r][t].y;
+  warp_reduce_scatter<V>(v, lane);
+  const bool writer = (lane & ((1 << (5 - S)) - 1)) == 0;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int vi = (lane >> (5 - S)) * R + i;
+    const int r = vi / NT, t = vi % NT;
+    if (PHASE == 1) {
+      // lanes < 16 hold gate rows (r < 4); lane ^ 16 holds the up row of the same (i, token)
+      const float other = __shfl_xor_sync(kFull, v[i], 16);
+      if (writer && lane < 16 && t < U.nt) {
+        const float hh = v[i] * tscale[r];
+        const float uu = other * tscale[r + 4];
+        P.a_ws[static_cast<size_t>(U.q0 + U.tb + t) * P.I + 4 * U.tile + r] = silu(hh) * uu;
+      }
+    } else if (writer && t < U.nt) {
+      const int q = U.q0 + U.tb + t;
+      const int row = 8 * U.tile + r;
+      const float y = v[i] * tscale[r];
+      if (P.y_perm != nullptr) {
+        P.y_perm[static_cast<size_t>(q) * P.d + row] = y;
+      } else {
+        const int p = __ldg(P.perm + q);
+        if (p >= 0 && p < P.T * P.k)
+          atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * y);
+      }
     }
   }
 }
 
 template <int FMT, int PHASE>
-__global__ void __launch_bounds__(kWarps * 32) ffn_decode_kernel(FfnParams P) {
+__global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ int16_t s_act[1024];
+  __shared__ int32_t s_ustart[1025];
   __shared__ int s_ws[36];
+  __shared__ __align__(8) uint64_t s_bar[kWarps * kStages];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  // compact the active experts (tokens > 0, resident) in expert order
+  const int tiles_per_e = (PHASE == 1) ? P.I / 4 : P.d / kRW;
+  // active experts (tokens > 0, resident) in expert order, with their unit counts
   const int per = (P.E + blockDim.x - 1) / blockDim.x;
   const int e0 = threadIdx.x * per;
-  int cnt = 0;
-  uint32_t mask = 0;   // per <= 8
+  int cnt = 0, units = 0;
+  uint32_t mask = 0;   // per <= 4
   const int npairs = P.T * P.k;
-  for (int j = 0; j < per; ++j) {
-    const int e = e0 + j;
+  for (int jx = 0; jx < per; ++jx) {
+    const int e = e0 + jx;
     if (e >= P.E) break;
     const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
     if (b <= a) continue;
@@ -397,58 +516,88 @@ __global__ void __launch_bounds__(kWarps * 32) ffn_decode_kernel(FfnParams P) {
       report(P.status, MOE_ERR_DEVICE);
       continue;
     }
-    mask |= 1u << j;
+    mask |= 1u << jx;
     ++cnt;
   }
   int n_act;
   int pos = block_scan(cnt, s_ws, &n_act);
-  for (int j = 0; j < per; ++j)
-    if (mask & (1u << j)) s_act[pos++] = static_cast<int16_t>(e0 + j);
+  for (int jx = 0; jx < per; ++jx)
+    if (mask & (1u << jx)) {
+      const int e = e0 + jx;
+      const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
+      s_act[pos++] = static_cast<int16_t>(e);
+      units += tiles_per_e * ((ne + kNTMax - 1) / kNTMax);
+    }
+  int total_units;
+  int ustart = block_scan(units, s_ws, &total_units);
+  pos -= cnt;
+  for (int jx = 0; jx < per; ++jx)
+    if (mask & (1u << jx)) {
+      const int e = e0 + jx;
+      const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
+      s_ustart[pos++] = ustart;
+      ustart += tiles_per_e * ((ne + kNTMax - 1) / kNTMax);
+    }
+  if (threadIdx.x < kWarps * kStages) mbar_init(&s_bar[threadIdx.x], 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
 
-  const int tiles_per_e = (PHASE == 1) ? P.I / 2 : P.d / kRW;
-  const long long total = static_cast<long long>(n_act) * tiles_per_e;
+  const int K = (PHASE == 1) ? P.d : P.I;
+  const size_t row_bytes = (FMT == MOE_W_BF16) ? static_cast<size_t>(K) * 2 : static_cast<size_t>(K) / 2;
   const long long nw = static_cast<long long>(gridDim.x) * kWarps;
   const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
-  const long long beg = total * gw / nw, end = total * (gw + 1) / nw;
-  for (long long w = beg; w < end; ++w) {
-    const int e = s_act[w / tiles_per_e];
-    const int tile = static_cast<int>(w % tiles_per_e);
-    const int q0 = __ldg(P.offsets + e);
-    const int ne = __ldg(P.offsets + e + 1) - q0;
-    const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + e)) * P.blob_bytes;
-    for (int tb = 0; tb < ne; tb += kNTMax) {
-      const int nt = min(kNTMax, ne - tb);
-      if (nt == 1) run_tile<FMT, PHASE, 1>(P, blob, tile, q0, tb, nt, lane);
-      else if (nt == 2) run_tile<FMT, PHASE, 2>(P, blob, tile, q0, tb, nt, lane);
-      else if (nt <= 4) run_tile<FMT, PHASE, 4>(P, blob, tile, q0, tb, nt, lane);
-      else run_tile<FMT, PHASE, 8>(P, blob, tile, q0, tb, nt, lane);
+  Pipe pp;
+  pp.ring = smem_raw + static_cast<size_t>(warp) * kStages * kStageBytes;
+  pp.bar = s_bar + warp * kStages;
+  pp.beg = total_units * gw / nw;
+  pp.n_units = total_units * (gw + 1) / nw - pp.beg;
+  pp.slices = static_cast<int>((row_bytes + kSlice - 1) / kSlice);
+  pp.n_items = pp.n_units * pp.slices;
+  pp.next_issue = 0;
+  pp.ok = true;
+  // prime the ring with kStages - 1 items
+  for (int i = 0; i < kStages - 1 && pp.next_issue < pp.n_items; ++i)
+    issue_item<FMT, PHASE>(P, s_act, s_ustart, n_act, pp, row_bytes, lane);
+  long long j = 0;
+  for (long long u = 0; u < pp.n_units && pp.ok; ++u) {
+    const Unit U = decode_unit<PHASE>(P, s_act, s_ustart, n_act, pp.beg + u);
+    if (U.nt == 1) run_unit<FMT, PHASE, 1>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
+    else if (U.nt == 2) run_unit<FMT, PHASE, 2>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
+    else run_unit<FMT, PHASE, 4>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
+  }
+  if (!pp.ok) {
+    report(P.status, MOE_ERR_TIMEOUT);
+  }
+  // every issued copy has landed before the CTA leaves (bounded)
+  for (long long i = j; i < pp.next_issue; ++i) {
+    const uint64_t t0 = now_ns();
+    while (!mbar_try(&pp.bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1)) && now_ns() - t0 <= kWaitNs) {
     }
   }
 }
 
 template <int FMT, int PHASE>
 moe_status launch_phase(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
-  static int occ[64] = {};
-  if (occ[dev.id] == 0) {
-    int o = 0;
-    MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, ffn_decode_kernel<FMT, PHASE>,
-                                                               kWarps * 32, 0));
-    occ[dev.id] = o > 0 ? o : 1;
+  static bool attr[64] = {};
+  if (!attr[dev.id]) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_decode_kernel<FMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(kSmemBytes)));
+    attr[dev.id] = true;
   }
-  const int tiles_per_e = (PHASE == 1) ? P.I / 2 : P.d / kRW;
-  const long long most = static_cast<long long>(min(P.E, P.T * P.k)) * tiles_per_e;
+  const int tiles_per_e = (PHASE == 1) ? P.I / 4 : P.d / kRW;
+  const long long most = static_cast<long long>(min(P.E, P.T * P.k)) * tiles_per_e *
+                         ((P.T * P.k + kNTMax - 1) / kNTMax);
   long long blocks = (most + kWarps - 1) / kWarps;
-  const long long cap = static_cast<long long>(dev.sm_count) * occ[dev.id];
-  if (blocks > cap) blocks = cap;
+  if (blocks > dev.sm_count) blocks = dev.sm_count;
   if (blocks < 1) blocks = 1;
-  ffn_decode_kernel<FMT, PHASE><<<static_cast<int>(blocks), kWarps * 32, 0, s>>>(P);
+  ffn_decode_kernel<FMT, PHASE><<<static_cast<int>(blocks), kWarps * 32, kSmemBytes, s>>>(P);
   MOE_LAUNCH_CHECK("ffn_decode_kernel");
   return MOE_OK;
 }
 
 template <int FMT>
 moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
+  if (kSmemBytes > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "needs %zu bytes of shared memory", kSmemBytes);
   moe_status st = launch_phase<FMT, 1>(P, dev, s);
   if (st != MOE_OK) return st;
   return launch_phase<FMT, 2>(P, dev, s);

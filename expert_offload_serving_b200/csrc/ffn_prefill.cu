@@ -1,19 +1,801 @@
-// Step 3 (FP4 tensor-core path, MOE_FFN_ACT_NVFP4): not built yet.
+// Step 3 (FP4 tensor-core path, MOE_FFN_ACT_NVFP4): the grouped SwiGLU expert
+// FFN as two block-scaled FP4 GEMMs on the 5th-generation tensor cores.
+//
+// In prefill many tokens of a layer reach nearly every expert, so each
+// expert's FFN is a dense contraction over a group of ~100 token rows
+// (ainewsfeed.tech, second paragraph; explainx.ai hardware guide, "Prefill:
+// load almost every expert without idling the GPU").  The pages give no
+// kernel; on B200 the contraction belongs on tcgen05 with NVFP4 operands.
+//
+// Launches (one stream):
+//   quant_x      x rows, gathered in expert order, -> NVFP4 (E2M1 codes, one
+//                E4M3 scale per 16, unit tensor scale) in an expert-padded
+//                layout: expert e's rows start at a multiple of 128, so every
+//                128-row B tile and its scale atoms align.
+//   gemm<1>      D[128 x N] = W_gu tile (64 gate + 64 up rows) x X^T over K = d;
+//                epilogue: a = silu(g_g * D_gate) * (g_u * D_up), requantised
+//                to NVFP4 into the padded A matrix.
+//   gemm<2>      D = W_d tile (128 rows of d) x A^T over K = I; epilogue:
+//                out[t][row] += gate * g_d * D  (red.global.add, the combine).
+// gemm is a persistent kernel, one CTA per SM, warp-specialised:
+//   warp 0      TMA producer: 128x128-byte A and B tiles (SWIZZLE_128B, no
+//               multicast) plus the 2 KB scale-atom slices by bulk copy, into
+//               a 5-stage ring guarded by mbarriers;
+//   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp of the scale
+//               atoms into TMEM, then 4 tcgen05.mma kind::mxf4nvf4 block16
+//               (K = 64 each) into one of two TMEM accumulators;
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp its 32
+//               TMEM lanes), overlapped with the next tile's main loop.
+// Every wait is bounded; on expiry the CTA records MOE_ERR_TIMEOUT in the
+// status word, stops issuing, drains what it issued and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace moe {
+namespace {
 
-size_t prefill_workspace_bytes(moe_shape s, int T, int k) {
-  (void)s;
-  (void)T;
-  (void)k;
-  return 0;
+constexpr int BM = 128;                 // weight rows per tile
+constexpr int BN = 128;                 // token rows per tile (max MMA N used)
+constexpr int BKB = 128;                // bytes of K per stage (256 FP4 elements)
+constexpr int STAGES = 5;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN * BKB;       // 16 KB
+constexpr int SF_BYTES = 2048;          // 4 atoms of 128 rows x 4 scales
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr int EPI_BYTES = 16 * 128 * 4 + 2 * 128 * 4;   // transposed 16-column slab + column info
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = 128;           // per accumulator buffer
+constexpr int SFA_COL = 256, SFB_COL = 272;
+constexpr int THREADS = 192;
+constexpr uint64_t kWaitNs = 2000000000ull;   // every wait gives up after 2 s
+
+struct GemmParams {
+  int E, d, I, T, k, n_slots, max_chunks;
+  const int32_t* offsets;
+  const int32_t* perm;
+  const int32_t* slot;
+  const float* gate;
+  const uint8_t* pool;       // slot pool
+  size_t blob_bytes;
+  BlobLayout L;
+  const uint8_t* act_sf;     // scale atoms of the B operand
+  uint8_t* aq;               // gemm<1> output codes  [rows][I/2]
+  uint8_t* aq_sf;            // gemm<1> output scale atoms
+  float* out;                // gemm<2> output [T][d]
+  int32_t* status;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-moe_status launch_ffn_prefill(moe_shape, const void*, int, int, const int32_t*, const int32_t*,
-                              const int32_t*, const void*, int, const float*, float*, void*, int32_t*,
-                              const DeviceInfo&, cudaStream_t) {
-  return fail(MOE_ERR_UNSUPPORTED, "the NVFP4 tensor-core path is not built in this version");
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: false when 2 s pass (or another role gave up first).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255u) == 255u) {
+      if (*abort_flag) return false;
+      if (now_ns() - t0 > kWaitNs) return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (teardown drains).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try(bar, parity) && now_ns() - t0 <= kWaitNs) {
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{ .reg .pred p; .reg .b32 r; elect.sync r|p, 0xffffffff; selp.u32 %0, 1, 0, p; }"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand tile, SWIZZLE_128B: rows of 128 bytes, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);   // start address
+  d |= static_cast<uint64_t>(1) << 16;                   // leading byte offset (unused, 16 B)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;           // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                   // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;                   // layout: SWIZZLE_128B
+  return d;
+}
+
+// One scale-factor atom (32 rows x 16 bytes, contiguous): no swizzle,
+// 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Instruction descriptor: kind::mxf4nvf4, A and B E2M1 (packed), K-major,
+// UE4M3 scales, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_fp4(int n) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t tmem, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %6, 0; "
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p; }" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// ------------------------------------------------------------------ NVFP4 quantisation
+// 16 values -> E4M3 scale byte s = e4m3_rn_satfinite(amax / 6) and 8 code
+// bytes q_i = e2m1_rn_satfinite(v_i / s) (IEEE fp32 division; all zero when s
+// is 0).  Element 2i goes to the low nibble.
+__device__ __forceinline__ uint32_t e4m3_byte(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xffu;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t byte) {
+  uint32_t h;
+  asm("{ .reg .b16 s; cvt.u16.u32 s, %1; cvt.rn.f16x2.e4m3x2 %0, s; }" : "=r"(h) : "r"(byte));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xffffu)));
+}
+
+__device__ __forceinline__ uint32_t e2m1x2_byte(float lo, float hi) {
+  uint32_t r;
+  asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u32.u8 %0, b; }" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// codes of 8 values (already divided by the scale) -> 4 bytes
+__device__ __forceinline__ uint32_t pack8(const float (&q)[8]) {
+  return e2m1x2_byte(q[0], q[1]) | (e2m1x2_byte(q[2], q[3]) << 8) | (e2m1x2_byte(q[4], q[5]) << 16) |
+         (e2m1x2_byte(q[6], q[7]) << 24);
+}
+
+// ------------------------------------------------------------------ shared prologue
+// Chunks: 128-row pieces of each evaluated expert's group (tokens > 0,
+// slot >= 0).  chunk_start[e] = exclusive prefix of the chunk counts; chunk c
+// occupies padded rows [128 c, 128 c + 128).
+__device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot, int E,
+                            int n_pairs, int n_slots, int32_t* chunk_start, int* ws, int32_t* status) {
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int cnt = 0;
+  for (int j = 0; j < per; ++j) {
+    const int e = e0 + j;
+    if (e >= E) break;
+    const int a = offsets[e], b = offsets[e + 1];
+    int c = 0;
+    if (b > a) {
+      if (a < 0 || b > n_pairs) {
+        report(status, MOE_ERR_DEVICE);
+      } else {
+        const int s = slot[e];
+        if (s >= n_slots) report(status, MOE_ERR_DEVICE);
+        else if (s >= 0) c = (b - a + BN - 1) / BN;
+      }
+    }
+    cnt += c;
+  }
+  // block exclusive scan of cnt
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) ws[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    const int w = (lane < nw) ? ws[lane] : 0;
+    int s = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, s, o);
+      if (lane >= o) s += y;
+    }
+    ws[lane] = s - w;
+    if (lane == 31) ws[32] = s;
+  }
+  __syncthreads();
+  int run = ws[warp] + x - cnt;
+  for (int j = 0; j < per; ++j) {
+    const int e = e0 + j;
+    if (e >= E) break;
+    chunk_start[e] = run;
+    const int a = offsets[e], b = offsets[e + 1];
+    if (b > a && a >= 0 && b <= n_pairs) {
+      const int s = slot[e];
+      if (s >= 0 && s < n_slots) run += (b - a + BN - 1) / BN;
+    }
+  }
+  const int total = ws[32];
+  if (threadIdx.x == 0) chunk_start[E] = total;
+  __syncthreads();
+  return total;
+}
+
+// expert of chunk c: the last e with chunk_start[e] <= c
+__device__ __forceinline__ int chunk_expert(const int32_t* chunk_start, int E, int c) {
+  int lo = 0, hi = E;   // invariant: chunk_start[lo] <= c < chunk_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (chunk_start[mid] <= c) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------------------ quant_x
+// One warp per real token row of a chunk: NVFP4 codes into xq[128 c + r][d/2]
+// and scale bytes into the atom layout of the padded matrix.
+__global__ void __launch_bounds__(256) quant_x_kernel(const uint16_t* __restrict__ x, int d, int T, int k,
+                                                     int E, int n_slots, const int32_t* __restrict__ offsets,
+                                                     const int32_t* __restrict__ perm,
+                                                     const int32_t* __restrict__ slot, uint8_t* __restrict__ xq,
+                                                     uint8_t* __restrict__ xsf, int32_t* status) {
+  __shared__ int32_t chunk_start[1025];
+  __shared__ int ws[36];
+  const int n_pairs = T * k;
+  const int n_chunks = build_chunks(offsets, slot, E, n_pairs, n_slots, chunk_start, ws, status);
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long rows = static_cast<long long>(n_chunks) * BN;
+  for (long long w = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); w < rows;
+       w += static_cast<long long>(gridDim.x) * warps) {
+    const int c = static_cast<int>(w / BN), r = static_cast<int>(w % BN);
+    const int e = chunk_expert(chunk_start, E, c);
+    const int q = offsets[e] + (c - chunk_start[e]) * BN + r;
+    if (q >= offsets[e + 1]) continue;                      // padding row: never read back
+    int p = perm[q];
+    if (p < 0 || p >= n_pairs) {
+      report(status, MOE_ERR_DEVICE);
+      p = 0;
+    }
+    const uint16_t* xr = x + static_cast<size_t>(p / k) * d;
+    const int prow = c * BN + r;
+    const int nb = d / 16;
+    for (int b = lane; b < nb; b += 32) {
+      const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
+      const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b + 8));
+      const uint32_t w32[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[2 * j] = __uint_as_float(w32[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w32[j] & 0xffff0000u);
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      const uint32_t sb = e4m3_byte(__fdiv_rn(amax, 6.0f));
+      const float s = e4m3_value(sb);
+      float q0[8], q1[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        q0[j] = (s > 0.f) ? __fdiv_rn(v[j], s) : 0.f;
+        q1[j] = (s > 0.f) ? __fdiv_rn(v[8 + j], s) : 0.f;
+      }
+      uint2 codes = make_uint2(pack8(q0), pack8(q1));
+      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(prow) * (d / 2) + 8 * b) = codes;
+      xsf[sf_atom_offset(prow, b, d)] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ the GEMMs
+template <int PHASE>
+__global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_constant__ CUtensorMap tm_w,
+                                                              const __grid_constant__ CUtensorMap tm_act,
+                                                              GemmParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  int32_t* col_t = reinterpret_cast<int32_t*>(epi + 16 * 128);
+  float* col_g = reinterpret_cast<float*>(col_t + 128);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
+  uint64_t* full = bars;                   // [STAGES]
+  uint64_t* empty = bars + STAGES;         // [STAGES]
+  uint64_t* tfull = bars + 2 * STAGES;     // [2]
+  uint64_t* tempty = bars + 2 * STAGES + 2;// [2]
+  uint64_t* drain = bars + 2 * STAGES + 4; // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int32_t* chunk_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E+1]
+  __shared__ int ws[36];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = (PHASE == 1) ? P.d : P.I;
+  const int KS = K / (2 * BKB);                 // stages of 256 elements
+  const int MT = (PHASE == 1) ? (2 * P.I) / BM : P.d / BM;
+  const int n_pairs = P.T * P.k;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  const int n_chunks = build_chunks(P.offsets, P.slot, P.E, n_pairs, P.n_slots, chunk_start, ws, P.status);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int n_units = min(n_chunks, P.max_chunks) * MT;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int c = u / MT, m = u % MT;
+      const int e = chunk_expert(chunk_start, P.E, c);
+      const int sl = P.slot[e];
+      const uint8_t* sfa_src = P.pool + static_cast<size_t>(sl) * P.blob_bytes +
+                               (PHASE == 1 ? P.L.sg : P.L.sd) + static_cast<size_t>(m) * (K / 64) * 512;
+      const uint8_t* sfb_src = P.act_sf + static_cast<size_t>(c) * (K / 64) * 512;
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (elect_one()) {
+          uint8_t* sA = stage_base + stage * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          uint8_t* sSFA = sB + B_BYTES;
+          uint8_t* sSFB = sSFA + SF_BYTES;
+          mbar_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl);
+          tma_load_2d(sB, &tm_act, &full[stage], ks * BKB, c * BN);
+          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage]);
+          bulk_load(sSFB, sfb_src + ks * SF_BYTES, SF_BYTES, &full[stage]);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // drain: wait (bounded) until the copies last issued into the ring have
+    // landed, so none is in flight when the CTA exits
+    const int outstanding = issued < STAGES ? issued : STAGES;
+    int s = stage;
+    uint32_t ph = phase;
+    for (int i = 0; i < outstanding; ++i) {
+      if (--s < 0) {
+        s = STAGES - 1;
+        ph ^= 1u;
+      }
+      mbar_drain(&full[s], ph);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+      const int c = u / MT;
+      const int e = chunk_expert(chunk_start, P.E, c);
+      const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
+      const int nvalid = min(BN, P.offsets[e + 1] - row0);
+      const int nmma = (nvalid + 15) & ~15;
+      const uint32_t idesc = idesc_fp4(nmma);
+      const int acc = it & 1;
+      if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + acc * ACC_COLS;
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          uint8_t* sA = stage_base + stage * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          uint8_t* sSFA = sB + B_BYTES;
+          uint8_t* sSFB = sSFA + SF_BYTES;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tc_cp_sf(tmem + SFA_COL + 4 * j, desc_sf(smem_u32(sSFA + 512 * j)));
+            tc_cp_sf(tmem + SFB_COL + 4 * j, desc_sf(smem_u32(sSFB + 512 * j)));
+          }
+          const uint64_t da = desc_sw128(smem_u32(sA));
+          const uint64_t db = desc_sw128(smem_u32(sB));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc_mma_fp4(d_tmem, da + 2 * j, db + 2 * j, idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 4 * j,
+                       (ks > 0 || j > 0) ? 1u : 0u);
+          tc_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&tfull[acc]);
+      __syncwarp();
+    }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // every MMA this thread issued has completed before TMEM is released
+    if (elect_one()) tc_commit(drain);
+    __syncwarp();
+    mbar_drain(drain, 0);
+  } else {
+    // ---------------------------------------------------------- epilogue (warps 2..5)
+    const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
+    const int et = (warp - 2) * 32 + lane;      // 0..127 within the epilogue group
+    const float* ts = nullptr;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+      const int c = u / MT, m = u % MT;
+      const int e = chunk_expert(chunk_start, P.E, c);
+      const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
+      const int nvalid = min(BN, P.offsets[e + 1] - row0);
+      const uint8_t* blob = P.pool + static_cast<size_t>(P.slot[e]) * P.blob_bytes;
+      ts = reinterpret_cast<const float*>(blob + P.L.ts);
+      const int acc = it & 1;
+      if (PHASE == 2) {
+        // column c <-> pair at sorted position row0 + c: its token and gate
+        named_sync(1, 128);               // the previous tile's readers are done
+        if (et < nvalid) {
+          const int p = P.perm[row0 + et];
+          const bool good = p >= 0 && p < n_pairs;
+          if (!good) report(P.status, MOE_ERR_DEVICE);
+          col_t[et] = good ? p / P.k : -1;
+          col_g[et] = good ? P.gate[p] : 0.f;
+        }
+      }
+      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS;
+      if (PHASE == 2) named_sync(1, 128);
+      const float g_mat = (PHASE == 1) ? 0.f : __ldg(ts + 2);
+      const float g_gate = (PHASE == 1) ? __ldg(ts + 0) : 0.f, g_up = (PHASE == 1) ? __ldg(ts + 1) : 0.f;
+      for (int cc = 0; cc < nvalid; cc += 16) {
+        float v[16];
+        tmem_ld16(tbase + cc, v);
+        if (PHASE == 2) {
+          const int row = m * BM + 32 * quad + lane;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = cc + j;
+            if (col < nvalid) {
+              const int t = col_t[col];
+              if (t >= 0)
+                atomicAdd(P.out + static_cast<size_t>(t) * P.d + row, col_g[col] * (g_mat * v[j]));
+            }
+          }
+        } else {
+          // transpose the 16-column slab through shared memory: epi[col][row]
+#pragma unroll
+          for (int j = 0; j < 16; ++j) epi[j * 128 + 32 * quad + lane] = v[j];
+          named_sync(1, 128);
+          // item: column cl, 16-block b of the 64 intermediate indices, half h
+          const int cl = et >> 3, b = (et >> 1) & 3, h = et & 1;
+          const int col = cc + cl;
+          float a[8];
+          float amax = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int il = 16 * b + 8 * h + j;
+            const float hg = epi[cl * 128 + il] * g_gate;
+            const float hu = epi[cl * 128 + 64 + il] * g_up;
+            a[j] = __fdiv_rn(hg, 1.0f + expf(-hg)) * hu;
+            amax = fmaxf(amax, fabsf(a[j]));
+          }
+          amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+          const uint32_t sb = e4m3_byte(__fdiv_rn(amax, 6.0f));
+          const float s = e4m3_value(sb);
+          float q[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) q[j] = (s > 0.f) ? __fdiv_rn(a[j], s) : 0.f;
+          const uint32_t codes = pack8(q);
+          if (col < nvalid) {
+            const int prow = c * BN + col;
+            const int i0 = m * 64;                       // first intermediate index of the tile
+            *reinterpret_cast<uint32_t*>(P.aq + static_cast<size_t>(prow) * (P.I / 2) + (i0 + 16 * b + 8 * h) / 2) =
+                codes;
+            if (h == 0) P.aq_sf[sf_atom_offset(prow, i0 / 16 + b, P.I)] = static_cast<uint8_t>(sb);
+          }
+          named_sync(1, 128);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Byte-element tensor map, box 128 (bytes of K) x 128 rows, 128-byte swizzle.
+moe_status make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t gdim[3], gstr[2];
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(BKB), 128u, 1u}, estr[3] = {1u, 1u, 1u};
+  for (int i = 0; i < rank; ++i) gdim[i] = dims[i];
+  for (int i = 0; i < rank - 1; ++i) gstr[i] = strides[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), gdim, gstr, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MOE_OK;
+}
+
+struct PrefillWs {
+  size_t rows;            // padded row capacity (multiple of 128)
+  size_t xq, xsf, aq, asf, bytes;
+};
+
+PrefillWs prefill_ws(moe_shape s, int T, int k) {
+  PrefillWs w{};
+  const size_t n = static_cast<size_t>(T) * k;
+  const size_t act = n < static_cast<size_t>(s.E) ? n : static_cast<size_t>(s.E);
+  w.rows = round_up(n + act * (BN - 1), BN);
+  size_t o = 0;
+  w.xq = o; o = round_up(o + w.rows * (s.d / 2), 1024);
+  w.xsf = o; o = round_up(o + w.rows * (s.d / 16), 1024);
+  w.aq = o; o = round_up(o + w.rows * (s.I / 2), 1024);
+  w.asf = o; o = round_up(o + w.rows * (s.I / 16), 1024);
+  w.bytes = o;
+  return w;
+}
+
+constexpr size_t kGemmSmem = STAGES * STAGE_BYTES + EPI_BYTES + 256 + 1025 * 4 + 1024;
+static_assert((2 * STAGES + 5) * 8 + 16 <= 256, "barrier area");
+
+}  // namespace
+
+size_t prefill_workspace_bytes(moe_shape s, int T, int k) { return prefill_ws(s, T, k).bytes; }
+
+moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
+                              const int32_t* perm, const int32_t* slot, const void* pool, int n_slots,
+                              const float* gate, float* out, void* ws_ptr, int32_t* status,
+                              const DeviceInfo& dev, cudaStream_t stream) {
+  MOE_REQUIRE(s.d % 256 == 0 && s.I % 256 == 0, "the FP4 tensor-core path needs d, I multiples of 256");
+  if (kGemmSmem > dev.smem_optin)
+    return fail(MOE_ERR_UNSUPPORTED, "needs %zu bytes of shared memory per CTA", kGemmSmem);
+  const PrefillWs w = prefill_ws(s, T, k);
+  uint8_t* base = static_cast<uint8_t*>(ws_ptr);
+  uint8_t* xq = base + w.xq;
+  uint8_t* xsf = base + w.xsf;
+  uint8_t* aq = base + w.aq;
+  uint8_t* asf = base + w.asf;
+  const BlobLayout L = blob_layout(s.fmt, s.d, s.I);
+  const int max_chunks = static_cast<int>(w.rows / BN);
+
+  static bool attr_done[64] = {};
+  if (!attr_done[dev.id]) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(gemm_fp4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(kGemmSmem)));
+    MOE_CUDA_TRY(cudaFuncSetAttribute(gemm_fp4_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(kGemmSmem)));
+    attr_done[dev.id] = true;
+  }
+
+  // tensor maps: weights [slot][rows][K bytes], activations [rows][K bytes]
+  CUtensorMap tm_gu, tm_d, tm_x, tm_a;
+  const uint8_t* pool8 = static_cast<const uint8_t*>(pool);
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.d / 2), static_cast<uint64_t>(2 * s.I),
+                              static_cast<uint64_t>(n_slots)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.d / 2), L.bytes};
+    moe_status st = make_map(&tm_gu, pool8 + L.wg, 3, dims, str);
+    if (st != MOE_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.I / 2), static_cast<uint64_t>(s.d),
+                              static_cast<uint64_t>(n_slots)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.I / 2), L.bytes};
+    moe_status st = make_map(&tm_d, pool8 + L.wd, 3, dims, str);
+    if (st != MOE_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.d / 2), w.rows};
+    const uint64_t str[1] = {static_cast<uint64_t>(s.d / 2)};
+    moe_status st = make_map(&tm_x, xq, 2, dims, str);
+    if (st != MOE_OK) return st;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.I / 2), w.rows};
+    const uint64_t str[1] = {static_cast<uint64_t>(s.I / 2)};
+    moe_status st = make_map(&tm_a, aq, 2, dims, str);
+    if (st != MOE_OK) return st;
+  }
+
+  {
+    const long long rows = static_cast<long long>(w.rows);
+    long long blocks = (rows + 7) / 8;
+    const long long cap = static_cast<long long>(dev.sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    quant_x_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), s.d, T, k,
+                                                                 s.E, n_slots, offsets, perm, slot, xq, xsf,
+                                                                 status);
+    MOE_LAUNCH_CHECK("quant_x_kernel");
+  }
+  GemmParams P{};
+  P.E = s.E;
+  P.d = s.d;
+  P.I = s.I;
+  P.T = T;
+  P.k = k;
+  P.n_slots = n_slots;
+  P.max_chunks = max_chunks;
+  P.offsets = offsets;
+  P.perm = perm;
+  P.slot = slot;
+  P.gate = gate;
+  P.pool = pool8;
+  P.blob_bytes = L.bytes;
+  P.L = L;
+  P.status = status;
+  P.out = out;
+  const int grid = dev.sm_count;
+  P.act_sf = xsf;
+  P.aq = aq;
+  P.aq_sf = asf;
+  gemm_fp4_kernel<1><<<grid, THREADS, kGemmSmem, stream>>>(tm_gu, tm_x, P);
+  MOE_LAUNCH_CHECK("gemm_fp4_kernel<1>");
+  P.act_sf = asf;
+  gemm_fp4_kernel<2><<<grid, THREADS, kGemmSmem, stream>>>(tm_d, tm_a, P);
+  MOE_LAUNCH_CHECK("gemm_fp4_kernel<2>");
+  return MOE_OK;
 }
 
 }  // namespace moe

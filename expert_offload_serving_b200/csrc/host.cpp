@@ -95,25 +95,36 @@ extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* w
     return MOE_OK;
   }
   MOE_REQUIRE(sg && su && sd, "null scale pointer for an FP4 format");
-  std::memcpy(b + L.wg, wg, m / 2);
-  std::memcpy(b + L.wu, wu, m / 2);
-  std::memcpy(b + L.wd, wd, m / 2);
   if (s.fmt == MOE_W_MXFP4) {
+    std::memcpy(b + L.wg, wg, m / 2);
+    std::memcpy(b + L.wu, wu, m / 2);
+    std::memcpy(b + L.wd, wd, m / 2);
     std::memcpy(b + L.sg, sg, m / 32);
     std::memcpy(b + L.su, su, m / 32);
     std::memcpy(b + L.sd, sd, m / 32);
     return MOE_OK;
   }
   MOE_REQUIRE(tensor_scales != nullptr, "NVFP4 needs 3 tensor scales");
-  // scale bytes move from row-major [R][K/16] into the MMA atom layout
-  struct M { const uint8_t* src; size_t off; int R, K; } mats[3] = {
-      {sg, L.sg, s.I, s.d}, {su, L.su, s.I, s.d}, {sd, L.sd, s.d, s.I}};
-  for (const M& mt : mats) {
-    const int nb = mt.K / 16;
-    for (int r = 0; r < mt.R; ++r)
-      for (int blk = 0; blk < nb; ++blk)
-        b[mt.off + sf_atom_offset(r, blk, mt.K)] = mt.src[static_cast<size_t>(r) * nb + blk];
+  // W_gu: gate and up rows interleaved in blocks of 64; scale bytes move from
+  // row-major [R][K/16] into the MMA atom layout
+  const size_t gate_row_bytes = static_cast<size_t>(s.d) / 2;
+  const int nbd = s.d / 16;
+  for (int i = 0; i < s.I; ++i) {
+    const int rg = gu_row(i, false), ru = gu_row(i, true);
+    std::memcpy(b + L.wg + rg * gate_row_bytes, static_cast<const uint8_t*>(wg) + i * gate_row_bytes,
+                gate_row_bytes);
+    std::memcpy(b + L.wg + ru * gate_row_bytes, static_cast<const uint8_t*>(wu) + i * gate_row_bytes,
+                gate_row_bytes);
+    for (int blk = 0; blk < nbd; ++blk) {
+      b[L.sg + sf_atom_offset(rg, blk, s.d)] = sg[static_cast<size_t>(i) * nbd + blk];
+      b[L.sg + sf_atom_offset(ru, blk, s.d)] = su[static_cast<size_t>(i) * nbd + blk];
+    }
   }
+  std::memcpy(b + L.wd, wd, m / 2);
+  const int nbi = s.I / 16;
+  for (int r = 0; r < s.d; ++r)
+    for (int blk = 0; blk < nbi; ++blk)
+      b[L.sd + sf_atom_offset(r, blk, s.I)] = sd[static_cast<size_t>(r) * nbi + blk];
   std::memcpy(b + L.ts, tensor_scales, 3 * sizeof(float));
   return MOE_OK;
 }

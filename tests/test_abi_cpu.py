@@ -104,9 +104,9 @@ def _canonical(name, E=3):
 
 @pytest.mark.parametrize("name", ["tiny", "decode_mxfp4", "prefill_nvfp4"])
 def test_pack_expert_layout(moe, name):
-    """Blob regions hold the canonical tensors (scales of NVFP4 in the MMA
-    atom layout: row r, block b at ((r/128)*(K/64) + b/4)*512 + (r%32)*16 +
-    ((r/32)%4)*4 + b%4)."""
+    """Blob regions hold the canonical tensors (NVFP4: gate/up rows interleaved
+    in blocks of 64, scales in the MMA atom layout: row r, block b at
+    ((r/128)*(K/64) + b/4)*512 + (r%32)*16 + ((r/32)%4)*4 + b%4)."""
     from expert_offload_serving_b200.layer import pack_pool
     cfg, w = _canonical(name)
     pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w, range(cfg.E), pin=False).numpy()
@@ -118,23 +118,33 @@ def test_pack_expert_layout(moe, name):
                 ref = w[key][e].contiguous().view(torch.uint8).numpy().ravel()
                 assert np.array_equal(b[n * 2 * m:(n + 1) * 2 * m], ref)
             continue
-        for n, key in enumerate(("wg", "wu", "wd")):
-            assert np.array_equal(b[n * m // 2:(n + 1) * m // 2], w[key][e].numpy().ravel())
-        base = 3 * m // 2
         if cfg.fmt == "mxfp4":
+            for n, key in enumerate(("wg", "wu", "wd")):
+                assert np.array_equal(b[n * m // 2:(n + 1) * m // 2], w[key][e].numpy().ravel())
+            base = 3 * m // 2
             for n, key in enumerate(("sg", "su", "sd")):
                 assert np.array_equal(b[base + n * m // 32: base + (n + 1) * m // 32], w[key][e].numpy().ravel())
-        else:
-            for n, key in enumerate(("sg", "su", "sd")):
-                sc = w[key][e].numpy()
-                R, nb = sc.shape
-                K = nb * 16
-                reg = b[base + n * m // 16: base + (n + 1) * m // 16]
-                rr, bb = np.meshgrid(np.arange(R), np.arange(nb), indexing="ij")
-                off = ((rr // 128) * (K // 64) + bb // 4) * 512 + (rr % 32) * 16 + ((rr // 32) % 4) * 4 + bb % 4
-                assert np.array_equal(reg[off], sc)
-            ts = b[base + 3 * m // 16: base + 3 * m // 16 + 12].view(np.float32)
-            assert np.array_equal(ts, w["ts"][e].numpy())
+            continue
+        # NVFP4: W_gu interleaves gate and up rows in blocks of 64
+        rb = cfg.d // 2
+        gu = b[:m].reshape(2 * cfg.I, rb)
+        i = np.arange(cfg.I)
+        rg = (i // 64) * 128 + i % 64
+        assert np.array_equal(gu[rg], w["wg"][e].numpy())
+        assert np.array_equal(gu[rg + 64], w["wu"][e].numpy())
+        assert np.array_equal(b[m:m + m // 2], w["wd"][e].numpy().ravel())
+
+        def atoms(reg, R, K):
+            rr, bb = np.meshgrid(np.arange(R), np.arange(K // 16), indexing="ij")
+            off = ((rr // 128) * (K // 64) + bb // 4) * 512 + (rr % 32) * 16 + ((rr // 32) % 4) * 4 + bb % 4
+            return reg[off]
+        sgu = atoms(b[3 * m // 2: 3 * m // 2 + m // 8], 2 * cfg.I, cfg.d)
+        assert np.array_equal(sgu[rg], w["sg"][e].numpy())
+        assert np.array_equal(sgu[rg + 64], w["su"][e].numpy())
+        base = 3 * m // 2 + m // 8
+        assert np.array_equal(atoms(b[base: base + m // 16], cfg.d, cfg.I), w["sd"][e].numpy())
+        ts = b[base + m // 16: base + m // 16 + 12].view(np.float32)
+        assert np.array_equal(ts, w["ts"][e].numpy())
 
 
 def test_cache_planner_matches_oracle_lru(moe):
