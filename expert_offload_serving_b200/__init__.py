@@ -47,6 +47,7 @@ _SIGS = {
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "moe_permute_scratch_bytes": (_SZ, [_I, _I, _I]),
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_expert_ffn_workspace_bytes": (_SZ, [moe_shape, _I, _I, _I]),
     "moe_expert_ffn": (_I, [moe_shape, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P, _P]),
     "moe_combine_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
@@ -134,6 +135,17 @@ def moe_permute(idx, E: int, offsets, perm, inv_perm, scratch=None, dev_status=N
     nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
     _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv_perm),
                              _ptr(scratch), nbytes, _ptr(dev_status), _stream(stream)))
+
+
+MOE_PERMUTE_NOALLOC_MAX_SCRATCH = 262144
+
+
+def moe_permute_noalloc(idx, E: int, offsets, perm, inv_perm, dev_status=None, stream=None):
+    """moe_permute without a scratch argument: for callers that cannot
+    allocate device memory (the library's fixed scratch array is used)."""
+    T, k = idx.shape
+    _check(lib().moe_permute_noalloc(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv_perm),
+                                     _ptr(dev_status), _stream(stream)))
 
 
 def moe_expert_ffn_workspace_bytes(s: moe_shape, T: int, k: int, flags: int = 0) -> int:

@@ -15,6 +15,8 @@
 // step) is a single fused launch with no scratch.  More tiles take three
 // launches: per-tile histograms -> one scan over (tile, expert) that yields
 // offsets and per-tile bases -> the ranked scatter.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -261,4 +263,62 @@ extern "C" moe_status moe_permute(const int32_t* idx, int T, int k, int E, int32
   permute_scatter_kernel<<<ntiles, kTile, smem, stream>>>(idx, n, E, counts, perm, inv_perm, dev_status);
   MOE_LAUNCH_CHECK("permute_scatter_kernel");
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: moe_permute with its scratch taken from a fixed array
+// compiled into the library, for callers that cannot allocate device memory.
+// The array lives in every device's memory for as long as the library is
+// loaded.  Its device address is looked up once per device, by the first call
+// made with that device current.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = MOE_PERMUTE_NOALLOC_MAX_SCRATCH;
+static_assert(kNoAllocScratchBytes % 256 == 0, "scratch size must keep 256-byte alignment");
+
+static __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_permute_scratch on the current device.  In host code the
+// symbol itself is only a host-side stand-in, never a device address.
+moe_status noalloc_scratch(const DeviceInfo& dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev.id] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress(permute scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev.id] = p;
+  }
+  *out = g_noalloc_addr[dev.id];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E, int32_t* offsets,
+                                          int32_t* perm, int32_t* inv_perm, int32_t* dev_status,
+                                          cudaStream_t stream) {
+  clear_error();
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= 32, "T=%d, k=%d", T, k);
+  MOE_REQUIRE(E >= 1 && E <= 1024, "E=%d outside [1, 1024]", E);
+  MOE_REQUIRE(static_cast<long long>(T) * k <= (1 << 24), "T*k too large");
+  const size_t need = moe_permute_scratch_bytes(T, k, E);
+  if (need > kNoAllocScratchBytes)
+    return fail(MOE_ERR_CAPACITY,
+                "moe_permute_noalloc: T=%d, k=%d, E=%d needs %zu bytes of scratch; its fixed array holds %zu "
+                "(use moe_permute with caller scratch)",
+                T, k, E, need, kNoAllocScratchBytes);
+  DeviceInfo dev;
+  moe_status st = current_device(&dev);
+  if (st != MOE_OK) return st;
+  void* scratch = nullptr;
+  if (need > 0) {
+    st = noalloc_scratch(dev, &scratch);
+    if (st != MOE_OK) return st;
+  }
+  return moe_permute(idx, T, k, E, offsets, perm, inv_perm, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+                     dev_status, stream);
 }

@@ -134,6 +134,31 @@ moe_status moe_permute(const int32_t* idx, int T, int k, int E,
                        void* scratch, size_t scratch_bytes, int32_t* dev_status,
                        cudaStream_t stream);
 
+/* moe_permute_noalloc -- the same permutation as moe_permute, for callers
+ * that cannot allocate device memory: for example a caller embedded in a host
+ * engine that has already reserved the device's memory for its own pool (a
+ * separate cudaMalloc there can fail, or stall the engine), or a caller on a
+ * latency-critical path that cannot afford an allocation call.  It takes no
+ * scratch argument and makes no allocation of any kind; its scratch is a
+ * fixed array of MOE_PERMUTE_NOALLOC_MAX_SCRATCH bytes compiled into the
+ * library, which every device that loads the library holds until the process
+ * exits.  The paper has no counterpart to this call.
+ *   Limits: moe_permute_scratch_bytes(T, k, E) <= MOE_PERMUTE_NOALLOC_MAX_SCRATCH
+ *     (e.g. T*k <= 65536 pairs at E = 1024, <= 262144 at E = 256); larger
+ *     problems return MOE_ERR_CAPACITY with nothing enqueued.
+ *   Set-up: the first call on a device (with that device current) looks up
+ *     the array's device address once; make that first call before any
+ *     stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *     call's contents (the kernels overwrite every entry they read, so nothing
+ *     has to start at zero).  Calls that overlap on the GPU -- on different
+ *     streams, or from several host threads without ordering -- race on it.
+ *   Arguments, outputs and errors are those of moe_permute. */
+#define MOE_PERMUTE_NOALLOC_MAX_SCRATCH 262144
+moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E,
+                               int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                               int32_t* dev_status, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Step 3 -- grouped SwiGLU expert FFN over the expert cache.  For every
  * expert e with slot_of_expert[e] >= 0 and every pair at sorted position q in
