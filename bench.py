@@ -36,6 +36,22 @@ METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill FP4 TFLOPS vs B200 pea
 L2_BYTES = 126 * 1024 * 1024
 
 
+def kernel_traffic(kernel_file, key):
+    """DRAM bytes (read + write) per launch of a kernel from the ncu capture
+    recorded in profiles/traffic.json -- only while the kernel's source file
+    still has the hash recorded there (None once the kernel has changed)."""
+    import hashlib
+    rec_path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "expert_offload_serving_b200", "csrc", kernel_file)
+    if not (os.path.exists(rec_path) and os.path.exists(src)):
+        return None
+    rec = json.load(open(rec_path)).get(key)
+    if not rec:
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if rec.get("source_sha256_16") == h else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -158,6 +174,46 @@ def experts_touched(layer):
     return int(((off[1:] - off[:-1]) > 0).sum())
 
 
+def decode_point(cfg, T, R, warmup, steps, stream):
+    """Device-timed decode_bf16 layer steps at T tokens (graph replay over R
+    replicas) and the expert-FFN time alone, for the secondary T points."""
+    import expert_offload_serving_b200 as moe
+    blob = moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
+    reps = build_replicas(cfg, T, R, seed0=500 + T)
+    U = []
+    for r in reps:
+        r["layer"].forward(r["logits"], r["x"])
+        torch.cuda.synchronize()
+        U.append(experts_touched(r["layer"]))
+    graphs = []
+    with torch.cuda.stream(stream):
+        for r in reps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                r["layer"].forward(r["logits"], r["x"])
+            graphs.append(g)
+        for i in range(warmup):
+            graphs[i % R].replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            graphs[i % R].replay()
+        e1.record(stream)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(steps):
+            reps[i % R]["layer"].ffn(reps[i % R]["x"])
+        f1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    ffn_ms = f0.elapsed_time(f1) / steps
+    gbs = sum(U) / R * blob / (ffn_ms / 1e3) / 1e9
+    hbm, _ = peaks()
+    del graphs, reps
+    return {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5), "ffn_ms": round(ffn_ms, 5),
+            "ffn_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4), "experts_touched": U}
+
+
 def run_gpu(args, rank, world, local):
     import expert_offload_serving_b200 as moe
     moe.lib()
@@ -268,6 +324,22 @@ def run_gpu(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg, T)
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill()
+    sweep = None
+    if not args.no_sweep and world == 1:
+        sweep = {}
+        for t in (1, 16):
+            if t == T:
+                continue
+            sweep[f"T{t}"] = decode_point(cfg, t, R, args.warmup, min(args.steps, 2000), stream)
+    cached = None
+    if not args.no_cached:
+        hp = cached_host_pool()
+        cached = [run_cached_decode(hp, T=t) for t in (1, 8)]
+        del hp
+
     result = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -299,7 +371,7 @@ def run_gpu(args, rank, world, local):
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
-            "traffic": None,
+            "traffic": kernel_traffic("ffn_decode.cu", f"decode_bf16_T{T}"),
             "algorithmic_bytes_per_launch": int(alg_bytes),
             "avg_launch_ms": round(ffn_avg_ms, 5),
         },
@@ -310,7 +382,149 @@ def run_gpu(args, rank, world, local):
     }
     if cpu is not None:
         result["cpu_baseline"] = cpu
+    if prefill is not None:
+        result["prefill"] = prefill
+    if cached is not None:
+        result["decode_mxfp4_cached"] = cached
+    if sweep:
+        result["decode_bf16_T_sweep"] = sweep
     return result
+
+
+# ---------------------------------------------------------------- prefill (FP4 tensor cores)
+def run_prefill(iters=20, warmup=5, T=4096):
+    """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, T tokens, NVFP4
+    activations on tcgen05): whole-layer time and the expert-FFN time alone.
+    The 3.6 GB of weights exceed L2 many times over, so no replicas."""
+    import expert_offload_serving_b200 as moe
+    from expert_offload_serving_b200.layer import MoeLayer, pack_pool
+    cfg = synth.CONFIGS["prefill_nvfp4"]
+    logits, x = synth.make_routing(cfg, T, 0)
+    w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
+    pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()}, range(cfg.E),
+                     pin=False).cuda()
+    del w
+    layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=pool, act="nvfp4")
+    lg, xx = logits.cuda(), x.cuda()
+    stream = torch.cuda.Stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            layer.forward(lg, xx)
+        e0.record(stream)
+        for _ in range(iters):
+            layer.forward(lg, xx)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        layer_ms = e0.elapsed_time(e1) / iters
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(iters):
+            layer.ffn(xx)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    ffn_ms = f0.elapsed_time(f1) / iters
+    moe.moe_check_status(layer.status)
+    flops = 2.0 * 3 * cfg.d * cfg.I * T * cfg.k
+    off = layer.offsets.cpu()
+    U = int(((off[1:] - off[:-1]) > 0).sum())
+    wbytes = U * moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
+    d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    bf16 = d.get("bf16_tflops", 1590.0)
+    fp4_peak = 4.0 * bf16          # dense FP4 = 4 x dense BF16 (nominal 9 / 2.25 PFLOP/s)
+    hbm, _ = peaks()
+    tf = flops / (ffn_ms / 1e3) / 1e12
+    gbs = wbytes / (ffn_ms / 1e3) / 1e9
+    roof_ms = max(wbytes / (hbm * 1e9), flops / (fp4_peak * 1e12)) * 1e3
+    return {
+        "workload": f"prefill_nvfp4: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, NVFP4 weights and activations",
+        "tokens_per_s": round(T / (layer_ms / 1e3), 1),
+        "layer_ms": round(layer_ms, 4),
+        "ffn_ms": round(ffn_ms, 4),
+        "tflops": round(tf, 1),
+        "fp4_peak_tflops": round(fp4_peak, 1),
+        "fp4_peak_source": "4 x measured bf16 (MEASURED_PEAKS.json bf16_tflops)",
+        "frac_fp4_peak": round(tf / fp4_peak, 4),
+        "weight_gbs": round(gbs, 1),
+        "frac_hbm": round(gbs / hbm, 4),
+        "roofline_ms": round(roof_ms, 4),
+        "frac_roofline": round(roof_ms / ffn_ms, 4),
+        "experts_touched": U,
+        "kernels": "quant_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2>",
+    }
+
+
+# ---------------------------------------------------------------- decode with the expert cache
+def cached_host_pool():
+    """The 256 MXFP4 experts of the cached-decode workload, packed into one
+    pinned host pool in expert order."""
+    from expert_offload_serving_b200.layer import pack_pool
+    cfg = synth.CONFIGS["decode_mxfp4"]
+    w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
+    return pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()}, range(cfg.E), pin=True)
+
+
+def run_cached_decode(host_pool, T=1, steps=64, warm=32):
+    """MXFP4 decode with 64 GPU slots over a drifting routing trace (E=256,
+    k=6, d=4096, I=2048): per step the host reads the routing, the LRU fills
+    misses from the pinned host pool over PCIe on a side stream, then
+    permute -> FFN -> combine.  Timed on the device over `steps` steps after
+    `warm` warm-up steps (fills included)."""
+    import expert_offload_serving_b200 as moe
+    from expert_offload_serving_b200.layer import MoeLayer
+    cfg = synth.CONFIGS["decode_mxfp4"]
+    B = host_pool.shape[1]
+    # pinned host -> device copy bandwidth of whole blobs (the fill path)
+    dst = torch.empty((8, B), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        for i in range(8):
+            dst[i].copy_(host_pool[i], non_blocking=True)
+        e0.record(s)
+        for rep in range(4):
+            for i in range(8):
+                dst[i].copy_(host_pool[8 * rep + i], non_blocking=True)
+        e1.record(s)
+    torch.cuda.synchronize()
+    h2d_gbs = 32 * B / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del dst
+    layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, host_pool=host_pool, n_slots=cfg.n_slots)
+    trace = synth.make_trace(cfg, T, steps=warm + steps, seed=0)
+    lgs = [lg.cuda() for lg, _ in trace]
+    xs = [x.cuda() for _, x in trace]
+    main = torch.cuda.Stream()
+    hits = misses = 0
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(main):
+        for t in range(warm + steps):
+            if t == warm:
+                t0.record(main)
+            layer.route(lgs[t])
+            U = sorted(set(layer.idx[:T].cpu().numpy().ravel().tolist()))
+            fills = layer.prepare(t, U, stream=main)
+            layer.permute(T)
+            layer.ffn(xs[t])
+            layer.combine(T)
+            if t >= warm:
+                misses += len(fills)
+                hits += len(U) - len(fills)
+        t1.record(main)
+    torch.cuda.synchronize()
+    moe.moe_check_status(layer.status)
+    ms = t0.elapsed_time(t1) / steps
+    return {
+        "workload": f"decode_mxfp4: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, {cfg.n_slots} slots, "
+                    f"AR(1) drifting trace, LRU fills from pinned host memory",
+        "tokens_per_s": round(T / (ms / 1e3), 1),
+        "ms_per_step": round(ms, 4),
+        "miss_rate": round(misses / max(1, hits + misses), 4),
+        "fills_per_step": round(misses / steps, 2),
+        "fill_mb_per_step": round(misses / steps * B / 1e6, 2),
+        "h2d_pinned_gbs": round(h2d_gbs, 1),
+        "steps": steps,
+    }
 
 
 # ---------------------------------------------------------------- CPU oracle arms
@@ -406,10 +620,17 @@ def main(argv=None):
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the FP4 prefill measurement")
+    ap.add_argument("--only-prefill", action="store_true", help="print only the FP4 prefill measurement")
+    ap.add_argument("--no-cached", action="store_true", help="skip the expert-cache decode measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the T=1 and T=16 decode points")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = dist_setup(args.gpus)
+    if args.only_prefill:
+        print(json.dumps(run_prefill(iters=max(3, min(args.steps, 50)), warmup=args.warmup)), flush=True)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
     else:

@@ -102,6 +102,17 @@ def _stream(s):
     return s.cuda_stream
 
 
+def _event(ev):
+    """cudaEvent_t of a torch.cuda.Event.  torch creates the CUDA event only on
+    its first record, so an event that was never recorded has no handle yet."""
+    if ev is None:
+        return None
+    h = ev.cuda_event
+    if not h:
+        raise ValueError("torch.cuda.Event has no CUDA event yet: record it once before passing it")
+    return h
+
+
 def shape(E: int, d: int, I: int, fmt) -> moe_shape:
     return moe_shape(E, d, I, FORMATS[fmt] if isinstance(fmt, str) else int(fmt))
 
@@ -192,9 +203,7 @@ class MoeCache:
         nf = ctypes.c_int32(0)
         side_h = None if side is None else _stream(side)
         _check(lib().moe_cache_fill(self.h, ex, len(experts), step, pr, len(protect), side_h,
-                                    None if reads_done is None else reads_done.cuda_event,
-                                    None if fill_done is None else fill_done.cuda_event,
-                                    fills, ctypes.byref(nf)))
+                                    _event(reads_done), _event(fill_done), fills, ctypes.byref(nf)))
         return [(fills[3 * i], fills[3 * i + 1], fills[3 * i + 2]) for i in range(nf.value)]
 
     def query(self):

@@ -47,16 +47,20 @@ extern "C" moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k, c
     MOE_REQUIRE(out != nullptr && gate != nullptr, "y_perm is NULL: out and gate are required");
     MOE_REQUIRE(aligned(out, 16) && aligned(gate, 4), "misaligned out or gate");
   }
+  if (flags & MOE_FFN_ACT_NVFP4) {
+    MOE_REQUIRE(s.fmt == MOE_W_NVFP4, "MOE_FFN_ACT_NVFP4 needs NVFP4 weights");
+    MOE_REQUIRE(y_perm == nullptr, "MOE_FFN_ACT_NVFP4 writes out (fused combine); y_perm must be NULL");
+    MOE_REQUIRE(s.d % 256 == 0 && s.I % 256 == 0, "the FP4 tensor-core path needs d, I multiples of 256");
+  }
   const size_t need = moe_expert_ffn_workspace_bytes(s, T, k, flags);
   if (need > 0 && (workspace == nullptr || ws_bytes < need))
     return fail(MOE_ERR_CAPACITY, "workspace needs %zu bytes, got %zu", need, ws_bytes);
   MOE_REQUIRE(workspace == nullptr || aligned(workspace, 256), "workspace must be 256-byte aligned");
+  // every argument check is done: only now touch the device
   DeviceInfo dev;
   st = current_device(&dev);
   if (st != MOE_OK) return st;
   if (flags & MOE_FFN_ACT_NVFP4) {
-    MOE_REQUIRE(s.fmt == MOE_W_NVFP4, "MOE_FFN_ACT_NVFP4 needs NVFP4 weights");
-    MOE_REQUIRE(y_perm == nullptr, "MOE_FFN_ACT_NVFP4 writes out (fused combine); y_perm must be NULL");
     return launch_ffn_prefill(s, x, T, k, offsets, perm, slot_of_expert, slot_pool, n_slots, gate, out,
                               workspace, dev_status, dev, stream);
   }

@@ -10,12 +10,12 @@
 // Two launches:
 //   phase 1  rows of W_g and W_u -> a[q][i] (fp32 workspace, q = sorted pair)
 //   phase 2  rows of W_d         -> y_perm[q][c]  or  out[t][c] += gate * y
-// Work unit = (active expert, warp tile of 8 weight rows, pass of <= 4 token
-// rows).  Phase 1 tiles hold gate rows i..i+3 and up rows i..i+3, so the
-// SwiGLU is formed in registers; phase 2 tiles hold 8 rows of W_d.
+// Work unit = (active expert, warp tile of 4 weight rows, pass of <= 4 (bf16)
+// or <= 2 (FP4) token rows).  Phase 1 tiles hold gate rows i, i+1 and up rows i, i+1, so the
+// SwiGLU is formed in registers; phase 2 tiles hold 4 rows of W_d.
 // Weights are streamed HBM -> shared memory by cp.async.bulk into a 3-stage
-// ring per warp (8 rows x 1 KB per stage, mbarrier-completed), so the number
-// of bytes in flight (up to 128 KB per SM) does not depend on registers.
+// ring per warp (4 rows x 1 KB per stage, mbarrier-completed; 16 warps per
+// SM), so the bytes in flight (up to 128 KB per SM) do not depend on registers.
 // Lanes split each 1 KB row slice in 16-byte chunks (8 bf16 or 32 FP4
 // weights): conflict-free 128-bit shared loads, dequantisation in registers
 // (E2M1 -> f16x2 by cvt, times the E8M0 or E4M3 block scale), packed fp32
@@ -31,12 +31,12 @@
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;                  // warps per CTA (each its own pipeline)
-constexpr int kRW = 8;                     // weight rows per warp tile
-constexpr int kNTMax = 4;                  // token rows per pass
+constexpr int kWarps = 16;                 // warps per CTA (each its own pipeline)
+constexpr int kRW = 4;                      // weight rows per warp tile
+constexpr int kNTMaxCap = 8;               // token rows per pass, upper bound
 constexpr int kSlice = 1024;               // bytes of one row per stage
 constexpr int kStages = 3;                 // ring depth per warp
-constexpr int kStageBytes = kRW * kSlice;  // 8 KB
+constexpr int kStageBytes = kRW * kSlice;  // 4 KB
 constexpr size_t kSmemBytes = static_cast<size_t>(kWarps) * kStages * kStageBytes + 1024;
 
 struct FfnParams {
@@ -56,14 +56,7 @@ struct FfnParams {
 };
 
 // ------------------------------------------------------------ small helpers
-__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
-  unsigned long long A, B, C;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(acc.x), "f"(acc.y));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(C));
-}
+__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) { acc = __ffma2_rn(a, b, acc); }
 
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
@@ -188,11 +181,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((i & 255u) == 255u && now_ns() - t0 > kWaitNs) return false;
   }
 }
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+// Weights are read once per layer call: stream them through L2 with an
+// evict-first policy so the activations and the SwiGLU workspace stay cached.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -229,7 +230,7 @@ struct Weights<MOE_W_MXFP4> {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float2 f = f16x2_to_float2(e2m1x2_to_f16x2((word >> (8 * j)) & 0xffu));
-      w[j] = make_float2(f.x * sc.s, f.y * sc.s);
+      w[j] = __fmul2_rn(f, make_float2(sc.s, sc.s));
     }
   }
 };
@@ -284,13 +285,19 @@ struct XF32 {
 //   wrow[r]: byte address of row r's codes; srow/rg: scale region and global
 //   row index of row r (FP4); xrows[t]: row index into xs.
 // ------------------------------------------------------------ work decomposition
+// Token rows per pass: 4 for bf16, 2 for FP4 (whose dequantisation keeps more
+// registers live); larger passes would spill at 128 registers per thread.
+template <int FMT>
+__host__ __device__ constexpr int nt_max() { return FMT == MOE_W_BF16 ? 4 : 2; }
+
 struct Unit {
   int e, tile, q0, tb, nt;   // expert, warp tile, first sorted row, first token row of the pass, rows
 };
 
-template <int PHASE>
+template <int FMT, int PHASE>
 __device__ __forceinline__ Unit decode_unit(const FfnParams& P, const int16_t* act, const int32_t* ustart,
                                             int n_act, long long u) {
+  constexpr int kNTMax = nt_max<FMT>();
   int lo = 0, hi = n_act;   // last a with ustart[a] <= u
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -315,14 +322,15 @@ template <int FMT, int PHASE>
 __device__ __forceinline__ const uint8_t* tile_row(const FfnParams& P, const uint8_t* blob, int tile, int r,
                                                    size_t row_bytes, int* grow, int* mat) {
   if (PHASE == 1) {
-    const bool up = r >= 4;
-    const int i = 4 * tile + (r & 3);
+    constexpr int H = kRW / 2;   // gate rows first, then the up rows of the same indices
+    const bool up = r >= H;
+    const int i = H * tile + (up ? r - H : r);
     const int row = (FMT == MOE_W_NVFP4) ? gu_row(i, up) : i;
     *grow = row;
     *mat = up ? 1 : 0;
     return blob + (up ? P.L.wu : P.L.wg) + static_cast<size_t>(row) * row_bytes;
   }
-  const int row = 8 * tile + r;
+  const int row = kRW * tile + r;
   *grow = row;
   *mat = 2;
   return blob + P.L.wd + static_cast<size_t>(row) * row_bytes;
@@ -330,12 +338,17 @@ __device__ __forceinline__ const uint8_t* tile_row(const FfnParams& P, const uin
 
 // The warp's pipeline state: items are (unit, slice) in order; item j lives
 // in stage j % kStages and completes phase (j / kStages) & 1 of its barrier.
+// Issuing: lane r (< 8) holds the address of weight row r of the unit being
+// issued, so one warp instruction issues the 8 row copies of a stage.
 struct Pipe {
   uint8_t* ring;       // kStages * kStageBytes
   uint64_t* bar;       // kStages
   long long beg, n_units, next_issue, n_items;
   int slices;
   bool ok;
+  long long issue_unit;        // unit whose row addresses lane_row holds (-1: none)
+  const uint8_t* lane_row;     // this lane's weight row of issue_unit (lanes < kRW)
+  uint64_t policy;             // L2 policy of the weight copies
 };
 
 template <int FMT, int PHASE>
@@ -345,24 +358,22 @@ __device__ __forceinline__ void issue_item(const FfnParams& P, const int16_t* ac
   const long long u = pp.beg + j / pp.slices;
   const int sl = static_cast<int>(j % pp.slices);
   const int st = static_cast<int>(j % kStages);
-  __syncwarp();
-  if (lane == 0) {
-    const Unit U = decode_unit<PHASE>(P, act, ustart, n_act, u);
+  if (u != pp.issue_unit) {
+    const Unit U = decode_unit<FMT, PHASE>(P, act, ustart, n_act, u);
     const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-    const size_t off = static_cast<size_t>(sl) * kSlice;
-    const uint32_t bytes = static_cast<uint32_t>(min(static_cast<size_t>(kSlice), row_bytes - off));
-    // the stage was last read by this warp's generic loads; order them before the async writes
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_expect_tx(&pp.bar[st], bytes * kRW);
-    uint8_t* dst = pp.ring + st * kStageBytes;
-#pragma unroll
-    for (int r = 0; r < kRW; ++r) {
-      int g, m;
-      const uint8_t* src = tile_row<FMT, PHASE>(P, blob, U.tile, r, row_bytes, &g, &m);
-      bulk_load(dst + r * kSlice, src + off, bytes, &pp.bar[st]);
-    }
+    int g, m;
+    pp.lane_row = tile_row<FMT, PHASE>(P, blob, U.tile, lane & (kRW - 1), row_bytes, &g, &m);
+    pp.issue_unit = u;
   }
+  const size_t off = static_cast<size_t>(sl) * kSlice;
+  const uint32_t bytes = static_cast<uint32_t>(min(static_cast<size_t>(kSlice), row_bytes - off));
+  // the stage was last read by this warp's generic loads; order them before the async writes
   __syncwarp();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (lane == 0) mbar_expect_tx(&pp.bar[st], bytes * kRW);
+  __syncwarp();
+  if (lane < kRW)
+    bulk_load(pp.ring + st * kStageBytes + lane * kSlice, pp.lane_row + off, bytes, &pp.bar[st], pp.policy);
 }
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
@@ -416,32 +427,48 @@ __device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* 
     }
     const uint8_t* stage = pp.ring + st * kStageBytes;
     const int valid = static_cast<int>(min(static_cast<size_t>(kSlice), row_bytes - static_cast<size_t>(sl) * kSlice));
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < 2; ++h) {
       const int c = lane + 32 * h;                 // 16-byte chunk inside the 1 KB slice
       if (c * 16 >= valid) break;
       const int k0 = (sl * kSlice + c * 16) * W::EPC / 16;   // first K element of the chunk
-      uint4 raw[kRW];
+      // FP4 reuses a row's 16 bytes for 4 sub-chunks: keep them; bf16 uses each once
+      constexpr int kHeld = (W::SUB > 1) ? kRW : 1;
+      uint4 raw[kHeld];
       typename W::Scale sc[kRW];
 #pragma unroll
       for (int r = 0; r < kRW; ++r) {
-        raw[r] = *reinterpret_cast<const uint4*>(stage + r * kSlice + c * 16);
+        if constexpr (W::SUB > 1) raw[r < kHeld ? r : 0] = *reinterpret_cast<const uint4*>(stage + r * kSlice + c * 16);
         sc[r] = W::scale(sreg[r], grow[r], k0 / W::EPC, K);
       }
 #pragma unroll
       for (int m = 0; m < W::SUB; ++m) {
-        float2 w[kRW][4];
+        // activations of at most 4 tokens are live at a time; weights are
+        // decoded once per 4-token group
+        constexpr int GS = NT < 4 ? NT : 4;
 #pragma unroll
-        for (int r = 0; r < kRW; ++r) W::decode(raw[r], m, sc[r], w[r]);
+        for (int g = 0; g < NT / GS; ++g) {
+          float2 xf[GS][4];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          float2 xf[4];
-          if (PHASE == 1) XBf16{P.x, P.d}.load(xrows[t], k0 + 8 * m, xf);
-          else XF32{P.a_ws, P.I}.load(xrows[t], k0 + 8 * m, xf);
+          for (int t = 0; t < GS; ++t) {
+            if (PHASE == 1) XBf16{P.x, P.d}.load(xrows[g * GS + t], k0 + 8 * m, xf[t]);
+            else XF32{P.a_ws, P.I}.load(xrows[g * GS + t], k0 + 8 * m, xf[t]);
+          }
 #pragma unroll
-          for (int r = 0; r < kRW; ++r)
+          for (int r = 0; r < kRW; ++r) {
+            float2 w[4];
+            if constexpr (W::SUB > 1) {
+              W::decode(raw[r < kHeld ? r : 0], m, sc[r], w);
+            } else {
+              const uint4 one = *reinterpret_cast<const uint4*>(stage + r * kSlice + c * 16);
+              W::decode(one, m, sc[r], w);
+            }
+            // q outer, tokens inner: consecutive FMAs update different accumulators
 #pragma unroll
-            for (int q = 0; q < 4; ++q) ffma2(acc[r][t], w[r][q], xf[q]);
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int t = 0; t < GS; ++t) ffma2(acc[r][g * GS + t], w[q], xf[t][q]);
+          }
         }
       }
     }
@@ -463,16 +490,16 @@ __device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* 
     const int vi = (lane >> (5 - S)) * R + i;
     const int r = vi / NT, t = vi % NT;
     if (PHASE == 1) {
-      // lanes < 16 hold gate rows (r < 4); lane ^ 16 holds the up row of the same (i, token)
+      // lanes < 16 hold gate rows (r < kRW/2); lane ^ 16 holds the up row of the same (i, token)
       const float other = __shfl_xor_sync(kFull, v[i], 16);
       if (writer && lane < 16 && t < U.nt) {
         const float hh = v[i] * tscale[r];
-        const float uu = other * tscale[r + 4];
-        P.a_ws[static_cast<size_t>(U.q0 + U.tb + t) * P.I + 4 * U.tile + r] = silu(hh) * uu;
+        const float uu = other * tscale[r + kRW / 2];
+        P.a_ws[static_cast<size_t>(U.q0 + U.tb + t) * P.I + (kRW / 2) * U.tile + r] = silu(hh) * uu;
       }
     } else if (writer && t < U.nt) {
       const int q = U.q0 + U.tb + t;
-      const int row = 8 * U.tile + r;
+      const int row = kRW * U.tile + r;
       const float y = v[i] * tscale[r];
       if (P.y_perm != nullptr) {
         P.y_perm[static_cast<size_t>(q) * P.d + row] = y;
@@ -487,6 +514,7 @@ __device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* 
 
 template <int FMT, int PHASE>
 __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P) {
+  static_assert(kWarps * kStages <= 64, "barrier array");
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ int16_t s_act[1024];
   __shared__ int32_t s_ustart[1025];
@@ -494,12 +522,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
   __shared__ __align__(8) uint64_t s_bar[kWarps * kStages];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int tiles_per_e = (PHASE == 1) ? P.I / 4 : P.d / kRW;
+  const int tiles_per_e = (PHASE == 1) ? P.I / (kRW / 2) : P.d / kRW;
   // active experts (tokens > 0, resident) in expert order, with their unit counts
   const int per = (P.E + blockDim.x - 1) / blockDim.x;
   const int e0 = threadIdx.x * per;
   int cnt = 0, units = 0;
-  uint32_t mask = 0;   // per <= 4
+  uint32_t mask = 0;   // per <= 2
   const int npairs = P.T * P.k;
   for (int jx = 0; jx < per; ++jx) {
     const int e = e0 + jx;
@@ -526,7 +554,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
       const int e = e0 + jx;
       const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
       s_act[pos++] = static_cast<int16_t>(e);
-      units += tiles_per_e * ((ne + kNTMax - 1) / kNTMax);
+      units += tiles_per_e * ((ne + nt_max<FMT>() - 1) / nt_max<FMT>());
     }
   int total_units;
   int ustart = block_scan(units, s_ws, &total_units);
@@ -536,7 +564,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
       const int e = e0 + jx;
       const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
       s_ustart[pos++] = ustart;
-      ustart += tiles_per_e * ((ne + kNTMax - 1) / kNTMax);
+      ustart += tiles_per_e * ((ne + nt_max<FMT>() - 1) / nt_max<FMT>());
     }
   if (threadIdx.x < kWarps * kStages) mbar_init(&s_bar[threadIdx.x], 1);
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -555,15 +583,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
   pp.n_items = pp.n_units * pp.slices;
   pp.next_issue = 0;
   pp.ok = true;
+  pp.issue_unit = -1;
+  pp.lane_row = nullptr;
+  pp.policy = policy_evict_first();
   // prime the ring with kStages - 1 items
   for (int i = 0; i < kStages - 1 && pp.next_issue < pp.n_items; ++i)
     issue_item<FMT, PHASE>(P, s_act, s_ustart, n_act, pp, row_bytes, lane);
   long long j = 0;
   for (long long u = 0; u < pp.n_units && pp.ok; ++u) {
-    const Unit U = decode_unit<PHASE>(P, s_act, s_ustart, n_act, pp.beg + u);
+    const Unit U = decode_unit<FMT, PHASE>(P, s_act, s_ustart, n_act, pp.beg + u);
     if (U.nt == 1) run_unit<FMT, PHASE, 1>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
-    else if (U.nt == 2) run_unit<FMT, PHASE, 2>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
-    else run_unit<FMT, PHASE, 4>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
+    else if (nt_max<FMT>() == 2 || U.nt == 2) run_unit<FMT, PHASE, 2>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
+    else run_unit<FMT, PHASE, (nt_max<FMT>() > 2 ? 4 : 2)>(P, s_act, s_ustart, n_act, pp, U, row_bytes, j, lane);
   }
   if (!pp.ok) {
     report(P.status, MOE_ERR_TIMEOUT);
@@ -584,9 +615,9 @@ moe_status launch_phase(const FfnParams& P, const DeviceInfo& dev, cudaStream_t 
                                       static_cast<int>(kSmemBytes)));
     attr[dev.id] = true;
   }
-  const int tiles_per_e = (PHASE == 1) ? P.I / 4 : P.d / kRW;
+  const int tiles_per_e = (PHASE == 1) ? P.I / (kRW / 2) : P.d / kRW;
   const long long most = static_cast<long long>(min(P.E, P.T * P.k)) * tiles_per_e *
-                         ((P.T * P.k + kNTMax - 1) / kNTMax);
+                         ((P.T * P.k + nt_max<FMT>() - 1) / nt_max<FMT>());
   long long blocks = (most + kWarps - 1) / kWarps;
   if (blocks > dev.sm_count) blocks = dev.sm_count;
   if (blocks < 1) blocks = 1;

@@ -8,9 +8,10 @@
 // kernel; on B200 the contraction belongs on tcgen05 with NVFP4 operands.
 //
 // Launches (one stream):
-//   quant_x      x rows, gathered in expert order, -> NVFP4 (E2M1 codes, one
-//                E4M3 scale per 16, unit tensor scale) in an expert-padded
-//                layout: expert e's rows start at a multiple of 128, so every
+//   quant_tokens x rows -> NVFP4 (E2M1 codes, one E4M3 scale per 16, unit
+//                tensor scale), once per token;
+//   gather_x     copies them in expert order into an expert-padded layout:
+//                expert e's rows start at a multiple of 128, so every
 //                128-row B tile and its scale atoms align.
 //   gemm<1>      D[128 x N] = W_gu tile (64 gate + 64 up rows) x X^T over K = d;
 //                epilogue: a = silu(g_g * D_gate) * (g_u * D_up), requantised
@@ -24,8 +25,9 @@
 //   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp of the scale
 //               atoms into TMEM, then 4 tcgen05.mma kind::mxf4nvf4 block16
 //               (K = 64 each) into one of two TMEM accumulators;
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp its 32
-//               TMEM lanes), overlapped with the next tile's main loop.
+//   warps 2-9   epilogue, two groups of four warps (each warp reads its 32
+//               TMEM lanes; the groups take alternate 16-column slabs),
+//               overlapped with the next tile's main loop.
 // Every wait is bounded; on expiry the CTA records MOE_ERR_TIMEOUT in the
 // status word, stops issuing, drains what it issued and frees its TMEM.
 #include <cuda.h>
@@ -45,11 +47,13 @@ constexpr int A_BYTES = BM * BKB;       // 16 KB
 constexpr int B_BYTES = BN * BKB;       // 16 KB
 constexpr int SF_BYTES = 2048;          // 4 atoms of 128 rows x 4 scales
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
-constexpr int EPI_BYTES = 16 * 128 * 4 + 2 * 128 * 4;   // transposed 16-column slab + column info
+constexpr int EPI_GROUPS = 2;           // epilogue warp groups (each covers the 4 TMEM lane quadrants)
+constexpr int EPI_THREADS = 128 * EPI_GROUPS;
+constexpr int EPI_BYTES = EPI_GROUPS * 16 * 128 * 4 + 2 * 128 * 4;   // a transposed 16-column slab per group + column info
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 128;           // per accumulator buffer
 constexpr int SFA_COL = 256, SFB_COL = 272;
-constexpr int THREADS = 192;
+constexpr int THREADS = 64 + EPI_THREADS;   // producer, MMA, epilogue groups
 constexpr uint64_t kWaitNs = 2000000000ull;   // every wait gives up after 2 s
 
 struct GemmParams {
@@ -121,28 +125,43 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// L2 policies: weights are streamed once (evict first); activation tiles are
+// re-read by every M tile of their group (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                            int z) {
+                                            int z, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -314,6 +333,21 @@ __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* 
   return total;
 }
 
+// Unit u -> (chunk, M tile).  GEMM1 runs chunk-major (the CTAs working at the
+// same time share one activation tile); GEMM2 runs M-tile-major, so the
+// tiles in flight all add into the same 128-column slab of out, which stays
+// in L2 while its ~6 contributions per element arrive.
+template <int PHASE>
+__device__ __forceinline__ void unit_coords(int u, int n_chunks, int MT, int* c, int* m) {
+  if (PHASE == 1) {
+    *c = u / MT;
+    *m = u % MT;
+  } else {
+    *m = u / n_chunks;
+    *c = u % n_chunks;
+  }
+}
+
 // expert of chunk c: the last e with chunk_start[e] <= c
 __device__ __forceinline__ int chunk_expert(const int32_t* chunk_start, int E, int c) {
   int lo = 0, hi = E;   // invariant: chunk_start[lo] <= c < chunk_start[hi]
@@ -326,34 +360,15 @@ __device__ __forceinline__ int chunk_expert(const int32_t* chunk_start, int E, i
 }
 
 // ------------------------------------------------------------------ quant_x
-// One warp per real token row of a chunk: NVFP4 codes into xq[128 c + r][d/2]
-// and scale bytes into the atom layout of the padded matrix.
-__global__ void __launch_bounds__(256) quant_x_kernel(const uint16_t* __restrict__ x, int d, int T, int k,
-                                                     int E, int n_slots, const int32_t* __restrict__ offsets,
-                                                     const int32_t* __restrict__ perm,
-                                                     const int32_t* __restrict__ slot, uint8_t* __restrict__ xq,
-                                                     uint8_t* __restrict__ xsf, int32_t* status) {
-  __shared__ int32_t chunk_start[1025];
-  __shared__ int ws[36];
-  const int n_pairs = T * k;
-  const int n_chunks = build_chunks(offsets, slot, E, n_pairs, n_slots, chunk_start, ws, status);
+// NVFP4 quantisation of each token row once (T rows, not T*k): codes into
+// xt[t][d/2] and scale bytes into xts[t][d/16], one warp per row.
+__global__ void __launch_bounds__(256) quant_tokens_kernel(const uint16_t* __restrict__ x, int d, int T,
+                                                          uint8_t* __restrict__ xt, uint8_t* __restrict__ xts) {
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
-  const long long rows = static_cast<long long>(n_chunks) * BN;
-  for (long long w = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); w < rows;
-       w += static_cast<long long>(gridDim.x) * warps) {
-    const int c = static_cast<int>(w / BN), r = static_cast<int>(w % BN);
-    const int e = chunk_expert(chunk_start, E, c);
-    const int q = offsets[e] + (c - chunk_start[e]) * BN + r;
-    if (q >= offsets[e + 1]) continue;                      // padding row: never read back
-    int p = perm[q];
-    if (p < 0 || p >= n_pairs) {
-      report(status, MOE_ERR_DEVICE);
-      p = 0;
-    }
-    const uint16_t* xr = x + static_cast<size_t>(p / k) * d;
-    const int prow = c * BN + r;
-    const int nb = d / 16;
+  const int nb = d / 16;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    const uint16_t* xr = x + static_cast<size_t>(t) * d;
     for (int b = lane; b < nb; b += 32) {
       const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b));
       const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(xr + 16 * b + 8));
@@ -375,10 +390,48 @@ __global__ void __launch_bounds__(256) quant_x_kernel(const uint16_t* __restrict
         q0[j] = (s > 0.f) ? __fdiv_rn(v[j], s) : 0.f;
         q1[j] = (s > 0.f) ? __fdiv_rn(v[8 + j], s) : 0.f;
       }
-      uint2 codes = make_uint2(pack8(q0), pack8(q1));
-      *reinterpret_cast<uint2*>(xq + static_cast<size_t>(prow) * (d / 2) + 8 * b) = codes;
-      xsf[sf_atom_offset(prow, b, d)] = static_cast<uint8_t>(sb);
+      *reinterpret_cast<uint2*>(xt + static_cast<size_t>(t) * (d / 2) + 8 * b) = make_uint2(pack8(q0), pack8(q1));
+      xts[static_cast<size_t>(t) * nb + b] = static_cast<uint8_t>(sb);
     }
+  }
+}
+
+// Gather: every real row of every chunk copies its token's codes into
+// xq[128 c + r][d/2] and its scale bytes, 4 blocks (one atom row) at a
+// time, into the atom layout of the padded matrix.  One warp per row.
+__global__ void __launch_bounds__(256) gather_x_kernel(const uint8_t* __restrict__ xt,
+                                                      const uint8_t* __restrict__ xts, int d, int T, int k, int E,
+                                                      int n_slots, const int32_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ perm,
+                                                      const int32_t* __restrict__ slot, uint8_t* __restrict__ xq,
+                                                      uint8_t* __restrict__ xsf, int32_t* status) {
+  __shared__ int32_t chunk_start[1025];
+  __shared__ int ws[36];
+  const int n_pairs = T * k;
+  const int n_chunks = build_chunks(offsets, slot, E, n_pairs, n_slots, chunk_start, ws, status);
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long rows = static_cast<long long>(n_chunks) * BN;
+  const int row_bytes = d / 2, nb = d / 16;
+  for (long long w = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); w < rows;
+       w += static_cast<long long>(gridDim.x) * warps) {
+    const int c = static_cast<int>(w / BN), r = static_cast<int>(w % BN);
+    const int e = chunk_expert(chunk_start, E, c);
+    const int q = offsets[e] + (c - chunk_start[e]) * BN + r;
+    if (q >= offsets[e + 1]) continue;                      // padding row: never read back
+    int p = perm[q];
+    if (p < 0 || p >= n_pairs) {
+      report(status, MOE_ERR_DEVICE);
+      p = 0;
+    }
+    const int t = p / k;
+    const int prow = c * BN + r;
+    const uint4* src = reinterpret_cast<const uint4*>(xt + static_cast<size_t>(t) * row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(prow) * row_bytes);
+    for (int i = lane; i < row_bytes / 16; i += 32) dst[i] = __ldg(src + i);
+    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(xts + static_cast<size_t>(t) * nb);
+    for (int g = lane; g < nb / 4; g += 32)
+      *reinterpret_cast<uint32_t*>(xsf + sf_atom_offset(prow, 4 * g, d)) = __ldg(ssrc + g);
   }
 }
 
@@ -390,8 +443,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
-  int32_t* col_t = reinterpret_cast<int32_t*>(epi + 16 * 128);
+  float* epi_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  int32_t* col_t = reinterpret_cast<int32_t*>(epi_all + EPI_GROUPS * 16 * 128);
   float* col_g = reinterpret_cast<float*>(col_t + 128);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
   uint64_t* full = bars;                   // [STAGES]
@@ -417,7 +470,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], EPI_THREADS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -433,16 +486,19 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int n_units = min(n_chunks, P.max_chunks) * MT;
+  const int n_chunks_used = min(n_chunks, P.max_chunks);
+  const int n_units = n_chunks_used * MT;
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
+    const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int c = u / MT, m = u % MT;
+      int c, m;
+      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int sl = P.slot[e];
       const uint8_t* sfa_src = P.pool + static_cast<size_t>(sl) * P.blob_bytes +
@@ -459,10 +515,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           uint8_t* sSFA = sB + B_BYTES;
           uint8_t* sSFB = sSFA + SF_BYTES;
           mbar_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl);
-          tma_load_2d(sB, &tm_act, &full[stage], ks * BKB, c * BN);
-          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage]);
-          bulk_load(sSFB, sfb_src + ks * SF_BYTES, SF_BYTES, &full[stage]);
+          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl, pol_stream);
+          tma_load_2d(sB, &tm_act, &full[stage], ks * BKB, c * BN, pol_keep);
+          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_stream);
+          bulk_load(sSFB, sfb_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_keep);
         }
         __syncwarp();
         ++issued;
@@ -495,7 +551,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const int c = u / MT;
+      int c, m_unused;
+      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m_unused);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
       const int nvalid = min(BN, P.offsets[e + 1] - row0);
@@ -551,14 +608,19 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     __syncwarp();
     mbar_drain(drain, 0);
   } else {
-    // ---------------------------------------------------------- epilogue (warps 2..5)
+    // ---------------------------------------------------------- epilogue (warps 2..9)
     const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
-    const int et = (warp - 2) * 32 + lane;      // 0..127 within the epilogue group
+    const int grp = (warp - 2) >> 2;            // column group: slabs grp, grp+2, ...
+    const int et = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
+    const int eall = (warp - 2) * 32 + lane;       // 0..255 over both groups
+    float* epi = epi_all + grp * 16 * 128;
+    const int bar_grp = 1 + grp, bar_all = 3;
     const float* ts = nullptr;
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const int c = u / MT, m = u % MT;
+      int c, m;
+      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
       const int nvalid = min(BN, P.offsets[e + 1] - row0);
@@ -567,13 +629,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       const int acc = it & 1;
       if (PHASE == 2) {
         // column c <-> pair at sorted position row0 + c: its token and gate
-        named_sync(1, 128);               // the previous tile's readers are done
-        if (et < nvalid) {
-          const int p = P.perm[row0 + et];
+        named_sync(bar_all, EPI_THREADS);       // the previous tile's readers are done
+        if (eall < nvalid) {
+          const int p = P.perm[row0 + eall];
           const bool good = p >= 0 && p < n_pairs;
           if (!good) report(P.status, MOE_ERR_DEVICE);
-          col_t[et] = good ? p / P.k : -1;
-          col_g[et] = good ? P.gate[p] : 0.f;
+          col_t[eall] = good ? p / P.k : -1;
+          col_g[eall] = good ? P.gate[p] : 0.f;
         }
       }
       if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag)) {
@@ -582,10 +644,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       }
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS;
-      if (PHASE == 2) named_sync(1, 128);
+      if (PHASE == 2) named_sync(bar_all, EPI_THREADS);
       const float g_mat = (PHASE == 1) ? 0.f : __ldg(ts + 2);
       const float g_gate = (PHASE == 1) ? __ldg(ts + 0) : 0.f, g_up = (PHASE == 1) ? __ldg(ts + 1) : 0.f;
-      for (int cc = 0; cc < nvalid; cc += 16) {
+      for (int cc = 16 * grp; cc < nvalid; cc += 16 * EPI_GROUPS) {
         float v[16];
         tmem_ld16(tbase + cc, v);
         if (PHASE == 2) {
@@ -603,7 +665,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           // transpose the 16-column slab through shared memory: epi[col][row]
 #pragma unroll
           for (int j = 0; j < 16; ++j) epi[j * 128 + 32 * quad + lane] = v[j];
-          named_sync(1, 128);
+          named_sync(bar_grp, 128);
           // item: column cl, 16-block b of the 64 intermediate indices, half h
           const int cl = et >> 3, b = (et >> 1) & 3, h = et & 1;
           const int col = cc + cl;
@@ -614,7 +676,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
             const int il = 16 * b + 8 * h + j;
             const float hg = epi[cl * 128 + il] * g_gate;
             const float hu = epi[cl * 128 + 64 + il] * g_up;
-            a[j] = __fdiv_rn(hg, 1.0f + expf(-hg)) * hu;
+            a[j] = __fdividef(hg, 1.0f + __expf(-hg)) * hu;
             amax = fmaxf(amax, fabsf(a[j]));
           }
           amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
@@ -631,7 +693,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
                 codes;
             if (h == 0) P.aq_sf[sf_atom_offset(prow, i0 / 16 + b, P.I)] = static_cast<uint8_t>(sb);
           }
-          named_sync(1, 128);
+          named_sync(bar_grp, 128);
         }
       }
       tc_fence_before();
@@ -680,7 +742,7 @@ moe_status make_map(CUtensorMap* map, const void* base, int rank, const uint64_t
 
 struct PrefillWs {
   size_t rows;            // padded row capacity (multiple of 128)
-  size_t xq, xsf, aq, asf, bytes;
+  size_t xt, xts, xq, xsf, aq, asf, bytes;
 };
 
 PrefillWs prefill_ws(moe_shape s, int T, int k) {
@@ -689,6 +751,8 @@ PrefillWs prefill_ws(moe_shape s, int T, int k) {
   const size_t act = n < static_cast<size_t>(s.E) ? n : static_cast<size_t>(s.E);
   w.rows = round_up(n + act * (BN - 1), BN);
   size_t o = 0;
+  w.xt = o; o = round_up(o + static_cast<size_t>(T) * (s.d / 2), 1024);
+  w.xts = o; o = round_up(o + static_cast<size_t>(T) * (s.d / 16), 1024);
   w.xq = o; o = round_up(o + w.rows * (s.d / 2), 1024);
   w.xsf = o; o = round_up(o + w.rows * (s.d / 16), 1024);
   w.aq = o; o = round_up(o + w.rows * (s.I / 2), 1024);
@@ -764,10 +828,14 @@ moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const in
     long long blocks = (rows + 7) / 8;
     const long long cap = static_cast<long long>(dev.sm_count) * 8;
     if (blocks > cap) blocks = cap;
-    quant_x_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), s.d, T, k,
-                                                                 s.E, n_slots, offsets, perm, slot, xq, xsf,
-                                                                 status);
-    MOE_LAUNCH_CHECK("quant_x_kernel");
+    long long tb = (static_cast<long long>(T) + 7) / 8;
+    if (tb > cap) tb = cap;
+    quant_tokens_kernel<<<static_cast<int>(tb), 256, 0, stream>>>(static_cast<const uint16_t*>(x), s.d, T,
+                                                                 base + w.xt, base + w.xts);
+    MOE_LAUNCH_CHECK("quant_tokens_kernel");
+    gather_x_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(base + w.xt, base + w.xts, s.d, T, k, s.E,
+                                                                  n_slots, offsets, perm, slot, xq, xsf, status);
+    MOE_LAUNCH_CHECK("gather_x_kernel");
   }
   GemmParams P{};
   P.E = s.E;

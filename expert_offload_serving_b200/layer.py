@@ -84,8 +84,11 @@ class MoeLayer:
             self.slot = torch.full((E,), -1, **i32)
             self.cache = MoeCache(self.s, n_slots, self.pool, host_pool, self.slot)
             self.side = torch.cuda.Stream(device=self.dev)
+            # torch creates a CUDA event lazily on first record: record both now
+            # so that their handles exist when the library records and waits on them
             self.fill_done = torch.cuda.Event()
             self.reads_done = torch.cuda.Event()
+            self.fill_done.record(self.side)
             self.reads_done.record()
 
     # -- steps -----------------------------------------------------------------

@@ -65,9 +65,15 @@ def _host_ptr(a):
 
 
 def test_argument_errors_before_any_cuda_call(moe):
+    """Every check runs before the first CUDA call: on a machine without a GPU
+    each bad call returns MOE_ERR_INVALID_ARG (never MOE_ERR_CUDA).  The buffer
+    is 256-byte aligned so that only the intended argument is wrong."""
     L_ = moe.lib()
-    buf = np.zeros(1024, dtype=np.float32)
+    raw = np.zeros(2048, dtype=np.float32)
+    shift = (-_host_ptr(raw)) % 256 // 4
+    buf = raw[shift: shift + 1024]
     p = _host_ptr(buf)
+    assert p % 256 == 0
     assert L_.moe_route_topk(p, 4, 8, 9, p, p, None) == moe.MOE_ERR_INVALID_ARG      # k > E
     assert L_.moe_route_topk(p, 4, 2000, 2, p, p, None) == moe.MOE_ERR_INVALID_ARG   # E > 1024
     assert L_.moe_route_topk(p, 4, 64, 33, p, p, None) == moe.MOE_ERR_INVALID_ARG    # k > 32
@@ -84,6 +90,12 @@ def test_argument_errors_before_any_cuda_call(moe):
                              None) == moe.MOE_ERR_INVALID_ARG                          # misaligned x
     assert L_.moe_expert_ffn(s, p, 4, 2, p, p, p, p, 8, p, p, None, 1, p, 1 << 20, None,
                              None) == moe.MOE_ERR_INVALID_ARG                          # act flag, bf16
+    assert b"NVFP4" in L_.moe_last_error()
+    s_nv = moe.shape(8, 384, 256, "nvfp4")
+    assert L_.moe_expert_ffn(s_nv, p, 4, 2, p, p, p, p, 8, p, None, p, 1, p, 1 << 30, None,
+                             None) == moe.MOE_ERR_INVALID_ARG                          # d % 256 != 0
+    assert L_.moe_expert_ffn(s, p, 4, 2, p, p, p, p, 8, p, p, None, 0, p, 16, None,
+                             None) == moe.MOE_ERR_CAPACITY                             # workspace too small
     assert L_.moe_combine_merge(p, p, p, p, None, None, 4, 2, 6, 8, p, None) == moe.MOE_ERR_INVALID_ARG
     assert L_.moe_cache_fill(None, None, 0, 0, None, 0, None, None, None, None, None) == \
         moe.MOE_ERR_INVALID_ARG

@@ -242,6 +242,9 @@ def test_cached_layer_trace(moe):
         layer.permute(T)
         layer.ffn(x.cuda())
         layer.combine(T)
+        # the main stream waited for this step's fills: once it drains, the side stream is idle
+        torch.cuda.current_stream().synchronize()
+        assert layer.side.query()
         out = layer.out[:T].cpu().numpy()
         ref = M.moe_layer(x.double().numpy(), logits.numpy(), cfg.k, weights)["out"]
         check_tol(out, ref, 1e-4, 1e-5)

@@ -67,3 +67,26 @@ def test_prefill_full_size_sampled(moe):
     toks = [0, 1, 2047, 4095]
     ref = b.oracle(tokens=toks)["out"]
     check_tol(out[toks], ref[toks])
+
+
+def test_activation_codes_bit_exact(moe):
+    """The NVFP4 quantisation of x (first stage of the tensor-core path) takes
+    its decisions in fp32 exactly as the oracle does: every per-token scale
+    and dequantised code must match bit for bit.  Reads the workspace's
+    per-token region (codes [T][d/2], then scales [T][d/16] at the next
+    1024-byte boundary)."""
+    from oracle import formats as F
+    cfg = _cfg("pf_codes", 8, 2, 512, 256)
+    T = 96
+    b = Built(cfg, T, seed=21, act="nvfp4")
+    b.run()
+    ws = b.layer.workspace.cpu().numpy()
+    d = cfg.d
+    codes = ws[: T * d // 2].reshape(T, d // 2)
+    off = (T * d // 2 + 1023) // 1024 * 1024
+    scales = ws[off: off + T * d // 16].reshape(T, d // 16)
+    deq_ref, s_ref, _ = F.nvfp4_quantize_rows(b.x.float().numpy())
+    got_s = F.e4m3_decode(scales)
+    assert np.array_equal(got_s, s_ref)
+    got = F.e2m1_decode(F.unpack_nibbles(codes)) * np.repeat(got_s, 16, axis=1)
+    assert np.array_equal(got, deq_ref)
