@@ -150,18 +150,28 @@ def barrier(world):
 
 
 # ---------------------------------------------------------------- workload
-def build_replicas(cfg, T, R, seed0=0):
-    """R independent resident layers with their inputs on the device."""
+def build_replicas(cfg, T, R, seed0=0, routed_only=False):
+    """R independent resident layers with their inputs on the device.
+    routed_only: materialise only the experts the batch's top-k selects (the
+    slot table maps them; the others are never read)."""
     from expert_offload_serving_b200.layer import MoeLayer, pack_pool
     reps = []
     for r in range(R):
         seed = seed0 + r
         logits, x = synth.make_routing(cfg, T, seed)
-        w = synth.make_experts(cfg, range(cfg.E), seed, device="cuda")
+        if routed_only:
+            experts = sorted(set(torch.topk(logits, cfg.k, dim=1).indices.ravel().tolist()))
+        else:
+            experts = list(range(cfg.E))
+        w = synth.make_experts(cfg, experts, seed, device="cuda")
         pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()},
-                         range(cfg.E), pin=False).cuda()
+                         experts, pin=False).cuda()
         del w
         layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=pool)
+        if routed_only:
+            layer.slot.fill_(-1)
+            layer.slot[torch.tensor(experts, device=layer.slot.device)] = torch.arange(
+                len(experts), dtype=torch.int32, device=layer.slot.device)
         reps.append(dict(layer=layer, logits=logits.cuda(), x=x.cuda(), logits_h=logits.pin_memory(),
                          x_h=x.pin_memory()))
     return reps
@@ -174,12 +184,12 @@ def experts_touched(layer):
     return int(((off[1:] - off[:-1]) > 0).sum())
 
 
-def decode_point(cfg, T, R, warmup, steps, stream):
+def decode_point(cfg, T, R, warmup, steps, stream, routed_only=False):
     """Device-timed decode_bf16 layer steps at T tokens (graph replay over R
     replicas) and the expert-FFN time alone, for the secondary T points."""
     import expert_offload_serving_b200 as moe
     blob = moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
-    reps = build_replicas(cfg, T, R, seed0=500 + T)
+    reps = build_replicas(cfg, T, R, seed0=500 + T, routed_only=routed_only)
     U = []
     for r in reps:
         r["layer"].forward(r["logits"], r["x"])
@@ -326,14 +336,21 @@ def run_gpu(args, rank, world, local):
 
     prefill = None
     if not args.no_prefill:
-        prefill = run_prefill()
+        prefill = run_prefill(Ts=(4096,) if (args.no_sweep or world > 1) else (4096, 16384, 32768))
     sweep = None
     if not args.no_sweep and world == 1:
         sweep = {}
         for t in (1, 16):
             if t == T:
                 continue
-            sweep[f"T{t}"] = decode_point(cfg, t, R, args.warmup, min(args.steps, 2000), stream)
+            # T=1 touches ~75 MB: 8 replicas stream >= 4x L2 between two uses of one
+            sweep[f"T{t}"] = decode_point(cfg, t, max(R, 8) if t == 1 else R, args.warmup,
+                                          min(args.steps, 2000), stream)
+    mx = None
+    if not args.no_sweep and world == 1:
+        cmx = synth.CONFIGS["decode_mxfp4"]
+        mx = {f"T{t}": decode_point(cmx, t, 8, args.warmup, min(args.steps, 1000), stream, routed_only=True)
+              for t in cmx.T}
     cached = None
     if not args.no_cached:
         hp = cached_host_pool()
@@ -383,76 +400,88 @@ def run_gpu(args, rank, world, local):
     if cpu is not None:
         result["cpu_baseline"] = cpu
     if prefill is not None:
-        result["prefill"] = prefill
+        result["prefill"] = prefill[0]
+        if len(prefill) > 1:
+            result["prefill_T_sweep"] = prefill[1:]
     if cached is not None:
         result["decode_mxfp4_cached"] = cached
     if sweep:
         result["decode_bf16_T_sweep"] = sweep
+    if mx:
+        result["decode_mxfp4_resident"] = mx
     return result
 
 
 # ---------------------------------------------------------------- prefill (FP4 tensor cores)
-def run_prefill(iters=20, warmup=5, T=4096):
-    """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, T tokens, NVFP4
-    activations on tcgen05): whole-layer time and the expert-FFN time alone.
-    The 3.6 GB of weights exceed L2 many times over, so no replicas."""
+def run_prefill(iters=20, warmup=5, Ts=(4096,)):
+    """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, NVFP4 activations
+    on tcgen05) at each token count in Ts: whole-layer time and the expert-FFN
+    time alone.  The 3.6 GB of weights exceed L2 many times over, so no
+    replicas.  T=4096 is bound by the weight read; at 16384 and 32768 tokens
+    the FP4 contraction dominates."""
     import expert_offload_serving_b200 as moe
     from expert_offload_serving_b200.layer import MoeLayer, pack_pool
     cfg = synth.CONFIGS["prefill_nvfp4"]
-    logits, x = synth.make_routing(cfg, T, 0)
     w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
     pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()}, range(cfg.E),
                      pin=False).cuda()
     del w
-    layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=pool, act="nvfp4")
-    lg, xx = logits.cuda(), x.cuda()
-    stream = torch.cuda.Stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for _ in range(warmup):
-            layer.forward(lg, xx)
-        e0.record(stream)
-        for _ in range(iters):
-            layer.forward(lg, xx)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        layer_ms = e0.elapsed_time(e1) / iters
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(iters):
-            layer.ffn(xx)
-        f1.record(stream)
-    torch.cuda.synchronize()
-    ffn_ms = f0.elapsed_time(f1) / iters
-    moe.moe_check_status(layer.status)
-    flops = 2.0 * 3 * cfg.d * cfg.I * T * cfg.k
-    off = layer.offsets.cpu()
-    U = int(((off[1:] - off[:-1]) > 0).sum())
-    wbytes = U * moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
+    layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, max(Ts), device_pool=pool, act="nvfp4")
     d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     bf16 = d.get("bf16_tflops", 1590.0)
     fp4_peak = 4.0 * bf16          # dense FP4 = 4 x dense BF16 (nominal 9 / 2.25 PFLOP/s)
     hbm, _ = peaks()
-    tf = flops / (ffn_ms / 1e3) / 1e12
-    gbs = wbytes / (ffn_ms / 1e3) / 1e9
-    roof_ms = max(wbytes / (hbm * 1e9), flops / (fp4_peak * 1e12)) * 1e3
-    return {
-        "workload": f"prefill_nvfp4: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, NVFP4 weights and activations",
-        "tokens_per_s": round(T / (layer_ms / 1e3), 1),
-        "layer_ms": round(layer_ms, 4),
-        "ffn_ms": round(ffn_ms, 4),
-        "tflops": round(tf, 1),
-        "fp4_peak_tflops": round(fp4_peak, 1),
-        "fp4_peak_source": "4 x measured bf16 (MEASURED_PEAKS.json bf16_tflops)",
-        "frac_fp4_peak": round(tf / fp4_peak, 4),
-        "weight_gbs": round(gbs, 1),
-        "frac_hbm": round(gbs / hbm, 4),
-        "roofline_ms": round(roof_ms, 4),
-        "frac_roofline": round(roof_ms / ffn_ms, 4),
-        "experts_touched": U,
-        "kernels": "quant_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2>",
-    }
+    out = []
+    for T in Ts:
+        logits, x = synth.make_routing(cfg, T, 0)
+        lg, xx = logits.cuda(), x.cuda()
+        stream = torch.cuda.Stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = iters if T <= 4096 else max(3, iters // 4)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                layer.forward(lg, xx)
+            e0.record(stream)
+            for _ in range(n):
+                layer.forward(lg, xx)
+            e1.record(stream)
+            f0.record(stream)
+            for _ in range(n):
+                layer.ffn(xx)
+            f1.record(stream)
+        torch.cuda.synchronize()
+        layer_ms = e0.elapsed_time(e1) / n
+        ffn_ms = f0.elapsed_time(f1) / n
+        moe.moe_check_status(layer.status)
+        flops = 2.0 * 3 * cfg.d * cfg.I * T * cfg.k
+        off = layer.offsets.cpu()
+        U = int(((off[1:] - off[:-1]) > 0).sum())
+        wbytes = U * moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
+        tf = flops / (ffn_ms / 1e3) / 1e12
+        gbs = wbytes / (ffn_ms / 1e3) / 1e9
+        roof_ms = max(wbytes / (hbm * 1e9), flops / (fp4_peak * 1e12)) * 1e3
+        out.append({
+            "workload": f"prefill_nvfp4: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, "
+                        "NVFP4 weights and activations",
+            "tokens_per_s": round(T / (layer_ms / 1e3), 1),
+            "layer_ms": round(layer_ms, 4),
+            "ffn_ms": round(ffn_ms, 4),
+            "tflops": round(tf, 1),
+            "fp4_peak_tflops": round(fp4_peak, 1),
+            "fp4_peak_source": "4 x measured bf16 (MEASURED_PEAKS.json bf16_tflops)",
+            "frac_fp4_peak": round(tf / fp4_peak, 4),
+            "weight_gbs": round(gbs, 1),
+            "frac_hbm": round(gbs / hbm, 4),
+            "roofline_ms": round(roof_ms, 4),
+            "frac_roofline": round(roof_ms / ffn_ms, 4),
+            "experts_touched": U,
+            "timed_iters": n,
+            "kernels": "quant_tokens_kernel, gather_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2>",
+        })
+        del lg, xx
+    return out
 
 
 # ---------------------------------------------------------------- decode with the expert cache
@@ -629,7 +658,9 @@ def main(argv=None):
         args.warmup = 3
     rank, world, local = dist_setup(args.gpus)
     if args.only_prefill:
-        print(json.dumps(run_prefill(iters=max(3, min(args.steps, 50)), warmup=args.warmup)), flush=True)
+        res = run_prefill(iters=max(3, min(args.steps, 50)), warmup=args.warmup,
+                          Ts=(4096,) if args.no_sweep else (4096, 16384, 32768))
+        print(json.dumps(res[0] if len(res) == 1 else res), flush=True)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)

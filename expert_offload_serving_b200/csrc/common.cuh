@@ -41,7 +41,8 @@ moe_status current_device(DeviceInfo* out);
 
 // ---------------------------------------------------------------- blob layout
 // One expert = one blob; every region starts on a 256-byte boundary.
-//   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16, row-major).
+//   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16; row-major, or blocked when
+//          bf16_blocked(d, I) -- see blocked_offset).
 //   MXFP4: codes wg [I][d/2], wu [I][d/2], wd [d][I/2] (low nibble = even
 //          element), then E8M0 scales sg [I][d/32], su [I][d/32], sd [d][I/32].
 //   NVFP4: codes of W_gu [2I][d/2] -- gate and up rows interleaved in blocks
@@ -82,6 +83,34 @@ __host__ __device__ inline BlobLayout blob_layout(int fmt, int d, int I) {
   }
   L.bytes = o;
   return L;
+}
+
+// bf16 blobs whose d and I are multiples of 256 store each matrix in blocks
+// for the decode MMA path: block (rb, ks) = rows [RB*rb, RB*rb + RB) x
+// elements [kBlockK*ks, kBlockK*ks + kBlockK), RB = 16 for W_g and W_u, 32 for
+// W_d; the blocks of a matrix are ordered [rb][ks], each block holds its rows
+// as lines of 2*kBlockK bytes, and inside a line the 16-byte chunk c (8 elements) sits at position
+// c ^ (row % 8) -- so one stage of the decode pipeline is one contiguous copy
+// and ldmatrix reads of 8 rows hit 8 different bank groups.  Inside every
+// group of 32 elements along K the elements are stored in the order
+// kpos32: the MMA k-steps 2j and 2j+1 then see, in the B-fragment slots of
+// lane group t, the 8 contiguous activations 32j + 8t .. 32j + 8t + 7, which
+// the lane fetches with one 16-byte load.
+__host__ __device__ inline bool bf16_blocked(int d, int I) { return d % 256 == 0 && I % 256 == 0; }
+constexpr int kBlockK = 128;   // elements per line of a block
+
+// Stored position of element k (0..31) of a 32-element group: MMA k-step
+// (k >> 2) & 1, fragment register (k >> 1) & 1, lane group k >> 3, half k & 1.
+__host__ __device__ inline int kpos32(int k) {
+  return ((k >> 2) & 1) * 16 + ((k >> 1) & 1) * 8 + (k >> 3) * 2 + (k & 1);
+}
+
+// Byte offset, inside a blocked matrix with K columns, of element (r, k).
+__host__ __device__ inline size_t blocked_offset(int r, int k, int K, int RB) {
+  const int p = (k & ~31) | kpos32(k & 31);
+  const size_t block = static_cast<size_t>(r / RB) * (K / kBlockK) + p / kBlockK;
+  const int rr = r % RB, c = (p % kBlockK) >> 3;
+  return (block * RB + rr) * (2 * kBlockK) + ((c ^ (rr & 7)) << 4) + (p & 7) * 2;
 }
 
 // Row of W_gu holding gate row i (up = false) or up row i (up = true).

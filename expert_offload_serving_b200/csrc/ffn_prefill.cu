@@ -17,7 +17,8 @@
 //                epilogue: a = silu(g_g * D_gate) * (g_u * D_up), requantised
 //                to NVFP4 into the padded A matrix.
 //   gemm<2>      D = W_d tile (128 rows of d) x A^T over K = I; epilogue:
-//                out[t][row] += gate * g_d * D  (red.global.add, the combine).
+//                out[t][row] += gate * g_d * D  (red.global.add.v4 on 4
+//                consecutive rows after a shared-memory transpose: the combine).
 // gemm is a persistent kernel, one CTA per SM, warp-specialised:
 //   warp 0      TMA producer: 128x128-byte A and B tiles (SWIZZLE_128B, no
 //               multicast) plus the 2 KB scale-atom slices by bulk copy, into
@@ -651,16 +652,30 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
         float v[16];
         tmem_ld16(tbase + cc, v);
         if (PHASE == 2) {
-          const int row = m * BM + 32 * quad + lane;
+          // transpose the slab through shared memory (epi[col][row]), then each
+          // thread adds 4 consecutive output rows of one column with one
+          // vector reduction: out[t][row .. row+3] += gate * g_d * y
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = cc + j;
+          for (int j = 0; j < 16; ++j) epi[j * 128 + 32 * quad + lane] = v[j];
+          named_sync(bar_grp, 128);
+#pragma unroll
+          for (int it2 = 0; it2 < 4; ++it2) {
+            const int item = et + 128 * it2;          // 16 columns x 32 row quads
+            const int cl = item >> 5, rq = item & 31;
+            const int col = cc + cl;
             if (col < nvalid) {
               const int t = col_t[col];
-              if (t >= 0)
-                atomicAdd(P.out + static_cast<size_t>(t) * P.d + row, col_g[col] * (g_mat * v[j]));
+              if (t >= 0) {
+                const float gm = col_g[col] * g_mat;
+                const float4 y = *reinterpret_cast<const float4*>(epi + cl * 128 + 4 * rq);
+                float* dst = P.out + static_cast<size_t>(t) * P.d + m * BM + 4 * rq;
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(gm * y.x),
+                             "f"(gm * y.y), "f"(gm * y.z), "f"(gm * y.w)
+                             : "memory");
+              }
             }
           }
+          named_sync(bar_grp, 128);
         } else {
           // transpose the 16-column slab through shared memory: epi[col][row]
 #pragma unroll

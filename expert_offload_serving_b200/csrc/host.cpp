@@ -89,9 +89,23 @@ extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* w
   std::memset(b, 0, L.bytes);
   const size_t m = static_cast<size_t>(s.I) * s.d;
   if (s.fmt == MOE_W_BF16) {
-    std::memcpy(b + L.wg, wg, m * 2);
-    std::memcpy(b + L.wu, wu, m * 2);
-    std::memcpy(b + L.wd, wd, m * 2);
+    if (!bf16_blocked(s.d, s.I)) {
+      std::memcpy(b + L.wg, wg, m * 2);
+      std::memcpy(b + L.wu, wu, m * 2);
+      std::memcpy(b + L.wd, wd, m * 2);
+      return MOE_OK;
+    }
+    // blocked layout: every element to its place (blocks, k order, swizzle)
+    struct Mt { const uint16_t* src; size_t off; int R, K, RB; } mats[3] = {
+        {static_cast<const uint16_t*>(wg), L.wg, s.I, s.d, 16},
+        {static_cast<const uint16_t*>(wu), L.wu, s.I, s.d, 16},
+        {static_cast<const uint16_t*>(wd), L.wd, s.d, s.I, 32}};
+    for (const Mt& mt : mats)
+      for (int r = 0; r < mt.R; ++r) {
+        const uint16_t* row = mt.src + static_cast<size_t>(r) * mt.K;
+        for (int k = 0; k < mt.K; ++k)
+          std::memcpy(b + mt.off + blocked_offset(r, k, mt.K, mt.RB), row + k, 2);
+      }
     return MOE_OK;
   }
   MOE_REQUIRE(sg && su && sd, "null scale pointer for an FP4 format");

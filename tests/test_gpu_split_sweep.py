@@ -48,7 +48,7 @@ def test_q_sweep(moe):
         return deq[e]
 
     report = []
-    for q in (0.0, 0.25, 0.5, 0.75, 1.0):
+    for q in [i / 10 for i in range(11)]:
         layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, host_pool=host_pool, n_slots=cfg.n_slots)
         lru = L.LRUCache(cfg.n_slots, cfg.E)
         gpu_ms = host_ms = 0.0
