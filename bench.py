@@ -16,6 +16,7 @@ Multi-GPU: launch with torchrun; every rank runs its own replica set
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -413,7 +414,7 @@ def run_gpu(args, rank, world, local):
 
 
 # ---------------------------------------------------------------- prefill (FP4 tensor cores)
-def run_prefill(iters=20, warmup=5, Ts=(4096,)):
+def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None):
     """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, NVFP4 activations
     on tcgen05) at each token count in Ts: whole-layer time and the expert-FFN
     time alone.  The 3.6 GB of weights exceed L2 many times over, so no
@@ -422,6 +423,9 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,)):
     import expert_offload_serving_b200 as moe
     from expert_offload_serving_b200.layer import MoeLayer, pack_pool
     cfg = synth.CONFIGS["prefill_nvfp4"]
+    if E is not None and E != cfg.E:
+        # a smaller expert count at the same d, I, k (for short profiler captures)
+        cfg = dataclasses.replace(cfg, E=E)
     w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
     pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()}, range(cfg.E),
                      pin=False).cuda()
@@ -651,6 +655,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the FP4 prefill measurement")
     ap.add_argument("--only-prefill", action="store_true", help="print only the FP4 prefill measurement")
+    ap.add_argument("--prefill-T", type=int, default=0, help="with --only-prefill: this token count only")
+    ap.add_argument("--prefill-E", type=int, default=None,
+                    help="with --only-prefill: this many experts instead of 256 (smaller captures)")
     ap.add_argument("--no-cached", action="store_true", help="skip the expert-cache decode measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the T=1 and T=16 decode points")
     args = ap.parse_args(argv)
@@ -658,8 +665,8 @@ def main(argv=None):
         args.warmup = 3
     rank, world, local = dist_setup(args.gpus)
     if args.only_prefill:
-        res = run_prefill(iters=max(3, min(args.steps, 50)), warmup=args.warmup,
-                          Ts=(4096,) if args.no_sweep else (4096, 16384, 32768))
+        Ts = (args.prefill_T,) if args.prefill_T else ((4096,) if args.no_sweep else (4096, 16384, 32768))
+        res = run_prefill(iters=max(3, min(args.steps, 50)), warmup=args.warmup, Ts=Ts, E=args.prefill_E)
         print(json.dumps(res[0] if len(res) == 1 else res), flush=True)
         return
     if args.impl == "reference":

@@ -41,8 +41,8 @@ moe_status current_device(DeviceInfo* out);
 
 // ---------------------------------------------------------------- blob layout
 // One expert = one blob; every region starts on a 256-byte boundary.
-//   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16; row-major, or blocked when
-//          bf16_blocked(d, I) -- see blocked_offset).
+//   BF16 : wg [I][d], wu [I][d], wd [d][I] (bf16; row-major, or in the
+//          tensor-core tile layout when bf16_blocked(d, I) -- sw128_offset).
 //   MXFP4: codes wg [I][d/2], wu [I][d/2], wd [d][I/2] (low nibble = even
 //          element), then E8M0 scales sg [I][d/32], su [I][d/32], sd [d][I/32].
 //   NVFP4: codes of W_gu [2I][d/2] -- gate and up rows interleaved in blocks
@@ -85,32 +85,21 @@ __host__ __device__ inline BlobLayout blob_layout(int fmt, int d, int I) {
   return L;
 }
 
-// bf16 blobs whose d and I are multiples of 256 store each matrix in blocks
-// for the decode MMA path: block (rb, ks) = rows [RB*rb, RB*rb + RB) x
-// elements [kBlockK*ks, kBlockK*ks + kBlockK), RB = 16 for W_g and W_u, 32 for
-// W_d; the blocks of a matrix are ordered [rb][ks], each block holds its rows
-// as lines of 2*kBlockK bytes, and inside a line the 16-byte chunk c (8 elements) sits at position
-// c ^ (row % 8) -- so one stage of the decode pipeline is one contiguous copy
-// and ldmatrix reads of 8 rows hit 8 different bank groups.  Inside every
-// group of 32 elements along K the elements are stored in the order
-// kpos32: the MMA k-steps 2j and 2j+1 then see, in the B-fragment slots of
-// lane group t, the 8 contiguous activations 32j + 8t .. 32j + 8t + 7, which
-// the lane fetches with one 16-byte load.
+// bf16 blobs whose d and I are multiples of 256 store their matrices in the
+// tensor-core tile layout of the decode GEMV: W_gu = the gate and up rows
+// interleaved in blocks of 64 (gu_row), occupying the wg and wu regions as one
+// [2I][d] matrix, and W_d [d][I]; each as tiles of 128 rows x 64 elements
+// (16 KB), ordered [row / 128][k / 64], so a tile's K range is contiguous and
+// one pipeline stage is one bulk copy.  Inside a tile row r is a 128-byte line
+// whose 16-byte chunk c (8 elements) sits at c ^ (r % 8): the canonical
+// 128-byte-swizzled K-major operand layout of tcgen05.mma.
 __host__ __device__ inline bool bf16_blocked(int d, int I) { return d % 256 == 0 && I % 256 == 0; }
-constexpr int kBlockK = 128;   // elements per line of a block
 
-// Stored position of element k (0..31) of a 32-element group: MMA k-step
-// (k >> 2) & 1, fragment register (k >> 1) & 1, lane group k >> 3, half k & 1.
-__host__ __device__ inline int kpos32(int k) {
-  return ((k >> 2) & 1) * 16 + ((k >> 1) & 1) * 8 + (k >> 3) * 2 + (k & 1);
-}
-
-// Byte offset, inside a blocked matrix with K columns, of element (r, k).
-__host__ __device__ inline size_t blocked_offset(int r, int k, int K, int RB) {
-  const int p = (k & ~31) | kpos32(k & 31);
-  const size_t block = static_cast<size_t>(r / RB) * (K / kBlockK) + p / kBlockK;
-  const int rr = r % RB, c = (p % kBlockK) >> 3;
-  return (block * RB + rr) * (2 * kBlockK) + ((c ^ (rr & 7)) << 4) + (p & 7) * 2;
+// Byte offset of element (r, k) of a tile-layout matrix with K columns.
+__host__ __device__ inline size_t sw128_offset(int r, int k, int K) {
+  const size_t tile = static_cast<size_t>(r >> 7) * (K >> 6) + (k >> 6);
+  const int rr = r & 127, c = (k >> 3) & 7;
+  return tile * 16384 + static_cast<size_t>(rr) * 128 + ((c ^ (rr & 7)) << 4) + (k & 7) * 2;
 }
 
 // Row of W_gu holding gate row i (up = false) or up row i (up = true).
@@ -129,10 +118,41 @@ __host__ __device__ inline size_t sf_atom_offset(int r, int b, int K) {
 moe_status check_shape(moe_shape s);
 
 // ---------------------------------------------------------------- device helpers
+constexpr unsigned kFull = 0xffffffffu;
+
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
-constexpr unsigned kFull = 0xffffffffu;
+// Exclusive block scan (blockDim <= 1024); ws >= 33 ints of shared memory.
+__device__ inline int block_scan(int v, int* ws, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) ws[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    const int w = (lane < nw) ? ws[lane] : 0;
+    int s = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, s, o);
+      if (lane >= o) s += y;
+    }
+    ws[lane] = s - w;
+    if (lane == 31) ws[32] = s;
+  }
+  __syncthreads();
+  const int r = ws[warp] + x - v;
+  *total = ws[32];
+  __syncthreads();
+  return r;
+}
+
 
 }  // namespace moe

@@ -23,9 +23,9 @@
 // 16-byte chunks (32 FP4 weights): conflict-free 128-bit shared loads, E2M1 ->
 // f16x2 by cvt, times the E8M0 or E4M3 block scale, packed fp32 FMAs against
 // the activations (read through L1), and a warp reduce-scatter at the end.
-// bf16 weights (warp MMA, mmap namespace below): 32-row tiles multiplied by
-// ldmatrix + mma.sync.m16n8k16 (bf16 x bf16 -> fp32), <= 32 token rows per
-// pass.
+// bf16 weights: the same CUDA-core scheme with 8 bf16 weights per 16 bytes,
+// for shapes outside the tensor-core tile layout; bf16 blobs in that layout
+// (d, I multiples of 256) go to the tcgen05 GEMV in ffn_decode_tc.cu.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -91,36 +91,6 @@ __device__ __forceinline__ float e8m0_to_float(uint32_t b) {
   if (b == 0u) return __uint_as_float(0x00400000u);   // 2^-127
   if (b == 255u) return __uint_as_float(0x7fc00000u); // NaN
   return __uint_as_float(b << 23);
-}
-
-// Exclusive block scan (blockDim <= 1024); ws >= 33 ints of shared memory.
-__device__ int block_scan(int v, int* ws, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) ws[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = (blockDim.x + 31) >> 5;
-    const int w = (lane < nw) ? ws[lane] : 0;
-    int s = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, s, o);
-      if (lane >= o) s += y;
-    }
-    ws[lane] = s - w;
-    if (lane == 31) ws[32] = s;
-  }
-  __syncthreads();
-  const int r = ws[warp] + x - v;
-  *total = ws[32];
-  __syncthreads();
-  return r;
 }
 
 // Reduce-scatter of V partial sums across the warp.  After it, the lane holds
@@ -648,389 +618,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
 //   B     activations straight from global/L1 in fragment layout; phase 2
 //         splits the fp32 SwiGLU output into bf16 hi + lo parts (two MMAs),
 //         which keeps its error near 2^-17 relative.
-namespace mmap {
-
-constexpr int kWarps = 8;
-constexpr int kRows = 32;                     // weight rows per warp tile
-constexpr int kSlice = 2 * kBlockK;          // bytes of a row per stage: one block line
-constexpr int kStages = 3;
-constexpr int kStageBytes = kRows * kSlice;   // one block of 32 rows (gate + up, or down)
-constexpr int kTok = 32;                      // token rows per pass (4 MMA n-tiles)
-constexpr size_t kSmemBytes = static_cast<size_t>(kWarps) * kStages * kStageBytes + 1024;
-
-struct Unit {
-  int e, tile, q0, tb, nt;
-};
-
-template <int PHASE>
-__device__ __forceinline__ Unit decode_unit(const FfnParams& P, const int16_t* act, const int32_t* ustart,
-                                            int n_act, long long u) {
-  int lo = 0, hi = n_act;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (ustart[mid] <= u) lo = mid;
-    else hi = mid;
-  }
-  Unit U;
-  U.e = act[lo];
-  U.q0 = __ldg(P.offsets + U.e);
-  const int ne = __ldg(P.offsets + U.e + 1) - U.q0;
-  const int passes = (ne + kTok - 1) / kTok;
-  const int local = static_cast<int>(u - ustart[lo]);
-  U.tile = local / passes;
-  U.tb = (local % passes) * kTok;
-  U.nt = min(kTok, ne - U.tb);
-  return U;
-}
-
-// First block of a unit's tile in the blocked bf16 layout; the next blocks
-// along K follow at kStageBytes / 2 (gate, up) or kStageBytes (down).
-template <int PHASE>
-__device__ __forceinline__ const uint8_t* tile_block(const FfnParams& P, const uint8_t* blob, int tile, bool up) {
-  if (PHASE == 1)
-    return blob + (up ? P.L.wu : P.L.wg) + static_cast<size_t>(tile) * (P.d / kBlockK) * (kStageBytes / 2);
-  return blob + P.L.wd + static_cast<size_t>(tile) * (P.I / kBlockK) * kStageBytes;
-}
-
-struct Pipe {
-  uint8_t* ring;
-  uint64_t* bar;
-  long long beg, n_units, next_issue, n_items;
-  int slices;
-  bool ok;
-  long long issue_unit;
-  const uint8_t* blk0;       // issue_unit's first gate (phase 1) or down block
-  const uint8_t* blk1;       // issue_unit's first up block (phase 1)
-  uint64_t policy;
-  // L2 prefetch cursor, kPrefetch items ahead of the shared-memory ring
-  long long next_pf, pf_unit;
-  const uint8_t* pf0;
-  const uint8_t* pf1;
-  bool pf_on;
-};
-
-// Items requested from DRAM into L2 ahead of the ring: the ring alone keeps
-// too few bytes in flight per SM to cover the loaded memory latency.
-constexpr int kPrefetch = 4;
-
-template <int PHASE>
-__device__ __forceinline__ void prefetch_to(const FfnParams& P, const int16_t* act, const int32_t* ustart,
-                                            int n_act, Pipe& pp, long long upto) {
-  if (upto > pp.n_items) upto = pp.n_items;
-  while (pp.next_pf < upto) {
-    const long long j = pp.next_pf++;
-    const long long u = pp.beg + j / pp.slices;
-    const int sl = static_cast<int>(j % pp.slices);
-    if (u != pp.pf_unit) {
-      const Unit U = decode_unit<PHASE>(P, act, ustart, n_act, u);
-      const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-      pp.pf0 = tile_block<PHASE>(P, blob, U.tile, false);
-      pp.pf1 = tile_block<PHASE>(P, blob, U.tile, true);
-      pp.pf_unit = u;
-    }
-    if (PHASE == 1) {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(pp.pf0 + static_cast<size_t>(sl) * (kStageBytes / 2)),
-                   "r"(kStageBytes / 2) : "memory");
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(pp.pf1 + static_cast<size_t>(sl) * (kStageBytes / 2)),
-                   "r"(kStageBytes / 2) : "memory");
-    } else {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(pp.pf0 + static_cast<size_t>(sl) * kStageBytes),
-                   "r"(kStageBytes) : "memory");
-    }
-  }
-}
-
-template <int PHASE>
-__device__ __forceinline__ void issue_item(const FfnParams& P, const int16_t* act, const int32_t* ustart,
-                                           int n_act, Pipe& pp, int lane) {
-  const long long j = pp.next_issue++;
-  const long long u = pp.beg + j / pp.slices;
-  const int sl = static_cast<int>(j % pp.slices);
-  const int st = static_cast<int>(j % kStages);
-  if (u != pp.issue_unit) {
-    const Unit U = decode_unit<PHASE>(P, act, ustart, n_act, u);
-    const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-    pp.blk0 = tile_block<PHASE>(P, blob, U.tile, false);
-    pp.blk1 = tile_block<PHASE>(P, blob, U.tile, true);
-    pp.issue_unit = u;
-  }
-  __syncwarp();
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  if (lane == 0) {
-    uint8_t* dst = pp.ring + st * kStageBytes;
-    mbar_expect_tx(&pp.bar[st], kStageBytes);
-    if (PHASE == 1) {
-      bulk_load(dst, pp.blk0 + static_cast<size_t>(sl) * (kStageBytes / 2), kStageBytes / 2, &pp.bar[st], pp.policy);
-      bulk_load(dst + kStageBytes / 2, pp.blk1 + static_cast<size_t>(sl) * (kStageBytes / 2), kStageBytes / 2,
-                &pp.bar[st], pp.policy);
-    } else {
-      bulk_load(dst, pp.blk0 + static_cast<size_t>(sl) * kStageBytes, kStageBytes, &pp.bar[st], pp.policy);
-    }
-    if (pp.pf_on) prefetch_to<PHASE>(P, act, ustart, n_act, pp, j + 1 + kPrefetch);
-  }
-  __syncwarp();
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// two fp32 -> bf16x2 (low half = first argument), round to nearest even
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-// NTT n-tiles of 8 token rows.
-template <int PHASE, int NTT>
-__device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* ustart, int n_act, Pipe& pp,
-                         const Unit& U, long long& j, int lane) {
-  const int g = lane >> 2, tq = lane & 3;   // fragment group and thread-in-group
-  // this lane's B-fragment token row for each n-tile (padding repeats the last real row)
-  const uint16_t* xb[NTT];
-  const float* af[NTT];
-#pragma unroll
-  for (int n = 0; n < NTT; ++n) {
-    const int q = U.q0 + U.tb + min(n * 8 + g, U.nt - 1);
-    if (PHASE == 1) {
-      int p = __ldg(P.perm + q);
-      if (p < 0 || p >= P.T * P.k) {
-        report(P.status, MOE_ERR_DEVICE);
-        p = 0;
-      }
-      xb[n] = P.x + static_cast<size_t>(p / P.k) * P.d;
-      af[n] = nullptr;
-    } else {
-      xb[n] = nullptr;
-      af[n] = P.a_ws + static_cast<size_t>(q) * P.I;
-    }
-  }
-  float acc[2][NTT][4];
-#pragma unroll
-  for (int m = 0; m < 2; ++m)
-#pragma unroll
-    for (int n = 0; n < NTT; ++n)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[m][n][c] = 0.f;
-  // ldmatrix: lane l addresses row (l & 7) + 8 ((l >> 3) & 1) of the m-tile,
-  // 16-byte chunk 2 kk + ((l >> 4) & 1), stored at chunk ^ (row % 8); m-tile 1
-  // (up rows, or down rows 16..31) sits 8 KB after m-tile 0
-  const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int lhi = (lane >> 4) & 1;
-  const int lsw = lrow & 7;
-  for (int sl = 0; sl < pp.slices; ++sl, ++j) {
-    if (pp.next_issue < pp.n_items) issue_item<PHASE>(P, act, ustart, n_act, pp, lane);
-    const int st = static_cast<int>(j % kStages);
-    if (!mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1))) {
-      pp.ok = false;
-      return;
-    }
-    const uint32_t sbase = smem_u32(pp.ring + st * kStageBytes) + lrow * kSlice;
-    const int kbase = sl * (kSlice / 2);
-    // pairs of k-steps: the blocked layout's k order puts this lane's B
-    // fragments of both k-steps in 8 contiguous activations
-#pragma unroll 2
-    for (int kp = 0; kp < kSlice / 64; ++kp) {
-      uint32_t a0[2][4], a1[2][4];
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t coff = static_cast<uint32_t>(((4 * kp + 2 * ks + lhi) ^ lsw) << 4);
-        ldsm_x4(a0[ks], sbase + coff);
-        ldsm_x4(a1[ks], sbase + kStageBytes / 2 + coff);
-      }
-      const int k0 = kbase + kp * 32 + 8 * tq;
-#pragma unroll
-      for (int n = 0; n < NTT; ++n) {
-        if (PHASE == 1) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(xb[n] + k0));
-          mma_bf16(acc[0][n], a0[0], v.x, v.y);
-          mma_bf16(acc[1][n], a1[0], v.x, v.y);
-          mma_bf16(acc[0][n], a0[1], v.z, v.w);
-          mma_bf16(acc[1][n], a1[1], v.z, v.w);
-        } else {
-          const float4 f0 = __ldg(reinterpret_cast<const float4*>(af[n] + k0));
-          const float4 f1 = __ldg(reinterpret_cast<const float4*>(af[n] + k0 + 4));
-          const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-          uint32_t h[4], l[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            h[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-            l[i] = pack_bf16x2(f[2 * i] - bf16_lo(h[i]), f[2 * i + 1] - bf16_hi(h[i]));
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            mma_bf16(acc[0][n], a0[ks], h[2 * ks], h[2 * ks + 1]);
-            mma_bf16(acc[1][n], a1[ks], h[2 * ks], h[2 * ks + 1]);
-            mma_bf16(acc[0][n], a0[ks], l[2 * ks], l[2 * ks + 1]);
-            mma_bf16(acc[1][n], a1[ks], l[2 * ks], l[2 * ks + 1]);
-          }
-        }
-      }
-    }
-  }
-  // fragments: acc[m][n][c]: row = 16 m + g + 8 (c >> 1), token col = 8 n + 2 tq + (c & 1)
-#pragma unroll
-  for (int n = 0; n < NTT; ++n)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int col = n * 8 + 2 * tq + (c & 1);
-      if (col >= U.nt) continue;
-      const int q = U.q0 + U.tb + col;
-      const int r = g + 8 * (c >> 1);
-      if (PHASE == 1) {
-        // acc[0] = gate rows, acc[1] = up rows of the same 16 indices
-        const float h = acc[0][n][c], u = acc[1][n][c];
-        P.a_ws[static_cast<size_t>(q) * P.I + 16 * U.tile + r] = silu(h) * u;
-      } else {
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int row = 32 * U.tile + 16 * m + r;
-          const float y = acc[m][n][c];
-          if (P.y_perm != nullptr) {
-            P.y_perm[static_cast<size_t>(q) * P.d + row] = y;
-          } else {
-            const int p = __ldg(P.perm + q);
-            if (p >= 0 && p < P.T * P.k)
-              atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * y);
-          }
-        }
-      }
-    }
-}
-
-template <int PHASE>
-__global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_mma_kernel(FfnParams P) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ int16_t s_act[1024];
-  __shared__ int32_t s_ustart[1025];
-  __shared__ int s_ws[36];
-  __shared__ __align__(8) uint64_t s_bar[kWarps * kStages];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int tiles_per_e = (PHASE == 1) ? P.I / 16 : P.d / 32;
-  const int per = (P.E + blockDim.x - 1) / blockDim.x;   // <= 8
-  const int e0 = threadIdx.x * per;
-  int cnt = 0;
-  uint32_t mask = 0;
-  const int npairs = P.T * P.k;
-  for (int jx = 0; jx < per; ++jx) {
-    const int e = e0 + jx;
-    if (e >= P.E) break;
-    const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
-    if (b <= a) continue;
-    if (a < 0 || b > npairs) {
-      report(P.status, MOE_ERR_DEVICE);
-      continue;
-    }
-    const int s = __ldg(P.slot + e);
-    if (s < 0) continue;
-    if (s >= P.n_slots) {
-      report(P.status, MOE_ERR_DEVICE);
-      continue;
-    }
-    mask |= 1u << jx;
-    ++cnt;
-  }
-  int n_act;
-  int pos = block_scan(cnt, s_ws, &n_act);
-  int units = 0;
-  for (int jx = 0; jx < per; ++jx)
-    if (mask & (1u << jx)) {
-      const int e = e0 + jx;
-      const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
-      s_act[pos++] = static_cast<int16_t>(e);
-      units += tiles_per_e * ((ne + kTok - 1) / kTok);
-    }
-  int total_units;
-  int ustart = block_scan(units, s_ws, &total_units);
-  pos -= cnt;
-  for (int jx = 0; jx < per; ++jx)
-    if (mask & (1u << jx)) {
-      const int e = e0 + jx;
-      const int ne = __ldg(P.offsets + e + 1) - __ldg(P.offsets + e);
-      s_ustart[pos++] = ustart;
-      ustart += tiles_per_e * ((ne + kTok - 1) / kTok);
-    }
-  if (threadIdx.x < kWarps * kStages) mbar_init(&s_bar[threadIdx.x], 1);
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  __syncthreads();
-
-  const int K = (PHASE == 1) ? P.d : P.I;
-  const long long nw = static_cast<long long>(gridDim.x) * kWarps;
-  const long long gw = static_cast<long long>(blockIdx.x) * kWarps + warp;
-  Pipe pp;
-  pp.ring = smem_raw + static_cast<size_t>(warp) * kStages * kStageBytes;
-  pp.bar = s_bar + warp * kStages;
-  pp.beg = total_units * gw / nw;
-  pp.n_units = total_units * (gw + 1) / nw - pp.beg;
-  pp.slices = K / kBlockK;
-  pp.n_items = pp.n_units * pp.slices;
-  pp.next_issue = 0;
-  pp.ok = true;
-  pp.issue_unit = -1;
-  pp.blk0 = pp.blk1 = nullptr;
-  pp.policy = policy_evict_first();
-  pp.next_pf = 0;
-  pp.pf_unit = -1;
-  pp.pf0 = pp.pf1 = nullptr;
-  // small expert sets are prefetched whole by phase 1; larger ones by the cursor
-  pp.pf_on = static_cast<size_t>(n_act) * P.blob_bytes > kPrefetchCap;
-  if (PHASE == 1) prefetch_active_blobs(P, s_act, n_act);
-  for (int i = 0; i < kStages - 1 && pp.next_issue < pp.n_items; ++i)
-    issue_item<PHASE>(P, s_act, s_ustart, n_act, pp, lane);
-  long long j = 0;
-  for (long long u = 0; u < pp.n_units && pp.ok; ++u) {
-    const Unit U = decode_unit<PHASE>(P, s_act, s_ustart, n_act, pp.beg + u);
-    const int ntt = (U.nt + 7) / 8;
-    if (ntt == 1) run_unit<PHASE, 1>(P, s_act, s_ustart, n_act, pp, U, j, lane);
-    else if (ntt == 2) run_unit<PHASE, 2>(P, s_act, s_ustart, n_act, pp, U, j, lane);
-    else if (ntt == 3) run_unit<PHASE, 3>(P, s_act, s_ustart, n_act, pp, U, j, lane);
-    else run_unit<PHASE, 4>(P, s_act, s_ustart, n_act, pp, U, j, lane);
-  }
-  if (!pp.ok) report(P.status, MOE_ERR_TIMEOUT);
-  for (long long i = j; i < pp.next_issue; ++i) {
-    const uint64_t t0 = now_ns();
-    while (!mbar_try(&pp.bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1)) && now_ns() - t0 <= kWaitNs) {
-    }
-  }
-}
-
-template <int PHASE>
-moe_status launch(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
-  static bool attr[64] = {};
-  if (!attr[dev.id]) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(ffn_decode_mma_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(kSmemBytes)));
-    attr[dev.id] = true;
-  }
-  const int tiles_per_e = (PHASE == 1) ? P.I / 16 : P.d / 32;
-  const long long most = static_cast<long long>(min(P.E, P.T * P.k)) * tiles_per_e *
-                         ((P.T * P.k + kTok - 1) / kTok);
-  long long blocks = (most + kWarps - 1) / kWarps;
-  if (blocks > dev.sm_count) blocks = dev.sm_count;
-  if (blocks < 1) blocks = 1;
-  ffn_decode_mma_kernel<PHASE><<<static_cast<int>(blocks), kWarps * 32, kSmemBytes, s>>>(P);
-  MOE_LAUNCH_CHECK("ffn_decode_mma_kernel");
-  return MOE_OK;
-}
-
-}  // namespace mmap
-
-// bf16 blobs in the blocked layout (d, I multiples of 256) take the MMA path.
-bool mma_shape_ok(const FfnParams& P) { return bf16_blocked(P.d, P.I); }
 
 template <int FMT, int PHASE>
 moe_status launch_phase(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
@@ -1054,11 +641,6 @@ moe_status launch_phase(const FfnParams& P, const DeviceInfo& dev, cudaStream_t 
 template <int FMT>
 moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
   if (kSmemBytes > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "needs %zu bytes of shared memory", kSmemBytes);
-  if (FMT == MOE_W_BF16 && mma_shape_ok(P) && mmap::kSmemBytes <= dev.smem_optin) {
-    moe_status st = mmap::launch<1>(P, dev, s);
-    if (st != MOE_OK) return st;
-    return mmap::launch<2>(P, dev, s);
-  }
   moe_status st = launch_phase<FMT, 1>(P, dev, s);
   if (st != MOE_OK) return st;
   return launch_phase<FMT, 2>(P, dev, s);
@@ -1070,10 +652,17 @@ size_t decode_workspace_bytes(moe_shape s, int T, int k) {
   return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256);
 }
 
+moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
+                            const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
+                            float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream);
+
 moe_status launch_ffn_decode(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
                              const int32_t* perm, const int32_t* slot, const void* pool, int n_slots,
                              const float* gate, float* y_perm, float* out, void* ws,
                              int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
+  if (s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I))
+    return launch_decode_tc(s, x, T, k, offsets, perm, slot, pool, n_slots, gate, y_perm, out, ws, status, dev,
+                            stream);
   FfnParams P{};
   P.E = s.E;
   P.d = s.d;

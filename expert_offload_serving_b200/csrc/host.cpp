@@ -95,17 +95,20 @@ extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* w
       std::memcpy(b + L.wd, wd, m * 2);
       return MOE_OK;
     }
-    // blocked layout: every element to its place (blocks, k order, swizzle)
-    struct Mt { const uint16_t* src; size_t off; int R, K, RB; } mats[3] = {
-        {static_cast<const uint16_t*>(wg), L.wg, s.I, s.d, 16},
-        {static_cast<const uint16_t*>(wu), L.wu, s.I, s.d, 16},
-        {static_cast<const uint16_t*>(wd), L.wd, s.d, s.I, 32}};
-    for (const Mt& mt : mats)
-      for (int r = 0; r < mt.R; ++r) {
-        const uint16_t* row = mt.src + static_cast<size_t>(r) * mt.K;
-        for (int k = 0; k < mt.K; ++k)
-          std::memcpy(b + mt.off + blocked_offset(r, k, mt.K, mt.RB), row + k, 2);
+    // tile layout: gate/up rows interleaved into W_gu, 16-byte chunks to their
+    // swizzled places
+    const uint8_t* g8 = static_cast<const uint8_t*>(wg);
+    const uint8_t* u8 = static_cast<const uint8_t*>(wu);
+    const uint8_t* d8 = static_cast<const uint8_t*>(wd);
+    for (int i = 0; i < s.I; ++i)
+      for (int k = 0; k < s.d; k += 8) {
+        const size_t src = (static_cast<size_t>(i) * s.d + k) * 2;
+        std::memcpy(b + L.wg + sw128_offset(gu_row(i, false), k, s.d), g8 + src, 16);
+        std::memcpy(b + L.wg + sw128_offset(gu_row(i, true), k, s.d), u8 + src, 16);
       }
+    for (int r = 0; r < s.d; ++r)
+      for (int k = 0; k < s.I; k += 8)
+        std::memcpy(b + L.wd + sw128_offset(r, k, s.I), d8 + (static_cast<size_t>(r) * s.I + k) * 2, 16);
     return MOE_OK;
   }
   MOE_REQUIRE(sg && su && sd, "null scale pointer for an FP4 format");

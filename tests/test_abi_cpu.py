@@ -114,57 +114,38 @@ def _canonical(name, E=3):
     return cfg, synth.make_experts(cfg, range(E), seed=3)
 
 
-def _kpos32(k):
-    """Stored position of element k of a 32-element group: the two MMA
-    k-steps (16 positions each) hold, in lane group t's B-fragment slots
-    (positions 2t, 2t+1 and 2t+8, 2t+9), the elements 8t..8t+3 (first k-step)
-    and 8t+4..8t+7 (second)."""
-    t, r = divmod(k, 8)
-    step, r = divmod(r, 4)
-    reg, half = divmod(r, 2)
-    return 16 * step + 8 * reg + 2 * t + half
-
-
-def test_kpos32_is_fragment_order():
-    # lane group t, k-step s, register b: positions 16 s + 8 b + 2 t + (0, 1)
-    # must hold the contiguous elements 8 t + 4 s + 2 b + (0, 1)
-    inv = {_kpos32(k): k for k in range(32)}
-    assert sorted(inv) == list(range(32))
-    for t in range(4):
-        got = [inv[16 * s + 8 * b + 2 * t + h] for s in range(2) for b in range(2) for h in range(2)]
-        assert got == list(range(8 * t, 8 * t + 8))
-
-
-BLOCK_K = 128   # elements per line of a blocked bf16 matrix
-
-
-def test_pack_bf16_blocked_layout(moe):
-    """bf16 blobs with d, I multiples of 256: blocks of RB rows x BLOCK_K
-    elements (RB = 16 for gate/up, 32 for down), ordered [row block][K block],
-    rows of 2 * BLOCK_K bytes; inside each 32-element group element k sits at
-    position _kpos32(k), and 16-byte chunk c of row r at chunk position
-    c ^ (r % 8)."""
+def test_pack_bf16_tile_layout(moe):
+    """bf16 blobs with d, I multiples of 256 hold W_gu (gate and up rows
+    interleaved in blocks of 64: row 128b + j = gate row 64b + j, row
+    128b + 64 + j = up row 64b + j) in the wg + wu regions and W_d in the wd
+    region, each as tiles of 128 rows x 64 elements (16 KB) ordered
+    [row / 128][k / 64]; in a tile, row r is a 128-byte line whose 16-byte
+    chunk c sits at chunk position c ^ (r % 8)."""
     from expert_offload_serving_b200.layer import pack_pool
     cfg = synth.LayerConfig("blk", E=2, k=1, d=512, I=256, fmt="bf16")
     w = synth.make_experts(cfg, range(2), seed=4)
     pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w, range(2), pin=False).numpy()
     m = cfg.I * cfg.d
+
+    def unpack(region, R, K):
+        words = region.view(np.uint16)
+        out = np.empty((R, K), dtype=np.uint16)
+        k = np.arange(K)
+        for r in range(R):
+            tile = (r // 128) * (K // 64) + k // 64
+            rr = r % 128
+            pos = tile * 16384 + rr * 128 + (((k // 8) % 8) ^ (rr % 8)) * 16 + (k % 8) * 2
+            out[r] = words[pos // 2]
+        return out
+
     for e in range(2):
         b = pool[e]
-        for n, (key, R, K, RB) in enumerate((("wg", cfg.I, cfg.d, 16), ("wu", cfg.I, cfg.d, 16),
-                                            ("wd", cfg.d, cfg.I, 32))):
-            region = b[n * 2 * m:(n + 1) * 2 * m]
-            src = w[key][e].contiguous().view(torch.int16).numpy().view(np.uint16)
-            words = region.view(np.uint16)
-            got = np.empty((R, K), dtype=np.uint16)
-            kp = np.array([32 * (k // 32) + _kpos32(k % 32) for k in range(K)])
-            for r in range(R):
-                blk = (r // RB) * (K // BLOCK_K) + kp // BLOCK_K
-                chunk = (kp % BLOCK_K) // 8
-                line = 2 * BLOCK_K
-                pos = blk * RB * line + (r % RB) * line + (chunk ^ ((r % RB) % 8)) * 16 + (kp % 8) * 2
-                got[r] = words[pos // 2]
-            assert np.array_equal(got, src)
+        src = {key: w[key][e].contiguous().view(torch.int16).numpy().view(np.uint16) for key in ("wg", "wu", "wd")}
+        gu = unpack(b[:2 * 2 * m], 2 * cfg.I, cfg.d)
+        for i in range(cfg.I):
+            assert np.array_equal(gu[(i // 64) * 128 + i % 64], src["wg"][i])
+            assert np.array_equal(gu[(i // 64) * 128 + 64 + i % 64], src["wu"][i])
+        assert np.array_equal(unpack(b[2 * 2 * m:3 * 2 * m], cfg.d, cfg.I), src["wd"])
 
 
 @pytest.mark.parametrize("name", ["tiny", "decode_mxfp4", "prefill_nvfp4"])
