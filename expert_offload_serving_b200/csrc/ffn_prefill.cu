@@ -190,19 +190,14 @@ __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* 
   return total;
 }
 
-// Unit u -> (chunk, M tile).  GEMM1 runs chunk-major (the CTAs working at the
-// same time share one activation tile); GEMM2 runs M-tile-major, so the
-// tiles in flight all add into the same 128-column slab of out, which stays
-// in L2 while its ~6 contributions per element arrive.
-template <int PHASE>
-__device__ __forceinline__ void unit_coords(int u, int n_chunks, int MT, int* c, int* m) {
-  if (PHASE == 1) {
-    *c = u / MT;
-    *m = u % MT;
-  } else {
-    *m = u / n_chunks;
-    *c = u % n_chunks;
-  }
+// Unit u -> (chunk, M tile), chunk-major for both GEMMs: the CTAs working at
+// the same time share one activation tile, and the M tiles of an expert with
+// several chunks are re-read while still in L2.  (Measured against M-tile-major
+// order for GEMM2, which keeps one 128-column slab of out hot for the fused
+// combine: equal at T = 4096, 8-9 % slower at T >= 16384.)
+__device__ __forceinline__ void unit_coords(int u, int MT, int* c, int* m) {
+  *c = u / MT;
+  *m = u % MT;
 }
 
 // expert of chunk c: the last e with chunk_start[e] <= c
@@ -355,12 +350,15 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       int c, m;
-      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m);
+      unit_coords(u, MT, &c, &m);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int sl = P.slot[e];
       const uint8_t* sfa_src = P.pool + static_cast<size_t>(sl) * P.blob_bytes +
                                (PHASE == 1 ? P.L.sg : P.L.sd) + static_cast<size_t>(m) * (K / 64) * 512;
       const uint8_t* sfb_src = P.act_sf + static_cast<size_t>(c) * (K / 64) * 512;
+      // a weight tile read by one chunk streams through L2; one that the
+      // expert's further chunks read again is kept
+      const uint64_t pol_a = (chunk_start[e + 1] - chunk_start[e] > 1) ? pol_keep : pol_stream;
       for (int ks = 0; ks < KS; ++ks) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           ok = false;
@@ -372,9 +370,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           uint8_t* sSFA = sB + B_BYTES;
           uint8_t* sSFB = sSFA + SF_BYTES;
           mbar_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl, pol_stream);
+          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl, pol_a);
           tma_load_2d(sB, &tm_act, &full[stage], ks * BKB, c * BN, pol_keep);
-          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_stream);
+          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_a);
           bulk_load(sSFB, sfb_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_keep);
         }
         __syncwarp();
@@ -409,7 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       int c, m_unused;
-      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m_unused);
+      unit_coords(u, MT, &c, &m_unused);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
       const int nvalid = min(BN, P.offsets[e + 1] - row0);
@@ -477,7 +475,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       int c, m;
-      unit_coords<PHASE>(u, n_chunks_used, MT, &c, &m);
+      unit_coords(u, MT, &c, &m);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
       const int nvalid = min(BN, P.offsets[e + 1] - row0);
