@@ -228,15 +228,16 @@ def decode_point(cfg, T, R, warmup, steps, stream, routed_only=False):
 def run_gpu(args, rank, world, local):
     import expert_offload_serving_b200 as moe
     moe.lib()
-    cfg = synth.CONFIGS["decode_bf16"]
+    cfg = synth.CONFIGS[args.config]
     T = args.tokens
+    routed_only = cfg.fmt != "bf16"   # the 256-expert MXFP4 layer: only the routed experts are materialised
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     blob = moe.moe_expert_blob_bytes(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt))
     # replicas: the bytes between two uses of one replica >= 4 x L2
     per_step = None
     R = args.replicas
-    reps = build_replicas(cfg, T, R, seed0=1000 * rank)
+    reps = build_replicas(cfg, T, R, seed0=1000 * rank, routed_only=routed_only)
     U = []
     for r in reps:
         r["layer"].forward(r["logits"], r["x"])
@@ -247,7 +248,9 @@ def run_gpu(args, rank, world, local):
         print(f"warning: replicas stream only {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
               "between reuses", file=sys.stderr)
     stream = torch.cuda.Stream(device=dev)
-    launches_per_step = 5   # route, permute, ffn gate/up, ffn down, combine
+    # route, permute, ffn gate/up, ffn down, combine; plus the split-sum kernel
+    # between the two GEMVs when T*k <= 32
+    launches_per_step = 5 + (1 if T * cfg.k <= 32 else 0)
 
     def step_fn(r):
         L = r["layer"]
@@ -369,10 +372,11 @@ def run_gpu(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if cfg.fmt == "bf16" else "mxfp4 weights x bf16 activations",
         "data": "synthetic",
         "config": {
-            "workload": f"decode_bf16: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, all experts resident",
+            "workload": f"{cfg.name}: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, "
+                        + ("the routed experts resident" if routed_only else "all experts resident"),
             "global_batch": T * world,
             "replicas": R,
             "l2": f"inputs larger than L2: {R} replicas, >= {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
@@ -382,14 +386,14 @@ def run_gpu(args, rank, world, local):
             "cuda_graph": True,
         },
         "roofline": {
-            "kernel": "moe_expert_ffn (ffn_decode gate/up + down)",
+            "kernel": "moe_expert_ffn (gemv_tc_kernel gate/up + down)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
-            "traffic": kernel_traffic("ffn_decode.cu", f"decode_bf16_T{T}"),
+            "traffic": kernel_traffic("ffn_decode_tc.cu", f"{cfg.name}_T{T}"),
             "algorithmic_bytes_per_launch": int(alg_bytes),
             "avg_launch_ms": round(ffn_avg_ms, 5),
         },
@@ -654,6 +658,8 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the FP4 prefill measurement")
+    ap.add_argument("--config", default="decode_bf16", choices=["decode_bf16", "decode_mxfp4"],
+                    help="decode workload of the main line (default: decode_bf16)")
     ap.add_argument("--only-prefill", action="store_true", help="print only the FP4 prefill measurement")
     ap.add_argument("--prefill-T", type=int, default=0, help="with --only-prefill: this token count only")
     ap.add_argument("--prefill-E", type=int, default=None,

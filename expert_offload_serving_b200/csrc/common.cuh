@@ -66,6 +66,12 @@ __host__ __device__ inline BlobLayout blob_layout(int fmt, int d, int I) {
     L.wu = o; o = round_up(o + m * 2, 256);
     L.wd = o; o = round_up(o + m * 2, 256);
     L.sg = L.su = L.sd = L.ts = o;
+  } else if (fmt == MOE_W_MXFP4 && d % 256 == 0 && I % 256 == 0) {
+    // stage-tiled (mx_tile_code_offset): W_gu tiles, then W_d tiles; the
+    // scale regions alias the code regions
+    L.wg = L.wu = L.sg = L.su = o; o = round_up(o + m + m / 16, 256);
+    L.wd = L.sd = o; o = round_up(o + m / 2 + m / 32, 256);
+    L.ts = o;
   } else if (fmt == MOE_W_MXFP4) {
     L.wg = o; o = round_up(o + m / 2, 256);
     L.wu = o; o = round_up(o + m / 2, 256);
@@ -101,6 +107,33 @@ __host__ __device__ inline size_t sw128_offset(int r, int k, int K) {
   const int rr = r & 127, c = (k >> 3) & 7;
   return tile * 16384 + static_cast<size_t>(rr) * 128 + ((c ^ (rr & 7)) << 4) + (k & 7) * 2;
 }
+
+// MXFP4 blobs whose d and I are multiples of 256 are stage-tiled for the
+// tensor-core decode GEMV: W_gu (gate and up rows interleaved as in gu_row)
+// and W_d are cut into tiles of 128 rows x 256 elements, ordered
+// [row / 128][k / 256], each 17408 bytes: the codes (row r = a 128-byte line
+// whose 16-byte chunk c sits at c ^ (r % 8), element 2i in the low nibble of
+// byte i), then the E8M0 scales (8 per row, row-major).  One tile is one
+// pipeline stage and one bulk copy.
+__host__ __device__ inline bool mx_tiled(int d, int I) { return d % 256 == 0 && I % 256 == 0; }
+constexpr int kMxTileBytes = 128 * 128 + 128 * 8;
+
+// Byte offsets of code byte b (elements 2b, 2b+1) and of the scale of 32-block
+// j of row r, in a stage-tiled matrix with K columns.
+__host__ __device__ inline size_t mx_tile_code_offset(int r, int b, int K) {
+  const size_t tile = static_cast<size_t>(r >> 7) * (K >> 8) + (b >> 7);
+  const int rr = r & 127, bb = b & 127;
+  return tile * kMxTileBytes + static_cast<size_t>(rr) * 128 + ((((bb >> 4) ^ (rr & 7)) << 4) | (bb & 15));
+}
+__host__ __device__ inline size_t mx_tile_scale_offset(int r, int j, int K) {
+  const size_t tile = static_cast<size_t>(r >> 7) * (K >> 8) + (j >> 3);
+  return tile * kMxTileBytes + 16384 + static_cast<size_t>(r & 127) * 8 + (j & 7);
+}
+
+// K splits of the decode GEMV for n = T*k routed pairs: few pairs give too few
+// (expert, tile) units to fill the SMs, so each tile's K range is split and
+// the partial sums are added afterwards.
+__host__ __device__ inline int decode_split(long long n) { return n <= 8 ? 4 : (n <= 32 ? 2 : 1); }
 
 // Row of W_gu holding gate row i (up = false) or up row i (up = true).
 __host__ __device__ inline int gu_row(int i, bool up) { return (i >> 6) * 128 + (up ? 64 : 0) + (i & 63); }

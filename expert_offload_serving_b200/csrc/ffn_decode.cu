@@ -649,7 +649,12 @@ moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t
 }  // namespace
 
 size_t decode_workspace_bytes(moe_shape s, int T, int k) {
-  return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256);
+  // a (fp32, or the two 16-bit planes of the tensor-core path); then the
+  // tensor-core path's split partial sums
+  const size_t n = static_cast<size_t>(T) * k;
+  const size_t a = round_up(n * s.I * sizeof(float), 256);
+  const int split = decode_split(static_cast<long long>(n));
+  return a + (split > 1 ? round_up(static_cast<size_t>(split) * n * 2 * s.I * sizeof(float), 256) : 0);
 }
 
 moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
@@ -660,7 +665,7 @@ moe_status launch_ffn_decode(moe_shape s, const void* x, int T, int k, const int
                              const int32_t* perm, const int32_t* slot, const void* pool, int n_slots,
                              const float* gate, float* y_perm, float* out, void* ws,
                              int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
-  if (s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I))
+  if ((s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I)) || (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)))
     return launch_decode_tc(s, x, T, k, offsets, perm, slot, pool, n_slots, gate, y_perm, out, ws, status, dev,
                             stream);
   FfnParams P{};

@@ -1,19 +1,30 @@
-// Step 3 on bf16 weights (moe_expert_ffn without MOE_FFN_ACT_NVFP4, bf16 blobs
-// in the tensor-core tile layout): the grouped SwiGLU expert FFN as two skinny
-// GEMMs on the 5th-generation tensor cores.
+// Step 3 at decode sizes on the 5th-generation tensor cores
+// (moe_expert_ffn without MOE_FFN_ACT_NVFP4; bf16 blobs in the tile layout and
+// MXFP4 blobs in the stage-tiled layout): the grouped SwiGLU expert FFN as two
+// skinny GEMMs.
 //
 // At decode sizes a layer call is bound by reading the routed experts' weights
 // from HBM (explainx.ai hardware guide, "Decode: decide whether to move an
-// expert or compute where it lives": one token touches few experts).  Here no
-// SM instruction is spent per weight element: bulk copies move 32 KB weight
-// stages into shared memory and one thread issues tcgen05.mma over them, with
-// the few token rows of the group as the N side and the accumulators in TMEM.
+// expert or compute where it lives": one token touches few experts).  Bulk
+// copies move whole weight stages into shared memory and one thread issues
+// tcgen05.mma over them, the few token rows of a group being the N side and
+// the accumulators living in TMEM:
+//   bf16   the stage (128 rows x 128 elements, 32 KB) is the A operand as it
+//          lands; no SM instruction is spent per weight element.
+//   MXFP4  no tensor-core kind multiplies FP4 by a 16-bit operand, so eight
+//          converter warps turn each stage (128 rows x 256 elements, 17 KB) into
+//          exact f16 values -- cvt of E2M1 pairs, times the power-of-two E8M0
+//          block scale -- stored into TMEM, where the MMA reads A; the token
+//          rows are converted bf16 -> f16 in shared memory.  f16 holds every
+//          E2M1 x 2^X exactly for X in [-23, 13] and every bf16 activation below
+//          65504 in magnitude; a scale or an activation outside is reported
+//          as MOE_ERR_UNSUPPORTED in the status word.
 //
 //   gemv<1>: D[128 x N] = W_gu tile (64 gate + 64 up rows of the same
 //            intermediate indices) x X^T over K = d, N <= 32 token rows
 //            gathered by one-row TMA loads of x.  Epilogue: a = silu(D_gate) *
-//            D_up, stored as two bf16 planes hi + lo (a - hi - lo ~ 2^-17 |a|)
-//            in the workspace, rows = sorted pair positions.
+//            D_up, stored as two 16-bit planes hi + lo (a - hi - lo ~ 2^-17 |a|
+//            for bf16, ~2^-22 |a| for f16) in the workspace, rows = sorted pairs.
 //   gemv<2>: D[128 x N] = W_d tile x (A_hi + A_lo)^T over K = I (two MMAs per
 //            k-step).  Epilogue: y_perm rows, or out[t] += gate * y (the fused
 //            combine).
@@ -21,11 +32,15 @@
 // Work unit = (expert, 128-row tile, chunk of <= 32 of the expert's pairs),
 // expert-major, chunks fastest, dealt round-robin to one persistent CTA per
 // SM.  Warp 0 produces (bulk copy of the weight stage, TMA loads of the token
-// rows, L2 prefetch of the weight stages a few items ahead), warp 1 owns TMEM
-// and issues the MMAs, warps 2-5 run the epilogue on double-buffered TMEM
-// accumulators.  Every wait is bounded: on expiry the CTA records
-// MOE_ERR_TIMEOUT, stops issuing, drains what it issued and frees its TMEM.
+// rows, L2 prefetch of weight stages a few items ahead), warp 1 owns TMEM and
+// issues the MMAs, [MXFP4: warps 2-9 convert], the last four warps run the
+// epilogue on double-buffered TMEM accumulators.  Every wait is bounded: on
+// expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains what it
+// issued and frees its TMEM.
+#include <algorithm>
+
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -35,6 +50,8 @@ namespace moe {
 struct TcDecodeParams {
   int E, d, I, T, k, n_slots;
   int a_box_rows;            // rows of one TMA box of the a planes (min(32, T*k))
+  int split1, split2;        // K splits of gemv<1> and gemv<2> (each <= its K stages)
+  float* part;               // split1 > 1: gemv<1> partial sums [split1][T*k][2I] fp32
   const int32_t* offsets;
   const int32_t* perm;
   const int32_t* slot;
@@ -42,7 +59,7 @@ struct TcDecodeParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  __nv_bfloat16* a_planes;   // [2][T*k][I]: hi, lo
+  uint16_t* a_planes;        // [2][T*k][I] 16-bit (bf16 or f16): hi, lo
   float* y_perm;             // [T*k][d] or null (then out)
   float* out;                // [T][d] (fused combine)
   int32_t* status;
@@ -54,42 +71,48 @@ using namespace ::moe::tc;
 
 constexpr int TM = 128;                  // weight rows per tile
 constexpr int TN = 32;                   // pairs per chunk (max MMA N)
-constexpr int A_ATOM = TM * 128;         // one 64-element atom of a tile: 16 KB
-constexpr int B_ATOM = TN * 128;         // one atom of the token rows: 4 KB
-constexpr int ATOMS = 2;                 // atoms per stage: K = 128
-constexpr int A_STAGE = ATOMS * A_ATOM;  // 32 KB, one bulk copy
-constexpr int THREADS = 192;             // producer, MMA, 4 epilogue warps
+constexpr int B_ATOM = TN * 128;         // one 64-element atom of the token rows: 4 KB
 constexpr int ACC_COLS = 32;             // TMEM columns per accumulator
-constexpr int TMEM_COLS = 64;            // two accumulators
 constexpr int PF_ITEMS = 4;              // L2 prefetch distance (stages)
 constexpr size_t kBlobPrefetchCap = 96ull << 20;
 
-template <int PHASE> struct Cfg;
-template <> struct Cfg<1> {
-  static constexpr int B_BYTES = ATOMS * B_ATOM;              // x rows
-  static constexpr int STAGE = A_STAGE + B_BYTES;             // 40 KB
-  static constexpr int STAGES = 5;
-  static constexpr int UP_BYTES = 64 * 33 * 4;                // up-row exchange
-};
-template <> struct Cfg<2> {
-  static constexpr int B_BYTES = 2 * ATOMS * B_ATOM;          // a hi + lo rows
-  static constexpr int STAGE = A_STAGE + B_BYTES;             // 48 KB
-  static constexpr int STAGES = 4;
-  static constexpr int UP_BYTES = 0;
+// Per (format, phase) geometry of a pipeline stage.
+template <int FMT, int PHASE>
+struct Cfg {
+  static constexpr bool MX = (FMT == MOE_W_MXFP4);
+  static constexpr int KSTAGE = MX ? 256 : 128;                  // K elements per stage
+  static constexpr int ATOMS = KSTAGE / 64;                      // B atoms per plane
+  static constexpr int A_STAGE = MX ? kMxTileBytes : 2 * TM * 128;   // weight bytes per stage
+  static constexpr int B_BYTES = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
+  static constexpr int STAGE = A_STAGE + B_BYTES;                // multiple of 1024
+  static constexpr int STAGES = PHASE == 1 ? (MX ? 6 : 5) : 4;
+  static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
+  static constexpr int CONV_WARPS = MX ? 8 : 0;                  // two per TMEM lane quadrant
+  static constexpr int THREADS = (2 + CONV_WARPS + 4) * 32;
+  static constexpr int EPI_WARP0 = 2 + CONV_WARPS;
+  static constexpr int ASLOTS = 3;                               // TMEM A buffers (MXFP4)
+  static constexpr int A_COL0 = 2 * ACC_COLS;                    // first TMEM column of the A buffers
+  static constexpr int A_COLS = KSTAGE / 2;                      // TMEM columns per A buffer
+  static constexpr int TMEM_COLS = MX ? 512 : 64;
+  static constexpr int N_BARS = 2 * STAGES + 5 + (MX ? 2 * ASLOTS : 0);
+  static_assert(STAGE % 1024 == 0 && A_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(!MX || A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(N_BARS * 8 + 16 <= 256, "barrier area");
 };
 
-template <int PHASE>
+template <int FMT, int PHASE>
 constexpr size_t smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(Cfg<PHASE>::STAGES) * Cfg<PHASE>::STAGE + Cfg<PHASE>::UP_BYTES + 256 +
-         static_cast<size_t>(E + 1) * 4;
+  using C = Cfg<FMT, PHASE>;
+  return 1024 + static_cast<size_t>(C::STAGES) * C::STAGE + C::UP_BYTES + 256 + static_cast<size_t>(E + 1) * 4;
 }
 
 struct Unit {
-  int e, m, q0, nvalid;
+  int e, m, q0, nvalid, ks0, ks1;   // K stages [ks0, ks1) of the unit's split
 };
 
-// unit u -> (expert, tile, chunk); ustart[e] = first unit of expert e
-__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int u) {
+// unit u -> (expert, tile, chunk, K split); ustart[e] = first unit of expert e
+__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int S, int KS,
+                                        int u) {
   int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -100,20 +123,23 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
   U.e = lo;
   const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
   const int chunks = (ne + TN - 1) / TN;
-  const int local = u - ustart[lo];
+  const int local = (u - ustart[lo]) / S, sp = (u - ustart[lo]) % S;
   U.m = local / chunks;
   const int c = local % chunks;
+  U.ks0 = sp * KS / S;
+  U.ks1 = (sp + 1) * KS / S;
   U.q0 = q_begin + c * TN;
   U.nvalid = min(TN, ne - c * TN);
   return U;
 }
 
 // First byte of unit U's weight tile (its K stages follow at A_STAGE).
-template <int PHASE>
+template <int FMT, int PHASE>
 __device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, const Unit& U) {
+  using C = Cfg<FMT, PHASE>;
   const int K = (PHASE == 1) ? P.d : P.I;
   const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-  return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / 64) * A_ATOM;
+  return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / C::KSTAGE) * C::A_STAGE;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -122,10 +148,67 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
-template <int PHASE>
-__global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_constant__ CUtensorMap tm_b,
-                                                               TcDecodeParams P) {
-  using C = Cfg<PHASE>;
+// E2M1 pair (one byte, element 2i in the low nibble) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{ .reg .b8 b; cvt.u8.u32 b, %1; cvt.rn.f16x2.e2m1x2 %0, b; }" : "=r"(r) : "r"(byte));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// E8M0 scale byte -> 2^(byte - 127) as f16x2, exact for exponents -24..15;
+// false when E2M1 x 2^X would not be exact in f16 (X outside [-23, 13]).
+__device__ __forceinline__ bool e8m0_f16x2(uint32_t byte, uint32_t* out) {
+  const int x = static_cast<int>(byte) - 127;
+  if (x < -23 || x > 13) {
+    *out = 0;
+    return false;
+  }
+  const uint32_t h = (x >= -14) ? static_cast<uint32_t>(x + 15) << 10 : 1u << (x + 24);
+  *out = h | (h << 16);
+  return true;
+}
+
+// 8 bf16 -> 8 f16 in place (one 16-byte chunk); false if one is beyond f16.
+__device__ __forceinline__ bool bf16x8_to_f16x8(uint4* p) {
+  uint4 v = *p;
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+    ok = ok && fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
+    const __half2 h = __floats2half2_rn(lo, hi);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *p = make_uint4(w[0], w[1], w[2], w[3]);
+  return ok;
+}
+
+__device__ __forceinline__ void split16(float a, bool mx, uint16_t* hi, uint16_t* lo) {
+  if (mx) {
+    const __half h = __float2half_rn(a);
+    const __half l = __float2half_rn(a - __half2float(h));
+    *hi = __half_as_ushort(h);
+    *lo = __half_as_ushort(l);
+  } else {
+    const __nv_bfloat16 h = __float2bfloat16_rn(a);
+    const __nv_bfloat16 l = __float2bfloat16_rn(a - __bfloat162float(h));
+    *hi = __bfloat16_as_ushort(h);
+    *lo = __bfloat16_as_ushort(l);
+  }
+}
+
+template <int FMT, int PHASE>
+__global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
+    gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_b, TcDecodeParams P) {
+  using C = Cfg<FMT, PHASE>;
+  constexpr int THREADS = C::THREADS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* up_buf = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE);
@@ -135,7 +218,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
   uint64_t* tfull = bars + 2 * C::STAGES;       // [2]
   uint64_t* tempty = bars + 2 * C::STAGES + 2;  // [2]
   uint64_t* drain = bars + 2 * C::STAGES + 4;   // [1]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint64_t* cvt_done = bars + 2 * C::STAGES + 5;               // [ASLOTS] (MXFP4)
+  uint64_t* afree = bars + 2 * C::STAGES + 5 + C::ASLOTS;      // [ASLOTS] (MXFP4)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
   int32_t* ustart = reinterpret_cast<int32_t*>(smem + C::STAGES * C::STAGE + C::UP_BYTES + 256);
@@ -143,8 +228,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = (PHASE == 1) ? P.d : P.I;
-  const int KS = K / (64 * ATOMS);
+  const int KS = K / C::KSTAGE;
   const int MT = (PHASE == 1) ? P.I / 64 : P.d / TM;
+  const int S = PHASE == 1 ? P.split1 : P.split2;   // K splits per tile
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
@@ -157,13 +243,19 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    if (C::MX) {
+      for (int a = 0; a < C::ASLOTS; ++a) {
+        mbar_init(&cvt_done[a], 32 * C::CONV_WARPS);
+        mbar_init(&afree[a], 1);
+      }
+    }
     *abort_flag = 0;
     *epi_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                 "r"(TMEM_COLS));
+                 "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
 
@@ -186,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
       continue;
     }
     if (s < 0) continue;
-    cnt += MT * ((b - a + TN - 1) / TN);
+    cnt += MT * S * ((b - a + TN - 1) / TN);
     ++act;
   }
   int total = 0;
@@ -199,7 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
     ustart[e] = run;
     const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
     const int s = __ldg(P.slot + e);
-    if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * ((b - a + TN - 1) / TN);
+    if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * S * ((b - a + TN - 1) / TN);
   }
   if (threadIdx.x == 0) ustart[P.E] = total;
   tc_fence_before();
@@ -235,47 +327,55 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
     int issued = 0;
     bool ok = true;
     // L2 prefetch cursor over this CTA's (unit, stage) items
-    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
+    int pf_u = blockIdx.x, pf_ks = 0, pf_ks1 = 0, pf_ahead = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_on && pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of(P, ustart, MT, pf_u));
+    if (pf_on && pf_u < n_units) {
+      const Unit V = unit_of(P, ustart, MT, S, KS, pf_u);
+      pf_base = tile_base<FMT, PHASE>(P, V);
+      pf_ks = V.ks0;
+      pf_ks1 = V.ks1;
+    }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of(P, ustart, MT, u);
-      const uint8_t* abase = tile_base<PHASE>(P, U);
+      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
       int tok = 0;
       if (PHASE == 1 && lane < U.nvalid) {
         const int p = __ldg(P.perm + U.q0 + lane);
         if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
         else tok = p / P.k;
       }
-      for (int ks = 0; ks < KS; ++ks) {
+      for (int ks = U.ks0; ks < U.ks1; ++ks) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         uint8_t* sA = smem + stage * C::STAGE;
-        uint8_t* sB = sA + A_STAGE;
+        uint8_t* sB = sA + C::A_STAGE;
         if (lane == 0) {
-          const uint32_t bytes =
-              A_STAGE + (PHASE == 1 ? 2u * U.nvalid : 2u * ATOMS * static_cast<uint32_t>(P.a_box_rows)) * 128u;
-          mbar_expect_tx(&full[stage], bytes);
-          bulk_load(sA, abase + static_cast<size_t>(ks) * A_STAGE, A_STAGE, &full[stage], pol_stream);
+          const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * P.a_box_rows;
+          mbar_expect_tx(&full[stage], C::A_STAGE + rows * C::ATOMS * 128u);
+          bulk_load(sA, abase + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE, &full[stage], pol_stream);
           if (PHASE == 2) {
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-              for (int a = 0; a < ATOMS; ++a)
-                tma_load_3d(sB + (pl * ATOMS + a) * B_ATOM, &tm_b, &full[stage], ks * 128 + 64 * a, U.q0, pl,
-                            pol_keep);
+              for (int a = 0; a < C::ATOMS; ++a)
+                tma_load_3d(sB + (pl * C::ATOMS + a) * B_ATOM, &tm_b, &full[stage], ks * C::KSTAGE + 64 * a, U.q0,
+                            pl, pol_keep);
           }
           // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one
           if (pf_on) {
             while (pf_u < n_units && pf_ahead < PF_ITEMS) {
-              prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * A_STAGE, A_STAGE);
+              prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
               ++pf_ahead;
-              if (++pf_ks == KS) {
-                pf_ks = 0;
+              if (++pf_ks == pf_ks1) {
                 pf_u += gridDim.x;
-                if (pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of(P, ustart, MT, pf_u));
+                if (pf_u < n_units) {
+                  const Unit V = unit_of(P, ustart, MT, S, KS, pf_u);
+                  pf_base = tile_base<FMT, PHASE>(P, V);
+                  pf_ks = V.ks0;
+                  pf_ks1 = V.ks1;
+                }
               }
             }
             --pf_ahead;
@@ -284,8 +384,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
         __syncwarp();
         if (PHASE == 1 && lane < U.nvalid) {
 #pragma unroll
-          for (int a = 0; a < ATOMS; ++a)
-            tma_load_2d(sB + a * B_ATOM + lane * 128, &tm_b, &full[stage], ks * 128 + 64 * a, tok, pol_keep);
+          for (int a = 0; a < C::ATOMS; ++a)
+            tma_load_2d(sB + a * B_ATOM + lane * 128, &tm_b, &full[stage], ks * C::KSTAGE + 64 * a, tok, pol_keep);
         }
         __syncwarp();
         ++issued;
@@ -314,11 +414,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    int it = 0;
+    int it = 0, j = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, u);
-      const uint32_t idesc = idesc_bf16(TM, U.nvalid <= 16 ? 16 : 32);
+      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      const int n_mma = U.nvalid <= 16 ? 16 : 32;
+      const uint32_t idesc = C::MX ? idesc_f16(TM, n_mma) : idesc_bf16(TM, n_mma);
       const int acc = it & 1;
       if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
         ok = false;
@@ -326,26 +427,37 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
-      for (int ks = 0; ks < KS; ++ks) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) {
+      for (int ks = U.ks0; ks < U.ks1; ++ks, ++j) {
+        const int aslot = j % C::ASLOTS;
+        // the stage has landed; MXFP4: and its A buffer (and, phase 1, the
+        // token rows) is converted
+        const bool got = mbar_wait(&full[stage], phase, abort_flag) &&
+                         (!C::MX || mbar_wait(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag));
+        if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (elect_one()) {
           uint8_t* sA = smem + stage * C::STAGE;
-          uint8_t* sB = sA + A_STAGE;
+          uint8_t* sB = sA + C::A_STAGE;
 #pragma unroll
-          for (int a = 0; a < ATOMS; ++a) {
-            const uint64_t da = desc_sw128(smem_u32(sA + a * A_ATOM));
-            const uint64_t dh = desc_sw128(smem_u32(sB + a * B_ATOM));
-            const uint64_t dl = desc_sw128(smem_u32(sB + (ATOMS + a) * B_ATOM));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {   // K = 16 per MMA: +32 bytes
-              tc_mma_bf16(d_tmem, da + 2 * kk, dh + 2 * kk, idesc, (ks > 0 || a > 0 || kk > 0) ? 1u : 0u);
-              if (PHASE == 2) tc_mma_bf16(d_tmem, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+          for (int kk = 0; kk < C::KSTAGE / 16; ++kk) {   // K = 16 per MMA: +32 bytes
+            const int a = kk >> 2;
+            const uint64_t dh = desc_sw128(smem_u32(sB + a * B_ATOM)) + 2 * (kk & 3);
+            const uint64_t dl = desc_sw128(smem_u32(sB + (C::ATOMS + a) * B_ATOM)) + 2 * (kk & 3);
+            const uint32_t first = (ks > U.ks0 || kk > 0) ? 1u : 0u;
+            if (C::MX) {
+              const uint32_t ta = tmem + C::A_COL0 + aslot * C::A_COLS + 8 * kk;
+              tc_mma_f16_ts(d_tmem, ta, dh, idesc, first);
+              if (PHASE == 2) tc_mma_f16_ts(d_tmem, ta, dl, idesc, 1u);
+            } else {
+              const uint64_t da = desc_sw128(smem_u32(sA + a * TM * 128)) + 2 * (kk & 3);
+              tc_mma_bf16(d_tmem, da, dh, idesc, first);
+              if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
             }
           }
+          if (C::MX) tc_commit(&afree[aslot]);
           tc_commit(&empty[stage]);
         }
         __syncwarp();
@@ -365,12 +477,77 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
     if (elect_one()) tc_commit(drain);
     __syncwarp();
     mbar_drain(drain, 0);
+  } else if (warp < C::EPI_WARP0) {
+    // ------------------------------------------------------------ MXFP4 converters (warps 2..9)
+    if constexpr (C::MX) {
+    const int quad = warp & 3;
+    const int r = 32 * quad + lane;                 // tile row = TMEM lane
+    const int half = (warp - 2) >> 2;               // this warp's half of the row's 256 elements
+    const int ct = threadIdx.x - 64;                // 0..255
+    bool ok = true;
+    bool range_ok = true;
+    int j = 0;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      for (int ks = U.ks0; ks < U.ks1; ++ks, ++j) {
+        const int s = j % C::STAGES, aslot = j % C::ASLOTS;
+        if (!mbar_wait(&full[s], (j / C::STAGES) & 1, abort_flag) ||
+            !mbar_wait(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* sA = smem + s * C::STAGE;
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(sA + 16384 + r * 8 + 4 * half);
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(32 * quad) << 16) + C::A_COL0 + aslot * C::A_COLS + 64 * half;
+        {
+          // chunks 4 half .. 4 half + 3 of the row: 128 elements -> 64 columns
+          uint4 q[4];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = 4 * half + cc;
+            q[cc] = *reinterpret_cast<const uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4));
+          }
+          uint32_t v[64];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t scl;
+            range_ok &= e8m0_f16x2((sc >> (8 * cc)) & 0xffu, &scl);
+            const uint32_t w[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
+#pragma unroll
+            for (int b = 0; b < 16; ++b) v[16 * cc + b] = hmul2(e2m1x2_f16x2((w[b >> 2] >> (8 * (b & 3))) & 0xffu), scl);
+          }
+          tmem_st64(taddr, v);
+        }
+        if (PHASE == 1) {
+          // token rows bf16 -> f16 in place (the swizzle only moves whole chunks)
+          uint8_t* sB = sA + C::A_STAGE;
+          const int n_chunks = U.nvalid * C::ATOMS * 8;
+          for (int idx = ct; idx < n_chunks; idx += 32 * C::CONV_WARPS) {
+            const int rr = idx / (C::ATOMS * 8), rem = idx % (C::ATOMS * 8);
+            range_ok &= bf16x8_to_f16x8(reinterpret_cast<uint4*>(sB + (rem >> 3) * B_ATOM + rr * 128 + (rem & 7) * 16));
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&cvt_done[aslot]);
+      }
+    }
+    if (!range_ok) report(P.status, MOE_ERR_UNSUPPORTED);
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (last four warps)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
+    bool range_ok = true;
     int it = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, u);
+      const Unit U = unit_of(P, ustart, MT, S, KS, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
@@ -385,7 +562,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (PHASE == 1) {
+      if (PHASE == 1 && S > 1) {
+        // a K split: the tile's partial gate (rows 0..63) and up (64..127) sums
+        const int r = 32 * quad + lane;
+        const int sp = (u - ustart[U.e]) % S;
+        const size_t col = (r < 64) ? static_cast<size_t>(64) * U.m + r : static_cast<size_t>(P.I) + 64 * U.m + (r - 64);
+        float* dst = P.part + (static_cast<size_t>(sp) * n_pairs + U.q0) * (2 * P.I) + col;
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c < U.nvalid) dst[static_cast<size_t>(c) * (2 * P.I)] = v[c];
+      } else if (PHASE == 1) {
         // rows 0..63 of the tile are gate rows, 64..127 the matching up rows
         if (quad >= 2) {
           const int i = 32 * (quad - 2) + lane;
@@ -401,8 +587,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
           for (int c = 0; c < 32; ++c) {
             if (c < U.nvalid) {
               const float a = silu(v[c]) * up_buf[i * 33 + c];
-              const __nv_bfloat16 hi = __float2bfloat16_rn(a);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(a - __bfloat162float(hi));
+              if (C::MX) range_ok &= fabsf(a) <= 65504.f;
+              uint16_t hi, lo;
+              split16(a, C::MX, &hi, &lo);
               const size_t o = static_cast<size_t>(U.q0 + c) * P.I + col;
               P.a_planes[o] = hi;
               P.a_planes[plane + o] = lo;
@@ -417,7 +604,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
           if (c < U.nvalid) {
             const int q = U.q0 + c;
             if (P.y_perm != nullptr) {
-              P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
+              // with K splits y_perm was zeroed and receives the split sums
+              if (S > 1) atomicAdd(P.y_perm + static_cast<size_t>(q) * P.d + row, v[c]);
+              else P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
             } else {
               const int p = __ldg(P.perm + q);
               if (p >= 0 && p < n_pairs)
@@ -427,34 +616,84 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_bf16_kernel(const __grid_cons
         }
       }
     }
+    if (!range_ok) report(P.status, MOE_ERR_UNSUPPORTED);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
   }
 }
 
-template <int PHASE>
+// After a split gemv<1>: a = silu(sum of gate partials) * (sum of up
+// partials) into the two 16-bit planes; and, when gemv<2> splits into y_perm,
+// y_perm zeroed for its split sums.
+template <bool MX>
+__global__ void __launch_bounds__(256) finish_swiglu_kernel(const float* __restrict__ part, int S, int n, int I,
+                                                            uint16_t* __restrict__ planes, float* y_zero, int n_y,
+                                                            int d, int32_t* status) {
+  const size_t tot = static_cast<size_t>(n) * I;   // n = 0: no split of gemv<1>
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  bool ok = true;
+  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < tot; idx += stride) {
+    const size_t q = idx / I, i = idx % I;
+    float h = 0.f, u = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float* p = part + (static_cast<size_t>(sp) * n + q) * (2 * static_cast<size_t>(I));
+      h += p[i];
+      u += p[I + i];
+    }
+    const float a = silu(h) * u;
+    if (MX) ok &= fabsf(a) <= 65504.f;
+    uint16_t hi, lo;
+    split16(a, MX, &hi, &lo);
+    planes[idx] = hi;
+    planes[tot + idx] = lo;
+  }
+  if (y_zero != nullptr) {
+    const size_t n4 = static_cast<size_t>(n_y) * d / 4;
+    for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n4; idx += stride)
+      reinterpret_cast<float4*>(y_zero)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (!ok) report(status, MOE_ERR_UNSUPPORTED);
+}
+
+template <int FMT, int PHASE>
 moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const DeviceInfo& dev, cudaStream_t s) {
-  const size_t smem = smem_bytes<PHASE>(P.E);
+  const size_t smem = smem_bytes<FMT, PHASE>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
   if (attr[dev.id] < smem) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(gemv_bf16_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MOE_CUDA_TRY(cudaFuncSetAttribute(gemv_tc_kernel<FMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(smem)));
     attr[dev.id] = smem;
   }
-  gemv_bf16_kernel<PHASE><<<dev.sm_count, THREADS, smem, s>>>(tm, P);
-  MOE_LAUNCH_CHECK("gemv_bf16_kernel");
+  gemv_tc_kernel<FMT, PHASE><<<dev.sm_count, Cfg<FMT, PHASE>::THREADS, smem, s>>>(tm, P);
+  MOE_LAUNCH_CHECK("gemv_tc_kernel");
   return MOE_OK;
+}
+
+template <int FMT>
+moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap& tm_a,
+                       const DeviceInfo& dev, cudaStream_t stream) {
+  moe_status st = launch_phase<FMT, 1>(P, tm_x, dev, stream);
+  if (st != MOE_OK) return st;
+  float* y_zero = (P.split2 > 1) ? P.y_perm : nullptr;
+  if (P.split1 > 1 || y_zero != nullptr) {
+    const size_t tot = static_cast<size_t>(P.T) * P.k * std::max(P.I, P.d);
+    const int blocks = static_cast<int>(std::min<size_t>((tot + 255) / 256, static_cast<size_t>(4) * dev.sm_count));
+    finish_swiglu_kernel<FMT == MOE_W_MXFP4><<<blocks, 256, 0, stream>>>(
+        P.part, P.split1, P.split1 > 1 ? P.T * P.k : 0, P.I, P.a_planes, y_zero, P.T * P.k, P.d, P.status);
+    MOE_LAUNCH_CHECK("finish_swiglu_kernel");
+  }
+  return launch_phase<FMT, 2>(P, tm_a, dev, stream);
 }
 
 }  // namespace
 
-// bf16 blobs in the tile layout: both GEMV launches.  ws holds the a planes
-// (T*k*I*4 bytes).
+// Both GEMV launches for bf16 blobs in the tile layout or MXFP4 blobs in the
+// stage-tiled layout.  ws holds the a planes (T*k*I*4 bytes).
 moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
                             const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
@@ -472,7 +711,16 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
   P.pool = static_cast<const uint8_t*>(pool);
   P.L = blob_layout(s.fmt, s.d, s.I);
   P.blob_bytes = P.L.bytes;
-  P.a_planes = static_cast<__nv_bfloat16*>(ws);
+  P.a_planes = static_cast<uint16_t*>(ws);
+  const size_t n_pairs = static_cast<size_t>(T) * k;
+  {
+    // K stages per tile: bf16 128 elements, MXFP4 256
+    const int kstage = s.fmt == MOE_W_MXFP4 ? 256 : 128;
+    const int split = decode_split(static_cast<long long>(n_pairs));
+    P.split1 = std::min(split, s.d / kstage);
+    P.split2 = std::min(std::min(split, 2), s.I / kstage);
+  }
+  P.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round_up(n_pairs * s.I * sizeof(float), 256));
   P.y_perm = y_perm;
   P.out = out;
   P.status = status;
@@ -490,12 +738,13 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
     const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, 2};
     const uint64_t str[2] = {static_cast<uint64_t>(s.I) * 2, n * s.I * 2};
     const uint32_t box[3] = {64u, static_cast<uint32_t>(P.a_box_rows), 1u};
-    const CUresult r = encode_tiled_sw128(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ws, dims, str, box);
+    const CUtensorMapDataType type =
+        s.fmt == MOE_W_MXFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUresult r = encode_tiled_sw128(&tm_a, type, 3, ws, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a planes failed (%d)", static_cast<int>(r));
   }
-  moe_status st = launch_phase<1>(P, tm_x, dev, stream);
-  if (st != MOE_OK) return st;
-  return launch_phase<2>(P, tm_a, dev, stream);
+  if (s.fmt == MOE_W_MXFP4) return launch_both<MOE_W_MXFP4>(P, tm_x, tm_a, dev, stream);
+  return launch_both<MOE_W_BF16>(P, tm_x, tm_a, dev, stream);
 }
 
 }  // namespace moe

@@ -148,6 +148,42 @@ def test_pack_bf16_tile_layout(moe):
         assert np.array_equal(unpack(b[2 * 2 * m:3 * 2 * m], cfg.d, cfg.I), src["wd"])
 
 
+def test_pack_mxfp4_tiled_layout(moe):
+    """MXFP4 blobs with d, I multiples of 256 hold W_gu (gate and up rows
+    interleaved in blocks of 64) and then W_d as tiles of 128 rows x 256
+    elements ordered [row / 128][k / 256], 17408 bytes each: the codes (row r
+    = a 128-byte line, 16-byte chunk c at chunk position c ^ (r % 8)), then
+    the 8 E8M0 scales of each row."""
+    from expert_offload_serving_b200.layer import pack_pool
+    cfg = synth.LayerConfig("mxt", E=1, k=1, d=512, I=256, fmt="mxfp4")
+    w = synth.make_experts(cfg, range(1), seed=6)
+    blob = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w, range(1), pin=False).numpy()[0]
+    tile_bytes = 128 * 128 + 128 * 8
+
+    def unpack(region, R, K):
+        codes = np.empty((R, K // 2), dtype=np.uint8)
+        scales = np.empty((R, K // 32), dtype=np.uint8)
+        b = np.arange(K // 2)
+        jj = np.arange(K // 32)
+        for r in range(R):
+            rr = r % 128
+            tile = (r // 128) * (K // 256) + b // 128
+            bb = b % 128
+            codes[r] = region[tile * tile_bytes + rr * 128 + (((bb // 16) ^ (rr % 8)) * 16) + bb % 16]
+            stile = (r // 128) * (K // 256) + jj // 8
+            scales[r] = region[stile * tile_bytes + 16384 + rr * 8 + jj % 8]
+        return codes, scales
+
+    gu_bytes = 2 * cfg.I * (cfg.d // 2 + cfg.d // 32)
+    gc, gs = unpack(blob[:gu_bytes], 2 * cfg.I, cfg.d)
+    for i in range(cfg.I):
+        rg, ru = (i // 64) * 128 + i % 64, (i // 64) * 128 + 64 + i % 64
+        assert np.array_equal(gc[rg], w["wg"][0][i].numpy()) and np.array_equal(gs[rg], w["sg"][0][i].numpy())
+        assert np.array_equal(gc[ru], w["wu"][0][i].numpy()) and np.array_equal(gs[ru], w["su"][0][i].numpy())
+    dc, ds = unpack(blob[gu_bytes:], cfg.d, cfg.I)
+    assert np.array_equal(dc, w["wd"][0].numpy()) and np.array_equal(ds, w["sd"][0].numpy())
+
+
 @pytest.mark.parametrize("name", ["tiny", "decode_mxfp4", "prefill_nvfp4"])
 def test_pack_expert_layout(moe, name):
     """Blob regions hold the canonical tensors (NVFP4: gate/up rows interleaved

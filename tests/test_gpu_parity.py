@@ -147,12 +147,14 @@ def test_layer_ragged_shapes(moe, fmt, d, I):
     check_tol(b.run().cpu().numpy(), b.oracle()["out"], 1e-4, 1e-5)
 
 
-def test_many_tokens_per_expert(moe):
-    """Groups larger than one 8-row pass (skewed routing, T=64, E=8)."""
-    cfg = synth.LayerConfig("skew", E=8, k=2, d=512, I=256, fmt="bf16", bias_std=2.0)
+@pytest.mark.parametrize("fmt", ["bf16", "mxfp4"])
+def test_many_tokens_per_expert(moe, fmt):
+    """Groups of more than one 32-pair chunk on the tensor-core path (skewed
+    routing, T=64, E=8; d, I multiples of 256)."""
+    cfg = synth.LayerConfig("skew", E=8, k=2, d=512, I=256, fmt=fmt, bias_std=2.0)
     b = Built(cfg, 64, seed=2)
     check_tol(b.run().cpu().numpy(), b.oracle()["out"], 1e-4, 1e-5)
-    assert (np.diff(b.layer.offsets.cpu().numpy()) > 16).any()
+    assert (np.diff(b.layer.offsets.cpu().numpy()) > 32).any()
 
 
 def test_y_perm_rows_match_pairs(moe):
@@ -165,9 +167,12 @@ def test_y_perm_rows_match_pairs(moe):
     check_tol(y[inv], ref, 1e-4, 1e-5)
 
 
-def test_fused_out_matches_combine(moe):
+@pytest.mark.parametrize("T", [1, 16])
+def test_fused_out_matches_combine(moe, T):
+    """out += gate * y in the FFN epilogue equals y_perm + combine (T=1 runs
+    the K-split GEMVs, whose partial sums meet in out)."""
     cfg = synth.CONFIGS["decode_bf16"]
-    b = Built(cfg, 16, seed=6)
+    b = Built(cfg, T, seed=6)
     ref = b.run().clone()
     L_ = b.layer
     out = torch.zeros_like(ref)
@@ -209,7 +214,9 @@ def test_host_partial_merge_and_q_sweep(moe):
             hp = b.oracle(experts=host_now)["out"].astype(np.float32)
             out = b.run(host_partial=torch.from_numpy(hp).cuda()).cpu().numpy()
             check_tol(out, ref)
-            check_tol(out, full, 1e-5, 1e-6)
+            # the merge itself adds the host partial exactly; merged and all-GPU
+            # outputs differ by the GPU path's own rounding on the host share
+            check_tol(out, full, 1e-4, 1e-5)
         b.layer.slot.copy_(slot_save)
 
 
