@@ -178,6 +178,25 @@ def build_replicas(cfg, T, R, seed0=0, routed_only=False):
     return reps
 
 
+def steps_per_graph(K, R, cap=32):
+    """Steps captured into one CUDA graph: the largest divisor of K that is a
+    multiple of R and at most cap (1 when there is none), so that K steps are
+    exactly K / G replays and one launch covers several small steps."""
+    for g in range(min(K, cap), 0, -1):
+        if K % g == 0 and g % R == 0:
+            return g
+    return 1
+
+
+def capture_cycle(fns, G, stream):
+    """One CUDA graph running G calls fns[0], fns[1], ... (cycling)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(G):
+            fns[i % len(fns)]()
+    return g
+
+
 def experts_touched(layer):
     """Distinct experts of the last step (non-empty groups of the layer's
     offsets): the algorithmic weight bytes are this count x blob bytes."""
@@ -196,31 +215,35 @@ def decode_point(cfg, T, R, warmup, steps, stream, routed_only=False):
         r["layer"].forward(r["logits"], r["x"])
         torch.cuda.synchronize()
         U.append(experts_touched(r["layer"]))
-    graphs = []
+    G = steps_per_graph(steps, R)
     with torch.cuda.stream(stream):
-        for r in reps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                r["layer"].forward(r["logits"], r["x"])
-            graphs.append(g)
-        for i in range(warmup):
-            graphs[i % R].replay()
+        step_fns = [lambda r=r: r["layer"].forward(r["logits"], r["x"]) for r in reps]
+        ffn_fns = [lambda r=r: r["layer"].ffn(r["x"]) for r in reps]
+        for f in step_fns + ffn_fns:
+            f()
+        stream.synchronize()
+        g_step = capture_cycle(step_fns, G, stream)
+        g_ffn = capture_cycle(ffn_fns, G, stream)
+        for _ in range(max(1, warmup // G)):
+            g_step.replay()
+            g_ffn.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(steps):
-            graphs[i % R].replay()
+        for _ in range(steps // G):
+            g_step.replay()
         e1.record(stream)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
-        for i in range(steps):
-            reps[i % R]["layer"].ffn(reps[i % R]["x"])
+        for _ in range(steps // G):
+            g_ffn.replay()
         f1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     ffn_ms = f0.elapsed_time(f1) / steps
+    del g_step, g_ffn
     gbs = sum(U) / R * blob / (ffn_ms / 1e3) / 1e9
     hbm, _ = peaks()
-    del graphs, reps
+    del reps
     return {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5), "ffn_ms": round(ffn_ms, 5),
             "ffn_gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4), "experts_touched": U}
 
@@ -256,22 +279,21 @@ def run_gpu(args, rank, world, local):
         L = r["layer"]
         L.forward(r["logits"], r["x"])
 
-    # CUDA graph per replica
-    graphs = []
+    # one CUDA graph of G consecutive steps cycling over the replicas (G divides
+    # K, so the K timed steps are K / G replays; small steps are not bound by
+    # the host's launch rate)
+    G = steps_per_graph(args.steps, R)
     with torch.cuda.stream(stream):
         for r in reps:                      # warm the code paths once before capture
             step_fn(r)
         stream.synchronize()
-        for r in reps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step_fn(r)
-            graphs.append(g)
+        g_steps = capture_cycle([lambda r=r: step_fn(r) for r in reps], G, stream)
     torch.cuda.synchronize()
 
-    # ---- device-timed steps
-    for i in range(args.warmup):
-        graphs[i % R].replay()
+    # ---- device-timed steps (W warm-up steps, rounded up to whole graphs)
+    with torch.cuda.stream(stream):
+        for _ in range((args.warmup + G - 1) // G):
+            g_steps.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -281,8 +303,8 @@ def run_gpu(args, rank, world, local):
     with ClockSampler(smi_id) as clk:
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            for i in range(args.steps):
-                graphs[i % R].replay()
+            for _ in range(args.steps // G):
+                g_steps.replay()
             ev1.record(stream)
         torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
@@ -290,18 +312,21 @@ def run_gpu(args, rank, world, local):
     ms_max = max_over_ranks(ms, world)
     value = world * args.steps * T / (ms_max / 1e3)
 
-    # ---- dominant kernel: moe_expert_ffn (gate/up + down launches), timed alone
-    ffn_ms = []
+    # ---- dominant kernel: moe_expert_ffn (gate/up + down launches), timed alone,
+    # as graph replays of G calls on the bench stream
     with torch.cuda.stream(stream):
-        for i in range(max(3, args.warmup)):
-            reps[i % R]["layer"].ffn(reps[i % R]["x"])
-        n_ffn = max(20, args.steps)
+        g_ffn = capture_cycle([lambda r=r: r["layer"].ffn(r["x"]) for r in reps], G, stream)
+        for _ in range(max(1, (max(3, args.warmup) + G - 1) // G)):
+            g_ffn.replay()
+        n_rep = max(1, (max(20, args.steps) + G - 1) // G)
+        n_ffn = n_rep * G
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(n_ffn):
-            reps[i % R]["layer"].ffn(reps[i % R]["x"])
+        for _ in range(n_rep):
+            g_ffn.replay()
         e1.record(stream)
     torch.cuda.synchronize()
+    del g_ffn
     ffn_avg_ms = e0.elapsed_time(e1) / n_ffn
     alg_bytes = sum(per_step[i % R] for i in range(n_ffn)) / n_ffn
     hbm_peak, peak_src = peaks()
@@ -383,7 +408,7 @@ def run_gpu(args, rank, world, local):
                   "read between reuses" if R > 1 else "single replica",
             "experts_touched_per_step": U,
             "parallelism": f"dp{world} (independent batches)",
-            "cuda_graph": True,
+            "cuda_graph": f"{G} steps per graph, cycling the replicas",
         },
         "roofline": {
             "kernel": "moe_expert_ffn (gemv_tc_kernel gate/up + down)",

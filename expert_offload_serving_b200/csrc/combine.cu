@@ -26,21 +26,39 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int c4 = blockIdx.x * blockDim.x + threadIdx.x;   // index of a float4 in the row
   if (t >= T || c4 * 4 >= d) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int p = t * k + j;
-    const int e = __ldg(idx + p);
-    if (slot != nullptr) {
-      if (e < 0 || e >= E_bound) continue;
-      if (__ldg(slot + e) < 0) continue;
+  // groups of 8 pairs: each level of the index chain (idx -> slot, inv_perm ->
+  // y_perm row) is loaded for the whole group before the next, so a token
+  // waits on ~4 dependent loads instead of 4 k; the sum keeps the order j = 0..k-1
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    int e[8], q[8];
+    float g[8];
+    bool use[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int p = t * k + j0 + jj;
+      use[jj] = j0 + jj < k;
+      e[jj] = use[jj] ? __ldg(idx + p) : 0;
+      q[jj] = use[jj] ? __ldg(inv_perm + p) : -1;
+      g[jj] = use[jj] ? __ldg(gate + p) : 0.f;
     }
-    const int q = __ldg(inv_perm + p);
-    if (q < 0 || q >= nq) continue;
-    const float g = __ldg(gate + p);
-    const float4 y = __ldg(reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(q) * d) + c4);
-    acc.x = fmaf(g, y.x, acc.x);
-    acc.y = fmaf(g, y.y, acc.y);
-    acc.z = fmaf(g, y.z, acc.z);
-    acc.w = fmaf(g, y.w, acc.w);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (slot != nullptr && use[jj]) use[jj] = e[jj] >= 0 && e[jj] < E_bound && __ldg(slot + e[jj]) >= 0;
+      use[jj] = use[jj] && q[jj] >= 0 && q[jj] < nq;
+    }
+    float4 y[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      y[jj] = use[jj] ? __ldg(reinterpret_cast<const float4*>(y_perm + static_cast<size_t>(q[jj]) * d) + c4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (!use[jj]) continue;
+      acc.x = fmaf(g[jj], y[jj].x, acc.x);
+      acc.y = fmaf(g[jj], y[jj].y, acc.y);
+      acc.z = fmaf(g[jj], y[jj].z, acc.z);
+      acc.w = fmaf(g[jj], y[jj].w, acc.w);
+    }
   }
   if (host_partial != nullptr) {
     const float4 h = reinterpret_cast<const float4*>(host_partial + static_cast<size_t>(t) * d)[c4];

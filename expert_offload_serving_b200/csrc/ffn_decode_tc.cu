@@ -32,7 +32,7 @@
 // Work unit = (expert, 128-row tile, chunk of <= 32 of the expert's pairs),
 // expert-major, chunks fastest, dealt round-robin to one persistent CTA per
 // SM.  Warp 0 produces (bulk copy of the weight stage, TMA loads of the token
-// rows, L2 prefetch of weight stages a few items ahead), warp 1 owns TMEM and
+// rows, L2 prefetch of the weight stages four items ahead), warp 1 owns TMEM and
 // issues the MMAs, [MXFP4: warps 2-9 convert], the last four warps run the
 // epilogue on double-buffered TMEM accumulators.  Every wait is bounded: on
 // expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains what it
@@ -74,7 +74,6 @@ constexpr int TN = 32;                   // pairs per chunk (max MMA N)
 constexpr int B_ATOM = TN * 128;         // one 64-element atom of the token rows: 4 KB
 constexpr int ACC_COLS = 32;             // TMEM columns per accumulator
 constexpr int PF_ITEMS = 4;              // L2 prefetch distance (stages)
-constexpr size_t kBlobPrefetchCap = 96ull << 20;
 
 // Per (format, phase) geometry of a pipeline stage.
 template <int FMT, int PHASE>
@@ -87,7 +86,8 @@ struct Cfg {
   static constexpr int STAGE = A_STAGE + B_BYTES;                // multiple of 1024
   static constexpr int STAGES = PHASE == 1 ? (MX ? 6 : 5) : 4;
   static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
-  static constexpr int CONV_WARPS = MX ? 8 : 0;                  // two per TMEM lane quadrant
+  static constexpr int CONV_PER_ROW = 2;                         // converter warps per TMEM lane quadrant
+  static constexpr int CONV_WARPS = MX ? 4 * CONV_PER_ROW : 0;
   static constexpr int THREADS = (2 + CONV_WARPS + 4) * 32;
   static constexpr int EPI_WARP0 = 2 + CONV_WARPS;
   static constexpr int ASLOTS = 3;                               // TMEM A buffers (MXFP4)
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   // ---- units per expert (evaluated experts only) and their exclusive prefix
   const int per = (P.E + THREADS - 1) / THREADS;
   const int e0 = threadIdx.x * per;
-  int cnt = 0, act = 0;
+  int cnt = 0;
   for (int j = 0; j < per; ++j) {
     const int e = e0 + j;
     if (e >= P.E) break;
@@ -279,12 +279,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     }
     if (s < 0) continue;
     cnt += MT * S * ((b - a + TN - 1) / TN);
-    ++act;
   }
   int total = 0;
   int run = block_scan(cnt, ws, &total);
-  int n_act = 0;
-  block_scan(act, ws, &n_act);
   for (int j = 0; j < per; ++j) {
     const int e = e0 + j;
     if (e >= P.E) break;
@@ -300,28 +297,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   const uint32_t tmem = *tmem_holder;
   const int n_units = total;
 
-  // small expert sets: request every active blob into L2 up front (all of the
-  // layer's DRAM reads in flight at once); the weights come through L2 anyway
-  if (PHASE == 1 && static_cast<size_t>(n_act) * P.blob_bytes <= kBlobPrefetchCap) {
-    const size_t chunk = 16384;
-    const size_t per_blob = (P.blob_bytes + chunk - 1) / chunk;
-    const size_t stride = static_cast<size_t>(gridDim.x) * THREADS;
-    size_t idx = static_cast<size_t>(blockIdx.x) * THREADS + threadIdx.x;
-    for (int e = 0; e < P.E; ++e) {
-      if (ustart[e + 1] == ustart[e]) continue;
-      const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + e)) * P.blob_bytes;
-      for (; idx < per_blob; idx += stride) {
-        const size_t off = idx * chunk;
-        prefetch_l2(blob + off, static_cast<uint32_t>(min(chunk, P.blob_bytes - off)));
-      }
-      idx -= per_blob;
-    }
-  }
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
-    const bool pf_on = static_cast<size_t>(n_act) * P.blob_bytes > kBlobPrefetchCap;
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
@@ -329,7 +307,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     // L2 prefetch cursor over this CTA's (unit, stage) items
     int pf_u = blockIdx.x, pf_ks = 0, pf_ks1 = 0, pf_ahead = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_on && pf_u < n_units) {
+    if (pf_u < n_units) {
       const Unit V = unit_of(P, ustart, MT, S, KS, pf_u);
       pf_base = tile_base<FMT, PHASE>(P, V);
       pf_ks = V.ks0;
@@ -363,8 +341,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
                 tma_load_3d(sB + (pl * C::ATOMS + a) * B_ATOM, &tm_b, &full[stage], ks * C::KSTAGE + 64 * a, U.q0,
                             pl, pol_keep);
           }
-          // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one
-          if (pf_on) {
+          // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one (the
+          // bulk copies of a CTA complete in order, so prefetching whole blobs
+          // up front would queue ahead of the stages the pipeline waits for)
+          {
             while (pf_u < n_units && pf_ahead < PF_ITEMS) {
               prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
               ++pf_ahead;
@@ -482,7 +462,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     if constexpr (C::MX) {
     const int quad = warp & 3;
     const int r = 32 * quad + lane;                 // tile row = TMEM lane
-    const int half = (warp - 2) >> 2;               // this warp's half of the row's 256 elements
+    constexpr int CPR = C::CONV_PER_ROW;            // warps sharing a row's 256 elements
+    constexpr int CH = 8 / CPR;                     // 16-byte chunks (32 elements) per warp
+    const int part = (warp - 2) >> 2;               // this warp's part of the row
     const int ct = threadIdx.x - 64;                // 0..255
     bool ok = true;
     bool range_ok = true;
@@ -498,27 +480,29 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         }
         tc_fence_after();
         uint8_t* sA = smem + s * C::STAGE;
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(sA + 16384 + r * 8 + 4 * half);
+        const uint2 sc2 = *reinterpret_cast<const uint2*>(sA + 16384 + r * 8);
         const uint32_t taddr =
-            tmem + (static_cast<uint32_t>(32 * quad) << 16) + C::A_COL0 + aslot * C::A_COLS + 64 * half;
+            tmem + (static_cast<uint32_t>(32 * quad) << 16) + C::A_COL0 + aslot * C::A_COLS + 16 * CH * part;
         {
-          // chunks 4 half .. 4 half + 3 of the row: 128 elements -> 64 columns
-          uint4 q[4];
+          // chunks CH part .. CH part + CH - 1 of the row: 32 CH elements -> 16 CH columns
+          uint4 q[CH];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int c = 4 * half + cc;
+          for (int cc = 0; cc < CH; ++cc) {
+            const int c = CH * part + cc;
             q[cc] = *reinterpret_cast<const uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4));
           }
-          uint32_t v[64];
+          uint32_t v[16 * CH];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < CH; ++cc) {
+            const int c = CH * part + cc;
             uint32_t scl;
-            range_ok &= e8m0_f16x2((sc >> (8 * cc)) & 0xffu, &scl);
+            range_ok &= e8m0_f16x2(((c < 4 ? sc2.x : sc2.y) >> (8 * (c & 3))) & 0xffu, &scl);
             const uint32_t w[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
 #pragma unroll
             for (int b = 0; b < 16; ++b) v[16 * cc + b] = hmul2(e2m1x2_f16x2((w[b >> 2] >> (8 * (b & 3))) & 0xffu), scl);
           }
-          tmem_st64(taddr, v);
+          if constexpr (CH == 4) tmem_st64(taddr, v);
+          else tmem_st32(taddr, v);
         }
         if (PHASE == 1) {
           // token rows bf16 -> f16 in place (the swizzle only moves whole chunks)
