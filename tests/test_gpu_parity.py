@@ -271,3 +271,57 @@ def test_ffn_reports_bad_slot(moe):
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_check_status(b.layer.status)
     assert ei.value.status == moe.MOE_ERR_DEVICE
+
+
+def test_ffn_reports_bad_slot_tensor_core_path(moe):
+    """The same error from the tcgen05 decode GEMV (bf16 tile layout)."""
+    cfg = synth.LayerConfig("tc_bad_slot", E=8, k=2, d=512, I=256, fmt="bf16")
+    b = Built(cfg, 4)
+    b.layer.slot[b.used[0]] = 10_000
+    b.run()
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_check_status(b.layer.status)
+    assert ei.value.status == moe.MOE_ERR_DEVICE
+
+
+def test_layer_max_experts_and_k(moe):
+    """E = 1024 and k = 32, the ABI's upper bounds, on the tensor-core path
+    (a 1025-entry unit table in shared memory)."""
+    cfg = synth.LayerConfig("maxek", E=1024, k=32, d=256, I=256, fmt="bf16", bias_std=0.5)
+    b = Built(cfg, 3, seed=8)
+    check_tol(b.run().cpu().numpy(), b.oracle()["out"], 1e-4, 1e-5)
+
+
+def _mx_layer_with(scale_byte=None, x_scale=None, which="sg"):
+    cfg = synth.LayerConfig("mx_range", E=8, k=2, d=512, I=256, fmt="mxfp4")
+    logits, x = synth.make_routing(cfg, 2, 4)
+    if x_scale is not None:
+        x = (x.float() * x_scale).to(torch.bfloat16)
+    b = Built(cfg, 2, seed=4, logits=logits, x=x)
+    if scale_byte is not None:
+        from expert_offload_serving_b200.layer import pack_pool
+        b.w_cpu[which][0].fill_(scale_byte)
+        b.layer.pool.copy_(pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, b.w_cpu, b.order, pin=False))
+    return b
+
+
+@pytest.mark.parametrize("scale_byte,x_scale", [(127 + 14, None), (127 - 24, None), (None, 1e5)])
+def test_mxfp4_outside_f16_range_is_reported(moe, scale_byte, x_scale):
+    """The MXFP4 tensor-core path multiplies in f16: an E8M0 scale outside
+    2^[-23, 13] or an activation beyond 65504 is reported as
+    MOE_ERR_UNSUPPORTED instead of being rounded silently."""
+    b = _mx_layer_with(scale_byte, x_scale)
+    b.run()
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_check_status(b.layer.status)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_mxfp4_edge_of_f16_range_is_exact(moe):
+    """Scales 2^-23 (gate) and 2^13 (down projection: its output stays fp32),
+    the ends of the exact range, still match the oracle."""
+    for byte, which in ((127 - 23, "sg"), (127 + 13, "sd")):
+        b = _mx_layer_with(byte, None, which)
+        out = b.run().cpu().numpy()
+        moe.moe_check_status(b.layer.status)
+        check_tol(out, b.oracle()["out"], 1e-4, 1e-5)
