@@ -131,6 +131,8 @@ class MoeLayer:
         """All steps for a resident pool; returns out [T, d] (a view of an
         internal buffer, overwritten by the next call)."""
         T = x.shape[0]
+        # resolve the current stream once for the four calls
+        stream = torch.cuda.current_stream() if stream is None else stream
         self.route(logits, stream)
         self.permute(T, stream)
         if self.act == "nvfp4":
