@@ -148,11 +148,13 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
-// E2M1 pair (one byte, element 2i in the low nibble) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
-  uint32_t r;
-  asm("{ .reg .b8 b; cvt.u8.u32 b, %1; cvt.rn.f16x2.e2m1x2 %0, b; }" : "=r"(r) : "r"(byte));
-  return r;
+// Four E2M1 pairs (the bytes of w, low byte first) -> four f16x2, exact.
+__device__ __forceinline__ void e2m1x8_f16x2(uint32_t w, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;"
+      " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;"
+      " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
@@ -499,7 +501,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
             range_ok &= e8m0_f16x2(((c < 4 ? sc2.x : sc2.y) >> (8 * (c & 3))) & 0xffu, &scl);
             const uint32_t w[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
 #pragma unroll
-            for (int b = 0; b < 16; ++b) v[16 * cc + b] = hmul2(e2m1x2_f16x2((w[b >> 2] >> (8 * (b & 3))) & 0xffu), scl);
+            for (int i = 0; i < 4; ++i) {
+              uint32_t h0, h1, h2, h3;
+              e2m1x8_f16x2(w[i], h0, h1, h2, h3);
+              v[16 * cc + 4 * i + 0] = hmul2(h0, scl);
+              v[16 * cc + 4 * i + 1] = hmul2(h1, scl);
+              v[16 * cc + 4 * i + 2] = hmul2(h2, scl);
+              v[16 * cc + 4 * i + 3] = hmul2(h3, scl);
+            }
           }
           if constexpr (CH == 4) tmem_st64(taddr, v);
           else tmem_st32(taddr, v);
