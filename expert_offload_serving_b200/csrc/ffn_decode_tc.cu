@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         else tok = p / P.k;
       }
       for (int ks = U.ks0; ks < U.ks1; ++ks) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+        if (!mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const uint32_t idesc = C::MX ? idesc_f16(TM, n_mma) : idesc_bf16(TM, n_mma);
       const int acc = it & 1;
-      if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+      if (!mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
@@ -413,8 +413,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         const int aslot = j % C::ASLOTS;
         // the stage has landed; MXFP4: and its A buffer (and, phase 1, the
         // token rows) is converted
-        const bool got = mbar_wait(&full[stage], phase, abort_flag) &&
-                         (!C::MX || mbar_wait(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag));
+        const bool got = mbar_wait<true>(&full[stage], phase, abort_flag) &&
+                         (!C::MX || mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag));
         if (!got) {
           ok = false;
           break;
@@ -475,8 +475,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       const Unit U = unit_of(P, ustart, MT, S, KS, u);
       for (int ks = U.ks0; ks < U.ks1; ++ks, ++j) {
         const int s = j % C::STAGES, aslot = j % C::ASLOTS;
-        if (!mbar_wait(&full[s], (j / C::STAGES) & 1, abort_flag) ||
-            !mbar_wait(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
+        if (!mbar_wait<true>(&full[s], (j / C::STAGES) & 1, abort_flag) ||
+            !mbar_wait<true>(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       const Unit U = unit_of(P, ustart, MT, S, KS, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
-      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
+      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
       named_sync(1, 128);
       if (*epi_fail) {
         report(P.status, MOE_ERR_TIMEOUT);

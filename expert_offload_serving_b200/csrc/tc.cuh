@@ -47,11 +47,28 @@ __device__ __forceinline__ uint64_t now_ns() {
   return t;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or ~20 us pass, instead of spinning and taking issue slots from
+// the warps that do the work.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: false when 2 s pass (or another role gave up first).
+// SLEEP: suspend between tries (measured better for the decode GEMVs, whose
+// waiting warps share issue slots with the converter warps; the prefill
+// GEMM's short stages keep the spinning form).
+template <bool SLEEP = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 0;; ++i) {
-    if (mbar_try(bar, parity)) return true;
+    if (SLEEP ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
     if ((i & 255u) == 255u) {
       if (*abort_flag) return false;
       if (now_ns() - t0 > kWaitNs) return false;
