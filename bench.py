@@ -271,9 +271,7 @@ def run_gpu(args, rank, world, local):
         print(f"warning: replicas stream only {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
               "between reuses", file=sys.stderr)
     stream = torch.cuda.Stream(device=dev)
-    # route, permute, ffn gate/up, ffn down, combine; plus the split-sum kernel
-    # between the two GEMVs when T*k <= 32
-    launches_per_step = 5 + (1 if T * cfg.k <= 32 else 0)
+    launches_per_step = 5   # route, permute, ffn gate/up, ffn down, combine
 
     def step_fn(r):
         L = r["layer"]
@@ -332,23 +330,58 @@ def run_gpu(args, rank, world, local):
     hbm_peak, peak_src = peaks()
     achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step
+    # uploads its logits and x from pinned host memory and downloads its out,
+    # pipelined as a serving loop would run it -- the copies go on a copy
+    # stream (uploads one step ahead, downloads behind), ordered by events,
+    # and the timed region closes when the last download has landed
     e2e_steps = max(3, min(args.steps, 50))
     outs_h = [torch.empty((T, cfg.d), dtype=torch.float32, pin_memory=True) for _ in range(R)]
-    with torch.cuda.stream(stream):
-        def e2e_step(i):
-            r = reps[i % R]
+    copy = torch.cuda.Stream(device=dev)
+    in_ready = [torch.cuda.Event() for _ in range(R)]
+    out_done = [torch.cuda.Event() for _ in range(R)]
+    out_copied = [torch.cuda.Event() for _ in range(R)]
+    for ev in out_done + out_copied:
+        ev.record(stream)                   # give every event a handle before it is waited on
+
+    def upload(i):
+        r = reps[i % R]
+        with torch.cuda.stream(copy):
+            copy.wait_event(out_done[i % R])          # the replica's previous step has read its inputs
             r["logits"].copy_(r["logits_h"], non_blocking=True)
             r["x"].copy_(r["x_h"], non_blocking=True)
-            out = r["layer"].forward(r["logits"], r["x"])
-            outs_h[i % R].copy_(out, non_blocking=True)
-        for i in range(max(3, args.warmup)):
-            e2e_step(i)
+            in_ready[i % R].record(copy)
+
+    def compute(i):
+        r = reps[i % R]
+        stream.wait_event(in_ready[i % R])
+        stream.wait_event(out_copied[i % R])          # its previous out has been downloaded
+        r["out_dev"] = r["layer"].forward(r["logits"], r["x"], stream=stream)
+        out_done[i % R].record(stream)
+
+    def download(i):
+        r = reps[i % R]
+        with torch.cuda.stream(copy):
+            copy.wait_event(out_done[i % R])
+            outs_h[i % R].copy_(r["out_dev"], non_blocking=True)
+            out_copied[i % R].record(copy)
+
+    def run_e2e(n, first):
+        upload(first)
+        for i in range(first, first + n):
+            if i + 1 < first + n:
+                upload(i + 1)
+            compute(i)
+            download(i)
+
+    with torch.cuda.stream(stream):
+        run_e2e(max(3, args.warmup), 0)
         torch.cuda.synchronize()
         barrier(world)
         e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i)
+        copy.wait_event(e0)
+        run_e2e(e2e_steps, 0)
+        stream.wait_event(out_copied[(e2e_steps - 1) % R])
         e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)

@@ -130,11 +130,6 @@ __host__ __device__ inline size_t mx_tile_scale_offset(int r, int j, int K) {
   return tile * kMxTileBytes + 16384 + static_cast<size_t>(r & 127) * 8 + (j & 7);
 }
 
-// K splits of the decode GEMV for n = T*k routed pairs: few pairs give too few
-// (expert, tile) units to fill the SMs, so each tile's K range is split and
-// the partial sums are added afterwards.
-__host__ __device__ inline int decode_split(long long n) { return n <= 8 ? 4 : (n <= 32 ? 2 : 1); }
-
 // Row of W_gu holding gate row i (up = false) or up row i (up = true).
 __host__ __device__ inline int gu_row(int i, bool up) { return (i >> 6) * 128 + (up ? 64 : 0) + (i & 63); }
 

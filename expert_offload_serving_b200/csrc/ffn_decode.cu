@@ -649,12 +649,8 @@ moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t
 }  // namespace
 
 size_t decode_workspace_bytes(moe_shape s, int T, int k) {
-  // a (fp32, or the two 16-bit planes of the tensor-core path); then the
-  // tensor-core path's split partial sums
-  const size_t n = static_cast<size_t>(T) * k;
-  const size_t a = round_up(n * s.I * sizeof(float), 256);
-  const int split = decode_split(static_cast<long long>(n));
-  return a + (split > 1 ? round_up(static_cast<size_t>(split) * n * 2 * s.I * sizeof(float), 256) : 0);
+  // a: fp32 (CUDA-core path) or the two 16-bit planes of the tensor-core path
+  return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256);
 }
 
 moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,

@@ -37,8 +37,6 @@
 // epilogue on double-buffered TMEM accumulators.  Every wait is bounded: on
 // expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains what it
 // issued and frees its TMEM.
-#include <algorithm>
-
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -49,9 +47,7 @@ namespace moe {
 
 struct TcDecodeParams {
   int E, d, I, T, k, n_slots;
-  int a_box_rows;            // rows of one TMA box of the a planes (min(32, T*k))
-  int split1, split2;        // K splits of gemv<1> and gemv<2> (each <= its K stages)
-  float* part;               // split1 > 1: gemv<1> partial sums [split1][T*k][2I] fp32
+  int a_box_rows[3];         // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
   const int32_t* offsets;
   const int32_t* perm;
   const int32_t* slot;
@@ -107,12 +103,11 @@ constexpr size_t smem_bytes(int E) {
 }
 
 struct Unit {
-  int e, m, q0, nvalid, ks0, ks1;   // K stages [ks0, ks1) of the unit's split
+  int e, m, q0, nvalid;
 };
 
-// unit u -> (expert, tile, chunk, K split); ustart[e] = first unit of expert e
-__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int S, int KS,
-                                        int u) {
+// unit u -> (expert, tile, chunk); ustart[e] = first unit of expert e
+__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int u) {
   int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -123,11 +118,9 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
   U.e = lo;
   const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
   const int chunks = (ne + TN - 1) / TN;
-  const int local = (u - ustart[lo]) / S, sp = (u - ustart[lo]) % S;
+  const int local = u - ustart[lo];
   U.m = local / chunks;
   const int c = local % chunks;
-  U.ks0 = sp * KS / S;
-  U.ks1 = (sp + 1) * KS / S;
   U.q0 = q_begin + c * TN;
   U.nvalid = min(TN, ne - c * TN);
   return U;
@@ -144,6 +137,35 @@ __device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, con
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Issued by gemv<1>'s producer once its own stages are all out: L2 prefetches
+// of the first weight stages of the gemv<2> units this CTA will run (same
+// round-robin deal), up to `budget` bytes, so that gemv<2> starts on warm L2.
+// gemv<2>'s units of expert e are proportional to gemv<1>'s: both are
+// tiles x chunks(e), so ustart1 scales to the gemv<2> table.
+template <int FMT>
+__device__ void prefetch_down_units(const TcDecodeParams& P, const int32_t* ustart1, int per1, size_t budget) {
+  using C = Cfg<FMT, 2>;
+  const int MT2 = P.d / TM, KS2 = P.I / C::KSTAGE, per2 = MT2;
+  const int n2 = ustart1[P.E] / per1 * per2;
+  for (int u = blockIdx.x; u < n2 && budget > 0; u += gridDim.x) {
+    int lo = 0, hi = P.E;   // last e with ustart1[e] / per1 * per2 <= u
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ustart1[mid] / per1 * per2 <= u) lo = mid;
+      else hi = mid;
+    }
+    const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+    const int chunks = (ne + TN - 1) / TN;
+    const int m = (u - ustart1[lo] / per1 * per2) / chunks;
+    const uint8_t* base = P.pool + static_cast<size_t>(__ldg(P.slot + lo)) * P.blob_bytes + P.L.wd +
+                          static_cast<size_t>(m) * KS2 * C::A_STAGE;
+    for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
+      prefetch_l2(base + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE);
+      budget = budget > static_cast<size_t>(C::A_STAGE) ? budget - C::A_STAGE : 0;
+    }
+  }
 }
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
@@ -208,7 +230,8 @@ __device__ __forceinline__ void split16(float a, bool mx, uint16_t* hi, uint16_t
 
 template <int FMT, int PHASE>
 __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
-    gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_b, TcDecodeParams P) {
+    gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b16,
+                   const __grid_constant__ CUtensorMap tm_b8, TcDecodeParams P) {
   using C = Cfg<FMT, PHASE>;
   constexpr int THREADS = C::THREADS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -232,7 +255,6 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   const int K = (PHASE == 1) ? P.d : P.I;
   const int KS = K / C::KSTAGE;
   const int MT = (PHASE == 1) ? P.I / 64 : P.d / TM;
-  const int S = PHASE == 1 ? P.split1 : P.split2;   // K splits per tile
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
@@ -280,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       continue;
     }
     if (s < 0) continue;
-    cnt += MT * S * ((b - a + TN - 1) / TN);
+    cnt += MT * ((b - a + TN - 1) / TN);
   }
   int total = 0;
   int run = block_scan(cnt, ws, &total);
@@ -290,7 +312,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     ustart[e] = run;
     const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
     const int s = __ldg(P.slot + e);
-    if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * S * ((b - a + TN - 1) / TN);
+    if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * ((b - a + TN - 1) / TN);
   }
   if (threadIdx.x == 0) ustart[P.E] = total;
   tc_fence_before();
@@ -307,16 +329,11 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     int issued = 0;
     bool ok = true;
     // L2 prefetch cursor over this CTA's (unit, stage) items
-    int pf_u = blockIdx.x, pf_ks = 0, pf_ks1 = 0, pf_ahead = 0;
+    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_u < n_units) {
-      const Unit V = unit_of(P, ustart, MT, S, KS, pf_u);
-      pf_base = tile_base<FMT, PHASE>(P, V);
-      pf_ks = V.ks0;
-      pf_ks1 = V.ks1;
-    }
+    if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of(P, ustart, MT, pf_u));
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      const Unit U = unit_of(P, ustart, MT, u);
       const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
       int tok = 0;
       if (PHASE == 1 && lane < U.nvalid) {
@@ -324,7 +341,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
         else tok = p / P.k;
       }
-      for (int ks = U.ks0; ks < U.ks1; ++ks) {
+      for (int ks = 0; ks < KS; ++ks) {
         if (!mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -332,15 +349,19 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         uint8_t* sA = smem + stage * C::STAGE;
         uint8_t* sB = sA + C::A_STAGE;
         if (lane == 0) {
-          const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * P.a_box_rows;
+          // gemv<2>: the smallest a-plane box (8, 16 or 32 rows) that holds the
+          // unit's pairs; rows beyond them are never read back
+          const int bi = U.nvalid <= P.a_box_rows[0] ? 0 : (U.nvalid <= P.a_box_rows[1] ? 1 : 2);
+          const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * P.a_box_rows[bi];
           mbar_expect_tx(&full[stage], C::A_STAGE + rows * C::ATOMS * 128u);
           bulk_load(sA, abase + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE, &full[stage], pol_stream);
           if (PHASE == 2) {
+            const CUtensorMap* tm = bi == 0 ? &tm_b8 : (bi == 1 ? &tm_b16 : &tm_b);
 #pragma unroll
             for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
               for (int a = 0; a < C::ATOMS; ++a)
-                tma_load_3d(sB + (pl * C::ATOMS + a) * B_ATOM, &tm_b, &full[stage], ks * C::KSTAGE + 64 * a, U.q0,
+                tma_load_3d(sB + (pl * C::ATOMS + a) * B_ATOM, tm, &full[stage], ks * C::KSTAGE + 64 * a, U.q0,
                             pl, pol_keep);
           }
           // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one (the
@@ -350,14 +371,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
             while (pf_u < n_units && pf_ahead < PF_ITEMS) {
               prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
               ++pf_ahead;
-              if (++pf_ks == pf_ks1) {
+              if (++pf_ks == KS) {
+                pf_ks = 0;
                 pf_u += gridDim.x;
-                if (pf_u < n_units) {
-                  const Unit V = unit_of(P, ustart, MT, S, KS, pf_u);
-                  pf_base = tile_base<FMT, PHASE>(P, V);
-                  pf_ks = V.ks0;
-                  pf_ks1 = V.ks1;
-                }
+                if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of(P, ustart, MT, pf_u));
               }
             }
             --pf_ahead;
@@ -377,6 +394,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
         }
       }
     }
+    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<FMT>(P, ustart, MT, 256u << 10);
+    __syncwarp();
     if (!ok) {
       report(P.status, MOE_ERR_TIMEOUT);
       *abort_flag = 1;
@@ -399,7 +418,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     int it = 0, j = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      const Unit U = unit_of(P, ustart, MT, u);
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const uint32_t idesc = C::MX ? idesc_f16(TM, n_mma) : idesc_bf16(TM, n_mma);
       const int acc = it & 1;
@@ -409,7 +428,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
-      for (int ks = U.ks0; ks < U.ks1; ++ks, ++j) {
+      for (int ks = 0; ks < KS; ++ks, ++j) {
         const int aslot = j % C::ASLOTS;
         // the stage has landed; MXFP4: and its A buffer (and, phase 1, the
         // token rows) is converted
@@ -428,7 +447,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
             const int a = kk >> 2;
             const uint64_t dh = desc_sw128(smem_u32(sB + a * B_ATOM)) + 2 * (kk & 3);
             const uint64_t dl = desc_sw128(smem_u32(sB + (C::ATOMS + a) * B_ATOM)) + 2 * (kk & 3);
-            const uint32_t first = (ks > U.ks0 || kk > 0) ? 1u : 0u;
+            const uint32_t first = (ks > 0 || kk > 0) ? 1u : 0u;
             if (C::MX) {
               const uint32_t ta = tmem + C::A_COL0 + aslot * C::A_COLS + 8 * kk;
               tc_mma_f16_ts(d_tmem, ta, dh, idesc, first);
@@ -472,8 +491,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     bool range_ok = true;
     int j = 0;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of(P, ustart, MT, S, KS, u);
-      for (int ks = U.ks0; ks < U.ks1; ++ks, ++j) {
+      const Unit U = unit_of(P, ustart, MT, u);
+      for (int ks = 0; ks < KS; ++ks, ++j) {
         const int s = j % C::STAGES, aslot = j % C::ASLOTS;
         if (!mbar_wait<true>(&full[s], (j / C::STAGES) & 1, abort_flag) ||
             !mbar_wait<true>(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
@@ -540,7 +559,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     bool range_ok = true;
     int it = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, S, KS, u);
+      const Unit U = unit_of(P, ustart, MT, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
@@ -555,16 +574,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (PHASE == 1 && S > 1) {
-        // a K split: the tile's partial gate (rows 0..63) and up (64..127) sums
-        const int r = 32 * quad + lane;
-        const int sp = (u - ustart[U.e]) % S;
-        const size_t col = (r < 64) ? static_cast<size_t>(64) * U.m + r : static_cast<size_t>(P.I) + 64 * U.m + (r - 64);
-        float* dst = P.part + (static_cast<size_t>(sp) * n_pairs + U.q0) * (2 * P.I) + col;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (c < U.nvalid) dst[static_cast<size_t>(c) * (2 * P.I)] = v[c];
-      } else if (PHASE == 1) {
+      if (PHASE == 1) {
         // rows 0..63 of the tile are gate rows, 64..127 the matching up rows
         if (quad >= 2) {
           const int i = 32 * (quad - 2) + lane;
@@ -597,9 +607,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
           if (c < U.nvalid) {
             const int q = U.q0 + c;
             if (P.y_perm != nullptr) {
-              // with K splits y_perm was zeroed and receives the split sums
-              if (S > 1) atomicAdd(P.y_perm + static_cast<size_t>(q) * P.d + row, v[c]);
-              else P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
+              P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
             } else {
               const int p = __ldg(P.perm + q);
               if (p >= 0 && p < n_pairs)
@@ -619,41 +627,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   }
 }
 
-// After a split gemv<1>: a = silu(sum of gate partials) * (sum of up
-// partials) into the two 16-bit planes; and, when gemv<2> splits into y_perm,
-// y_perm zeroed for its split sums.
-template <bool MX>
-__global__ void __launch_bounds__(256) finish_swiglu_kernel(const float* __restrict__ part, int S, int n, int I,
-                                                            uint16_t* __restrict__ planes, float* y_zero, int n_y,
-                                                            int d, int32_t* status) {
-  const size_t tot = static_cast<size_t>(n) * I;   // n = 0: no split of gemv<1>
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  bool ok = true;
-  for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < tot; idx += stride) {
-    const size_t q = idx / I, i = idx % I;
-    float h = 0.f, u = 0.f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float* p = part + (static_cast<size_t>(sp) * n + q) * (2 * static_cast<size_t>(I));
-      h += p[i];
-      u += p[I + i];
-    }
-    const float a = silu(h) * u;
-    if (MX) ok &= fabsf(a) <= 65504.f;
-    uint16_t hi, lo;
-    split16(a, MX, &hi, &lo);
-    planes[idx] = hi;
-    planes[tot + idx] = lo;
-  }
-  if (y_zero != nullptr) {
-    const size_t n4 = static_cast<size_t>(n_y) * d / 4;
-    for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < n4; idx += stride)
-      reinterpret_cast<float4*>(y_zero)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  if (!ok) report(status, MOE_ERR_UNSUPPORTED);
-}
-
 template <int FMT, int PHASE>
-moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const DeviceInfo& dev, cudaStream_t s) {
+moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const CUtensorMap& tm16,
+                        const CUtensorMap& tm8, const DeviceInfo& dev, cudaStream_t s) {
   const size_t smem = smem_bytes<FMT, PHASE>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
@@ -662,25 +638,17 @@ moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const De
                                       static_cast<int>(smem)));
     attr[dev.id] = smem;
   }
-  gemv_tc_kernel<FMT, PHASE><<<dev.sm_count, Cfg<FMT, PHASE>::THREADS, smem, s>>>(tm, P);
+  gemv_tc_kernel<FMT, PHASE><<<dev.sm_count, Cfg<FMT, PHASE>::THREADS, smem, s>>>(tm, tm16, tm8, P);
   MOE_LAUNCH_CHECK("gemv_tc_kernel");
   return MOE_OK;
 }
 
 template <int FMT>
-moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap& tm_a,
+moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap (&tm_a)[3],
                        const DeviceInfo& dev, cudaStream_t stream) {
-  moe_status st = launch_phase<FMT, 1>(P, tm_x, dev, stream);
+  moe_status st = launch_phase<FMT, 1>(P, tm_x, tm_x, tm_x, dev, stream);
   if (st != MOE_OK) return st;
-  float* y_zero = (P.split2 > 1) ? P.y_perm : nullptr;
-  if (P.split1 > 1 || y_zero != nullptr) {
-    const size_t tot = static_cast<size_t>(P.T) * P.k * std::max(P.I, P.d);
-    const int blocks = static_cast<int>(std::min<size_t>((tot + 255) / 256, static_cast<size_t>(4) * dev.sm_count));
-    finish_swiglu_kernel<FMT == MOE_W_MXFP4><<<blocks, 256, 0, stream>>>(
-        P.part, P.split1, P.split1 > 1 ? P.T * P.k : 0, P.I, P.a_planes, y_zero, P.T * P.k, P.d, P.status);
-    MOE_LAUNCH_CHECK("finish_swiglu_kernel");
-  }
-  return launch_phase<FMT, 2>(P, tm_a, dev, stream);
+  return launch_phase<FMT, 2>(P, tm_a[2], tm_a[1], tm_a[0], dev, stream);
 }
 
 }  // namespace
@@ -705,21 +673,15 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
   P.L = blob_layout(s.fmt, s.d, s.I);
   P.blob_bytes = P.L.bytes;
   P.a_planes = static_cast<uint16_t*>(ws);
-  const size_t n_pairs = static_cast<size_t>(T) * k;
-  {
-    // K stages per tile: bf16 128 elements, MXFP4 256
-    const int kstage = s.fmt == MOE_W_MXFP4 ? 256 : 128;
-    const int split = decode_split(static_cast<long long>(n_pairs));
-    P.split1 = std::min(split, s.d / kstage);
-    P.split2 = std::min(std::min(split, 2), s.I / kstage);
-  }
-  P.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + round_up(n_pairs * s.I * sizeof(float), 256));
   P.y_perm = y_perm;
   P.out = out;
   P.status = status;
   const uint64_t n = static_cast<uint64_t>(T) * k;
-  P.a_box_rows = static_cast<int>(n < static_cast<uint64_t>(TN) ? n : static_cast<uint64_t>(TN));
-  CUtensorMap tm_x, tm_a;
+  for (int i = 0; i < 3; ++i) {
+    const uint64_t r = static_cast<uint64_t>(8) << i;   // 8, 16, 32 = TN
+    P.a_box_rows[i] = static_cast<int>(n < r ? n : r);
+  }
+  CUtensorMap tm_x, tm_a[3];
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T)};
     const uint64_t str[1] = {static_cast<uint64_t>(s.d) * 2};
@@ -727,13 +689,13 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
     const CUresult r = encode_tiled_sw128(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of x failed (%d)", static_cast<int>(r));
   }
-  {
+  for (int i = 0; i < 3; ++i) {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, 2};
     const uint64_t str[2] = {static_cast<uint64_t>(s.I) * 2, n * s.I * 2};
-    const uint32_t box[3] = {64u, static_cast<uint32_t>(P.a_box_rows), 1u};
+    const uint32_t box[3] = {64u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
     const CUtensorMapDataType type =
         s.fmt == MOE_W_MXFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const CUresult r = encode_tiled_sw128(&tm_a, type, 3, ws, dims, str, box);
+    const CUresult r = encode_tiled_sw128(&tm_a[i], type, 3, ws, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a planes failed (%d)", static_cast<int>(r));
   }
   if (s.fmt == MOE_W_MXFP4) return launch_both<MOE_W_MXFP4>(P, tm_x, tm_a, dev, stream);

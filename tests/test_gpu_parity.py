@@ -169,8 +169,7 @@ def test_y_perm_rows_match_pairs(moe):
 
 @pytest.mark.parametrize("T", [1, 16])
 def test_fused_out_matches_combine(moe, T):
-    """out += gate * y in the FFN epilogue equals y_perm + combine (T=1 runs
-    the K-split GEMVs, whose partial sums meet in out)."""
+    """out += gate * y in the FFN epilogue equals y_perm + combine."""
     cfg = synth.CONFIGS["decode_bf16"]
     b = Built(cfg, T, seed=6)
     ref = b.run().clone()
