@@ -178,8 +178,20 @@ moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E,
  *                     accumulated with atomic adds; the caller initialises out
  *                     (zeros, or the host partial).
  *   flags: 0 or MOE_FFN_ACT_NVFP4.
- *   workspace: device, >= moe_expert_ffn_workspace_bytes(s, T, k, flags).
- *   dev_status: device int32 word or NULL (slot or expert out of range).
+ *   workspace: device, 256-byte aligned, >= moe_expert_ffn_workspace_bytes(s,
+ *              T, k, flags); its contents need no initialisation.
+ *   dev_status: device int32 word or NULL.  Kernels record the first error
+ *              there (read it with moe_check_status after the stream):
+ *              MOE_ERR_DEVICE   a slot or expert index out of range;
+ *              MOE_ERR_TIMEOUT  a bounded wait on the copy pipeline ran out;
+ *              MOE_ERR_UNSUPPORTED  (MXFP4 on the tensor-core path, which
+ *                               multiplies in f16 exactly) an E8M0 scale
+ *                               outside 2^[-23, 13], or |x| or |a| above 65504.
+ * Paths (chosen from the shape, the same results up to rounding order):
+ *   BF16 with d, I multiples of 256 and MXFP4 with d, I multiples of 256: the
+ *   tcgen05 decode GEMVs over the tile layouts of moe_pack_expert; other
+ *   BF16/MXFP4 shapes and NVFP4 without MOE_FFN_ACT_NVFP4: CUDA cores;
+ *   MOE_FFN_ACT_NVFP4: the tcgen05 FP4 GEMMs (d, I multiples of 256).
  * Limits: T*k <= 1<<24. */
 size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int flags);
 moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k,
