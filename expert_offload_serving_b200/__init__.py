@@ -51,6 +51,8 @@ _SIGS = {
     "moe_expert_ffn_workspace_bytes": (_SZ, [moe_shape, _I, _I, _I]),
     "moe_expert_ffn": (_I, [moe_shape, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P, _P]),
     "moe_combine_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "moe_layer_forward": (_I, [moe_shape, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P, _P, _I, _P, _I, _P,
+                               _SZ, _P, _P, _P, _P]),
     "moe_cache_create": (_I, [moe_shape, _I, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_cache_fill": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
     "moe_cache_query": (_I, [_P, _P, _P, _P]),
@@ -179,6 +181,20 @@ def moe_combine_merge(y_perm, idx, gate, inv_perm, slot_of_expert, host_partial,
     _check(lib().moe_combine_merge(_ptr(y_perm), _ptr(idx), _ptr(gate), _ptr(inv_perm),
                                    _ptr(slot_of_expert), _ptr(host_partial), T, k, d, E, _ptr(out),
                                    _stream(stream)))
+
+
+def moe_layer_forward(s: moe_shape, logits, x, k: int, idx, gate, offsets, perm, inv_perm, scratch,
+                      slot_of_expert, slot_pool, n_slots: int, y_perm, flags, workspace, host_partial, out,
+                      dev_status=None, stream=None):
+    """All four steps in one call (moe_route_topk -> moe_permute ->
+    moe_expert_ffn -> moe_combine_merge); x [T, d] gives T."""
+    T = x.shape[0]
+    sb = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    wb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().moe_layer_forward(s, _ptr(logits), _ptr(x), T, k, _ptr(idx), _ptr(gate), _ptr(offsets), _ptr(perm),
+                                   _ptr(inv_perm), _ptr(scratch), sb, _ptr(slot_of_expert), _ptr(slot_pool),
+                                   n_slots, _ptr(y_perm), flags, _ptr(workspace), wb, _ptr(host_partial),
+                                   _ptr(out), _ptr(dev_status), _stream(stream)))
 
 
 def moe_check_status(dev_status, stream=None):

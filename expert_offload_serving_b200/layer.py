@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (MOE_FFN_ACT_NVFP4, FORMATS, MoeCache, moe_combine_merge, moe_expert_blob_bytes,
+from . import (MOE_FFN_ACT_NVFP4, FORMATS, MoeCache, _check, lib, moe_combine_merge, moe_expert_blob_bytes,
                moe_expert_ffn, moe_expert_ffn_workspace_bytes, moe_pack_expert, moe_permute,
                moe_permute_scratch_bytes, moe_route_topk, shape)
 
@@ -128,21 +128,21 @@ class MoeLayer:
                           self.E, out if out is not None else self.out[:T], stream)
 
     def forward(self, logits, x, host_partial=None, stream=None):
-        """All steps for a resident pool; returns out [T, d] (a view of an
-        internal buffer, overwritten by the next call)."""
+        """All steps for a resident pool through moe_layer_forward (one C
+        call); returns out [T, d] (a view of an internal buffer, overwritten by
+        the next call)."""
         T = x.shape[0]
-        # resolve the current stream once for the four calls
-        stream = torch.cuda.current_stream() if stream is None else stream
-        self.route(logits, stream)
-        self.permute(T, stream)
-        if self.act == "nvfp4":
-            o = self.out[:T]
-            if host_partial is None:
-                o.zero_()
-            else:
-                o.copy_(host_partial)
-            self.ffn(x, stream)
-        else:
-            self.ffn(x, stream)
-            self.combine(T, host_partial, stream)
+        if not hasattr(self, "_fwd_args"):
+            # device addresses of the layer's own buffers, resolved once
+            nb = lambda t: t.numel() * t.element_size()
+            self._fwd_args = (self.idx.data_ptr(), self.gate.data_ptr(), self.offsets.data_ptr(),
+                              self.perm.data_ptr(), self.inv_perm.data_ptr(), self.scratch.data_ptr(),
+                              nb(self.scratch), self.slot.data_ptr(), self.pool.data_ptr(), self.n_slots,
+                              0 if self.y_perm is None else self.y_perm.data_ptr(), self.flags,
+                              self.workspace.data_ptr(), nb(self.workspace))
+        s = (torch.cuda.current_stream() if stream is None else stream)
+        s = s if isinstance(s, int) else s.cuda_stream
+        hp = 0 if host_partial is None else host_partial.data_ptr()
+        _check(lib().moe_layer_forward(self.s, logits.data_ptr(), x.data_ptr(), T, self.k, *self._fwd_args, hp,
+                                       self.out.data_ptr(), self.status.data_ptr(), s))
         return self.out[:T]

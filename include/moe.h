@@ -220,6 +220,23 @@ moe_status moe_combine_merge(const float* y_perm, const int32_t* idx, const floa
                              cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* A whole layer call in one entry point: moe_route_topk -> moe_permute ->
+ * moe_expert_ffn -> moe_combine_merge, all enqueued on `stream`; with
+ * MOE_FFN_ACT_NVFP4, out is first set to host_partial (or zero) and the FFN
+ * adds the combine into it (y_perm is then unused and may be NULL).  Every
+ * buffer is the one the individual call takes, with the same meaning,
+ * layout, ownership and errors; the results are those of the four calls.
+ * It exists for the host cost of a decode step: one call instead of four.
+ * Returns the first failing step's status; nothing after it is enqueued. */
+moe_status moe_layer_forward(moe_shape s, const float* logits, const void* x, int T, int k,
+                             int32_t* idx, float* gate, int32_t* offsets, int32_t* perm,
+                             int32_t* inv_perm, void* scratch, size_t scratch_bytes,
+                             const int32_t* slot_of_expert, const void* slot_pool, int n_slots,
+                             float* y_perm, int flags, void* workspace, size_t ws_bytes,
+                             const float* host_partial, float* out, int32_t* dev_status,
+                             cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Step 5 -- the GPU expert cache: LRU residency of expert blobs in device
  * slots, filled from a pinned host pool (freetoken.wiki mechanism table:
  * "Global LRU expert cache"; explainx.ai hardware guide: experts are copied
