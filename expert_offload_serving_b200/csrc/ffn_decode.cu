@@ -29,9 +29,12 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace moe {
 namespace {
+
+using namespace ::moe::tc;
 
 constexpr int kWarps = 16;                 // warps per CTA (each its own pipeline)
 constexpr int kRW = 4;                      // weight rows per warp tile
@@ -121,53 +124,9 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[V], int lane) {
 }
 
 // ------------------------------------------------------------ bulk copies
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-constexpr uint64_t kWaitNs = 2000000000ull;   // a stage that has not landed in 2 s is an error
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = now_ns();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 255u) == 255u && now_ns() - t0 > kWaitNs) return false;
-  }
-}
-// Weights are read once per layer call: stream them through L2 with an
-// evict-first policy so the activations and the SwiGLU workspace stay cached.
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                                          uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
-      "%4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
+// (mbarrier, bulk-copy and L2-policy wrappers: tc.cuh).  Weights are read once
+// per layer call: they stream through L2 with an evict-first policy so the
+// activations and the SwiGLU workspace stay cached.
 
 // Small expert sets: when every active expert's blob together fits well
 // inside L2, the first launch asks L2 to fetch all of them at once (16 KB bulk
@@ -413,7 +372,7 @@ __device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* 
   for (int sl = 0; sl < pp.slices; ++sl, ++j) {
     if (pp.next_issue < pp.n_items) issue_item<FMT, PHASE>(P, act, ustart, n_act, pp, row_bytes, lane);
     const int st = static_cast<int>(j % kStages);
-    if (!mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1))) {
+    if (!mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1), nullptr)) {
       pp.ok = false;
       return;
     }

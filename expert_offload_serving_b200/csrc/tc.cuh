@@ -60,7 +60,8 @@ __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: false when 2 s pass (or another role gave up first).
+// Bounded wait: false when 2 s pass (or another role gave up first; no
+// abort flag: abort_flag == nullptr).
 // SLEEP: suspend between tries (measured better for the decode GEMVs, whose
 // waiting warps share issue slots with the converter warps; the prefill
 // GEMM's short stages keep the spinning form).
@@ -70,7 +71,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   for (uint32_t i = 0;; ++i) {
     if (SLEEP ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
     if ((i & 255u) == 255u) {
-      if (*abort_flag) return false;
+      if (abort_flag != nullptr && *abort_flag) return false;
       if (now_ns() - t0 > kWaitNs) return false;
     }
   }
