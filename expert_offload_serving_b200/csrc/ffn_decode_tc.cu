@@ -17,8 +17,10 @@
 //          block scale -- stored into TMEM, where the MMA reads A; the token
 //          rows are converted bf16 -> f16 in shared memory.  f16 holds every
 //          E2M1 x 2^X exactly for X in [-23, 13] and every bf16 activation below
-//          65504 in magnitude; a scale or an activation outside is reported
-//          as MOE_ERR_UNSUPPORTED in the status word.
+//          65504 in magnitude; a scale above, a scale below on a block with
+//          nonzero codes (blocks of zeros are exact at any scale), or an
+//          activation outside is reported as MOE_ERR_UNSUPPORTED in the status
+//          word.
 //
 //   gemv<1>: D[128 x N] = W_gu tile (64 gate + 64 up rows of the same
 //            intermediate indices) x X^T over K = d, N <= 32 token rows
@@ -185,13 +187,17 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   return r;
 }
 
-// E8M0 scale byte -> 2^(byte - 127) as f16x2, exact for exponents -24..15;
-// false when E2M1 x 2^X would not be exact in f16 (X outside [-23, 13]).
-__device__ __forceinline__ bool e8m0_f16x2(uint32_t byte, uint32_t* out) {
+// E8M0 scale byte -> 2^(byte - 127) as f16x2.  Exact for X = byte - 127 in
+// [-23, 13], where every E2M1 x 2^X is an f16.  Below, the products lie under
+// f16's smallest subnormal: the scale flushes to 0 and *tiny is set (exact for
+// an all-zero block, such as the ones encoded with byte 0); above, they would
+// overflow: false.
+__device__ __forceinline__ bool e8m0_f16x2(uint32_t byte, uint32_t* out, bool* tiny) {
   const int x = static_cast<int>(byte) - 127;
+  *tiny = x < -23;
   if (x < -23 || x > 13) {
     *out = 0;
-    return false;
+    return x <= 13;
   }
   const uint32_t h = (x >= -14) ? static_cast<uint32_t>(x + 15) << 10 : 1u << (x + 24);
   *out = h | (h << 16);
@@ -517,7 +523,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
           for (int cc = 0; cc < CH; ++cc) {
             const int c = CH * part + cc;
             uint32_t scl;
-            range_ok &= e8m0_f16x2(((c < 4 ? sc2.x : sc2.y) >> (8 * (c & 3))) & 0xffu, &scl);
+            bool tiny;
+            range_ok &= e8m0_f16x2(((c < 4 ? sc2.x : sc2.y) >> (8 * (c & 3))) & 0xffu, &scl, &tiny);
+            // a flushed scale is exact only for a block of zeros (E2M1 magnitude bits 0)
+            if (tiny) range_ok &= ((q[cc].x | q[cc].y | q[cc].z | q[cc].w) & 0x77777777u) == 0u;
             const uint32_t w[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {

@@ -186,7 +186,8 @@ moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E,
  *              MOE_ERR_TIMEOUT  a bounded wait on the copy pipeline ran out;
  *              MOE_ERR_UNSUPPORTED  (MXFP4 on the tensor-core path, which
  *                               multiplies in f16 exactly) an E8M0 scale
- *                               outside 2^[-23, 13], or |x| or |a| above 65504.
+ *                               above 2^13, or below 2^-23 on a block with
+ *                               nonzero codes, or |x| or |a| above 65504.
  * Paths (chosen from the shape, the same results up to rounding order):
  *   BF16 with d, I multiples of 256 and MXFP4 with d, I multiples of 256: the
  *   tcgen05 decode GEMVs over the tile layouts of moe_pack_expert; other

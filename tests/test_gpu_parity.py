@@ -324,3 +324,21 @@ def test_mxfp4_edge_of_f16_range_is_exact(moe):
         out = b.run().cpu().numpy()
         moe.moe_check_status(b.layer.status)
         check_tol(out, b.oracle()["out"], 1e-4, 1e-5)
+
+
+def test_mxfp4_zero_block_with_smallest_scale_is_exact(moe):
+    """A block of zero codes encoded with E8M0 byte 0 (2^-127, as MXFP4
+    writers emit for all-zero blocks) is exact on the f16 tensor-core path:
+    no error is reported and the output matches the oracle."""
+    cfg = synth.LayerConfig("mx_zero", E=8, k=2, d=512, I=256, fmt="mxfp4")
+    logits, x = synth.make_routing(cfg, 2, 4)
+    b = Built(cfg, 2, seed=4, logits=logits, x=x)
+    from expert_offload_serving_b200.layer import pack_pool
+    for key, sk in (("wg", "sg"), ("wd", "sd")):
+        b.w_cpu[key][0][:8, :16] = 0           # 8 rows: their first 32-element block is all zeros
+        b.w_cpu[sk][0][:8, 0] = 0              # with the smallest scale
+    b._deq.clear()
+    b.layer.pool.copy_(pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, b.w_cpu, b.order, pin=False))
+    out = b.run().cpu().numpy()
+    moe.moe_check_status(b.layer.status)
+    check_tol(out, b.oracle()["out"], 1e-4, 1e-5)
