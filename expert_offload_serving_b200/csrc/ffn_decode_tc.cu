@@ -31,14 +31,17 @@
 //            k-step).  Epilogue: y_perm rows, or out[t] += gate * y (the fused
 //            combine).
 //
-// Work unit = (expert, 128-row tile, chunk of <= 32 of the expert's pairs),
-// expert-major, chunks fastest, dealt round-robin to one persistent CTA per
-// SM.  Warp 0 produces (bulk copy of the weight stage, TMA loads of the token
-// rows, L2 prefetch of the weight stages four items ahead), warp 1 owns TMEM and
-// issues the MMAs, [MXFP4: warps 2-9 convert], the last four warps run the
-// epilogue on double-buffered TMEM accumulators.  Every wait is bounded: on
-// expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains what it
-// issued and frees its TMEM.
+// Work unit = (expert, 128-row tile, chunk of <= TN of the expert's pairs; TN
+// = 16 when T <= 16, else 32), expert-major, chunks fastest, dealt round-robin
+// to one persistent CTA per SM.  Warp 0 produces the weight stages (bulk copy,
+// L2 prefetch four stages ahead; bf16: with the token rows' TMA loads), warp
+// 1 owns TMEM and issues the MMAs, [MXFP4: warps 2-9 convert, the last warp
+// loads the token rows into a ring of their own], four warps run the epilogue
+// on double-buffered TMEM accumulators.  A decode GEMV moves as many bytes per
+// SM as it keeps in flight, so the weight ring takes every byte of shared
+// memory the rest leaves (MXFP4: 10 / 9 stages of 17 KB for TN = 16).  Every
+// wait is bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing,
+// drains what it issued and frees its TMEM.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -68,47 +71,70 @@ namespace {
 using namespace ::moe::tc;
 
 constexpr int TM = 128;                  // weight rows per tile
-constexpr int TN = 32;                   // pairs per chunk (max MMA N)
-constexpr int B_ATOM = TN * 128;         // one 64-element atom of the token rows: 4 KB
 constexpr int ACC_COLS = 32;             // TMEM columns per accumulator
 constexpr int PF_ITEMS = 4;              // L2 prefetch distance (stages)
+constexpr int kSmemBudget = 226 * 1024;  // opt-in shared memory of one CTA (227 KB) less the static 1 KB
+constexpr int kMaxE = 1024;              // experts the unit table is sized for
+constexpr int kBarBytes = 512;           // mbarriers, the TMEM address and two flags
 
-// Per (format, phase) geometry of a pipeline stage.
-template <int FMT, int PHASE>
+// Per (format, phase, chunk width) geometry.  TN = pairs per chunk (the MMA's
+// N is 16 or 32): 16 whenever T <= 16, since an expert holds at most one pair
+// per token, which halves the token-row buffers and frees room for weight stages.
+//
+// bf16: the MMA reads both operands from shared memory, so a weight stage and
+// its token rows are freed together: one ring of SA stages (B ring indexed alike).
+// MXFP4: the converters are done with a weight stage long before the MMA is
+// done with the token rows, so the weight stages (SA) and the token-row
+// stages (SB) are separate rings with their own producers, and the weight
+// ring takes every byte the token rows do not need.
+template <int FMT, int PHASE, int TN>
 struct Cfg {
   static constexpr bool MX = (FMT == MOE_W_MXFP4);
   static constexpr int KSTAGE = MX ? 256 : 128;                  // K elements per stage
   static constexpr int ATOMS = KSTAGE / 64;                      // B atoms per plane
+  static constexpr int B_ATOM = TN * 128;                        // one 64-element atom of TN token rows
   static constexpr int A_STAGE = MX ? kMxTileBytes : 2 * TM * 128;   // weight bytes per stage
-  static constexpr int B_BYTES = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
-  static constexpr int STAGE = A_STAGE + B_BYTES;                // multiple of 1024
-  static constexpr int STAGES = PHASE == 1 ? (MX ? 6 : 5) : 4;
+  static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
   static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
+  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
+  static constexpr int SB_MX = B_STAGE <= 8192 ? 5 : (B_STAGE >= 32768 ? 3 : 4);
+  static constexpr int SA_FIT = MX ? (kSmemBudget - FIXED - SB_MX * B_STAGE) / A_STAGE
+                                   : (kSmemBudget - FIXED) / (A_STAGE + B_STAGE);
+  static constexpr int SA = SA_FIT > 12 ? 12 : SA_FIT;           // weight stages
+  static constexpr int SB = MX ? SB_MX : SA;                     // token-row stages
+  static constexpr int A_RING = SA * A_STAGE;
+  static constexpr int B_RING = SB * B_STAGE;
   static constexpr int CONV_PER_ROW = 2;                         // converter warps per TMEM lane quadrant
   static constexpr int CONV_WARPS = MX ? 4 * CONV_PER_ROW : 0;
-  static constexpr int THREADS = (2 + CONV_WARPS + 4) * 32;
   static constexpr int EPI_WARP0 = 2 + CONV_WARPS;
+  static constexpr int BPROD_WARP = EPI_WARP0 + 4;               // MXFP4: the token-row producer
+  static constexpr int THREADS = (EPI_WARP0 + 4 + (MX ? 1 : 0)) * 32;
   static constexpr int ASLOTS = 3;                               // TMEM A buffers (MXFP4)
   static constexpr int A_COL0 = 2 * ACC_COLS;                    // first TMEM column of the A buffers
   static constexpr int A_COLS = KSTAGE / 2;                      // TMEM columns per A buffer
   static constexpr int TMEM_COLS = MX ? 512 : 64;
-  static constexpr int N_BARS = 2 * STAGES + 5 + (MX ? 2 * ASLOTS : 0);
-  static_assert(STAGE % 1024 == 0 && A_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
+  static constexpr int N_BARS = 2 * SA + (MX ? 2 * SB + 2 * ASLOTS : 0) + 5;
+  static_assert(TN == 16 || TN == 32, "chunk width");
+  static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(SA >= 3, "weight ring");
+  static_assert(FIXED + A_RING + B_RING <= kSmemBudget, "shared memory budget");
   static_assert(!MX || A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(N_BARS * 8 + 16 <= 256, "barrier area");
+  static_assert(N_BARS * 8 + 16 <= kBarBytes, "barrier area");
 };
 
-template <int FMT, int PHASE>
+template <int FMT, int PHASE, int TN>
 constexpr size_t smem_bytes(int E) {
-  using C = Cfg<FMT, PHASE>;
-  return 1024 + static_cast<size_t>(C::STAGES) * C::STAGE + C::UP_BYTES + 256 + static_cast<size_t>(E + 1) * 4;
+  using C = Cfg<FMT, PHASE, TN>;
+  return 1024 + static_cast<size_t>(C::A_RING) + C::B_RING + C::UP_BYTES + kBarBytes +
+         static_cast<size_t>(E + 1) * 4;
 }
 
 struct Unit {
   int e, m, q0, nvalid;
 };
 
-// unit u -> (expert, tile, chunk); ustart[e] = first unit of expert e
+// unit u -> (expert, tile, chunk of TN pairs); ustart[e] = first unit of expert e
+template <int TN>
 __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int u) {
   int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
   while (hi - lo > 1) {
@@ -131,7 +157,7 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
 // First byte of unit U's weight tile (its K stages follow at A_STAGE).
 template <int FMT, int PHASE>
 __device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, const Unit& U) {
-  using C = Cfg<FMT, PHASE>;
+  using C = Cfg<FMT, PHASE, 32>;   // the weight stages do not depend on TN
   const int K = (PHASE == 1) ? P.d : P.I;
   const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
   return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / C::KSTAGE) * C::A_STAGE;
@@ -146,9 +172,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 // round-robin deal), up to `budget` bytes, so that gemv<2> starts on warm L2.
 // gemv<2>'s units of expert e are proportional to gemv<1>'s: both are
 // tiles x chunks(e), so ustart1 scales to the gemv<2> table.
-template <int FMT>
+template <int FMT, int TN>
 __device__ void prefetch_down_units(const TcDecodeParams& P, const int32_t* ustart1, int per1, size_t budget) {
-  using C = Cfg<FMT, 2>;
+  using C = Cfg<FMT, 2, TN>;
   const int MT2 = P.d / TM, KS2 = P.I / C::KSTAGE, per2 = MT2;
   const int n2 = ustart1[P.E] / per1 * per2;
   for (int u = blockIdx.x; u < n2 && budget > 0; u += gridDim.x) {
@@ -234,27 +260,95 @@ __device__ __forceinline__ void split16(float a, bool mx, uint16_t* hi, uint16_t
   }
 }
 
-template <int FMT, int PHASE>
-__global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
+// gemv<1>: the token of each of the unit's pairs (lane q: pair q0 + q).
+template <int PHASE>
+__device__ __forceinline__ int token_of(const TcDecodeParams& P, const Unit& U, int lane, int n_pairs) {
+  int tok = 0;
+  if (PHASE == 1 && lane < U.nvalid) {
+    const int p = __ldg(P.perm + U.q0 + lane);
+    if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
+    else tok = p / P.k;
+  }
+  return tok;
+}
+
+// gemv<2>: the smallest a-plane box (8, 16 or 32 rows) that holds the unit's
+// pairs.  With TN = 16 a unit has at most min(16, T*k) pairs, box 1.
+template <int TN>
+__device__ __forceinline__ int a_box(const TcDecodeParams& P, int nvalid) {
+  if (nvalid <= P.a_box_rows[0]) return 0;
+  return (TN == 16 || nvalid <= P.a_box_rows[1]) ? 1 : 2;
+}
+
+// Bytes that land in a token-row stage of unit U.
+template <class C, int PHASE, int TN>
+__device__ __forceinline__ uint32_t b_bytes(const TcDecodeParams& P, const Unit& U) {
+  const uint32_t rows =
+      PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
+  return rows * C::ATOMS * 128u;
+}
+
+// Token rows of K stage ks of unit U into sB, completing on bar (whose
+// expected bytes lane 0 has posted): gemv<1> one row TMA of x per pair and
+// atom, lane q loading pair q0 + q; gemv<2> both planes of the a box, rows
+// past the unit's pairs never read back.  Called by all lanes of one warp.
+template <class C, int PHASE, int TN>
+__device__ __forceinline__ void load_b(const TcDecodeParams& P, const Unit& U, int ks, int tok, uint8_t* sB,
+                                       uint64_t* bar, const CUtensorMap* tm_b, const CUtensorMap* tm_b16,
+                                       const CUtensorMap* tm_b8, uint64_t pol, int lane) {
+  if (PHASE == 2) {
+    if (lane == 0) {
+      const int bi = a_box<TN>(P, U.nvalid);
+      const CUtensorMap* tm = bi == 0 ? tm_b8 : (bi == 1 ? tm_b16 : tm_b);
+#pragma unroll
+      for (int pl = 0; pl < 2; ++pl)
+#pragma unroll
+        for (int a = 0; a < C::ATOMS; ++a)
+          tma_load_3d(sB + (pl * C::ATOMS + a) * C::B_ATOM, tm, bar, ks * C::KSTAGE + 64 * a, U.q0, pl, pol);
+    }
+  } else if (lane < U.nvalid) {
+#pragma unroll
+    for (int a = 0; a < C::ATOMS; ++a)
+      tma_load_2d(sB + a * C::B_ATOM + lane * 128, tm_b, bar, ks * C::KSTAGE + 64 * a, tok, pol);
+  }
+}
+
+// Waits for the copies of the last min(issued, n) stages of a ring to land.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, int stage, uint32_t phase) {
+  const int outstanding = issued < n ? issued : n;
+  for (int i = 0; i < outstanding; ++i) {
+    if (--stage < 0) {
+      stage = n - 1;
+      phase ^= 1u;
+    }
+    mbar_drain(&full[stage], phase);
+  }
+}
+
+template <int FMT, int PHASE, int TN>
+__global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b16,
                    const __grid_constant__ CUtensorMap tm_b8, TcDecodeParams P) {
-  using C = Cfg<FMT, PHASE>;
+  using C = Cfg<FMT, PHASE, TN>;
   constexpr int THREADS = C::THREADS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* up_buf = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE + C::UP_BYTES);
-  uint64_t* full = bars;                        // [STAGES]
-  uint64_t* empty = bars + C::STAGES;           // [STAGES]
-  uint64_t* tfull = bars + 2 * C::STAGES;       // [2]
-  uint64_t* tempty = bars + 2 * C::STAGES + 2;  // [2]
-  uint64_t* drain = bars + 2 * C::STAGES + 4;   // [1]
-  uint64_t* cvt_done = bars + 2 * C::STAGES + 5;               // [ASLOTS] (MXFP4)
-  uint64_t* afree = bars + 2 * C::STAGES + 5 + C::ASLOTS;      // [ASLOTS] (MXFP4)
+  uint8_t* ring_b = smem + C::A_RING;           // token-row stages
+  float* up_buf = reinterpret_cast<float*>(ring_b + C::B_RING);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_b + C::B_RING + C::UP_BYTES);
+  uint64_t* full = bars;                        // [SA] weight stage landed (bf16: with its token rows)
+  uint64_t* empty = bars + C::SA;               // [SA] weight stage free
+  uint64_t* tfull = bars + 2 * C::SA;           // [2]
+  uint64_t* tempty = tfull + 2;                 // [2]
+  uint64_t* drain = tfull + 4;                  // [1]
+  uint64_t* cvt_done = tfull + 5;               // [ASLOTS] (MXFP4)
+  uint64_t* afree = cvt_done + C::ASLOTS;       // [ASLOTS] (MXFP4)
+  uint64_t* bfull = afree + C::ASLOTS;          // [SB] token rows landed (MXFP4)
+  uint64_t* bempty = bfull + C::SB;             // [SB] token rows free (MXFP4)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
-  int32_t* ustart = reinterpret_cast<int32_t*>(smem + C::STAGES * C::STAGE + C::UP_BYTES + 256);
+  int32_t* ustart = reinterpret_cast<int32_t*>(ring_b + C::B_RING + C::UP_BYTES + kBarBytes);
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -264,9 +358,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::SA; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], C::MX ? 32 * C::CONV_WARPS : 1);   // MXFP4: every converter thread has read it
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -277,6 +371,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       for (int a = 0; a < C::ASLOTS; ++a) {
         mbar_init(&cvt_done[a], 32 * C::CONV_WARPS);
         mbar_init(&afree[a], 1);
+      }
+      for (int s = 0; s < C::SB; ++s) {
+        mbar_init(&bfull[s], 1);
+        mbar_init(&bempty[s], 1);
       }
     }
     *abort_flag = 0;
@@ -328,7 +426,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   const int n_units = total;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight producer (bf16: and token rows)
     const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
@@ -337,94 +435,95 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     // L2 prefetch cursor over this CTA's (unit, stage) items
     int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of(P, ustart, MT, pf_u));
+    if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of<TN>(P, ustart, MT, pf_u));
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of(P, ustart, MT, u);
+      const Unit U = unit_of<TN>(P, ustart, MT, u);
       const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
-      int tok = 0;
-      if (PHASE == 1 && lane < U.nvalid) {
-        const int p = __ldg(P.perm + U.q0 + lane);
-        if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
-        else tok = p / P.k;
-      }
+      const int tok = C::MX ? 0 : token_of<PHASE>(P, U, lane, n_pairs);
       for (int ks = 0; ks < KS; ++ks) {
-        if (!mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag)) {
+        // one verdict for the warp: its lanes take the same path
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag))) {
           ok = false;
           break;
         }
-        uint8_t* sA = smem + stage * C::STAGE;
-        uint8_t* sB = sA + C::A_STAGE;
+        uint8_t* sA = smem + stage * C::A_STAGE;
         if (lane == 0) {
-          // gemv<2>: the smallest a-plane box (8, 16 or 32 rows) that holds the
-          // unit's pairs; rows beyond them are never read back
-          const int bi = U.nvalid <= P.a_box_rows[0] ? 0 : (U.nvalid <= P.a_box_rows[1] ? 1 : 2);
-          const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * P.a_box_rows[bi];
-          mbar_expect_tx(&full[stage], C::A_STAGE + rows * C::ATOMS * 128u);
+          mbar_expect_tx(&full[stage], C::A_STAGE + (C::MX ? 0u : b_bytes<C, PHASE, TN>(P, U)));
           bulk_load(sA, abase + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE, &full[stage], pol_stream);
-          if (PHASE == 2) {
-            const CUtensorMap* tm = bi == 0 ? &tm_b8 : (bi == 1 ? &tm_b16 : &tm_b);
-#pragma unroll
-            for (int pl = 0; pl < 2; ++pl)
-#pragma unroll
-              for (int a = 0; a < C::ATOMS; ++a)
-                tma_load_3d(sB + (pl * C::ATOMS + a) * B_ATOM, tm, &full[stage], ks * C::KSTAGE + 64 * a, U.q0,
-                            pl, pol_keep);
-          }
           // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one (the
           // bulk copies of a CTA complete in order, so prefetching whole blobs
           // up front would queue ahead of the stages the pipeline waits for)
-          {
-            while (pf_u < n_units && pf_ahead < PF_ITEMS) {
-              prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
-              ++pf_ahead;
-              if (++pf_ks == KS) {
-                pf_ks = 0;
-                pf_u += gridDim.x;
-                if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of(P, ustart, MT, pf_u));
-              }
+          while (pf_u < n_units && pf_ahead < PF_ITEMS) {
+            prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
+            ++pf_ahead;
+            if (++pf_ks == KS) {
+              pf_ks = 0;
+              pf_u += gridDim.x;
+              if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of<TN>(P, ustart, MT, pf_u));
             }
-            --pf_ahead;
           }
+          --pf_ahead;
         }
         __syncwarp();
-        if (PHASE == 1 && lane < U.nvalid) {
-#pragma unroll
-          for (int a = 0; a < C::ATOMS; ++a)
-            tma_load_2d(sB + a * B_ATOM + lane * 128, &tm_b, &full[stage], ks * C::KSTAGE + 64 * a, tok, pol_keep);
-        }
+        if constexpr (!C::MX)
+          load_b<C, PHASE, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &full[stage], &tm_b, &tm_b16, &tm_b8,
+                               pol_keep, lane);
         __syncwarp();
         ++issued;
-        if (++stage == C::STAGES) {
+        if (++stage == C::SA) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<FMT>(P, ustart, MT, 256u << 10);
+    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<FMT, TN>(P, ustart, MT, 256u << 10);
     __syncwarp();
     if (!ok) {
       report(P.status, MOE_ERR_TIMEOUT);
       *abort_flag = 1;
     }
     // drain: the copies last issued into the ring have landed before exit
-    const int outstanding = issued < C::STAGES ? issued : C::STAGES;
-    int s = stage;
-    uint32_t ph = phase;
-    for (int i = 0; i < outstanding; ++i) {
-      if (--s < 0) {
-        s = C::STAGES - 1;
-        ph ^= 1u;
+    drain_ring(full, C::SA, issued, stage, phase);
+  } else if (C::MX && warp == C::BPROD_WARP) {
+    // ------------------------------------------------------------ token-row producer (MXFP4)
+    const uint64_t pol_keep = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit U = unit_of<TN>(P, ustart, MT, u);
+      const int tok = token_of<PHASE>(P, U, lane, n_pairs);
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag))) {
+          ok = false;
+          break;
+        }
+        uint8_t* sB = ring_b + stage * C::B_STAGE;
+        if (lane == 0) mbar_expect_tx(&bfull[stage], b_bytes<C, PHASE, TN>(P, U));
+        __syncwarp();
+        load_b<C, PHASE, TN>(P, U, ks, tok, sB, &bfull[stage], &tm_b, &tm_b16, &tm_b8, pol_keep, lane);
+        __syncwarp();
+        ++issued;
+        if (++stage == C::SB) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      mbar_drain(&full[s], ph);
     }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    drain_ring(bfull, C::SB, issued, stage, phase);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
+    int stage = 0;                 // bf16: the shared ring; MXFP4: the token-row ring
     uint32_t phase = 0;
     int it = 0, j = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, u);
+      const Unit U = unit_of<TN>(P, ustart, MT, u);
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const uint32_t idesc = C::MX ? idesc_f16(TM, n_mma) : idesc_bf16(TM, n_mma);
       const int acc = it & 1;
@@ -436,23 +535,24 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
       for (int ks = 0; ks < KS; ++ks, ++j) {
         const int aslot = j % C::ASLOTS;
-        // the stage has landed; MXFP4: and its A buffer (and, phase 1, the
-        // token rows) is converted
-        const bool got = mbar_wait<true>(&full[stage], phase, abort_flag) &&
-                         (!C::MX || mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag));
+        // bf16: the stage has landed.  MXFP4: the token rows have landed and
+        // the A buffer (and, phase 1, the token rows) is converted
+        const bool got = C::MX ? (mbar_wait<true>(&bfull[stage], phase, abort_flag) &&
+                                  mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag))
+                               : mbar_wait<true>(&full[stage], phase, abort_flag);
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (elect_one()) {
-          uint8_t* sA = smem + stage * C::STAGE;
-          uint8_t* sB = sA + C::A_STAGE;
+          const uint8_t* sA = smem + stage * C::A_STAGE;   // bf16
+          const uint8_t* sB = ring_b + stage * C::B_STAGE;
 #pragma unroll
           for (int kk = 0; kk < C::KSTAGE / 16; ++kk) {   // K = 16 per MMA: +32 bytes
             const int a = kk >> 2;
-            const uint64_t dh = desc_sw128(smem_u32(sB + a * B_ATOM)) + 2 * (kk & 3);
-            const uint64_t dl = desc_sw128(smem_u32(sB + (C::ATOMS + a) * B_ATOM)) + 2 * (kk & 3);
+            const uint64_t dh = desc_sw128(smem_u32(sB + a * C::B_ATOM)) + 2 * (kk & 3);
+            const uint64_t dl = desc_sw128(smem_u32(sB + (C::ATOMS + a) * C::B_ATOM)) + 2 * (kk & 3);
             const uint32_t first = (ks > 0 || kk > 0) ? 1u : 0u;
             if (C::MX) {
               const uint32_t ta = tmem + C::A_COL0 + aslot * C::A_COLS + 8 * kk;
@@ -464,11 +564,15 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
               if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
             }
           }
-          if (C::MX) tc_commit(&afree[aslot]);
-          tc_commit(&empty[stage]);
+          if (C::MX) {
+            tc_commit(&afree[aslot]);
+            tc_commit(&bempty[stage]);
+          } else {
+            tc_commit(&empty[stage]);
+          }
         }
         __syncwarp();
-        if (++stage == C::STAGES) {
+        if (++stage == C::SB) {
           stage = 0;
           phase ^= 1u;
         }
@@ -495,18 +599,19 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     const int ct = threadIdx.x - 64;                // 0..255
     bool ok = true;
     bool range_ok = true;
-    int j = 0;
+    int j = 0, sa = 0, sb = 0;
+    uint32_t pa = 0, pb = 0;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of(P, ustart, MT, u);
+      const Unit U = unit_of<TN>(P, ustart, MT, u);
       for (int ks = 0; ks < KS; ++ks, ++j) {
-        const int s = j % C::STAGES, aslot = j % C::ASLOTS;
-        if (!mbar_wait<true>(&full[s], (j / C::STAGES) & 1, abort_flag) ||
+        const int aslot = j % C::ASLOTS;
+        if (!mbar_wait<true>(&full[sa], pa, abort_flag) ||
             !mbar_wait<true>(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint8_t* sA = smem + s * C::STAGE;
+        const uint8_t* sA = smem + sa * C::A_STAGE;
         const uint2 sc2 = *reinterpret_cast<const uint2*>(sA + 16384 + r * 8);
         const uint32_t taddr =
             tmem + (static_cast<uint32_t>(32 * quad) << 16) + C::A_COL0 + aslot * C::A_COLS + 16 * CH * part;
@@ -538,22 +643,37 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
               v[16 * cc + 4 * i + 3] = hmul2(h3, scl);
             }
           }
+          // every value read from the stage is in registers: hand it back to the producer
+          mbar_arrive(&empty[sa]);
           if constexpr (CH == 4) tmem_st64(taddr, v);
           else tmem_st32(taddr, v);
         }
         if (PHASE == 1) {
           // token rows bf16 -> f16 in place (the swizzle only moves whole chunks)
-          uint8_t* sB = sA + C::A_STAGE;
+          if (!mbar_wait<true>(&bfull[sb], pb, abort_flag)) {
+            tmem_wait_st();
+            ok = false;
+            break;
+          }
+          uint8_t* sB = ring_b + sb * C::B_STAGE;
           const int n_chunks = U.nvalid * C::ATOMS * 8;
           for (int idx = ct; idx < n_chunks; idx += 32 * C::CONV_WARPS) {
             const int rr = idx / (C::ATOMS * 8), rem = idx % (C::ATOMS * 8);
-            range_ok &= bf16x8_to_f16x8(reinterpret_cast<uint4*>(sB + (rem >> 3) * B_ATOM + rr * 128 + (rem & 7) * 16));
+            range_ok &= bf16x8_to_f16x8(reinterpret_cast<uint4*>(sB + (rem >> 3) * C::B_ATOM + rr * 128 + (rem & 7) * 16));
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&cvt_done[aslot]);
+        if (++sa == C::SA) {
+          sa = 0;
+          pa ^= 1u;
+        }
+        if (++sb == C::SB) {
+          sb = 0;
+          pb ^= 1u;
+        }
       }
     }
     if (!range_ok) report(P.status, MOE_ERR_UNSUPPORTED);
@@ -568,7 +688,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
     bool range_ok = true;
     int it = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
-      const Unit U = unit_of(P, ustart, MT, u);
+      const Unit U = unit_of<TN>(P, ustart, MT, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
@@ -636,28 +756,28 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE>::THREADS, 1)
   }
 }
 
-template <int FMT, int PHASE>
+template <int FMT, int PHASE, int TN>
 moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const CUtensorMap& tm16,
                         const CUtensorMap& tm8, const DeviceInfo& dev, cudaStream_t s) {
-  const size_t smem = smem_bytes<FMT, PHASE>(P.E);
+  const size_t smem = smem_bytes<FMT, PHASE, TN>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
   if (attr[dev.id] < smem) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(gemv_tc_kernel<FMT, PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MOE_CUDA_TRY(cudaFuncSetAttribute(gemv_tc_kernel<FMT, PHASE, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(smem)));
     attr[dev.id] = smem;
   }
-  gemv_tc_kernel<FMT, PHASE><<<dev.sm_count, Cfg<FMT, PHASE>::THREADS, smem, s>>>(tm, tm16, tm8, P);
+  gemv_tc_kernel<FMT, PHASE, TN><<<dev.sm_count, Cfg<FMT, PHASE, TN>::THREADS, smem, s>>>(tm, tm16, tm8, P);
   MOE_LAUNCH_CHECK("gemv_tc_kernel");
   return MOE_OK;
 }
 
-template <int FMT>
+template <int FMT, int TN>
 moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap (&tm_a)[3],
                        const DeviceInfo& dev, cudaStream_t stream) {
-  moe_status st = launch_phase<FMT, 1>(P, tm_x, tm_x, tm_x, dev, stream);
+  moe_status st = launch_phase<FMT, 1, TN>(P, tm_x, tm_x, tm_x, dev, stream);
   if (st != MOE_OK) return st;
-  return launch_phase<FMT, 2>(P, tm_a[2], tm_a[1], tm_a[0], dev, stream);
+  return launch_phase<FMT, 2, TN>(P, tm_a[2], tm_a[1], tm_a[0], dev, stream);
 }
 
 }  // namespace
@@ -687,7 +807,7 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
   P.status = status;
   const uint64_t n = static_cast<uint64_t>(T) * k;
   for (int i = 0; i < 3; ++i) {
-    const uint64_t r = static_cast<uint64_t>(8) << i;   // 8, 16, 32 = TN
+    const uint64_t r = static_cast<uint64_t>(8) << i;   // 8, 16, 32 (the widest chunk)
     P.a_box_rows[i] = static_cast<int>(n < r ? n : r);
   }
   CUtensorMap tm_x, tm_a[3];
@@ -707,8 +827,12 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
     const CUresult r = encode_tiled_sw128(&tm_a[i], type, 3, ws, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a planes failed (%d)", static_cast<int>(r));
   }
-  if (s.fmt == MOE_W_MXFP4) return launch_both<MOE_W_MXFP4>(P, tm_x, tm_a, dev, stream);
-  return launch_both<MOE_W_BF16>(P, tm_x, tm_a, dev, stream);
+  // an expert holds at most one pair per token: with T <= 16 every chunk fits 16 rows
+  if (s.fmt == MOE_W_MXFP4)
+    return T <= 16 ? launch_both<MOE_W_MXFP4, 16>(P, tm_x, tm_a, dev, stream)
+                   : launch_both<MOE_W_MXFP4, 32>(P, tm_x, tm_a, dev, stream);
+  return T <= 16 ? launch_both<MOE_W_BF16, 16>(P, tm_x, tm_a, dev, stream)
+                 : launch_both<MOE_W_BF16, 32>(P, tm_x, tm_a, dev, stream);
 }
 
 }  // namespace moe

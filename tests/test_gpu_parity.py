@@ -157,6 +157,18 @@ def test_many_tokens_per_expert(moe, fmt):
     assert (np.diff(b.layer.offsets.cpu().numpy()) > 32).any()
 
 
+@pytest.mark.parametrize("fmt", ["bf16", "mxfp4"])
+@pytest.mark.parametrize("T", [16, 17])
+def test_chunk_width_boundary(moe, fmt, T):
+    """T = 16 runs 16-pair chunks, T = 17 32-pair chunks; E = 4, k = 4 puts
+    every token on every expert, so the groups fill the chunk exactly (16) or
+    spill one pair past it (17)."""
+    cfg = synth.LayerConfig("full", E=4, k=4, d=512, I=256, fmt=fmt)
+    b = Built(cfg, T, seed=7)
+    check_tol(b.run().cpu().numpy(), b.oracle()["out"], 1e-4, 1e-5)
+    assert (np.diff(b.layer.offsets.cpu().numpy()) == T).all()
+
+
 def test_y_perm_rows_match_pairs(moe):
     cfg = synth.CONFIGS["decode_bf16"]
     b = Built(cfg, 16, seed=4)
@@ -324,6 +336,26 @@ def test_mxfp4_edge_of_f16_range_is_exact(moe):
         out = b.run().cpu().numpy()
         moe.moe_check_status(b.layer.status)
         check_tol(out, b.oracle()["out"], 1e-4, 1e-5)
+
+
+def test_mxfp4_mixed_block_scales_are_exact(moe):
+    """Every block of every routed expert gets its own E8M0 scale, gate rows in
+    2^[-23, 2] and the down projection across the whole exact range 2^[-23, 13],
+    so each warp's converters meet scales from both ends of f16 at once; the
+    output still matches the oracle."""
+    cfg = synth.LayerConfig("mx_mixed", E=8, k=2, d=512, I=256, fmt="mxfp4")
+    logits, x = synth.make_routing(cfg, 4, 4)
+    b = Built(cfg, 4, seed=4, logits=logits, x=x)
+    from expert_offload_serving_b200.layer import pack_pool
+    g = torch.Generator().manual_seed(9)
+    for key, hi in (("sg", 127 + 2), ("sd", 127 + 13)):
+        for t in b.w_cpu[key]:
+            t.copy_(torch.randint(127 - 23, hi + 1, t.shape, generator=g, dtype=torch.int64).to(t.dtype))
+    b._deq.clear()
+    b.layer.pool.copy_(pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, b.w_cpu, b.order, pin=False))
+    out = b.run().cpu().numpy()
+    moe.moe_check_status(b.layer.status)
+    check_tol(out, b.oracle()["out"], 1e-4, 1e-5)
 
 
 def test_mxfp4_zero_block_with_smallest_scale_is_exact(moe):
