@@ -34,12 +34,12 @@
 // Work unit = (expert, 128-row tile, chunk of <= TN of the expert's pairs; TN
 // = 16 when T <= 16, else 32), expert-major, chunks fastest, dealt round-robin
 // to one persistent CTA per SM.  Warp 0 produces the weight stages (bulk copy,
-// L2 prefetch four stages ahead; bf16: with the token rows' TMA loads), warp
-// 1 owns TMEM and issues the MMAs, [MXFP4: warps 2-9 convert, the last warp
-// loads the token rows into a ring of their own], four warps run the epilogue
-// on double-buffered TMEM accumulators.  A decode GEMV moves as many bytes per
-// SM as it keeps in flight, so the weight ring takes every byte of shared
-// memory the rest leaves (MXFP4: 10 / 9 stages of 17 KB for TN = 16).  Every
+// L2 prefetch four stages ahead), warp 1 owns TMEM and issues the MMAs,
+// [MXFP4: warps 2-9 convert], four warps run the epilogue on double-buffered
+// TMEM accumulators, and the last warp loads the token rows into a ring of
+// their own.  A decode GEMV moves as many bytes per SM as it keeps in flight,
+// so the weight ring takes every byte of shared memory the rest leaves (bf16:
+// 5-6 stages of 32 KB; MXFP4: 10 / 9 stages of 17 KB for TN = 16).  Every
 // wait is bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing,
 // drains what it issued and frees its TMEM.
 #include <cuda_bf16.h>
@@ -81,12 +81,11 @@ constexpr int kBarBytes = 512;           // mbarriers, the TMEM address and two 
 // N is 16 or 32): 16 whenever T <= 16, since an expert holds at most one pair
 // per token, which halves the token-row buffers and frees room for weight stages.
 //
-// bf16: the MMA reads both operands from shared memory, so a weight stage and
-// its token rows are freed together: one ring of SA stages (B ring indexed alike).
-// MXFP4: the converters are done with a weight stage long before the MMA is
-// done with the token rows, so the weight stages (SA) and the token-row
-// stages (SB) are separate rings with their own producers, and the weight
-// ring takes every byte the token rows do not need.
+// Weight stages (SA) and token-row stages (SB) are separate rings, each with
+// its own producer warp, and the weight ring takes every byte the token rows
+// leave: the token rows come from L2 (x, or the a planes just written), so a
+// few stages cover them.  MXFP4: the converters free a weight stage as soon
+// as they have read it; bf16: the MMA frees both.
 template <int FMT, int PHASE, int TN>
 struct Cfg {
   static constexpr bool MX = (FMT == MOE_W_MXFP4);
@@ -97,23 +96,22 @@ struct Cfg {
   static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
   static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
-  static constexpr int SB_MX = B_STAGE <= 8192 ? 5 : (B_STAGE >= 32768 ? 3 : 4);
-  static constexpr int SA_FIT = MX ? (kSmemBudget - FIXED - SB_MX * B_STAGE) / A_STAGE
-                                   : (kSmemBudget - FIXED) / (A_STAGE + B_STAGE);
+  static constexpr int SB = MX ? (B_STAGE <= 8192 ? 5 : (B_STAGE >= 32768 ? 3 : 4))            // token-row stages
+                               : (B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3);
+  static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_STAGE;
   static constexpr int SA = SA_FIT > 12 ? 12 : SA_FIT;           // weight stages
-  static constexpr int SB = MX ? SB_MX : SA;                     // token-row stages
   static constexpr int A_RING = SA * A_STAGE;
   static constexpr int B_RING = SB * B_STAGE;
   static constexpr int CONV_PER_ROW = 2;                         // converter warps per TMEM lane quadrant
   static constexpr int CONV_WARPS = MX ? 4 * CONV_PER_ROW : 0;
   static constexpr int EPI_WARP0 = 2 + CONV_WARPS;
-  static constexpr int BPROD_WARP = EPI_WARP0 + 4;               // MXFP4: the token-row producer
-  static constexpr int THREADS = (EPI_WARP0 + 4 + (MX ? 1 : 0)) * 32;
+  static constexpr int BPROD_WARP = EPI_WARP0 + 4;               // the token-row producer
+  static constexpr int THREADS = (EPI_WARP0 + 5) * 32;
   static constexpr int ASLOTS = 3;                               // TMEM A buffers (MXFP4)
   static constexpr int A_COL0 = 2 * ACC_COLS;                    // first TMEM column of the A buffers
   static constexpr int A_COLS = KSTAGE / 2;                      // TMEM columns per A buffer
   static constexpr int TMEM_COLS = MX ? 512 : 64;
-  static constexpr int N_BARS = 2 * SA + (MX ? 2 * SB + 2 * ASLOTS : 0) + 5;
+  static constexpr int N_BARS = 2 * SA + 2 * SB + 2 * ASLOTS + 5;
   static_assert(TN == 16 || TN == 32, "chunk width");
   static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
@@ -336,15 +334,15 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   uint8_t* ring_b = smem + C::A_RING;           // token-row stages
   float* up_buf = reinterpret_cast<float*>(ring_b + C::B_RING);
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring_b + C::B_RING + C::UP_BYTES);
-  uint64_t* full = bars;                        // [SA] weight stage landed (bf16: with its token rows)
+  uint64_t* full = bars;                        // [SA] weight stage landed
   uint64_t* empty = bars + C::SA;               // [SA] weight stage free
   uint64_t* tfull = bars + 2 * C::SA;           // [2]
   uint64_t* tempty = tfull + 2;                 // [2]
   uint64_t* drain = tfull + 4;                  // [1]
   uint64_t* cvt_done = tfull + 5;               // [ASLOTS] (MXFP4)
   uint64_t* afree = cvt_done + C::ASLOTS;       // [ASLOTS] (MXFP4)
-  uint64_t* bfull = afree + C::ASLOTS;          // [SB] token rows landed (MXFP4)
-  uint64_t* bempty = bfull + C::SB;             // [SB] token rows free (MXFP4)
+  uint64_t* bfull = afree + C::ASLOTS;          // [SB] token rows landed
+  uint64_t* bempty = bfull + C::SB;             // [SB] token rows free
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
@@ -372,10 +370,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
         mbar_init(&cvt_done[a], 32 * C::CONV_WARPS);
         mbar_init(&afree[a], 1);
       }
-      for (int s = 0; s < C::SB; ++s) {
-        mbar_init(&bfull[s], 1);
-        mbar_init(&bempty[s], 1);
-      }
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
     *abort_flag = 0;
     *epi_fail = 0;
@@ -426,8 +424,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   const int n_units = total;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ weight producer (bf16: and token rows)
-    const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
+    // ------------------------------------------------------------ weight producer
+    const uint64_t pol_stream = policy_evict_first();
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
@@ -439,7 +437,6 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<TN>(P, ustart, MT, u);
       const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
-      const int tok = C::MX ? 0 : token_of<PHASE>(P, U, lane, n_pairs);
       for (int ks = 0; ks < KS; ++ks) {
         // one verdict for the warp: its lanes take the same path
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag))) {
@@ -448,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
         }
         uint8_t* sA = smem + stage * C::A_STAGE;
         if (lane == 0) {
-          mbar_expect_tx(&full[stage], C::A_STAGE + (C::MX ? 0u : b_bytes<C, PHASE, TN>(P, U)));
+          mbar_expect_tx(&full[stage], C::A_STAGE);
           bulk_load(sA, abase + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE, &full[stage], pol_stream);
           // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one (the
           // bulk copies of a CTA complete in order, so prefetching whole blobs
@@ -465,10 +462,6 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
           --pf_ahead;
         }
         __syncwarp();
-        if constexpr (!C::MX)
-          load_b<C, PHASE, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &full[stage], &tm_b, &tm_b16, &tm_b8,
-                               pol_keep, lane);
-        __syncwarp();
         ++issued;
         if (++stage == C::SA) {
           stage = 0;
@@ -484,8 +477,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     }
     // drain: the copies last issued into the ring have landed before exit
     drain_ring(full, C::SA, issued, stage, phase);
-  } else if (C::MX && warp == C::BPROD_WARP) {
-    // ------------------------------------------------------------ token-row producer (MXFP4)
+  } else if (warp == C::BPROD_WARP) {
+    // ------------------------------------------------------------ token-row producer
     const uint64_t pol_keep = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
@@ -518,8 +511,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     drain_ring(bfull, C::SB, issued, stage, phase);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;                 // bf16: the shared ring; MXFP4: the token-row ring
-    uint32_t phase = 0;
+    int stage = 0, sa = 0;         // token-row ring; weight ring (bf16)
+    uint32_t phase = 0, pa = 0;
     int it = 0, j = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
@@ -535,18 +528,18 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
       for (int ks = 0; ks < KS; ++ks, ++j) {
         const int aslot = j % C::ASLOTS;
-        // bf16: the stage has landed.  MXFP4: the token rows have landed and
-        // the A buffer (and, phase 1, the token rows) is converted
-        const bool got = C::MX ? (mbar_wait<true>(&bfull[stage], phase, abort_flag) &&
-                                  mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag))
-                               : mbar_wait<true>(&full[stage], phase, abort_flag);
+        // the token rows have landed, and bf16: the weight stage; MXFP4: the
+        // A buffer is converted (phase 1: the token rows too)
+        const bool got = mbar_wait<true>(&bfull[stage], phase, abort_flag) &&
+                         (C::MX ? mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag)
+                                : mbar_wait<true>(&full[sa], pa, abort_flag));
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (elect_one()) {
-          const uint8_t* sA = smem + stage * C::A_STAGE;   // bf16
+          const uint8_t* sA = smem + sa * C::A_STAGE;      // bf16
           const uint8_t* sB = ring_b + stage * C::B_STAGE;
 #pragma unroll
           for (int kk = 0; kk < C::KSTAGE / 16; ++kk) {   // K = 16 per MMA: +32 bytes
@@ -564,17 +557,17 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
               if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
             }
           }
-          if (C::MX) {
-            tc_commit(&afree[aslot]);
-            tc_commit(&bempty[stage]);
-          } else {
-            tc_commit(&empty[stage]);
-          }
+          tc_commit(C::MX ? &afree[aslot] : &empty[sa]);
+          tc_commit(&bempty[stage]);
         }
         __syncwarp();
         if (++stage == C::SB) {
           stage = 0;
           phase ^= 1u;
+        }
+        if (++sa == C::SA) {
+          sa = 0;
+          pa ^= 1u;
         }
       }
       if (!ok) break;
