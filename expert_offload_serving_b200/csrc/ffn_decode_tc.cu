@@ -99,7 +99,7 @@ struct Cfg {
   static constexpr int SB = MX ? (B_STAGE <= 8192 ? 5 : (B_STAGE >= 32768 ? 3 : 4))            // token-row stages
                                : (B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3);
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_STAGE;
-  static constexpr int SA = SA_FIT > 12 ? 12 : SA_FIT;           // weight stages
+  static constexpr int SA = (!MX && TN == 16 && PHASE == 1) ? 5 : (SA_FIT > 12 ? 12 : SA_FIT);           // weight stages
   static constexpr int A_RING = SA * A_STAGE;
   static constexpr int B_RING = SB * B_STAGE;
   static constexpr int CONV_PER_ROW = 2;                         // converter warps per TMEM lane quadrant
