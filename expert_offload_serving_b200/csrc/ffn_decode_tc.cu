@@ -37,9 +37,10 @@
 // L2 prefetch four stages ahead), warp 1 owns TMEM and issues the MMAs,
 // [MXFP4: warps 2-9 convert], four warps run the epilogue on double-buffered
 // TMEM accumulators, and the last warp loads the token rows into a ring of
-// their own.  A decode GEMV moves as many bytes per SM as it keeps in flight,
-// so the weight ring takes every byte of shared memory the rest leaves (bf16:
-// 5-6 stages of 32 KB; MXFP4: 10 / 9 stages of 17 KB for TN = 16).  Every
+// their own.  The weight ring takes the shared memory the rest leaves (bf16:
+// 5 stages of 32 KB; MXFP4: 10 / 9 stages of 17 KB for TN = 16), so that
+// the bf16 GEMVs keep enough bytes in flight to run near the HBM rate; the
+// MXFP4 ones are bound by the conversion unit that executes cvt.  Every
 // wait is bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing,
 // drains what it issued and frees its TMEM.
 #include <cuda_bf16.h>
