@@ -69,7 +69,8 @@ enum {
   /* Quantise x and the SwiGLU output to NVFP4 (unit tensor scale, one E4M3
    * scale per 16 elements, round-to-nearest-even) before the two products and
    * run them on the FP4 tensor cores.  Requires MOE_W_NVFP4.  Without this
-   * flag activations stay in bf16/fp32 and the CUDA-core path runs. */
+   * flag NVFP4 weights run on the CUDA-core path with the activations kept in
+   * bf16/fp32 (BF16 and MXFP4 weights never quantise the activations). */
   MOE_FFN_ACT_NVFP4 = 1
 };
 
