@@ -75,11 +75,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 using namespace moe;
 
-extern "C" moe_status moe_combine_merge(const float* y_perm, const int32_t* idx, const float* gate,
-                                        const int32_t* inv_perm, const int32_t* slot_of_expert,
-                                        const float* host_partial, int T, int k, int d, int E,
-                                        float* out, cudaStream_t stream) {
-  clear_error();
+moe_status moe::check_combine_args(const float* y_perm, const int32_t* idx, const float* gate,
+                                   const int32_t* inv_perm, const float* host_partial, int T, int k, int d, int E,
+                                   const float* out) {
   MOE_REQUIRE(T >= 0 && k >= 1 && k <= 32 && d >= 4 && d % 4 == 0, "T=%d, k=%d, d=%d", T, k, d);
   MOE_REQUIRE(E >= 1 && E <= 1024, "E=%d outside [1, 1024]", E);
   MOE_REQUIRE(static_cast<long long>(T) * k <= (1 << 24), "T*k too large");
@@ -88,8 +86,18 @@ extern "C" moe_status moe_combine_merge(const float* y_perm, const int32_t* idx,
   MOE_REQUIRE(aligned(y_perm, 16) && aligned(out, 16) && (!host_partial || aligned(host_partial, 16)),
               "y_perm, out and host_partial must be 16-byte aligned");
   MOE_REQUIRE(T <= 65535, "T=%d above the grid limit 65535", T);
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_combine_merge(const float* y_perm, const int32_t* idx, const float* gate,
+                                        const int32_t* inv_perm, const int32_t* slot_of_expert,
+                                        const float* host_partial, int T, int k, int d, int E,
+                                        float* out, cudaStream_t stream) {
+  clear_error();
+  moe_status st = check_combine_args(y_perm, idx, gate, inv_perm, host_partial, T, k, d, E, out);
+  if (st != MOE_OK || T == 0) return st;
   DeviceInfo dev;
-  moe_status st = current_device(&dev);
+  st = current_device(&dev);
   if (st != MOE_OK) return st;
   const int threads = 256;
   dim3 grid((d / 4 + threads - 1) / threads, T);

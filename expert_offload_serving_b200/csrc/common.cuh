@@ -35,6 +35,20 @@ void clear_error();
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Argument checks of the four steps.  They touch no device: each entry point
+// runs its own before the first CUDA call, and moe_layer_forward runs all four
+// before it enqueues anything.
+moe_status check_route_args(const float* logits, int T, int E, int k, const int32_t* idx, const float* gate);
+moe_status check_permute_args(const int32_t* idx, int T, int k, int E, const int32_t* offsets,
+                              const int32_t* perm, const int32_t* inv_perm, const void* scratch,
+                              size_t scratch_bytes);
+moe_status check_ffn_args(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
+                          const int32_t* slot_of_expert, const void* slot_pool, int n_slots, const float* gate,
+                          const float* y_perm, const float* out, int flags, const void* workspace,
+                          size_t ws_bytes);
+moe_status check_combine_args(const float* y_perm, const int32_t* idx, const float* gate, const int32_t* inv_perm,
+                              const float* host_partial, int T, int k, int d, int E, const float* out);
+
 // Device attributes of the current device (cached per device id).
 struct DeviceInfo { int id, sm_count, cc_major, cc_minor; size_t smem_optin; };
 moe_status current_device(DeviceInfo* out);

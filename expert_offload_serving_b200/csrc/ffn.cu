@@ -24,12 +24,10 @@ extern "C" size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int 
   return decode_workspace_bytes(s, T, k);
 }
 
-extern "C" moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
-                                     const int32_t* perm, const int32_t* slot_of_expert,
-                                     const void* slot_pool, int n_slots, const float* gate,
-                                     float* y_perm, float* out, int flags, void* workspace,
-                                     size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
-  clear_error();
+moe_status moe::check_ffn_args(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
+                               const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
+                               int n_slots, const float* gate, const float* y_perm, const float* out, int flags,
+                               const void* workspace, size_t ws_bytes) {
   moe_status st = check_shape(s);
   if (st != MOE_OK) return st;
   MOE_REQUIRE(T >= 0 && k >= 1 && k <= 32 && k <= s.E, "T=%d, k=%d, E=%d", T, k, s.E);
@@ -56,6 +54,18 @@ extern "C" moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k, c
   if (need > 0 && (workspace == nullptr || ws_bytes < need))
     return fail(MOE_ERR_CAPACITY, "workspace needs %zu bytes, got %zu", need, ws_bytes);
   MOE_REQUIRE(workspace == nullptr || aligned(workspace, 256), "workspace must be 256-byte aligned");
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
+                                     const int32_t* perm, const int32_t* slot_of_expert,
+                                     const void* slot_pool, int n_slots, const float* gate,
+                                     float* y_perm, float* out, int flags, void* workspace,
+                                     size_t ws_bytes, int32_t* dev_status, cudaStream_t stream) {
+  clear_error();
+  moe_status st = check_ffn_args(s, x, T, k, offsets, perm, slot_of_expert, slot_pool, n_slots, gate, y_perm,
+                                 out, flags, workspace, ws_bytes);
+  if (st != MOE_OK || T == 0) return st;
   // every argument check is done: only now touch the device
   DeviceInfo dev;
   st = current_device(&dev);

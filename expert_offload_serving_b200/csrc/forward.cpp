@@ -1,7 +1,9 @@
 // moe_layer_forward: the layer's four steps from one host call (route ->
 // permute -> expert FFN -> combine, or the FFN's fused combine), enqueued on
-// one stream.  Each step is the public entry point itself, so arguments,
-// checks and results are exactly those of the individual calls.
+// one stream.  Every step's arguments are checked before the first one is
+// enqueued, so a rejected call leaves the stream untouched; each step is then
+// the public entry point itself, so checks and results are exactly those of
+// the individual calls.
 #include "common.cuh"
 
 extern "C" moe_status moe_layer_forward(moe_shape s, const float* logits, const void* x, int T, int k,
@@ -11,13 +13,23 @@ extern "C" moe_status moe_layer_forward(moe_shape s, const float* logits, const 
                                         float* y_perm, int flags, void* workspace, size_t ws_bytes,
                                         const float* host_partial, float* out, int32_t* dev_status,
                                         cudaStream_t stream) {
-  moe_status st = moe_route_topk(logits, T, s.E, k, idx, gate, stream);
+  ::moe::clear_error();
+  const bool fused = (flags & MOE_FFN_ACT_NVFP4) != 0;
+  moe_status st = ::moe::check_route_args(logits, T, s.E, k, idx, gate);
+  if (st == MOE_OK) st = ::moe::check_permute_args(idx, T, k, s.E, offsets, perm, inv_perm, scratch, scratch_bytes);
+  if (st == MOE_OK)
+    st = ::moe::check_ffn_args(s, x, T, k, offsets, perm, slot_of_expert, slot_pool, n_slots, gate,
+                        fused ? nullptr : y_perm, fused ? out : nullptr, flags, workspace, ws_bytes);
+  if (st == MOE_OK && !fused)
+    st = ::moe::check_combine_args(y_perm, idx, gate, inv_perm, host_partial, T, k, s.d, s.E, out);
+  if (st != MOE_OK) return st;
+  if (fused) MOE_REQUIRE(out != nullptr, "out is required");
+  st = moe_route_topk(logits, T, s.E, k, idx, gate, stream);
   if (st != MOE_OK) return st;
   st = moe_permute(idx, T, k, s.E, offsets, perm, inv_perm, scratch, scratch_bytes, dev_status, stream);
   if (st != MOE_OK) return st;
-  if (flags & MOE_FFN_ACT_NVFP4) {
+  if (fused) {
     ::moe::clear_error();
-    MOE_REQUIRE(out != nullptr, "out is required");
     if (T > 0) {
       const size_t bytes = static_cast<size_t>(T) * s.d * sizeof(float);
       if (host_partial != nullptr) {

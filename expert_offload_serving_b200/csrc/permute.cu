@@ -222,25 +222,38 @@ extern "C" size_t moe_permute_scratch_bytes(int T, int k, int E) {
   return static_cast<size_t>(ntiles) * E * sizeof(int32_t);
 }
 
-extern "C" moe_status moe_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets,
-                                  int32_t* perm, int32_t* inv_perm, void* scratch,
-                                  size_t scratch_bytes, int32_t* dev_status, cudaStream_t stream) {
-  clear_error();
+moe_status moe::check_permute_args(const int32_t* idx, int T, int k, int E, const int32_t* offsets,
+                                   const int32_t* perm, const int32_t* inv_perm, const void* scratch,
+                                   size_t scratch_bytes) {
   MOE_REQUIRE(T >= 0 && k >= 1 && k <= 32, "T=%d, k=%d", T, k);
   MOE_REQUIRE(E >= 1 && E <= 1024, "E=%d outside [1, 1024]", E);
   MOE_REQUIRE(static_cast<long long>(T) * k <= (1 << 24), "T*k too large");
   MOE_REQUIRE(offsets != nullptr, "null offsets");
   MOE_REQUIRE(aligned(offsets, 4), "misaligned offsets");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(idx && perm && inv_perm, "null pointer");
+  MOE_REQUIRE(aligned(idx, 4) && aligned(perm, 4) && aligned(inv_perm, 4), "misaligned pointer");
+  const size_t need = moe_permute_scratch_bytes(T, k, E);   // 0 when the pairs fit one tile
+  if (need > 0 && (scratch == nullptr || scratch_bytes < need))
+    return fail(MOE_ERR_CAPACITY, "moe_permute needs %zu bytes of scratch, got %zu", need, scratch_bytes);
+  MOE_REQUIRE(need == 0 || aligned(scratch, 4), "misaligned scratch");
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets,
+                                  int32_t* perm, int32_t* inv_perm, void* scratch,
+                                  size_t scratch_bytes, int32_t* dev_status, cudaStream_t stream) {
+  clear_error();
+  moe_status st = check_permute_args(idx, T, k, E, offsets, perm, inv_perm, scratch, scratch_bytes);
+  if (st != MOE_OK) return st;
   const int n = T * k;
   DeviceInfo dev;
-  moe_status st = current_device(&dev);
+  st = current_device(&dev);
   if (st != MOE_OK) return st;
   if (n == 0) {
     MOE_CUDA_TRY(cudaMemsetAsync(offsets, 0, (E + 1) * sizeof(int32_t), stream));
     return MOE_OK;
   }
-  MOE_REQUIRE(idx && perm && inv_perm, "null pointer");
-  MOE_REQUIRE(aligned(idx, 4) && aligned(perm, 4) && aligned(inv_perm, 4), "misaligned pointer");
   const size_t smem = rank_smem_bytes(E);
   MOE_REQUIRE(smem <= dev.smem_optin, "E=%d needs %zu bytes of shared memory", E, smem);
   st = ensure_smem_attr(dev);
@@ -251,10 +264,6 @@ extern "C" moe_status moe_permute(const int32_t* idx, int T, int k, int E, int32
     MOE_LAUNCH_CHECK("permute_fused_kernel");
     return MOE_OK;
   }
-  const size_t need = moe_permute_scratch_bytes(T, k, E);
-  if (scratch == nullptr || scratch_bytes < need)
-    return fail(MOE_ERR_CAPACITY, "moe_permute needs %zu bytes of scratch, got %zu", need, scratch_bytes);
-  MOE_REQUIRE(aligned(scratch, 4), "misaligned scratch");
   int32_t* counts = static_cast<int32_t*>(scratch);
   permute_count_kernel<<<ntiles, kTile, E * sizeof(int), stream>>>(idx, n, E, counts);
   MOE_LAUNCH_CHECK("permute_count_kernel");

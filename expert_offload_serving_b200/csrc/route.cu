@@ -89,9 +89,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* idx,
 
 using namespace moe;
 
-extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, int32_t* idx,
-                                     float* gate, cudaStream_t stream) {
-  clear_error();
+moe_status moe::check_route_args(const float* logits, int T, int E, int k, const int32_t* idx, const float* gate) {
   MOE_REQUIRE(T >= 0, "T=%d < 0", T);
   MOE_REQUIRE(E >= 1 && E <= 1024, "E=%d outside [1, 1024]", E);
   MOE_REQUIRE(k >= 1 && k <= E && k <= 32, "k=%d outside [1, min(E, 32)]", k);
@@ -99,8 +97,16 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(logits && idx && gate, "null pointer");
   MOE_REQUIRE(aligned(logits, 4) && aligned(idx, 4) && aligned(gate, 4), "misaligned pointer");
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, int32_t* idx,
+                                     float* gate, cudaStream_t stream) {
+  clear_error();
+  moe_status st = check_route_args(logits, T, E, k, idx, gate);
+  if (st != MOE_OK || T == 0) return st;
   DeviceInfo dev;
-  moe_status st = current_device(&dev);
+  st = current_device(&dev);
   if (st != MOE_OK) return st;
   cudaError_t err;
   if (E <= 32) err = launch_route<1>(logits, T, E, k, idx, gate, stream);

@@ -229,7 +229,10 @@ moe_status moe_combine_merge(const float* y_perm, const int32_t* idx, const floa
  * buffer is the one the individual call takes, with the same meaning,
  * layout, ownership and errors; the results are those of the four calls.
  * It exists for the host cost of a decode step: one call instead of four.
- * Returns the first failing step's status; nothing after it is enqueued. */
+ * The arguments of all four steps are checked first: a call rejected by a
+ * check (MOE_ERR_INVALID_ARG, MOE_ERR_CAPACITY) enqueues nothing.  After
+ * that, a step that fails at launch (MOE_ERR_CUDA, or a device-dependent
+ * limit) returns its status and nothing after it is enqueued. */
 moe_status moe_layer_forward(moe_shape s, const float* logits, const void* x, int T, int k,
                              int32_t* idx, float* gate, int32_t* offsets, int32_t* perm,
                              int32_t* inv_perm, void* scratch, size_t scratch_bytes,

@@ -101,6 +101,62 @@ def test_argument_errors_before_any_cuda_call(moe):
         moe.MOE_ERR_INVALID_ARG
 
 
+def _aligned_host_buffer(n_floats=1 << 16):
+    raw = np.zeros(n_floats + 64, dtype=np.float32)
+    shift = (-_host_ptr(raw)) % 256 // 4
+    buf = raw[shift: shift + n_floats]
+    assert _host_ptr(buf) % 256 == 0
+    return buf
+
+
+def _forward(moe, s, p, T, k, flags=0, scratch_bytes=1 << 20, out=None, y_perm=None):
+    out = p if out is None else out
+    y_perm = p if y_perm is None else y_perm
+    return moe.lib().moe_layer_forward(s, p, p, T, k, p, p, p, p, p, p, scratch_bytes, p, p, 8,
+                                       None if flags else y_perm, flags, p, 1 << 30, None, out, None, None)
+
+
+def test_layer_forward_checks_every_step_before_enqueueing(moe):
+    """moe_layer_forward rejects a bad argument of any of its four steps before
+    the first step is enqueued: no CUDA call happens, so on any machine the
+    status is the argument error itself, never MOE_ERR_CUDA."""
+    buf = _aligned_host_buffer()
+    p = _host_ptr(buf)
+    bf16 = moe.shape(8, 256, 256, "bf16")
+    assert _forward(moe, moe.shape(8, 60, 64, "bf16"), p, 4, 2) == moe.MOE_ERR_INVALID_ARG     # FFN shape
+    assert _forward(moe, bf16, p, 4, 9) == moe.MOE_ERR_INVALID_ARG                             # route: k > E
+    assert _forward(moe, bf16, p, 4, 2, out=p + 4) == moe.MOE_ERR_INVALID_ARG                  # combine: out
+    assert b"16-byte" in moe.lib().moe_last_error()
+    assert _forward(moe, bf16, p, 4, 2, y_perm=p + 4) == moe.MOE_ERR_INVALID_ARG               # FFN: y_perm
+    assert _forward(moe, bf16, p, 4, 2, flags=1) == moe.MOE_ERR_INVALID_ARG                    # act flag, bf16
+    assert b"NVFP4" in moe.lib().moe_last_error()
+    big = moe.shape(256, 256, 256, "bf16")
+    assert _forward(moe, big, p, 4096, 6, scratch_bytes=16) == moe.MOE_ERR_CAPACITY            # permute scratch
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="valid calls would launch on host pointers")
+def test_valid_arguments_pass_every_check(moe):
+    """The converse: arguments that are valid pass every check and reach the
+    device query, which is what fails on a host without a GPU (MOE_ERR_CUDA)."""
+    L_ = moe.lib()
+    buf = _aligned_host_buffer()
+    p = _host_ptr(buf)
+    s = moe.shape(8, 256, 256, "bf16")
+
+    def reached_device(st):
+        return st == moe.MOE_ERR_CUDA and b"cudaGetDevice" in L_.moe_last_error()
+
+    assert reached_device(L_.moe_route_topk(p, 4, 8, 2, p, p, None))
+    assert reached_device(L_.moe_permute(p, 4, 2, 8, p, p, p, None, 0, None, None))
+    need = moe.moe_permute_scratch_bytes(4096, 6, 256)
+    assert need > 0
+    assert reached_device(L_.moe_permute(p, 4096, 6, 256, p, p, p, p, need, None, None))
+    assert reached_device(L_.moe_expert_ffn(s, p, 4, 2, p, p, p, p, 8, p, p, None, 0, p, 1 << 20, None, None))
+    assert reached_device(L_.moe_combine_merge(p, p, p, p, p, None, 4, 2, 256, 8, p, None))
+    assert reached_device(_forward(moe, s, p, 4, 2))
+    assert reached_device(_forward(moe, moe.shape(8, 256, 256, "nvfp4"), p, 4, 2, flags=1))
+
+
 def test_workspace_and_scratch_sizes(moe):
     s = moe.shape(128, 2048, 768, "bf16")
     assert moe.moe_expert_ffn_workspace_bytes(s, 64, 8) >= 64 * 8 * 768 * 4
