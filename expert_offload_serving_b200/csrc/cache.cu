@@ -27,6 +27,10 @@ struct moe_cache {
   const uint8_t* host_pool;    // pinned host
   int32_t* slot_table_dev;     // device [E]
   std::vector<int32_t> expert_of_slot, last_used, slot_of_expert;
+  // set when enqueueing a fill failed part-way: a copy may have reached a
+  // victim slot whose table entry was never updated, so no later fill or FFN
+  // may trust the device state
+  bool broken = false;
 };
 
 namespace moe {
@@ -45,6 +49,36 @@ __global__ void apply_table_updates(int32_t* table, int E, TableUpdates u) {
   if (threadIdx.x == 0 && blockIdx.x == 0)
     for (int i = 0; i < u.n; ++i)
       if (u.expert[i] >= 0 && u.expert[i] < E) table[u.expert[i]] = u.value[i];
+}
+
+struct Fill {
+  int32_t e, s, old;
+};
+
+// The copies of a planned fill, then the kernels that write its slot-table
+// changes, on `side` after `reads_done`.
+moe_status enqueue_fills(moe_cache* c, const std::vector<Fill>& plan, cudaStream_t side,
+                         cudaEvent_t reads_done) {
+  if (reads_done != nullptr) MOE_CUDA_TRY(cudaStreamWaitEvent(side, reads_done, 0));
+  for (const Fill& f : plan)
+    MOE_CUDA_TRY(cudaMemcpyAsync(c->slot_pool + static_cast<size_t>(f.s) * c->blob_bytes,
+                                 c->host_pool + static_cast<size_t>(f.e) * c->blob_bytes, c->blob_bytes,
+                                 cudaMemcpyHostToDevice, side));
+  TableUpdates u{};
+  for (size_t i = 0; i < plan.size(); ++i) {
+    if (plan[i].old >= 0) {
+      u.expert[u.n] = plan[i].old;
+      u.value[u.n++] = -1;
+    }
+    u.expert[u.n] = plan[i].e;
+    u.value[u.n++] = plan[i].s;
+    if (u.n > kMaxUpdates - 2 || i + 1 == plan.size()) {
+      apply_table_updates<<<1, 32, 0, side>>>(c->slot_table_dev, c->shape.E, u);
+      MOE_LAUNCH_CHECK("apply_table_updates");
+      u.n = 0;
+    }
+  }
+  return MOE_OK;
 }
 
 }  // namespace
@@ -102,6 +136,8 @@ extern "C" moe_status moe_cache_fill(moe_cache* c, const int32_t* experts, int n
                                      int32_t* n_fills) {
   clear_error();
   MOE_REQUIRE(c != nullptr, "null cache");
+  if (c->broken)
+    return fail(MOE_ERR_CUDA, "an earlier fill failed part-way; the device slots are undefined: recreate the cache");
   MOE_REQUIRE(n >= 0 && n_protect >= 0, "negative count");
   MOE_REQUIRE(n == 0 || experts != nullptr, "null experts");
   MOE_REQUIRE(n_protect == 0 || protect != nullptr, "null protect list");
@@ -120,7 +156,6 @@ extern "C" moe_status moe_cache_fill(moe_cache* c, const int32_t* experts, int n
   std::vector<int32_t> eos = c->expert_of_slot, lu = c->last_used, soe = c->slot_of_expert;
   for (int32_t e : want)
     if (soe[e] >= 0) lu[soe[e]] = step;
-  struct Fill { int32_t e, s, old; };
   std::vector<Fill> plan;
   for (int32_t e : want) {
     if (soe[e] >= 0) continue;
@@ -144,28 +179,17 @@ extern "C" moe_status moe_cache_fill(moe_cache* c, const int32_t* experts, int n
     plan.push_back({e, s, old});
   }
   // enqueue the copies and the slot-table updates
-  if (!plan.empty() && c->slot_pool != nullptr) {
-    if (reads_done != nullptr) MOE_CUDA_TRY(cudaStreamWaitEvent(side, reads_done, 0));
-    for (const Fill& f : plan)
-      MOE_CUDA_TRY(cudaMemcpyAsync(c->slot_pool + static_cast<size_t>(f.s) * c->blob_bytes,
-                                   c->host_pool + static_cast<size_t>(f.e) * c->blob_bytes,
-                                   c->blob_bytes, cudaMemcpyHostToDevice, side));
-    TableUpdates u{};
-    for (size_t i = 0; i < plan.size(); ++i) {
-      if (plan[i].old >= 0) {
-        u.expert[u.n] = plan[i].old;
-        u.value[u.n++] = -1;
-      }
-      u.expert[u.n] = plan[i].e;
-      u.value[u.n++] = plan[i].s;
-      if (u.n > kMaxUpdates - 2 || i + 1 == plan.size()) {
-        apply_table_updates<<<1, 32, 0, side>>>(c->slot_table_dev, E, u);
-        MOE_LAUNCH_CHECK("apply_table_updates");
-        u.n = 0;
-      }
+  if (c->slot_pool != nullptr) {
+    moe_status st = plan.empty() ? MOE_OK : enqueue_fills(c, plan, side, reads_done);
+    if (st == MOE_OK && fill_done != nullptr) {
+      const cudaError_t e = cudaEventRecord(fill_done, side);
+      if (e != cudaSuccess) st = fail(MOE_ERR_CUDA, "cudaEventRecord(fill_done) failed: %s", cudaGetErrorString(e));
+    }
+    if (st != MOE_OK) {
+      c->broken = !plan.empty();
+      return st;
     }
   }
-  if (fill_done != nullptr && c->slot_pool != nullptr) MOE_CUDA_TRY(cudaEventRecord(fill_done, side));
   c->expert_of_slot.swap(eos);
   c->last_used.swap(lu);
   c->slot_of_expert.swap(soe);

@@ -268,7 +268,11 @@ moe_status moe_layer_forward(moe_shape s, const float* logits, const void* x, in
  *   non-NULL).  fills (host int32 [n][3] or NULL) receives
  *   (expert, slot, evicted expert or -1) per fill; *n_fills their count.
  *   If there are not enough evictable slots, MOE_ERR_CAPACITY is returned
- *   and the cache state is unchanged. */
+ *   and the cache state is unchanged.  If enqueueing fails (MOE_ERR_CUDA),
+ *   the host bookkeeping is unchanged but a copy may already have reached a
+ *   victim slot whose table entry was not rewritten: the handle then refuses
+ *   every later fill with MOE_ERR_CUDA; recreate the cache (and its slot
+ *   table) before the next FFN call. */
 typedef struct moe_cache moe_cache;
 moe_status moe_cache_create(moe_shape s, int n_slots, void* slot_pool, const void* host_pool,
                             int32_t* slot_of_expert_dev, moe_cache** out);

@@ -319,3 +319,26 @@ def test_cache_capacity_error_leaves_state(moe):
         c.fill([3, 4, 5], 1)
     assert ei.value.status == moe.MOE_ERR_CAPACITY
     assert c.query() == before
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="the copies would run")
+def test_cache_failed_fill_makes_the_cache_unusable(moe):
+    """A fill whose copies cannot be enqueued (here: no GPU) fails with
+    MOE_ERR_CUDA and leaves the host bookkeeping as it was; every later fill
+    fails the same way until the cache is recreated, since a copy may already
+    have reached a victim slot whose table entry was never rewritten."""
+    buf = _aligned_host_buffer()             # stands in for the pools; never touched
+    p = _host_ptr(buf)
+    s = moe.shape(16, 64, 64, "bf16")
+    c = moe.MoeCache(s, 2, slot_pool=p, host_pool=p, slot_of_expert_dev=p)
+    before = c.query()
+    with pytest.raises(moe.MoeError) as ei:
+        c.fill([1, 2], 0)
+    assert ei.value.status == moe.MOE_ERR_CUDA
+    assert c.query() == before
+    with pytest.raises(moe.MoeError) as ei:
+        c.fill([3], 1)
+    assert ei.value.status == moe.MOE_ERR_CUDA
+    assert b"recreate" in moe.lib().moe_last_error()
+    planner = moe.MoeCache(s, 2)             # a plan-only handle enqueues nothing and is unaffected
+    assert planner.fill([1, 2], 0) == [(1, 0, -1), (2, 1, -1)]
