@@ -91,9 +91,25 @@ class MoeLayer:
             self.fill_done.record(self.side)
             self.reads_done.record()
 
+    # -- argument checks ---------------------------------------------------------
+    # The C calls see plain pointers, so the sizes of the layer's own buffers
+    # (T_max tokens) are enforced here, before any call is made.
+    def _check_T(self, T: int) -> int:
+        if not 0 <= T <= self.T_max:
+            raise ValueError(f"T={T} outside [0, {self.T_max}]: the layer's buffers hold T_max={self.T_max} tokens")
+        return T
+
+    def _check_tensor(self, name, t, shape, dtype):
+        if t is None:
+            return
+        same_device = t.device.type == self.dev.type and (self.dev.index is None or t.device.index == self.dev.index)
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or not same_device:
+            raise ValueError(f"{name}: expected a contiguous {dtype} tensor of shape {tuple(shape)} on {self.dev}, "
+                             f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
     # -- steps -----------------------------------------------------------------
     def route(self, logits, stream=None):
-        T = logits.shape[0]
+        T = self._check_T(logits.shape[0])
         moe_route_topk(logits, self.k, self.idx[:T], self.gate[:T], stream)
 
     def prepare(self, step: int, gpu_experts, protect=(), stream=None):
@@ -107,11 +123,12 @@ class MoeLayer:
         return fills
 
     def permute(self, T, stream=None):
+        self._check_T(T)
         moe_permute(self.idx[:T], self.E, self.offsets, self.perm, self.inv_perm,
                     scratch=self.scratch, dev_status=self.status, stream=stream)
 
     def ffn(self, x, stream=None, out=None):
-        T = x.shape[0]
+        T = self._check_T(x.shape[0])
         if self.act == "nvfp4":
             moe_expert_ffn(self.s, x, self.k, self.offsets, self.perm, self.slot, self.pool, self.n_slots,
                            gate=self.gate, out=out if out is not None else self.out[:T], flags=self.flags,
@@ -124,14 +141,20 @@ class MoeLayer:
             self.reads_done.record(stream or torch.cuda.current_stream())
 
     def combine(self, T, host_partial=None, stream=None, out=None):
+        self._check_T(T)
+        self._check_tensor("host_partial", host_partial, (T, self.d), torch.float32)
         moe_combine_merge(self.y_perm, self.idx[:T], self.gate[:T], self.inv_perm, self.slot, host_partial,
                           self.E, out if out is not None else self.out[:T], stream)
 
     def forward(self, logits, x, host_partial=None, stream=None):
-        """All steps for a resident pool through moe_layer_forward (one C
-        call); returns out [T, d] (a view of an internal buffer, overwritten by
-        the next call)."""
-        T = x.shape[0]
+        """All steps through moe_layer_forward (one C call); returns out [T, d]
+        (a view of an internal buffer, overwritten by the next call).  Cached
+        mode: call prepare() first; the pool reads are then recorded for the
+        next fill to wait on, as ffn() does."""
+        T = self._check_T(x.shape[0])
+        self._check_tensor("logits", logits, (T, self.E), torch.float32)
+        self._check_tensor("x", x, (T, self.d), torch.bfloat16)
+        self._check_tensor("host_partial", host_partial, (T, self.d), torch.float32)
         if not hasattr(self, "_fwd_args"):
             # device addresses of the layer's own buffers, resolved once
             nb = lambda t: t.numel() * t.element_size()
@@ -145,4 +168,10 @@ class MoeLayer:
         hp = 0 if host_partial is None else host_partial.data_ptr()
         _check(lib().moe_layer_forward(self.s, logits.data_ptr(), x.data_ptr(), T, self.k, *self._fwd_args, hp,
                                        self.out.data_ptr(), self.status.data_ptr(), s))
+        if self.cache is not None:
+            if stream is None:
+                rs = torch.cuda.current_stream()
+            else:
+                rs = torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream
+            self.reads_done.record(rs)
         return self.out[:T]

@@ -342,3 +342,30 @@ def test_cache_failed_fill_makes_the_cache_unusable(moe):
     assert b"recreate" in moe.lib().moe_last_error()
     planner = moe.MoeCache(s, 2)             # a plan-only handle enqueues nothing and is unaffected
     assert planner.fill([1, 2], 0) == [(1, 0, -1), (2, 1, -1)]
+
+
+def test_layer_rejects_inputs_its_buffers_cannot_hold(moe):
+    """The C calls see plain pointers, so MoeLayer checks the sizes of its own
+    buffers (T_max tokens) and the input tensors before any call: a batch
+    larger than T_max, or logits / x / host_partial of the wrong shape or type,
+    raise ValueError instead of letting a kernel write past a buffer."""
+    from expert_offload_serving_b200.layer import MoeLayer
+    E, d, I, k, T_max = 8, 256, 256, 2, 4
+    B = moe.moe_expert_blob_bytes(moe.shape(E, d, I, "bf16"))
+    layer = MoeLayer(E, d, I, "bf16", k, T_max, device="cpu", device_pool=torch.zeros((E, B), dtype=torch.uint8))
+    logits = torch.zeros((T_max + 1, E), dtype=torch.float32)
+    x = torch.zeros((T_max + 1, d), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="T_max"):
+        layer.forward(logits, x)
+    with pytest.raises(ValueError, match="T_max"):
+        layer.route(logits)
+    with pytest.raises(ValueError, match="T_max"):
+        layer.permute(T_max + 1)
+    with pytest.raises(ValueError, match="logits"):
+        layer.forward(logits[:2].double(), x[:2])
+    with pytest.raises(ValueError, match="x:"):
+        layer.forward(logits[:2], x[:2].float())
+    with pytest.raises(ValueError, match="x:"):
+        layer.forward(logits[:2], torch.zeros((2, 2 * d), dtype=torch.bfloat16)[:, ::2])
+    with pytest.raises(ValueError, match="host_partial"):
+        layer.forward(logits[:2], x[:2], host_partial=torch.zeros((2, d), dtype=torch.float64))
