@@ -96,6 +96,19 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _dev(name, t, n, dtype):
+    """The C calls see plain pointers: a device buffer must be a contiguous CUDA
+    tensor of the documented dtype holding the n elements the call touches
+    (checked here, since the library cannot see sizes)."""
+    if t is None:
+        return
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+    if t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call touches {n}")
+
+
 def _stream(s):
     if s is None:
         return torch.cuda.current_stream().cuda_stream
@@ -136,6 +149,9 @@ def moe_pack_expert(s: moe_shape, wg, wu, wd, sg=None, su=None, sd=None, tensor_
 
 def moe_route_topk(logits, k: int, idx, gate, stream=None):
     T, E = logits.shape
+    _dev("logits", logits, T * E, torch.float32)
+    _dev("idx", idx, T * k, torch.int32)
+    _dev("gate", gate, T * k, torch.float32)
     _check(lib().moe_route_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(gate), _stream(stream)))
 
 
@@ -143,8 +159,17 @@ def moe_permute_scratch_bytes(T: int, k: int, E: int) -> int:
     return lib().moe_permute_scratch_bytes(T, k, E)
 
 
-def moe_permute(idx, E: int, offsets, perm, inv_perm, scratch=None, dev_status=None, stream=None):
+def _permute_buffers(idx, E, offsets, perm, inv_perm):
     T, k = idx.shape
+    _dev("idx", idx, T * k, torch.int32)
+    _dev("offsets", offsets, E + 1, torch.int32)
+    _dev("perm", perm, T * k, torch.int32)
+    _dev("inv_perm", inv_perm, T * k, torch.int32)
+    return T, k
+
+
+def moe_permute(idx, E: int, offsets, perm, inv_perm, scratch=None, dev_status=None, stream=None):
+    T, k = _permute_buffers(idx, E, offsets, perm, inv_perm)
     nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
     _check(lib().moe_permute(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv_perm),
                              _ptr(scratch), nbytes, _ptr(dev_status), _stream(stream)))
@@ -156,7 +181,7 @@ MOE_PERMUTE_NOALLOC_MAX_SCRATCH = 262144
 def moe_permute_noalloc(idx, E: int, offsets, perm, inv_perm, dev_status=None, stream=None):
     """moe_permute without a scratch argument: for callers that cannot
     allocate device memory (the library's fixed scratch array is used)."""
-    T, k = idx.shape
+    T, k = _permute_buffers(idx, E, offsets, perm, inv_perm)
     _check(lib().moe_permute_noalloc(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv_perm),
                                      _ptr(dev_status), _stream(stream)))
 
@@ -169,6 +194,14 @@ def moe_expert_ffn(s: moe_shape, x, k: int, offsets, perm, slot_of_expert, slot_
                    gate=None, y_perm=None, out=None, flags: int = 0, workspace=None,
                    dev_status=None, stream=None):
     T = x.shape[0]
+    _dev("x", x, T * s.d, torch.bfloat16)
+    _dev("offsets", offsets, s.E + 1, torch.int32)
+    _dev("perm", perm, T * k, torch.int32)
+    _dev("slot_of_expert", slot_of_expert, s.E, torch.int32)
+    _dev("slot_pool", slot_pool, n_slots * moe_expert_blob_bytes(s), torch.uint8)
+    _dev("gate", gate, T * k, torch.float32)
+    _dev("y_perm", y_perm, T * k * s.d, torch.float32)
+    _dev("out", out, T * s.d, torch.float32)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().moe_expert_ffn(s, _ptr(x), T, k, _ptr(offsets), _ptr(perm), _ptr(slot_of_expert),
                                 _ptr(slot_pool), n_slots, _ptr(gate), _ptr(y_perm), _ptr(out), flags,
@@ -178,6 +211,13 @@ def moe_expert_ffn(s: moe_shape, x, k: int, offsets, perm, slot_of_expert, slot_
 def moe_combine_merge(y_perm, idx, gate, inv_perm, slot_of_expert, host_partial, E: int, out, stream=None):
     T, k = idx.shape
     d = out.shape[1]
+    _dev("y_perm", y_perm, T * k * d, torch.float32)
+    _dev("idx", idx, T * k, torch.int32)
+    _dev("gate", gate, T * k, torch.float32)
+    _dev("inv_perm", inv_perm, T * k, torch.int32)
+    _dev("slot_of_expert", slot_of_expert, E, torch.int32)
+    _dev("host_partial", host_partial, T * d, torch.float32)
+    _dev("out", out, T * d, torch.float32)
     _check(lib().moe_combine_merge(_ptr(y_perm), _ptr(idx), _ptr(gate), _ptr(inv_perm),
                                    _ptr(slot_of_expert), _ptr(host_partial), T, k, d, E, _ptr(out),
                                    _stream(stream)))
@@ -189,6 +229,15 @@ def moe_layer_forward(s: moe_shape, logits, x, k: int, idx, gate, offsets, perm,
     """All four steps in one call (moe_route_topk -> moe_permute ->
     moe_expert_ffn -> moe_combine_merge); x [T, d] gives T."""
     T = x.shape[0]
+    n = T * k
+    for name, t, need, dt in (("logits", logits, T * s.E, torch.float32), ("x", x, T * s.d, torch.bfloat16),
+                              ("idx", idx, n, torch.int32), ("gate", gate, n, torch.float32),
+                              ("offsets", offsets, s.E + 1, torch.int32), ("perm", perm, n, torch.int32),
+                              ("inv_perm", inv_perm, n, torch.int32), ("slot_of_expert", slot_of_expert, s.E, torch.int32),
+                              ("slot_pool", slot_pool, n_slots * moe_expert_blob_bytes(s), torch.uint8),
+                              ("y_perm", y_perm, n * s.d, torch.float32),
+                              ("host_partial", host_partial, T * s.d, torch.float32), ("out", out, T * s.d, torch.float32)):
+        _dev(name, t, need, dt)
     sb = 0 if scratch is None else scratch.numel() * scratch.element_size()
     wb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().moe_layer_forward(s, _ptr(logits), _ptr(x), T, k, _ptr(idx), _ptr(gate), _ptr(offsets), _ptr(perm),

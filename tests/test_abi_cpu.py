@@ -369,3 +369,23 @@ def test_layer_rejects_inputs_its_buffers_cannot_hold(moe):
         layer.forward(logits[:2], torch.zeros((2, 2 * d), dtype=torch.bfloat16)[:, ::2])
     with pytest.raises(ValueError, match="host_partial"):
         layer.forward(logits[:2], x[:2], host_partial=torch.zeros((2, d), dtype=torch.float64))
+
+
+def test_bindings_check_buffers_before_the_call(moe):
+    """The bindings marshal tensors into plain pointers, so they first check
+    that each device buffer is a contiguous CUDA tensor of the documented
+    dtype large enough for the call: a host tensor or a short buffer raises
+    ValueError instead of reaching a kernel."""
+    idx = torch.zeros((4, 2), dtype=torch.int32)
+    with pytest.raises(ValueError, match="logits: expected a contiguous CUDA"):
+        moe.moe_route_topk(torch.zeros((4, 8)), 2, idx, torch.zeros((4, 2)))
+    with pytest.raises(ValueError, match="idx: expected a contiguous CUDA"):
+        moe.moe_permute(idx, 8, torch.zeros(9, dtype=torch.int32), idx.view(-1), idx.view(-1))
+    s = moe.shape(8, 256, 256, "bf16")
+    with pytest.raises(ValueError, match="x: expected"):
+        moe.moe_expert_ffn(s, torch.zeros((4, 256)), 2, None, None, None, None, 8)
+    if torch.cuda.is_available():
+        short = torch.zeros(7, dtype=torch.int32, device="cuda")
+        with pytest.raises(ValueError, match="holds 7 elements"):
+            moe.moe_route_topk(torch.zeros((4, 8), device="cuda"), 2, short,
+                               torch.zeros((4, 2), device="cuda"))
