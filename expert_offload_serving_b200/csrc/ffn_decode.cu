@@ -23,9 +23,10 @@
 // 16-byte chunks (32 FP4 weights): conflict-free 128-bit shared loads, E2M1 ->
 // f16x2 by cvt, times the E8M0 or E4M3 block scale, packed fp32 FMAs against
 // the activations (read through L1), and a warp reduce-scatter at the end.
-// bf16 weights: the same CUDA-core scheme with 8 bf16 weights per 16 bytes,
-// for shapes outside the tensor-core tile layout; bf16 blobs in that layout
-// (d, I multiples of 256) go to the tcgen05 GEMV in ffn_decode_tc.cu.
+// bf16 weights: the same CUDA-core scheme with 8 bf16 weights per 16 bytes.
+// This file serves NVFP4 weights and the shapes outside the tensor-core
+// layouts: bf16 blobs in the tile layout and MXFP4 blobs in the stage-tiled
+// layout (d, I multiples of 256) go to the tcgen05 GEMVs in ffn_decode_tc.cu.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -558,25 +559,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) ffn_decode_kernel(FfnParams P)
     }
   }
 }
-
-// ============================================================ bf16 weights: warp MMA path
-// With bf16 weights there is nothing to dequantise, and the FFN is a small
-// dense product per expert (weights x <= 32 token rows).  The CUDA-core path
-// above needs ~7 issued instructions per weight element at T=64 (unpack, FMA,
-// activation loads), more than the issue rate allows at HBM speed.  Here the
-// same shared-memory weight ring feeds warp-level tensor-core MMAs instead:
-// ldmatrix.x4 loads a 16x16 weight block, mma.sync.m16n8k16 (bf16 x bf16,
-// fp32 accumulate; products are exact in fp32) multiplies it with 8 token
-// rows, so ~0.5 instruction per weight element remains.
-//   tile  phase 1: gate rows i0..i0+15 and up rows i0..i0+15 (the SwiGLU is
-//         formed on matching accumulator fragments); phase 2: 32 rows of W_d.
-//   stage 32 rows x 512 B (256 K elements): with the blocked bf16 blob layout
-//         that is one 16 KB block (down) or two 8 KB blocks (gate, up), each
-//         one bulk copy; their 16-byte chunks are stored XOR-swizzled by row so
-//         the 8 row addresses of each ldmatrix hit distinct banks.
-//   B     activations straight from global/L1 in fragment layout; phase 2
-//         splits the fp32 SwiGLU output into bf16 hi + lo parts (two MMAs),
-//         which keeps its error near 2^-17 relative.
 
 template <int FMT, int PHASE>
 moe_status launch_phase(const FfnParams& P, const DeviceInfo& dev, cudaStream_t s) {
