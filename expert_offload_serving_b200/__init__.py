@@ -53,6 +53,8 @@ _SIGS = {
     "moe_combine_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "moe_layer_forward": (_I, [moe_shape, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P, _P, _I, _P, _I, _P,
                                _SZ, _P, _P, _P, _P]),
+    "moe_split_misses": (_I, [_P, _I, _P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double, _P, _P, _P,
+                              _P]),
     "moe_cache_create": (_I, [moe_shape, _I, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_cache_fill": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
     "moe_cache_query": (_I, [_P, _P, _P, _P]),
@@ -244,6 +246,22 @@ def moe_layer_forward(s: moe_shape, logits, x, k: int, idx, gate, offsets, perm,
                                    _ptr(inv_perm), _ptr(scratch), sb, _ptr(slot_of_expert), _ptr(slot_pool),
                                    n_slots, _ptr(y_perm), flags, _ptr(workspace), wb, _ptr(host_partial),
                                    _ptr(out), _ptr(dev_status), _stream(stream)))
+
+
+def moe_split_misses(misses, tokens_per_expert, q=None, bw_pcie=0.0, bw_host=0.0):
+    """The q split of a step's misses (host only): returns (filled, host), two
+    ascending lists of expert ids.  q=None selects the q* policy from the
+    bandwidths; otherwise floor(q*m + 0.5) misses are filled."""
+    m = len(misses)
+    E = len(tokens_per_expert)
+    ms = (ctypes.c_int32 * max(1, m))(*[int(e) for e in misses])
+    tok = (ctypes.c_int32 * max(1, E))(*[int(t) for t in tokens_per_expert])
+    f = (ctypes.c_int32 * max(1, m))()
+    h = (ctypes.c_int32 * max(1, m))()
+    nf, nh = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().moe_split_misses(ms, m, tok, E, -1.0 if q is None else float(q), float(bw_pcie), float(bw_host),
+                                  f, ctypes.byref(nf), h, ctypes.byref(nh)))
+    return [f[i] for i in range(nf.value)], [h[i] for i in range(nh.value)]
 
 
 def moe_check_status(dev_status, stream=None):

@@ -242,6 +242,29 @@ moe_status moe_layer_forward(moe_shape s, const float* logits, const void* x, in
                              cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* The q split of a decode step's cache misses (host only, no device call):
+ * each missed expert is either filled into the GPU cache over PCIe or run on
+ * the host, and the two partial sums merge exactly in moe_combine_merge
+ * (explainx.ai hardware guide, "Decode: decide whether to move an expert or
+ * compute where it lives"; futuresignalnews.com article, "Bandwidth-Adaptive
+ * Execution (The q* Policy)").
+ *   misses: host int32 [m], distinct expert ids in [0, E).
+ *   tokens_per_expert: host int32 [E], the step's routed tokens per expert.
+ *   q in [0, 1]: fill floor(q*m + 0.5) misses.  q < 0: the q* policy, which
+ *     fills floor(m*bw_pcie/(bw_pcie + bw_host) + 0.5) misses so that the
+ *     fills (over PCIe) and the host computation (through host memory), each
+ *     moving one blob per expert, take the same time; bw_pcie and bw_host
+ *     are the profiled bandwidths in any one unit.
+ *   The misses with the most routed tokens are filled (ties: lower id).
+ *   filled, host: host int32 [m] each, receive the two sets in ascending id;
+ *   *n_filled + *n_host = m.
+ * Errors: MOE_ERR_INVALID_ARG for an id out of range or listed twice, q > 1,
+ * or q < 0 without positive finite bandwidths. */
+moe_status moe_split_misses(const int32_t* misses, int m, const int32_t* tokens_per_expert, int E, double q,
+                            double bw_pcie, double bw_host, int32_t* filled, int32_t* n_filled,
+                            int32_t* host, int32_t* n_host);
+
+/* ------------------------------------------------------------------------ */
 /* Step 5 -- the GPU expert cache: LRU residency of expert blobs in device
  * slots, filled from a pinned host pool (freetoken.wiki mechanism table:
  * "Global LRU expert cache"; explainx.ai hardware guide: experts are copied

@@ -2,6 +2,7 @@
 host-only calls work, arguments are rejected before any CUDA call, and the
 cache's host bookkeeping makes the oracle's LRU decisions (no GPU needed)."""
 import ctypes
+import json
 import os
 import re
 
@@ -389,3 +390,30 @@ def test_bindings_check_buffers_before_the_call(moe):
         with pytest.raises(ValueError, match="holds 7 elements"):
             moe.moe_route_topk(torch.zeros((4, 8), device="cuda"), 2, short,
                                torch.zeros((4, 2), device="cuda"))
+
+
+def test_split_misses_matches_oracle(moe, golden_dir):
+    """moe_split_misses (host only) makes the oracle's choices: for q in
+    [0, 1] the floor(q*m + 0.5) misses with the most routed tokens, ties to
+    the lower id; for q* the oracle's count at the bandwidths the pages print
+    for their workstation (pinned host memory and PCIe)."""
+    fig = json.load(open(os.path.join(golden_dir, "pages_figures.json")))["glm_workstation_bandwidth"]
+    bw_pcie, bw_host = fig["pcie_gbs"], fig["host_gbs"]
+    rng = np.random.default_rng(5)
+    for trial in range(300):
+        E = int(rng.integers(1, 300))
+        m = int(rng.integers(0, min(E, 40) + 1))
+        misses = rng.choice(E, m, replace=False).tolist()
+        tok = rng.integers(0, 4, E).tolist()           # small counts: many ties
+        for q in (0.0, 0.3, 0.5, 1.0, float(rng.uniform())):
+            assert moe.moe_split_misses(misses, tok, q) == L.split_misses(misses, tok, q)
+        n = L.q_star(m, bw_pcie, bw_host)
+        filled, host = moe.moe_split_misses(misses, tok, None, bw_pcie, bw_host)
+        assert len(filled) == n and len(filled) + len(host) == m
+        if m:
+            assert (filled, host) == L.split_misses(misses, tok, n / m)
+    for bad in (dict(misses=[1, 1], q=0.5), dict(misses=[300], q=0.5), dict(misses=[1], q=1.5),
+                dict(misses=[1], q=None)):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_split_misses(bad["misses"], [1] * 16, bad["q"])
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG
