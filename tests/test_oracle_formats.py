@@ -157,8 +157,8 @@ def test_nvfp4_dequant_closed_form():
     w = F.dequant_nvfp4(packed, scales, np.float32(0.01))
     base = F.e2m1_decode(codes)
     g = float(np.float32(0.01))
-    assert np.allclose(w[0, :16], base[:16] * 0.75 * g, rtol=0, atol=0)
-    assert np.allclose(w[0, 16:], base[16:] * 3.5 * g, rtol=0, atol=0)
+    assert np.array_equal(w[0, :16], base[:16] * 0.75 * g)
+    assert np.array_equal(w[0, 16:], base[16:] * 3.5 * g)
 
 
 def test_bf16_decode():
