@@ -56,7 +56,10 @@ struct Fill {
 };
 
 // The copies of a planned fill, then the kernels that write its slot-table
-// changes, on `side` after `reads_done`.
+// changes, on `side` after `reads_done`.  That event must follow the last
+// kernel of the previous step that reads the pool or the slot table (the
+// combine reads the table), or a victim slot could be overwritten, or its
+// table entry cleared, while that step still uses it.
 moe_status enqueue_fills(moe_cache* c, const std::vector<Fill>& plan, cudaStream_t side,
                          cudaEvent_t reads_done) {
   if (reads_done != nullptr) MOE_CUDA_TRY(cudaStreamWaitEvent(side, reads_done, 0));

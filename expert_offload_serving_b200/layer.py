@@ -127,30 +127,58 @@ class MoeLayer:
         moe_permute(self.idx[:T], self.E, self.offsets, self.perm, self.inv_perm,
                     scratch=self.scratch, dev_status=self.status, stream=stream)
 
-    def ffn(self, x, stream=None, out=None):
+    def _record_reads_done(self, stream):
+        # the next fill's copies into a victim slot, and its slot-table update,
+        # wait on this event: it must follow the last kernel of the step that
+        # reads the pool or the slot table
+        if self.cache is not None:
+            if stream is None:
+                rs = torch.cuda.current_stream()
+            else:
+                rs = torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream
+            self.reads_done.record(rs)
+
+    def ffn(self, x, stream=None, out=None, host_partial=None):
+        """The expert FFN.  act="nvfp4": the FFN adds gate-weighted outputs
+        into `out` itself (fused combine), so `out` is first set to
+        host_partial, or to zero; combine() is then not called."""
         T = self._check_T(x.shape[0])
         if self.act == "nvfp4":
+            self._check_tensor("host_partial", host_partial, (T, self.d), torch.float32)
+            o = out if out is not None else self.out[:T]
+            s = torch.cuda.current_stream() if stream is None else (
+                torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream)
+            with torch.cuda.stream(s):
+                if host_partial is not None:
+                    o.copy_(host_partial)
+                else:
+                    o.zero_()
             moe_expert_ffn(self.s, x, self.k, self.offsets, self.perm, self.slot, self.pool, self.n_slots,
-                           gate=self.gate, out=out if out is not None else self.out[:T], flags=self.flags,
+                           gate=self.gate, out=o, flags=self.flags,
                            workspace=self.workspace, dev_status=self.status, stream=stream)
+            self._record_reads_done(stream)          # the fused FFN is the step's last reader
         else:
+            if host_partial is not None:
+                raise ValueError("host_partial belongs to combine() unless act='nvfp4'")
             moe_expert_ffn(self.s, x, self.k, self.offsets, self.perm, self.slot, self.pool, self.n_slots,
                            y_perm=self.y_perm, workspace=self.workspace, dev_status=self.status,
                            stream=stream)
-        if self.cache is not None:
-            self.reads_done.record(stream or torch.cuda.current_stream())
 
     def combine(self, T, host_partial=None, stream=None, out=None):
+        if self.act == "nvfp4":
+            raise RuntimeError("act='nvfp4' combines inside ffn() (fused into the down projection); "
+                               "pass host_partial to ffn() instead")
         self._check_T(T)
         self._check_tensor("host_partial", host_partial, (T, self.d), torch.float32)
         moe_combine_merge(self.y_perm, self.idx[:T], self.gate[:T], self.inv_perm, self.slot, host_partial,
                           self.E, out if out is not None else self.out[:T], stream)
+        self._record_reads_done(stream)              # combine reads the slot table
 
     def forward(self, logits, x, host_partial=None, stream=None):
         """All steps through moe_layer_forward (one C call); returns out [T, d]
         (a view of an internal buffer, overwritten by the next call).  Cached
-        mode: call prepare() first; the pool reads are then recorded for the
-        next fill to wait on, as ffn() does."""
+        mode: call prepare() first; the step's reads of the pool and the slot
+        table are then recorded for the next fill to wait on."""
         T = self._check_T(x.shape[0])
         self._check_tensor("logits", logits, (T, self.E), torch.float32)
         self._check_tensor("x", x, (T, self.d), torch.bfloat16)
@@ -168,10 +196,5 @@ class MoeLayer:
         hp = 0 if host_partial is None else host_partial.data_ptr()
         _check(lib().moe_layer_forward(self.s, logits.data_ptr(), x.data_ptr(), T, self.k, *self._fwd_args, hp,
                                        self.out.data_ptr(), self.status.data_ptr(), s))
-        if self.cache is not None:
-            if stream is None:
-                rs = torch.cuda.current_stream()
-            else:
-                rs = torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream
-            self.reads_done.record(rs)
+        self._record_reads_done(stream)
         return self.out[:T]

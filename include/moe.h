@@ -285,7 +285,9 @@ moe_status moe_split_misses(const int32_t* misses, int m, const int32_t* tokens_
  *   last_used (ties: lowest slot) whose expert is neither in `experts` nor in
  *   `protect` (the other experts of this step, e.g. the host-computed ones).
  *   For each fill it enqueues on `side`: a wait on `reads_done` (if non-NULL;
- *   the last kernel that read the pool), the blob copy host -> slot with
+ *   recorded after the last kernel of the previous step that reads the pool
+ *   OR the slot table -- moe_combine_merge reads the table, so on the unfused
+ *   path it is the combine, not the FFN), the blob copy host -> slot with
  *   cudaMemcpyAsync, and one kernel that writes the slot-table changes
  *   (evicted expert -> -1, new expert -> slot); then records `fill_done` (if
  *   non-NULL).  fills (host int32 [n][3] or NULL) receives

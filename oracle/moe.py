@@ -29,7 +29,11 @@ Readings where the pages are silent:
 Pins (tests/test_oracle_layer.py): brute force on tiny
 inputs in pure-Python loops; E=1, k=1 equals a dense SwiGLU from torch's silu
 and matmul; token-order invariance; subset A plus complement B equals the
-whole layer; top-k against a sorted() brute force with constructed ties.
+whole layer; top-k against a sorted() brute force with constructed ties;
+act="nvfp4" against a layer worked by hand (its quantised x and a written out,
+ties included), with planted misplacements of either quantisation failing it
+(tests/test_oracle_mutations.py); dequant_expert's NVFP4 tensor scales against
+hand-set, distinct gate / up / down scales.
 """
 from __future__ import annotations
 

@@ -219,3 +219,100 @@ def test_act_quant_mode_close_to_unquantised():
     b = M.moe_layer(x, logits, cfg.k, lambda e: deq[e], act="nvfp4")["out"]
     rel = np.abs(a - b).mean() / np.abs(a).mean()
     assert 0.005 < rel < 0.2
+
+
+# ---------------------------------------------------------------- act = "nvfp4"
+# A layer worked by hand for the FP4 x FP4 reading: x and the SwiGLU output a
+# are each quantised to NVFP4 (blocks of 16 along K, unit tensor scale, scale
+# = E4M3(amax/6), codes = E2M1 nearest with ties to the even mantissa) before
+# the product that consumes them.  T = 1, d = 32 (two x blocks), I = 16 (one a
+# block), one expert, k = 1 (gate 1).
+_X_B0 = [3.0, -1.25, 0.3, 0.75, -0.1, 2.2, 1.0, -3.0, 0.5, 0.26, -2.6, 1.74, 0.0, -0.74, 1.5, 2.5]
+# block 0: amax 3 -> s = 0.5 (exact E4M3).  x/s = 6, -2.5 (tie -> -2), 0.6 -> 0.5,
+# 1.5, -0.2 -> -0, 4.4 -> 4, 2, -6, 1, 0.52 -> 0.5, -5.2 -> -6, 3.48 -> 3, 0,
+# -1.48 -> -1.5, 3, 5 (tie -> 4); times s:
+_XQ_B0 = [3.0, -1.0, 0.25, 0.75, -0.0, 2.0, 1.0, -3.0, 0.5, 0.25, -3.0, 1.5, 0.0, -0.75, 1.5, 2.0]
+# block 1 = 4 x block 0: amax 12 -> s = 2, the same codes, values x 4.
+_C = [0.375, -0.15625, 0.0625, 0.21875, 0.34375, 0.046875, 0.015625, -0.09375]
+
+
+def _hand_layer():
+    d, I = 32, 16
+    x = np.array(_X_B0 + [4.0 * v for v in _X_B0])[None, :]
+    wg = np.zeros((I, d))
+    wu = np.zeros((I, d))
+    wd = np.zeros((d, I))
+    for i in range(I):
+        sgn = 1.0 if i % 2 == 0 else -1.0
+        # h = +-(64 xq0 + 64 xq1 + 256 xq2) = +-(192 - 64 + 64) = +-192: silu(192) = 192
+        # exactly in float64 and silu(-192) ~ -1e-81, which is -0 in fp32
+        wg[i, 0], wg[i, 1], wg[i, 2] = 64 * sgn, 64 * sgn, 256 * sgn
+        # u = xq5 * w = 2 * w: c_m on even rows, 1 on odd rows
+        wu[i, 5] = _C[i // 2] / 2 if i % 2 == 0 else 0.5
+        wd[i, i] = 1 / 8              # out[c] = a_q[c] / 8 for c < 16
+        wd[16, i] = 1 / 16            # out[16] = sum(a_q) / 16
+    return x, wg, wu, wd
+
+
+def _hand_expected():
+    # a (even rows) = 192 c = 72, -30, 12, 42, 66, 9, 3, -18; odd rows -0.
+    # amax 72 -> s = 12 (exact E4M3); a/s = 16 c = 6, -2.5 (tie -> -2), 1,
+    # 3.5 (tie -> 4), 5.5 -> 6, 0.75 (tie -> 1), 0.25 (tie -> 0), -1.5;
+    # a_q = 72, -24, 12, 48, 72, 12, 0, -18.
+    aq = [72.0, -24.0, 12.0, 48.0, 72.0, 12.0, 0.0, -18.0]
+    out = np.zeros(32)
+    for m, v in enumerate(aq):
+        out[2 * m] = v / 8
+    out[16] = sum(aq) / 16            # 174 / 16 = 10.875
+    return out
+
+
+def test_act_nvfp4_quantises_x_by_hand():
+    x, *_ = _hand_layer()
+    deq, s, _ = F.nvfp4_quantize_rows(x.astype(np.float32))
+    assert s.tolist() == [[0.5, 2.0]]
+    assert deq[0].tolist() == _XQ_B0 + [4.0 * v for v in _XQ_B0]
+    assert np.signbit(deq[0, 4]) and np.signbit(deq[0, 20])      # -0.1 keeps its sign bit
+
+
+def test_act_nvfp4_layer_hand_worked():
+    x, wg, wu, wd = _hand_layer()
+    y = M.swiglu_ffn(x, wg, wu, wd, act="nvfp4")
+    assert y[0].tolist() == _hand_expected().tolist()
+    res = M.moe_layer(x, np.zeros((1, 1), np.float32), 1, lambda e: (wg, wu, wd), act="nvfp4")
+    assert res["out"][0].tolist() == _hand_expected().tolist()
+
+
+def test_act_none_layer_differs_from_hand_worked():
+    """Without activation quantisation the same layer is not the hand-worked
+    result (h = 188.8, u = 1.1 c): the quantisation is what that pin checks."""
+    x, wg, wu, wd = _hand_layer()
+    y = M.swiglu_ffn(x, wg, wu, wd, act="none")
+    assert abs(y[0, 0] - 188.8 * 1.1 * _C[0] / 8) < 1e-9
+    assert y[0].tolist() != _hand_expected().tolist()
+
+
+# ---------------------------------------------------------------- NVFP4 weights
+_E2M1_MAG = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_nvfp4_dequant_expert_tensor_scale_order():
+    """dequant_expert applies the fp32 tensor scales to gate, up and down in
+    that order, and each E4M3 block scale to its own 16 elements of a row.
+    Codes: element (r, c) of every matrix holds magnitude (r + c) % 8 with the
+    sign bit set on odd rows; block b of every row has scale 2^b; tensor
+    scales gate 2, up 1/2, down 1/4."""
+    I, d = 16, 32
+    def mat(R, K):
+        codes = np.array([[((r + c) % 8) | (8 if r % 2 else 0) for c in range(K)] for r in range(R)], np.uint8)
+        packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+        sc = np.array([[0x38 + 8 * b for b in range(K // 16)] for _ in range(R)], np.uint8)   # 2^b
+        want = np.array([[(-1.0 if r % 2 else 1.0) * _E2M1_MAG[(r + c) % 8] * 2.0 ** (c // 16)
+                          for c in range(K)] for r in range(R)])
+        return packed[None], sc[None], want
+    (cg, sg, g), (cu, su, u), (cd, sd, dn) = mat(I, d), mat(I, d), mat(d, I)
+    w = dict(wg=cg, sg=sg, wu=cu, su=su, wd=cd, sd=sd, ts=np.array([[2.0, 0.5, 0.25]], np.float32))
+    G, U, D = M.dequant_expert("nvfp4", w, 0)
+    assert np.array_equal(G, 2.0 * g)
+    assert np.array_equal(U, 0.5 * u)
+    assert np.array_equal(D, 0.25 * dn)

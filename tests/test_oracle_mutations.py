@@ -109,3 +109,58 @@ def test_most_recent_victim_is_caught(monkeypatch):
     # the module's victim choice calls min(); planting max() picks the newest slot
     monkeypatch.setattr(L, "min", max, raising=False)
     assert _fails(PR.test_hand_worked_trace)
+
+
+# ---- act = "nvfp4": the FP4 prefill reading quantises x before GEMM1 and a
+# before GEMM2; each plausible misplacement must fail the hand-worked layer.
+def _q(v, block=16):
+    return F.nvfp4_quantize_rows(np.asarray(v, np.float32), block)[0]
+
+
+def _plant_ffn(monkeypatch, body):
+    def bad(xr, wg, wu, wd, act="none", dtype=np.float64):
+        if act != "nvfp4":
+            return M.__dict__["_orig_swiglu"](xr, wg, wu, wd, act=act, dtype=dtype)
+        return body(np.asarray(xr, np.float64), np.asarray(wg), np.asarray(wu), np.asarray(wd))
+    monkeypatch.setitem(M.__dict__, "_orig_swiglu", M.swiglu_ffn)
+    monkeypatch.setattr(M, "swiglu_ffn", bad)
+
+
+def test_nvfp4_x_quantised_but_not_a_is_caught(monkeypatch):
+    _plant_ffn(monkeypatch, lambda x, g, u, d: (M.silu(_q(x) @ g.T) * (_q(x) @ u.T)) @ d.T)
+    assert _fails(PL.test_act_nvfp4_layer_hand_worked)
+
+
+def test_nvfp4_a_quantised_but_not_x_is_caught(monkeypatch):
+    _plant_ffn(monkeypatch, lambda x, g, u, d: _q(M.silu(x @ g.T) * (x @ u.T)) @ d.T)
+    assert _fails(PL.test_act_nvfp4_layer_hand_worked)
+
+
+def test_nvfp4_a_quantised_before_the_product_is_caught(monkeypatch):
+    _plant_ffn(monkeypatch, lambda x, g, u, d: (_q(M.silu(_q(x) @ g.T)) * _q(_q(x) @ u.T)) @ d.T)
+    assert _fails(PL.test_act_nvfp4_layer_hand_worked)
+
+
+def test_nvfp4_x_blocks_of_32_is_caught(monkeypatch):
+    _plant_ffn(monkeypatch, lambda x, g, u, d: _q(M.silu(_q(x, 32) @ g.T) * (_q(x, 32) @ u.T)) @ d.T)
+    assert _fails(PL.test_act_nvfp4_layer_hand_worked)
+
+
+def test_nvfp4_scale_from_amax_over_4_is_caught(monkeypatch):
+    orig = F.e4m3_round
+    # the quantiser's only e4m3_round call takes amax/6; planting amax/4 there
+    monkeypatch.setattr(F, "e4m3_round", lambda v: orig(np.asarray(v, np.float32) * np.float32(1.5)))
+    assert _fails(PL.test_act_nvfp4_quantises_x_by_hand)
+    assert _fails(PL.test_act_nvfp4_layer_hand_worked)
+
+
+def test_nvfp4_tensor_scales_reversed_is_caught(monkeypatch):
+    orig = F.dequant_nvfp4
+    calls = []
+
+    def bad(codes, scales, ts):
+        calls.append(ts)
+        return orig(codes, scales, {2.0: 0.25, 0.25: 2.0}.get(float(ts), ts))   # gate <-> down
+    monkeypatch.setattr(F, "dequant_nvfp4", bad)
+    assert _fails(PL.test_nvfp4_dequant_expert_tensor_scale_order)
+    assert len(calls) == 3
