@@ -63,9 +63,11 @@ def peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples (every 100 ms, each with nvidia-smi's own timestamp)
+    of SM clock and throttle reasons while the bench runs; summary() keeps the
+    samples that fall inside the given wall-clock windows."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -78,7 +80,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -98,25 +100,64 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    @staticmethod
+    def now():
+        return time.time()
+
+    def _samples(self):
+        import datetime
+        out = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                out.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        return out
+
+    def summary(self, windows=None):
+        """Median SM clock, max clock and the throttle reasons seen, over the
+        samples inside `windows` ([(t0, t1)] wall-clock seconds; all if None)."""
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for ts, clk, cmax, flags in self._samples():
+            if windows is not None and not any(a - 0.05 <= ts <= b + 0.05 for a, b in windows):
+                continue
+            sm.append(clk)
+            mx.append(cmax)
+            for n, v in zip(names, flags):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def cpu_info():
+    """Host CPU model and its physical core count (unique (package, core)
+    pairs in /proc/cpuinfo), next to the threads this process may use."""
+    model, cores = None, set()
+    try:
+        phys = core = None
+        for ln in open("/proc/cpuinfo"):
+            k, _, v = ln.partition(":")
+            k, v = k.strip(), v.strip()
+            if k == "model name" and model is None:
+                model = v
+            elif k == "physical id":
+                phys = v
+            elif k == "core id":
+                core = v
+            elif not k and phys is not None:
+                cores.add((phys, core))
+                phys = core = None
+    except OSError:
+        pass
+    return {"cpu_model": model, "physical_cores": len(cores) or None, "threads_available": _cpu_cores()}
 
 
 # ---------------------------------------------------------------- distributed
@@ -249,6 +290,15 @@ def decode_point(cfg, T, R, warmup, steps, stream, routed_only=False):
 
 
 def run_gpu(args, rank, world, local):
+    """The GPU arm, with nvidia-smi sampling clocks over the whole run."""
+    idx = local if world > 1 else 0
+    props = torch.cuda.get_device_properties(idx)
+    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(idx)
+    with ClockSampler(smi_id) as clk:
+        return _run_gpu(args, rank, world, local, clk, [])
+
+
+def _run_gpu(args, rank, world, local, clk, timed_windows):
     import expert_offload_serving_b200 as moe
     moe.lib()
     cfg = synth.CONFIGS[args.config]
@@ -296,15 +346,14 @@ def run_gpu(args, rank, world, local):
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    props = torch.cuda.get_device_properties(dev)
-    smi_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(dev.index)
-    with ClockSampler(smi_id) as clk:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(args.steps // G):
-                g_steps.replay()
-            ev1.record(stream)
-        torch.cuda.synchronize()
+    w0 = ClockSampler.now()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps // G):
+            g_steps.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    timed_windows.append((w0, ClockSampler.now()))
     ms = ev0.elapsed_time(ev1)
     barrier(world)
     ms_max = max_over_ranks(ms, world)
@@ -312,21 +361,27 @@ def run_gpu(args, rank, world, local):
 
     # ---- dominant kernel: moe_expert_ffn (gate/up + down launches), timed alone,
     # as graph replays of G calls on the bench stream
+    # each replay (G calls cycling the R replicas) timed on its own; the line
+    # reports the median replay
     with torch.cuda.stream(stream):
         g_ffn = capture_cycle([lambda r=r: r["layer"].ffn(r["x"]) for r in reps], G, stream)
         for _ in range(max(1, (max(3, args.warmup) + G - 1) // G)):
             g_ffn.replay()
-        n_rep = max(1, (max(20, args.steps) + G - 1) // G)
-        n_ffn = n_rep * G
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_rep):
+        n_rep = max(20, (args.steps + G - 1) // G)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_rep)]
+        w0 = ClockSampler.now()
+        for a, b in evs:
+            a.record(stream)
             g_ffn.replay()
-        e1.record(stream)
+            b.record(stream)
     torch.cuda.synchronize()
+    timed_windows.append((w0, ClockSampler.now()))
     del g_ffn
-    ffn_avg_ms = e0.elapsed_time(e1) / n_ffn
-    alg_bytes = sum(per_step[i % R] for i in range(n_ffn)) / n_ffn
+    rep_ms = sorted(a.elapsed_time(b) for a, b in evs)
+    ffn_avg_ms = statistics.median(rep_ms) / G
+    ffn_spread = (round(rep_ms[0] / G, 5), round(rep_ms[-1] / G, 5))
+    alg_bytes = sum(per_step[i % R] for i in range(G)) / G
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     hbm_peak, peak_src = peaks()
     achieved = alg_bytes / (ffn_avg_ms / 1e3) / 1e9
 
@@ -398,7 +453,8 @@ def run_gpu(args, rank, world, local):
 
     prefill = None
     if not args.no_prefill:
-        prefill = run_prefill(Ts=(4096,) if (args.no_sweep or world > 1) else (4096, 16384, 32768))
+        prefill = run_prefill(Ts=(4096,) if (args.no_sweep or world > 1) else (4096, 16384, 32768),
+                              windows=timed_windows)
     sweep = None
     if not args.no_sweep and world == 1:
         sweep = {}
@@ -454,11 +510,14 @@ def run_gpu(args, rank, world, local):
             "traffic": kernel_traffic("ffn_decode_tc.cu", f"{cfg.name}_T{T}"),
             "algorithmic_bytes_per_launch": int(alg_bytes),
             "avg_launch_ms": round(ffn_avg_ms, 5),
+            "timing": f"median of {n_rep} graph replays of {G} calls (per-call min/max over replays: "
+                      f"{ffn_spread[0]} / {ffn_spread[1]} ms)",
         },
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clk.summary(timed_windows),
+        "clocks_whole_run": clk.summary(),
     }
     if cpu is not None:
         result["cpu_baseline"] = cpu
@@ -476,7 +535,7 @@ def run_gpu(args, rank, world, local):
 
 
 # ---------------------------------------------------------------- prefill (FP4 tensor cores)
-def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None):
+def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
     """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, NVFP4 activations
     on tcgen05) at each token count in Ts: whole-layer time and the expert-FFN
     time alone.  The 3.6 GB of weights exceed L2 many times over, so no
@@ -503,23 +562,29 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None):
         logits, x = synth.make_routing(cfg, T, 0)
         lg, xx = logits.cuda(), x.cuda()
         stream = torch.cuda.Stream()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n = iters if T <= 4096 else max(3, iters // 4)
+        n = max(20, iters)
+        ev = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        le = [ev() for _ in range(n)]
+        fe = [ev() for _ in range(n)]
         with torch.cuda.stream(stream):
             for _ in range(warmup):
                 layer.forward(lg, xx)
-            e0.record(stream)
-            for _ in range(n):
+            w0 = time.time()
+            for a, b in le:                     # each call timed on its own: the median is reported
+                a.record(stream)
                 layer.forward(lg, xx)
-            e1.record(stream)
-            f0.record(stream)
-            for _ in range(n):
+                b.record(stream)
+            for a, b in fe:
+                a.record(stream)
                 layer.ffn(xx)
-            f1.record(stream)
+                b.record(stream)
         torch.cuda.synchronize()
-        layer_ms = e0.elapsed_time(e1) / n
-        ffn_ms = f0.elapsed_time(f1) / n
+        if windows is not None:
+            windows.append((w0, time.time()))
+        layer_all = sorted(a.elapsed_time(b) for a, b in le)
+        ffn_all = sorted(a.elapsed_time(b) for a, b in fe)
+        layer_ms = statistics.median(layer_all)
+        ffn_ms = statistics.median(ffn_all)
         moe.moe_check_status(layer.status)
         flops = 2.0 * 3 * cfg.d * cfg.I * T * cfg.k
         off = layer.offsets.cpu()
@@ -544,6 +609,7 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None):
             "frac_roofline": round(roof_ms / ffn_ms, 4),
             "experts_touched": U,
             "timed_iters": n,
+            "timing": f"median of {n} individually timed calls (FFN min/max {ffn_all[0]:.4f} / {ffn_all[-1]:.4f} ms)",
             "kernels": "quant_tokens_kernel, gather_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2>",
         })
         del lg, xx
@@ -674,14 +740,18 @@ def cpu_baseline(cfg, T, seconds=10.0):
     return {"value": round(passes * T / dt, 2), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{passes} float64 oracle passes over one batch of T={T} tokens of the decode_bf16 "
                       f"workload ({len(cache)} experts; weights dequantised before timing)",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), **cpu_info()}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the float64 oracle on the host cores, on the GPU
+    arm's workload and batch (decode_bf16, T = --tokens), each step one batch
+    with fresh routing.  The timed steps are capped so that the arm ends
+    within a few minutes; the line reports how many ran."""
     if rank != 0:
         return None
     cfg = synth.CONFIGS["decode_bf16"]
-    T_s = args.cpu_tokens
+    T_s = args.tokens
     from oracle import moe as M
     # every expert generated and dequantised before timing (as for
     # cpu_baseline): the timed steps are the oracle's layer passes only
@@ -689,23 +759,29 @@ def run_reference(args, rank, world):
     for e in range(cfg.E):
         ww = synth.make_experts(cfg, [e], 0, device="cpu")
         cache[e] = M.dequant_expert(cfg.fmt, ww, 0)
-    for i in range(args.warmup):
+    for i in range(min(args.warmup, 3)):
         oracle_step(cfg, T_s, 5000 + i, cache)
+    budget_s = 150.0
     t0 = time.perf_counter()
+    done = 0
     for i in range(args.steps):
         oracle_step(cfg, T_s, 6000 + i, cache)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
     dt = time.perf_counter() - t0
-    v = args.steps * T_s / dt
+    v = done * T_s / dt
+    workload = f"{cfg.name}: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T_s}, all experts resident"
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "n_gpus": world, "steps": done, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"decode_bf16: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I}; each step a sample "
-                               f"of {T_s} tokens", "parallelism": "host cores"},
+        "config": {"workload": workload, "global_batch": T_s, "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-                         "sample": f"{T_s} tokens per step, fresh routing each step; all {cfg.E} experts' "
-                                   "weights generated and dequantised before timing"},
+                         "sample": f"{done} steps of {T_s} tokens (fresh routing each step, capped at "
+                                   f"{budget_s:.0f} s); all {cfg.E} experts' weights generated and dequantised "
+                                   "before timing", **cpu_info()},
         "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -718,7 +794,6 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--tokens", type=int, default=64, help="tokens per step (1, 16 or 64)")
     ap.add_argument("--replicas", type=int, default=4)
-    ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the FP4 prefill measurement")
     ap.add_argument("--config", default="decode_bf16", choices=["decode_bf16", "decode_mxfp4"],

@@ -55,6 +55,9 @@ _SIGS = {
                                _SZ, _P, _P, _P, _P]),
     "moe_split_misses": (_I, [_P, _I, _P, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double, _P, _P, _P,
                               _P]),
+    "moe_host_expert_ffn": (_I, [moe_shape, _P, _P, _I, _P, _P, _P, _I, _I, _P, _I]),
+    "moe_profile_bandwidth": (_I, [moe_shape, _P, _I, _P, _SZ, _I, _P, ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_double)]),
     "moe_cache_create": (_I, [moe_shape, _I, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_cache_fill": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
     "moe_cache_query": (_I, [_P, _P, _P, _P]),
@@ -262,6 +265,46 @@ def moe_split_misses(misses, tokens_per_expert, q=None, bw_pcie=0.0, bw_host=0.0
     _check(lib().moe_split_misses(ms, m, tok, E, -1.0 if q is None else float(q), float(bw_pcie), float(bw_host),
                                   f, ctypes.byref(nf), h, ctypes.byref(nh)))
     return [f[i] for i in range(nf.value)], [h[i] for i in range(nh.value)]
+
+
+def _host(name, t, n, dtype):
+    """A host buffer of the host-only calls: a contiguous CPU tensor of the
+    documented dtype holding n elements."""
+    if t.is_cuda or t.dtype != dtype or not t.is_contiguous() or t.numel() < n:
+        raise ValueError(f"{name}: expected a contiguous CPU {dtype} tensor of >= {n} elements, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def moe_host_expert_ffn(s: moe_shape, host_pool, experts, x, idx, gate, out, n_threads: int = 0):
+    """The host share of a split step (host only): out [T, d] fp32 = the
+    gate-weighted SwiGLU sum over the pairs whose expert is in `experts`,
+    computed on the CPU from the host pool's blobs.  x bf16 [T, d], idx int32
+    [T, k], gate fp32 [T, k]: CPU tensors.  Releases the GIL while it runs."""
+    T, k = idx.shape
+    B = moe_expert_blob_bytes(s)
+    _host("host_pool", host_pool, s.E * B, torch.uint8)
+    _host("x", x, T * s.d, torch.bfloat16)
+    _host("idx", idx, T * k, torch.int32)
+    _host("gate", gate, T * k, torch.float32)
+    _host("out", out, T * s.d, torch.float32)
+    ex = (ctypes.c_int32 * max(1, len(experts)))(*[int(e) for e in experts])
+    _check(lib().moe_host_expert_ffn(s, _ptr(host_pool), ex, len(experts), _ptr(x), _ptr(idx), _ptr(gate), T, k,
+                                     _ptr(out), int(n_threads)))
+
+
+def moe_profile_bandwidth(s: moe_shape, host_pool, n_blobs: int, dev_buf=None, n_threads: int = 0, stream=None):
+    """(pinned host -> device GB/s, host expert-kernel GB/s) measured on this
+    machine; dev_buf None skips the copy measurement."""
+    B = moe_expert_blob_bytes(s)
+    _host("host_pool", host_pool, n_blobs * B, torch.uint8)
+    if dev_buf is not None:
+        _dev("dev_buf", dev_buf, B, torch.uint8)
+    h2d, hst = ctypes.c_double(0), ctypes.c_double(0)
+    _check(lib().moe_profile_bandwidth(s, _ptr(host_pool), int(n_blobs), _ptr(dev_buf),
+                                       0 if dev_buf is None else dev_buf.numel(), int(n_threads),
+                                       _stream(stream) if dev_buf is not None else None,
+                                       ctypes.byref(h2d), ctypes.byref(hst)))
+    return h2d.value, hst.value
 
 
 def moe_check_status(dev_status, stream=None):

@@ -30,8 +30,19 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libmoe")
 
 
+def gxx_path() -> str:
+    for cand in (os.environ.get("CXX"), shutil.which("g++")):
+        if cand and shutil.which(cand):
+            return cand
+    raise RuntimeError("g++ not found: the host compiler is required to build libmoe")
+
+
+def cuda_include() -> str:
+    return os.path.join(os.path.dirname(os.path.dirname(nvcc_path())), "include")
+
+
 def _sources():
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp", ".cc")))
 
 
 def _headers():
@@ -45,7 +56,12 @@ def _compile(src, debug, verbose):
     newest_dep = max(os.path.getmtime(p) for p in [src] + _headers())
     if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
         return obj, ""
-    cmd = [nvcc_path()] + ARCH + COMMON + ["-c", src, "-o", obj]
+    if src.endswith(".cc"):
+        # host-only code that uses CPU vector intrinsics: the host compiler
+        cmd = [gxx_path(), "-O3", "-std=c++17", "-fPIC", "-pthread", "-Wall", "-I" + os.path.join(ROOT, "include"),
+               "-I" + cuda_include(), "-c", src, "-o", obj]
+    else:
+        cmd = [nvcc_path()] + ARCH + COMMON + ["-c", src, "-o", obj]
     if src.endswith(".cpp"):
         cmd += ["-x", "cu"]
     if debug:
@@ -70,7 +86,7 @@ def build(debug: bool = False, verbose: bool = False) -> str:
                 print(f"== {os.path.basename(o)}\n{log}")
     if os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs):
         return LIB
-    cmd = [nvcc_path()] + ARCH + ["-shared", "-o", LIB] + objs + ["-Xcompiler", "-fPIC"]
+    cmd = [nvcc_path()] + ARCH + ["-shared", "-o", LIB] + objs + ["-Xcompiler", "-fPIC", "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -589,8 +589,13 @@ moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t
 
 }  // namespace
 
+size_t decode_mx_workspace_bytes(moe_shape s, int T, int k);
+
 size_t decode_workspace_bytes(moe_shape s, int T, int k) {
-  // a: fp32 (CUDA-core path) or the two 16-bit planes of the tensor-core path
+  // MXFP4 tensor-core path: the E4M3 terms of x and a with their scales;
+  // otherwise a: fp32 (CUDA-core path) or the two 16-bit planes of the bf16
+  // tensor-core path
+  if (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)) return decode_mx_workspace_bytes(s, T, k);
   return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256);
 }
 
@@ -598,11 +603,18 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
                             const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream);
 
+moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
+                            const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
+                            float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream);
+
 moe_status launch_ffn_decode(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
                              const int32_t* perm, const int32_t* slot, const void* pool, int n_slots,
                              const float* gate, float* y_perm, float* out, void* ws,
                              int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
-  if ((s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I)) || (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)))
+  if (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I))
+    return launch_decode_mx(s, x, T, k, offsets, perm, slot, pool, n_slots, gate, y_perm, out, ws, status, dev,
+                            stream);
+  if (s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I))
     return launch_decode_tc(s, x, T, k, offsets, perm, slot, pool, n_slots, gate, y_perm, out, ws, status, dev,
                             stream);
   FfnParams P{};

@@ -1,0 +1,820 @@
+// Step 3 at decode sizes for MXFP4 weights on the 5th-generation tensor cores
+// (moe_expert_ffn without MOE_FFN_ACT_NVFP4, MXFP4 blobs in the stage-tiled
+// layout, i.e. d and I multiples of 256): the grouped SwiGLU expert FFN as two
+// skinny block-scaled GEMMs that read the E2M1 weights as stored.
+//
+// A decode layer call is bound by reading the routed experts' weights from HBM
+// (explainx.ai hardware guide, "Decode: decide whether to move an expert or
+// compute where it lives").  The weights are never converted on the SM: TMA
+// loads each stage's packed E2M1 codes with the 16U4_ALIGN16B expansion (16
+// codes into every 16-byte slot, the operand layout of
+// tcgen05.mma kind::mxf8f6f4), the E8M0 block scales go to TMEM by tcgen05.cp,
+// and the tensor core applies them (block_scale, one scale per 32 K elements).
+//
+// That kind multiplies FP8/FP6/FP4 by FP8/FP6/FP4, so the activations enter as
+// sums of E4M3 terms, each term with its own E8M0 scale per 32 elements
+// (chosen from the block's largest remaining magnitude, so no term saturates):
+//   x (bf16, 8 significant bits)  -> 2 terms, exact unless an element is more
+//                                     than ~2^18 below its block's maximum;
+//   a (fp32, the SwiGLU output)   -> 4 terms (16 significant bits), residual
+//                                     below 2^-16 of each block's maximum.
+// Each term is one MMA; the accumulator is fp32 in TMEM.
+//
+//   split_x:  x [T][d] -> 2 E4M3 planes + 2 scale planes, once per token.
+//   gemv<1>:  D[128 x N] = W_gu tile (64 gate + 64 up rows of the same
+//             intermediate indices) x X^T over K = d, N <= TN token rows
+//             gathered by one-row TMA loads.  Epilogue: a = silu(D_gate) *
+//             D_up split into 4 E4M3 planes + scales (warp-wide maxima over
+//             the 32 lanes = one 32-element block of I).
+//   gemv<2>:  D[128 x N] = W_d tile x A^T over K = I, 4 MMAs per K step.
+//             Epilogue: y_perm rows, or out[t] += gate * y (fused combine).
+//
+// Work unit = (expert, 128-row tile, chunk of <= TN pairs), expert-major,
+// dealt round-robin to one persistent CTA per SM.  Warp 0 produces the weight
+// stages (two TMA boxes + one bulk copy of the scale atoms per 17 KB tile,
+// with an L2 prefetch cursor PF_ITEMS tiles ahead), warp 1 owns TMEM and
+// issues tcgen05.cp + tcgen05.mma, warps 2-5 run the epilogue on
+// double-buffered accumulators, warp 6 loads the token-row terms and their
+// scale atoms.  Every wait is bounded: on expiry the CTA records
+// MOE_ERR_TIMEOUT, stops issuing, drains what it issued and frees its TMEM.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace ::moe::tc;
+
+constexpr int TM = 128;                    // weight rows per tile
+constexpr int KSTAGE = 256;                // K elements per stage (one blob tile)
+constexpr int A_BOX = 128 * 128;           // one TMA box: 128 rows x 128 padded codes
+constexpr int A_SMEM = 2 * A_BOX + 1024;   // codes (expanded) + 2 scale atoms
+constexpr uint32_t A_TX = 2 * A_BOX + 1024;
+constexpr int ACC_COLS = 32;
+constexpr int SFA_COL = 64;                // TMEM: 2 accumulators, then scale factors
+constexpr int SFB_COL = 72;
+constexpr int TMEM_COLS = 128;
+constexpr int NX = 2;                      // E4M3 terms of x
+constexpr int NA = 4;                      // E4M3 terms of a
+constexpr int PF_ITEMS = 8;                // L2 prefetch distance (tiles)
+constexpr int kSmemBudget = 226 * 1024;
+constexpr int kMaxE = 1024;
+constexpr int kBarBytes = 512;
+constexpr int THREADS = 7 * 32;
+constexpr int BPROD_WARP = 6;
+
+struct MxParams {
+  int E, d, I, T, k, n_slots;
+  int a_box_rows[3];       // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
+  const int32_t* offsets;
+  const int32_t* perm;
+  const int32_t* slot;
+  const float* gate;
+  const uint8_t* pool;
+  size_t blob_bytes;
+  BlobLayout L;
+  const uint8_t* xs;       // [NX][T][d/32] E8M0 scales of the x terms
+  uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
+  uint8_t* as;             // [NA][T*k][I/32] their E8M0 scales
+  float* y_perm;
+  float* out;
+  int32_t* status;
+};
+
+template <int PHASE, int TN>
+struct Cfg {
+  static constexpr int NT = PHASE == 1 ? NX : NA;                // terms of the B operand
+  static constexpr int B_ATOM = TN * 128;                        // TN rows x 128 E4M3 values
+  static constexpr int B_CODES = NT * 2 * B_ATOM;                // 2 atoms (256 K) per term
+  static constexpr int B_STAGE = B_CODES + NT * 1024;            // + 2 scale atoms per term
+  static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;
+  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
+  // token-row stages: gemv<2>'s come from the a terms gemv<1> just wrote (L2)
+  static constexpr int SB = PHASE == 2 ? 2 : (B_STAGE <= 12 * 1024 ? 4 : 3);
+  static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_SMEM;
+  static constexpr int SA = SA_FIT > 8 ? 8 : SA_FIT;
+  static constexpr int A_RING = SA * A_SMEM;
+  static constexpr int B_RING = SB * B_STAGE;
+  static constexpr int N_BARS = 2 * SA + 2 * SB + 5;
+  static_assert(TN == 16 || TN == 32, "chunk width");
+  static_assert(A_SMEM % 1024 == 0 && B_STAGE % 1024 == 0 && B_ATOM % 1024 == 0, "1024-byte alignment");
+  static_assert(SA >= 3, "weight ring");
+  static_assert(FIXED + A_RING + B_RING <= kSmemBudget, "shared memory budget");
+  static_assert(SFB_COL + 8 * NT <= TMEM_COLS, "TMEM budget");
+  static_assert(N_BARS * 8 + 16 <= kBarBytes, "barrier area");
+};
+
+template <int PHASE, int TN>
+constexpr size_t smem_bytes(int E) {
+  using C = Cfg<PHASE, TN>;
+  return 1024 + static_cast<size_t>(C::A_RING) + C::B_RING + C::UP_BYTES + kBarBytes +
+         static_cast<size_t>(E + 1) * 4;
+}
+
+struct Unit {
+  int e, m, q0, nvalid;
+};
+
+template <int TN>
+__device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart, int u) {
+  int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ustart[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit U;
+  U.e = lo;
+  const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+  const int chunks = (ne + TN - 1) / TN;
+  const int local = u - ustart[lo];
+  U.m = local / chunks;
+  const int c = local % chunks;
+  U.q0 = q_begin + c * TN;
+  U.nvalid = min(TN, ne - c * TN);
+  return U;
+}
+
+// First byte of the blob tile (expert U.e, row tile U.m, k tile 0) of a phase.
+template <int PHASE>
+__device__ __forceinline__ const uint8_t* tile_base(const MxParams& P, const Unit& U) {
+  const int K = (PHASE == 1) ? P.d : P.I;
+  const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
+  return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / KSTAGE) * kMxTileBytes;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// gemv<1>'s producer, once its own tiles are all issued: L2 prefetches of the
+// first tiles of the gemv<2> units this CTA will run (same round-robin deal),
+// up to `budget` bytes.  gemv<2>'s units of expert e are tiles x chunks(e) like
+// gemv<1>'s, so ustart1 scales to the gemv<2> table.
+template <int TN>
+__device__ void prefetch_down_units(const MxParams& P, const int32_t* ustart1, int per1, size_t budget) {
+  const int per2 = P.d / TM, KS2 = P.I / KSTAGE;
+  const int n2 = ustart1[P.E] / per1 * per2;
+  for (int u = blockIdx.x; u < n2 && budget > 0; u += gridDim.x) {
+    int lo = 0, hi = P.E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ustart1[mid] / per1 * per2 <= u) lo = mid;
+      else hi = mid;
+    }
+    const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+    const int chunks = (ne + TN - 1) / TN;
+    const int m = (u - ustart1[lo] / per1 * per2) / chunks;
+    const uint8_t* base = P.pool + static_cast<size_t>(__ldg(P.slot + lo)) * P.blob_bytes + P.L.wd +
+                          static_cast<size_t>(m) * KS2 * kMxTileBytes;
+    for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
+      prefetch_l2(base + static_cast<size_t>(ks) * kMxTileBytes, kMxTileBytes);
+      budget = budget > static_cast<size_t>(kMxTileBytes) ? budget - kMxTileBytes : 0;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ E4M3 / E8M0 terms
+// E8M0 byte of the smallest power of two 2^e with amax <= 448 * 2^e (448 =
+// 1.75 * 2^8 is the largest E4M3 value), so that amax / 2^e rounds to a
+// finite E4M3; byte 0 (2^-127) for zero, subnormal or small amax.
+__device__ __forceinline__ uint32_t e8m0_for(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int be = static_cast<int>((b >> 23) & 255u);
+  if (be == 0) return 0u;
+  const int byte = be - 8 + ((b & 0x7fffffu) > 0x600000u ? 1 : 0);
+  return static_cast<uint32_t>(byte < 0 ? 0 : byte);
+}
+
+// 2^-(byte - 127) (exact, normal fp32 for byte <= 253)
+__device__ __forceinline__ float inv_pow2(uint32_t byte) { return __uint_as_float((254u - byte) << 23); }
+
+// v * 2^(byte - 127), exact for the E4M3 values v multiplies here
+__device__ __forceinline__ float times_pow2(float v, uint32_t byte) {
+  if (byte >= 1u) return v * __uint_as_float(byte << 23);
+  return (v * 5.421010862427522e-20f) * 1.0842021724855044e-19f;   // 2^-64 * 2^-63
+}
+
+// fp32 -> E4M3 byte, round to nearest even, saturating to +-448
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return r & 0xffu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h;
+  asm("{ .reg .b16 s; cvt.u16.u32 s, %1; cvt.rn.f16x2.e4m3x2 %0, s; }" : "=r"(h) : "r"(byte));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xffffu)));
+}
+
+// ------------------------------------------------------------------ split_x
+// One thread per 32-element block of a token row: NX E4M3 terms of the
+// bf16 values, each term with the E8M0 scale of the block's remaining maximum.
+__global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                         uint8_t* __restrict__ xq, uint8_t* __restrict__ xs) {
+  const int nb = d / 32;
+  const long long n = static_cast<long long>(T) * nb;
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(g / nb), b = static_cast<int>(g % nb);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d + 32 * b);
+    float r[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = __ldg(src + i);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        r[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        r[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    }
+#pragma unroll
+    for (int term = 0; term < NX; ++term) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(r[i]));
+      const uint32_t sb = e8m0_for(amax);
+      const float inv = inv_pow2(sb);
+      uint32_t packed[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) packed[i] = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t q = e4m3_rn(r[i] * inv);
+        packed[i >> 2] |= q << (8 * (i & 3));
+        r[i] -= times_pow2(e4m3_to_f32(q), sb);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(xq + (static_cast<size_t>(term) * T + t) * d + 32 * b);
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      xs[(static_cast<size_t>(term) * T + t) * nb + b] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ the GEMVs
+template <int PHASE>
+__device__ __forceinline__ int token_of(const MxParams& P, const Unit& U, int lane, int n_pairs) {
+  int tok = 0;
+  if (PHASE == 1 && lane < U.nvalid) {
+    const int p = __ldg(P.perm + U.q0 + lane);
+    if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
+    else tok = p / P.k;
+  }
+  return tok;
+}
+
+template <int TN>
+__device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
+  if (nvalid <= P.a_box_rows[0]) return 0;
+  return (TN == 16 || nvalid <= P.a_box_rows[1]) ? 1 : 2;
+}
+
+// Token-row terms of K stage ks of unit U into the B stage at sB, and their
+// E8M0 scale atoms after them: gemv<1> one-row TMA loads of the x planes
+// (lane q loads pair q0 + q), gemv<2> one box of a-plane rows per term.
+// The scale bytes are plain loads and shared-memory stores (rows past the
+// unit's pairs get 2^0, their MMA columns are never read); they are made
+// visible to the tensor core's async proxy before lane 0 arrives.  Called by
+// all lanes of one warp.
+template <class C, int PHASE, int TN>
+__device__ __forceinline__ void load_b(const MxParams& P, const Unit& U, int ks, int tok, uint8_t* sB,
+                                       uint64_t* bar, const CUtensorMap* tm_b, const CUtensorMap* tm_b16,
+                                       const CUtensorMap* tm_b8, uint64_t pol, int lane, int n_pairs) {
+  uint8_t* sf = sB + C::B_CODES;
+  if (lane < TN) {
+    const int K = PHASE == 1 ? P.d : P.I;
+    const int nb = K / 32;
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j) {
+      uint2 v = make_uint2(0x7f7f7f7fu, 0x7f7f7f7fu);
+      if (lane < U.nvalid) {
+        const size_t row = PHASE == 1 ? static_cast<size_t>(j) * P.T + tok
+                                      : static_cast<size_t>(j) * n_pairs + U.q0 + lane;
+        const uint8_t* src = (PHASE == 1 ? P.xs : P.as) + row * nb + 8 * ks;
+        v = *reinterpret_cast<const uint2*>(src);
+      }
+      *reinterpret_cast<uint32_t*>(sf + (2 * j) * 512 + lane * 16) = v.x;
+      *reinterpret_cast<uint32_t*>(sf + (2 * j + 1) * 512 + lane * 16) = v.y;
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid)
+                                   : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
+  if (lane == 0) mbar_expect_tx(bar, rows * C::NT * 2 * 128u);
+  __syncwarp();
+  if (PHASE == 2) {
+    if (lane == 0) {
+      const int bi = a_box<TN>(P, U.nvalid);
+      const CUtensorMap* tm = bi == 0 ? tm_b8 : (bi == 1 ? tm_b16 : tm_b);
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(sB + (2 * j + h) * C::B_ATOM, tm, bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
+    }
+  } else if (lane < U.nvalid) {
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, tm_b, bar, ks * KSTAGE + 128 * h, tok, j, pol);
+  }
+}
+
+__device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, int stage, uint32_t phase) {
+  const int outstanding = issued < n ? issued : n;
+  for (int i = 0; i < outstanding; ++i) {
+    if (--stage < 0) {
+      stage = n - 1;
+      phase ^= 1u;
+    }
+    mbar_drain(&full[stage], phase);
+  }
+}
+
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+      "[%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t tmem, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4: A = E2M1 (weights), B = E4M3
+// (activation terms), both K-major, E8M0 scales, M = 128, N = n; sf = the
+// byte of each 32-bit scale cell (the 32-element block within the atom's 4).
+__device__ __forceinline__ uint32_t idesc_mx(int n, uint32_t sf) {
+  return (sf << 4) | (5u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(TM >> 4) << 24) | (sf << 29);
+}
+
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                          uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %6, 0; "
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%4], [%5], p; }" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
+
+template <int PHASE, int TN>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemv_mx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_b16, const __grid_constant__ CUtensorMap tm_b8,
+                   MxParams P) {
+  using C = Cfg<PHASE, TN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring_b = smem + C::A_RING;
+  float* up_buf = reinterpret_cast<float*>(ring_b + C::B_RING);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_b + C::B_RING + C::UP_BYTES);
+  uint64_t* full = bars;                        // [SA] weight tile landed
+  uint64_t* empty = bars + C::SA;               // [SA] weight tile free
+  uint64_t* tfull = bars + 2 * C::SA;           // [2]
+  uint64_t* tempty = tfull + 2;                 // [2]
+  uint64_t* drain = tfull + 4;                  // [1]
+  uint64_t* bfull = tfull + 5;                  // [SB] token-row terms landed
+  uint64_t* bempty = bfull + C::SB;             // [SB] token-row terms free
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  int32_t* ustart = reinterpret_cast<int32_t*>(ring_b + C::B_RING + C::UP_BYTES + kBarBytes);
+  __shared__ int ws[36];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = (PHASE == 1) ? P.d : P.I;
+  const int KS = K / KSTAGE;
+  const int MT = (PHASE == 1) ? P.I / 64 : P.d / TM;
+  const int n_pairs = P.T * P.k;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
+    }
+    *abort_flag = 0;
+    *epi_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+
+  // ---- units per expert (evaluated experts only) and their exclusive prefix
+  const int per = (P.E + THREADS - 1) / THREADS;
+  const int e0 = threadIdx.x * per;
+  int cnt = 0;
+  for (int j = 0; j < per; ++j) {
+    const int e = e0 + j;
+    if (e >= P.E) break;
+    const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
+    if (b <= a) continue;
+    if (a < 0 || b > n_pairs) {
+      report(P.status, MOE_ERR_DEVICE);
+      continue;
+    }
+    const int s = __ldg(P.slot + e);
+    if (s >= P.n_slots) {
+      report(P.status, MOE_ERR_DEVICE);
+      continue;
+    }
+    if (s < 0) continue;
+    cnt += MT * ((b - a + TN - 1) / TN);
+  }
+  int total = 0;
+  int run = block_scan(cnt, ws, &total);
+  for (int j = 0; j < per; ++j) {
+    const int e = e0 + j;
+    if (e >= P.E) break;
+    ustart[e] = run;
+    const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
+    const int s = __ldg(P.slot + e);
+    if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * ((b - a + TN - 1) / TN);
+  }
+  if (threadIdx.x == 0) ustart[P.E] = total;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int n_units = total;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weight producer
+    const uint64_t pol_stream = policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
+    const uint8_t* pf_base = nullptr;
+    if (pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of<TN>(P, ustart, pf_u));
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit U = unit_of<TN>(P, ustart, u);
+      const int sl = __ldg(P.slot + U.e);
+      const uint8_t* abase = tile_base<PHASE>(P, U);
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag))) {
+          ok = false;
+          break;
+        }
+        uint8_t* sA = smem + stage * A_SMEM;
+        if (lane == 0) {
+          mbar_expect_tx(&full[stage], A_TX);
+          // codes: two boxes of 128 rows x 128 codes, expanded by the TMA into
+          // 16-byte slots; coordinates (k in tile, row, k tile, row tile, slot)
+          tma_load_5d(sA, &tm_w, &full[stage], 0, 0, ks, U.m, sl, pol_stream);
+          tma_load_5d(sA + A_BOX, &tm_w, &full[stage], 128, 0, ks, U.m, sl, pol_stream);
+          bulk_load(sA + 2 * A_BOX, abase + static_cast<size_t>(ks) * kMxTileBytes + 16384, 1024, &full[stage],
+                    pol_stream);
+          while (pf_u < n_units && pf_ahead < PF_ITEMS) {
+            prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * kMxTileBytes, kMxTileBytes);
+            ++pf_ahead;
+            if (++pf_ks == KS) {
+              pf_ks = 0;
+              pf_u += gridDim.x;
+              if (pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of<TN>(P, ustart, pf_u));
+            }
+          }
+          --pf_ahead;
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == C::SA) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<TN>(P, ustart, MT, 256u << 10);
+    __syncwarp();
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    drain_ring(full, C::SA, issued, stage, phase);
+  } else if (warp == BPROD_WARP) {
+    // ------------------------------------------------------------ token-row producer
+    const uint64_t pol_keep = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit U = unit_of<TN>(P, ustart, u);
+      const int tok = token_of<PHASE>(P, U, lane, n_pairs);
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag))) {
+          ok = false;
+          break;
+        }
+        load_b<C, PHASE, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &bfull[stage], &tm_b, &tm_b16, &tm_b8,
+                             pol_keep, lane, n_pairs);
+        __syncwarp();
+        ++issued;
+        if (++stage == C::SB) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    drain_ring(bfull, C::SB, issued, stage, phase);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int sb = 0, sa = 0;
+    uint32_t pb = 0, pa = 0;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
+      const Unit U = unit_of<TN>(P, ustart, u);
+      const int n_mma = U.nvalid <= 16 ? 16 : 32;
+      const int acc = it & 1;
+      if (!mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + acc * ACC_COLS;
+      for (int ks = 0; ks < KS; ++ks) {
+        if (!(mbar_wait<true>(&bfull[sb], pb, abort_flag) && mbar_wait<true>(&full[sa], pa, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint8_t* sA = smem + sa * A_SMEM;
+          const uint8_t* sB = ring_b + sb * C::B_STAGE;
+          // scale atoms -> TMEM: weights (2 atoms = 8 blocks of 32), then each term's
+          tc_cp_sf(tmem + SFA_COL, desc_sf(smem_u32(sA + 2 * A_BOX)));
+          tc_cp_sf(tmem + SFA_COL + 4, desc_sf(smem_u32(sA + 2 * A_BOX + 512)));
+#pragma unroll
+          for (int j = 0; j < C::NT; ++j) {
+            tc_cp_sf(tmem + SFB_COL + 8 * j, desc_sf(smem_u32(sB + C::B_CODES + (2 * j) * 512)));
+            tc_cp_sf(tmem + SFB_COL + 8 * j + 4, desc_sf(smem_u32(sB + C::B_CODES + (2 * j + 1) * 512)));
+          }
+#pragma unroll
+          for (int kk = 0; kk < KSTAGE / 32; ++kk) {   // K = 32 per MMA: +32 bytes of the expanded rows
+            const int h = kk >> 2, sub = kk & 3;
+            const uint64_t da = desc_sw128(smem_u32(sA + h * A_BOX)) + 2 * sub;
+            const uint32_t idesc = idesc_mx(n_mma, static_cast<uint32_t>(sub));
+#pragma unroll
+            for (int j = 0; j < C::NT; ++j) {
+              const uint64_t db = desc_sw128(smem_u32(sB + (2 * j + h) * C::B_ATOM)) + 2 * sub;
+              const uint32_t first = (ks > 0 || kk > 0 || j > 0) ? 1u : 0u;
+              tc_mma_mx(d_tmem, da, db, idesc, tmem + SFA_COL + 4 * h, tmem + SFB_COL + 8 * j + 4 * h, first);
+            }
+          }
+          tc_commit(&empty[sa]);
+          tc_commit(&bempty[sb]);
+        }
+        __syncwarp();
+        if (++sb == C::SB) {
+          sb = 0;
+          pb ^= 1u;
+        }
+        if (++sa == C::SA) {
+          sa = 0;
+          pa ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(&tfull[acc]);
+      __syncwarp();
+    }
+    if (!ok) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (elect_one()) tc_commit(drain);
+    __syncwarp();
+    mbar_drain(drain, 0);
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+      const Unit U = unit_of<TN>(P, ustart, u);
+      const int acc = it & 1;
+      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
+      named_sync(1, 128);
+      if (*epi_fail) {
+        report(P.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      float v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (PHASE == 1) {
+        // rows 0..63 of the tile are gate rows, 64..127 the matching up rows
+        if (quad >= 2) {
+          const int i = 32 * (quad - 2) + lane;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) up_buf[i * 33 + c] = v[c];
+        }
+        named_sync(1, 128);
+        if (quad < 2) {
+          // this warp's 32 lanes hold one 32-element block of I for every pair
+          const int i = 32 * quad + lane;
+          const size_t col = static_cast<size_t>(64) * U.m + i;
+          const size_t blk = static_cast<size_t>(2) * U.m + quad;
+          const int nbi = P.I / 32;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < U.nvalid) {
+              float r = silu(v[c]) * up_buf[i * 33 + c];
+              const size_t q = static_cast<size_t>(U.q0 + c);
+#pragma unroll
+              for (int j = 0; j < NA; ++j) {
+                const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r)));
+                const uint32_t sb = e8m0_for(__uint_as_float(amax));
+                const uint32_t t = e4m3_rn(r * inv_pow2(sb));
+                r -= times_pow2(e4m3_to_f32(t), sb);
+                const size_t plane = static_cast<size_t>(j) * n_pairs;
+                P.aq[(plane + q) * P.I + col] = static_cast<uint8_t>(t);
+                if (lane == 0) P.as[(plane + q) * nbi + blk] = static_cast<uint8_t>(sb);
+              }
+            }
+          }
+        }
+        named_sync(1, 128);
+      } else {
+        const int row = TM * U.m + 32 * quad + lane;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c < U.nvalid) {
+            const int q = U.q0 + c;
+            if (P.y_perm != nullptr) {
+              P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
+            } else {
+              const int p = __ldg(P.perm + q);
+              if (p >= 0 && p < n_pairs)
+                atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * v[c]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+template <int PHASE, int TN>
+moe_status launch_phase(const MxParams& P, const CUtensorMap& tw, const CUtensorMap& tb, const CUtensorMap& tb16,
+                        const CUtensorMap& tb8, const DeviceInfo& dev, cudaStream_t s) {
+  const size_t smem = smem_bytes<PHASE, TN>(P.E);
+  if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "MXFP4 decode GEMV needs %zu bytes of shared memory", smem);
+  static size_t attr[64] = {};
+  if (attr[dev.id] < smem) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(gemv_mx_kernel<PHASE, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(smem)));
+    attr[dev.id] = smem;
+  }
+  gemv_mx_kernel<PHASE, TN><<<dev.sm_count, THREADS, smem, s>>>(tw, tb, tb16, tb8, P);
+  MOE_LAUNCH_CHECK("gemv_mx_kernel");
+  return MOE_OK;
+}
+
+// 5-D map over the stage tiles of one matrix of every slot: (k within the
+// tile: 256 codes, row within the tile: 128, k tile, row tile, slot); the box
+// is 128 codes x 128 rows, each 16 codes expanded into a 16-byte slot.
+CUresult encode_weight_map(CUtensorMap* map, const uint8_t* region0, int K, int R, int n_slots,
+                           size_t blob_bytes) {
+  auto fn = encode_tiled_fn();
+  if (!fn) return CUDA_ERROR_NOT_FOUND;
+  const int KT = K / KSTAGE, RT = R / TM;
+  cuuint64_t gdim[5] = {static_cast<cuuint64_t>(KSTAGE), static_cast<cuuint64_t>(TM), static_cast<cuuint64_t>(KT),
+                        static_cast<cuuint64_t>(RT), static_cast<cuuint64_t>(n_slots)};
+  cuuint64_t gstr[4] = {128, static_cast<cuuint64_t>(kMxTileBytes),
+                        static_cast<cuuint64_t>(KT) * kMxTileBytes, static_cast<cuuint64_t>(blob_bytes)};
+  cuuint32_t box[5] = {128, static_cast<cuuint32_t>(TM), 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 5, const_cast<uint8_t*>(region0), gdim, gstr, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+struct MxWorkspace {
+  size_t xq, xs, aq, as, bytes;
+};
+
+MxWorkspace mx_workspace(moe_shape s, int T, int k) {
+  MxWorkspace W{};
+  const size_t n = static_cast<size_t>(T) * k;
+  size_t o = 0;
+  W.xq = o; o = round_up(o + static_cast<size_t>(NX) * T * s.d, 256);
+  W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 32), 256);
+  W.aq = o; o = round_up(o + static_cast<size_t>(NA) * n * s.I, 256);
+  W.as = o; o = round_up(o + static_cast<size_t>(NA) * n * (s.I / 32), 256);
+  W.bytes = o;
+  return W;
+}
+
+template <int TN>
+moe_status launch_both(const MxParams& P, const CUtensorMap& tw1, const CUtensorMap& tw2, const CUtensorMap& tx,
+                       const CUtensorMap (&ta)[3], const DeviceInfo& dev, cudaStream_t stream) {
+  moe_status st = launch_phase<1, TN>(P, tw1, tx, tx, tx, dev, stream);
+  if (st != MOE_OK) return st;
+  return launch_phase<2, TN>(P, tw2, ta[2], ta[1], ta[0], dev, stream);
+}
+
+}  // namespace
+
+size_t decode_mx_workspace_bytes(moe_shape s, int T, int k) { return mx_workspace(s, T, k).bytes; }
+
+// Split x, then both GEMV launches, for MXFP4 blobs in the stage-tiled layout.
+moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
+                            const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
+                            float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
+  const MxWorkspace W = mx_workspace(s, T, k);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  MxParams P{};
+  P.E = s.E;
+  P.d = s.d;
+  P.I = s.I;
+  P.T = T;
+  P.k = k;
+  P.n_slots = n_slots;
+  P.offsets = offsets;
+  P.perm = perm;
+  P.slot = slot;
+  P.gate = gate;
+  P.pool = static_cast<const uint8_t*>(pool);
+  P.L = blob_layout(s.fmt, s.d, s.I);
+  P.blob_bytes = P.L.bytes;
+  P.xs = w8 + W.xs;
+  P.aq = w8 + W.aq;
+  P.as = w8 + W.as;
+  P.y_perm = y_perm;
+  P.out = out;
+  P.status = status;
+  const uint64_t n = static_cast<uint64_t>(T) * k;
+  for (int i = 0; i < 3; ++i) {
+    const uint64_t r = static_cast<uint64_t>(8) << i;
+    P.a_box_rows[i] = static_cast<int>(n < r ? n : r);
+  }
+  CUtensorMap tw1, tw2, tx, ta[3];
+  CUresult r = encode_weight_map(&tw1, P.pool + P.L.wg, s.d, 2 * s.I, n_slots, P.blob_bytes);
+  if (r == CUDA_SUCCESS) r = encode_weight_map(&tw2, P.pool + P.L.wd, s.I, s.d, n_slots, P.blob_bytes);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the MXFP4 weights failed (%d)", static_cast<int>(r));
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T), static_cast<uint64_t>(NX)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T) * s.d};
+    const uint32_t box[3] = {128u, 1u, 1u};
+    r = encode_tiled_sw128(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
+  }
+  for (int i = 0; i < 3; ++i) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, static_cast<uint64_t>(NA)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.I), n * s.I};
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
+    r = encode_tiled_sw128(&ta[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a terms failed (%d)", static_cast<int>(r));
+  }
+  {
+    const long long blocks = static_cast<long long>(T) * (s.d / 32);
+    const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
+    mx_split_x_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq, w8 + W.xs);
+    MOE_LAUNCH_CHECK("mx_split_x_kernel");
+  }
+  return T <= 16 ? launch_both<16>(P, tw1, tw2, tx, ta, dev, stream) : launch_both<32>(P, tw1, tw2, tx, ta, dev, stream);
+}
+
+}  // namespace moe

@@ -1,48 +1,35 @@
-// Step 3 at decode sizes on the 5th-generation tensor cores
-// (moe_expert_ffn without MOE_FFN_ACT_NVFP4; bf16 blobs in the tile layout and
-// MXFP4 blobs in the stage-tiled layout): the grouped SwiGLU expert FFN as two
-// skinny GEMMs.
+// Step 3 at decode sizes on the 5th-generation tensor cores for bf16 blobs in
+// the tile layout (moe_expert_ffn without MOE_FFN_ACT_NVFP4): the grouped
+// SwiGLU expert FFN as two skinny GEMMs.  (MXFP4 blobs run on the block-scaled
+// kind in ffn_decode_mx.cu.)
 //
 // At decode sizes a layer call is bound by reading the routed experts' weights
 // from HBM (explainx.ai hardware guide, "Decode: decide whether to move an
 // expert or compute where it lives": one token touches few experts).  Bulk
-// copies move whole weight stages into shared memory and one thread issues
-// tcgen05.mma over them, the few token rows of a group being the N side and
-// the accumulators living in TMEM:
-//   bf16   the stage (128 rows x 128 elements, 32 KB) is the A operand as it
-//          lands; no SM instruction is spent per weight element.
-//   MXFP4  no tensor-core kind multiplies FP4 by a 16-bit operand, so eight
-//          converter warps turn each stage (128 rows x 256 elements, 17 KB) into
-//          exact f16 values -- cvt of E2M1 pairs, times the power-of-two E8M0
-//          block scale -- stored into TMEM, where the MMA reads A; the token
-//          rows are converted bf16 -> f16 in shared memory.  f16 holds every
-//          E2M1 x 2^X exactly for X in [-23, 13] and every bf16 activation below
-//          65504 in magnitude; a scale above, a scale below on a block with
-//          nonzero codes (blocks of zeros are exact at any scale), or an
-//          activation outside is reported as MOE_ERR_UNSUPPORTED in the status
-//          word.
+// copies move whole weight stages (128 rows x 128 elements, 32 KB) into shared
+// memory, where the stage is the A operand of tcgen05.mma as it lands -- no SM
+// instruction is spent per weight element; one thread issues the MMAs, the few
+// token rows of a group being the N side and the accumulators living in TMEM.
 //
 //   gemv<1>: D[128 x N] = W_gu tile (64 gate + 64 up rows of the same
 //            intermediate indices) x X^T over K = d, N <= 32 token rows
 //            gathered by one-row TMA loads of x.  Epilogue: a = silu(D_gate) *
-//            D_up, stored as two 16-bit planes hi + lo (a - hi - lo ~ 2^-17 |a|
-//            for bf16, ~2^-22 |a| for f16) in the workspace, rows = sorted pairs.
+//            D_up, stored as two bf16 planes hi + lo (a - hi - lo ~ 2^-17 |a|)
+//            in the workspace, rows = sorted pairs.
 //   gemv<2>: D[128 x N] = W_d tile x (A_hi + A_lo)^T over K = I (two MMAs per
 //            k-step).  Epilogue: y_perm rows, or out[t] += gate * y (the fused
 //            combine).
 //
-// Work unit = (expert, 128-row tile, chunk of <= TN of the expert's pairs; TN
-// = 16 when T <= 16, else 32), expert-major, chunks fastest, dealt round-robin
-// to one persistent CTA per SM.  Warp 0 produces the weight stages (bulk copy,
-// L2 prefetch four stages ahead), warp 1 owns TMEM and issues the MMAs,
-// [MXFP4: warps 2-9 convert], four warps run the epilogue on double-buffered
-// TMEM accumulators, and the last warp loads the token rows into a ring of
-// their own.  The weight ring takes the shared memory the rest leaves (bf16:
-// 5 stages of 32 KB; MXFP4: 10 / 9 stages of 17 KB for TN = 16), so that
-// the bf16 GEMVs keep enough bytes in flight to run near the HBM rate; the
-// MXFP4 ones are bound by the conversion unit that executes cvt.  Every
-// wait is bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing,
-// drains what it issued and frees its TMEM.
+// Work unit = (expert, 128-row tile, chunk of <= TN pairs; TN = 16 when T <=
+// 16, else 32), expert-major, chunks fastest, dealt round-robin to one
+// persistent CTA per SM.  Warp 0 produces the weight stages (bulk copy, L2
+// prefetch four stages ahead), warp 1 owns TMEM and issues the MMAs, four
+// warps run the epilogue on double-buffered TMEM accumulators, and the last
+// warp loads the token rows into a ring of their own.  The weight ring takes
+// the shared memory the rest leaves (5 stages of 32 KB), so that the GEMVs
+// keep enough bytes in flight to run near the HBM rate.  Every wait is
+// bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains
+// what it issued and frees its TMEM.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -61,7 +48,7 @@ struct TcDecodeParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  uint16_t* a_planes;        // [2][T*k][I] 16-bit (bf16 or f16): hi, lo
+  uint16_t* a_planes;        // [2][T*k][I] bf16: hi, lo
   float* y_perm;             // [T*k][d] or null (then out)
   float* out;                // [T][d] (fused combine)
   int32_t* status;
@@ -78,46 +65,38 @@ constexpr int kSmemBudget = 226 * 1024;  // opt-in shared memory of one CTA (227
 constexpr int kMaxE = 1024;              // experts the unit table is sized for
 constexpr int kBarBytes = 512;           // mbarriers, the TMEM address and two flags
 
-// Per (format, phase, chunk width) geometry.  TN = pairs per chunk (the MMA's
-// N is 16 or 32): 16 whenever T <= 16, since an expert holds at most one pair
-// per token, which halves the token-row buffers and frees room for weight stages.
+// Per (phase, chunk width) geometry.  TN = pairs per chunk (the MMA's N is 16
+// or 32): 16 whenever T <= 16, since an expert holds at most one pair per
+// token, which halves the token-row buffers and frees room for weight stages.
 //
 // Weight stages (SA) and token-row stages (SB) are separate rings, each with
 // its own producer warp, and the weight ring takes every byte the token rows
 // leave: the token rows come from L2 (x, or the a planes just written), so a
-// few stages cover them.  MXFP4: the converters free a weight stage as soon
-// as they have read it; bf16: the MMA frees both.
+// few stages cover them.  The MMA frees both.
 template <int FMT, int PHASE, int TN>
 struct Cfg {
-  static constexpr bool MX = (FMT == MOE_W_MXFP4);
-  static constexpr int KSTAGE = MX ? 256 : 128;                  // K elements per stage
+  static_assert(FMT == MOE_W_BF16, "bf16 blobs only");
+  static constexpr int KSTAGE = 128;                             // K elements per stage
   static constexpr int ATOMS = KSTAGE / 64;                      // B atoms per plane
   static constexpr int B_ATOM = TN * 128;                        // one 64-element atom of TN token rows
-  static constexpr int A_STAGE = MX ? kMxTileBytes : 2 * TM * 128;   // weight bytes per stage
+  static constexpr int A_STAGE = 2 * TM * 128;                   // weight bytes per stage
   static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
   static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
-  static constexpr int SB = MX ? (B_STAGE <= 8192 ? 5 : (B_STAGE >= 32768 ? 3 : 4))            // token-row stages
-                               : (B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3);
+  static constexpr int SB = B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3;   // token-row stages
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_STAGE;
-  static constexpr int SA = (!MX && TN == 16 && PHASE == 1) ? 5 : (SA_FIT > 12 ? 12 : SA_FIT);           // weight stages
+  static constexpr int SA = (TN == 16 && PHASE == 1) ? 5 : (SA_FIT > 12 ? 12 : SA_FIT);   // weight stages
   static constexpr int A_RING = SA * A_STAGE;
   static constexpr int B_RING = SB * B_STAGE;
-  static constexpr int CONV_PER_ROW = 2;                         // converter warps per TMEM lane quadrant
-  static constexpr int CONV_WARPS = MX ? 4 * CONV_PER_ROW : 0;
-  static constexpr int EPI_WARP0 = 2 + CONV_WARPS;
+  static constexpr int EPI_WARP0 = 2;
   static constexpr int BPROD_WARP = EPI_WARP0 + 4;               // the token-row producer
   static constexpr int THREADS = (EPI_WARP0 + 5) * 32;
-  static constexpr int ASLOTS = 3;                               // TMEM A buffers (MXFP4)
-  static constexpr int A_COL0 = 2 * ACC_COLS;                    // first TMEM column of the A buffers
-  static constexpr int A_COLS = KSTAGE / 2;                      // TMEM columns per A buffer
-  static constexpr int TMEM_COLS = MX ? 512 : 64;
-  static constexpr int N_BARS = 2 * SA + 2 * SB + 2 * ASLOTS + 5;
+  static constexpr int TMEM_COLS = 64;
+  static constexpr int N_BARS = 2 * SA + 2 * SB + 5;
   static_assert(TN == 16 || TN == 32, "chunk width");
   static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
   static_assert(FIXED + A_RING + B_RING <= kSmemBudget, "shared memory budget");
-  static_assert(!MX || A_COL0 + ASLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(N_BARS * 8 + 16 <= kBarBytes, "barrier area");
 };
 
@@ -197,66 +176,11 @@ __device__ void prefetch_down_units(const TcDecodeParams& P, const int32_t* usta
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
-// Four E2M1 pairs (the bytes of w, low byte first) -> four f16x2, exact.
-__device__ __forceinline__ void e2m1x8_f16x2(uint32_t w, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm("{ .reg .b8 b0, b1, b2, b3; mov.b32 {b0, b1, b2, b3}, %4;"
-      " cvt.rn.f16x2.e2m1x2 %0, b0; cvt.rn.f16x2.e2m1x2 %1, b1;"
-      " cvt.rn.f16x2.e2m1x2 %2, b2; cvt.rn.f16x2.e2m1x2 %3, b3; }"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-      : "r"(w));
-}
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// E8M0 scale byte -> 2^(byte - 127) as f16x2.  Exact for X = byte - 127 in
-// [-23, 13], where every E2M1 x 2^X is an f16.  Below, the products lie under
-// f16's smallest subnormal: the scale flushes to 0 and *tiny is set (exact for
-// an all-zero block, such as the ones encoded with byte 0); above, they would
-// overflow: false.
-__device__ __forceinline__ bool e8m0_f16x2(uint32_t byte, uint32_t* out, bool* tiny) {
-  const int x = static_cast<int>(byte) - 127;
-  *tiny = x < -23;
-  if (x < -23 || x > 13) {
-    *out = 0;
-    return x <= 13;
-  }
-  const uint32_t h = (x >= -14) ? static_cast<uint32_t>(x + 15) << 10 : 1u << (x + 24);
-  *out = h | (h << 16);
-  return true;
-}
-
-// 8 bf16 -> 8 f16 in place (one 16-byte chunk); false if one is beyond f16.
-__device__ __forceinline__ bool bf16x8_to_f16x8(uint4* p) {
-  uint4 v = *p;
-  uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  bool ok = true;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-    ok = ok && fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
-    const __half2 h = __floats2half2_rn(lo, hi);
-    w[i] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-  *p = make_uint4(w[0], w[1], w[2], w[3]);
-  return ok;
-}
-
-__device__ __forceinline__ void split16(float a, bool mx, uint16_t* hi, uint16_t* lo) {
-  if (mx) {
-    const __half h = __float2half_rn(a);
-    const __half l = __float2half_rn(a - __half2float(h));
-    *hi = __half_as_ushort(h);
-    *lo = __half_as_ushort(l);
-  } else {
-    const __nv_bfloat16 h = __float2bfloat16_rn(a);
-    const __nv_bfloat16 l = __float2bfloat16_rn(a - __bfloat162float(h));
-    *hi = __bfloat16_as_ushort(h);
-    *lo = __bfloat16_as_ushort(l);
-  }
+__device__ __forceinline__ void split_bf16(float a, uint16_t* hi, uint16_t* lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(a);
+  const __nv_bfloat16 l = __float2bfloat16_rn(a - __bfloat162float(h));
+  *hi = __bfloat16_as_ushort(h);
+  *lo = __bfloat16_as_ushort(l);
 }
 
 // gemv<1>: the token of each of the unit's pairs (lane q: pair q0 + q).
@@ -340,9 +264,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   uint64_t* tfull = bars + 2 * C::SA;           // [2]
   uint64_t* tempty = tfull + 2;                 // [2]
   uint64_t* drain = tfull + 4;                  // [1]
-  uint64_t* cvt_done = tfull + 5;               // [ASLOTS] (MXFP4)
-  uint64_t* afree = cvt_done + C::ASLOTS;       // [ASLOTS] (MXFP4)
-  uint64_t* bfull = afree + C::ASLOTS;          // [SB] token rows landed
+  uint64_t* bfull = tfull + 5;                  // [SB] token rows landed
   uint64_t* bempty = bfull + C::SB;             // [SB] token rows free
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -359,19 +281,13 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::SA; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::MX ? 32 * C::CONV_WARPS : 1);   // MXFP4: every converter thread has read it
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
-    if (C::MX) {
-      for (int a = 0; a < C::ASLOTS; ++a) {
-        mbar_init(&cvt_done[a], 32 * C::CONV_WARPS);
-        mbar_init(&afree[a], 1);
-      }
-    }
     for (int s = 0; s < C::SB; ++s) {
       mbar_init(&bfull[s], 1);
       mbar_init(&bempty[s], 1);
@@ -512,14 +428,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     drain_ring(bfull, C::SB, issued, stage, phase);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0, sa = 0;         // token-row ring; weight ring (bf16)
+    int stage = 0, sa = 0;         // token-row ring; weight ring
     uint32_t phase = 0, pa = 0;
-    int it = 0, j = 0;
+    int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       const Unit U = unit_of<TN>(P, ustart, MT, u);
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
-      const uint32_t idesc = C::MX ? idesc_f16(TM, n_mma) : idesc_bf16(TM, n_mma);
+      const uint32_t idesc = idesc_bf16(TM, n_mma);
       const int acc = it & 1;
       if (!mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
         ok = false;
@@ -527,20 +443,17 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
-      for (int ks = 0; ks < KS; ++ks, ++j) {
-        const int aslot = j % C::ASLOTS;
-        // the token rows have landed, and bf16: the weight stage; MXFP4: the
-        // A buffer is converted (phase 1: the token rows too)
+      for (int ks = 0; ks < KS; ++ks) {
+        // the token rows and the weight stage have landed
         const bool got = mbar_wait<true>(&bfull[stage], phase, abort_flag) &&
-                         (C::MX ? mbar_wait<true>(&cvt_done[aslot], (j / C::ASLOTS) & 1, abort_flag)
-                                : mbar_wait<true>(&full[sa], pa, abort_flag));
+                         mbar_wait<true>(&full[sa], pa, abort_flag);
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (elect_one()) {
-          const uint8_t* sA = smem + sa * C::A_STAGE;      // bf16
+          const uint8_t* sA = smem + sa * C::A_STAGE;
           const uint8_t* sB = ring_b + stage * C::B_STAGE;
 #pragma unroll
           for (int kk = 0; kk < C::KSTAGE / 16; ++kk) {   // K = 16 per MMA: +32 bytes
@@ -548,17 +461,11 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
             const uint64_t dh = desc_sw128(smem_u32(sB + a * C::B_ATOM)) + 2 * (kk & 3);
             const uint64_t dl = desc_sw128(smem_u32(sB + (C::ATOMS + a) * C::B_ATOM)) + 2 * (kk & 3);
             const uint32_t first = (ks > 0 || kk > 0) ? 1u : 0u;
-            if (C::MX) {
-              const uint32_t ta = tmem + C::A_COL0 + aslot * C::A_COLS + 8 * kk;
-              tc_mma_f16_ts(d_tmem, ta, dh, idesc, first);
-              if (PHASE == 2) tc_mma_f16_ts(d_tmem, ta, dl, idesc, 1u);
-            } else {
-              const uint64_t da = desc_sw128(smem_u32(sA + a * TM * 128)) + 2 * (kk & 3);
-              tc_mma_bf16(d_tmem, da, dh, idesc, first);
-              if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
-            }
+            const uint64_t da = desc_sw128(smem_u32(sA + a * TM * 128)) + 2 * (kk & 3);
+            tc_mma_bf16(d_tmem, da, dh, idesc, first);
+            if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
           }
-          tc_commit(C::MX ? &afree[aslot] : &empty[sa]);
+          tc_commit(&empty[sa]);
           tc_commit(&bempty[stage]);
         }
         __syncwarp();
@@ -582,104 +489,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     if (elect_one()) tc_commit(drain);
     __syncwarp();
     mbar_drain(drain, 0);
-  } else if (warp < C::EPI_WARP0) {
-    // ------------------------------------------------------------ MXFP4 converters (warps 2..9)
-    if constexpr (C::MX) {
-    const int quad = warp & 3;
-    const int r = 32 * quad + lane;                 // tile row = TMEM lane
-    constexpr int CPR = C::CONV_PER_ROW;            // warps sharing a row's 256 elements
-    constexpr int CH = 8 / CPR;                     // 16-byte chunks (32 elements) per warp
-    const int part = (warp - 2) >> 2;               // this warp's part of the row
-    const int ct = threadIdx.x - 64;                // 0..255
-    bool ok = true;
-    bool range_ok = true;
-    int j = 0, sa = 0, sb = 0;
-    uint32_t pa = 0, pb = 0;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of<TN>(P, ustart, MT, u);
-      for (int ks = 0; ks < KS; ++ks, ++j) {
-        const int aslot = j % C::ASLOTS;
-        if (!mbar_wait<true>(&full[sa], pa, abort_flag) ||
-            !mbar_wait<true>(&afree[aslot], ((j / C::ASLOTS) & 1) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint8_t* sA = smem + sa * C::A_STAGE;
-        const uint2 sc2 = *reinterpret_cast<const uint2*>(sA + 16384 + r * 8);
-        const uint32_t taddr =
-            tmem + (static_cast<uint32_t>(32 * quad) << 16) + C::A_COL0 + aslot * C::A_COLS + 16 * CH * part;
-        {
-          // chunks CH part .. CH part + CH - 1 of the row: 32 CH elements -> 16 CH columns
-          uint4 q[CH];
-#pragma unroll
-          for (int cc = 0; cc < CH; ++cc) {
-            const int c = CH * part + cc;
-            q[cc] = *reinterpret_cast<const uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4));
-          }
-          uint32_t v[16 * CH];
-#pragma unroll
-          for (int cc = 0; cc < CH; ++cc) {
-            const int c = CH * part + cc;
-            uint32_t scl;
-            bool tiny;
-            range_ok &= e8m0_f16x2(((c < 4 ? sc2.x : sc2.y) >> (8 * (c & 3))) & 0xffu, &scl, &tiny);
-            // a flushed scale is exact only for a block of zeros (E2M1 magnitude bits 0)
-            if (tiny) range_ok &= ((q[cc].x | q[cc].y | q[cc].z | q[cc].w) & 0x77777777u) == 0u;
-            const uint32_t w[4] = {q[cc].x, q[cc].y, q[cc].z, q[cc].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint32_t h0, h1, h2, h3;
-              e2m1x8_f16x2(w[i], h0, h1, h2, h3);
-              v[16 * cc + 4 * i + 0] = hmul2(h0, scl);
-              v[16 * cc + 4 * i + 1] = hmul2(h1, scl);
-              v[16 * cc + 4 * i + 2] = hmul2(h2, scl);
-              v[16 * cc + 4 * i + 3] = hmul2(h3, scl);
-            }
-          }
-          // every value read from the stage is in registers: hand it back to the producer
-          mbar_arrive(&empty[sa]);
-          if constexpr (CH == 4) tmem_st64(taddr, v);
-          else tmem_st32(taddr, v);
-        }
-        if (PHASE == 1) {
-          // token rows bf16 -> f16 in place (the swizzle only moves whole chunks)
-          if (!mbar_wait<true>(&bfull[sb], pb, abort_flag)) {
-            tmem_wait_st();
-            ok = false;
-            break;
-          }
-          uint8_t* sB = ring_b + sb * C::B_STAGE;
-          const int n_chunks = U.nvalid * C::ATOMS * 8;
-          for (int idx = ct; idx < n_chunks; idx += 32 * C::CONV_WARPS) {
-            const int rr = idx / (C::ATOMS * 8), rem = idx % (C::ATOMS * 8);
-            range_ok &= bf16x8_to_f16x8(reinterpret_cast<uint4*>(sB + (rem >> 3) * C::B_ATOM + rr * 128 + (rem & 7) * 16));
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&cvt_done[aslot]);
-        if (++sa == C::SA) {
-          sa = 0;
-          pa ^= 1u;
-        }
-        if (++sb == C::SB) {
-          sb = 0;
-          pb ^= 1u;
-        }
-      }
-    }
-    if (!range_ok) report(P.status, MOE_ERR_UNSUPPORTED);
-    if (!ok) {
-      report(P.status, MOE_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    }
   } else {
     // ------------------------------------------------------------ epilogue (last four warps)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
-    bool range_ok = true;
     int it = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
       const Unit U = unit_of<TN>(P, ustart, MT, u);
@@ -713,9 +525,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
           for (int c = 0; c < 32; ++c) {
             if (c < U.nvalid) {
               const float a = silu(v[c]) * up_buf[i * 33 + c];
-              if (C::MX) range_ok &= fabsf(a) <= 65504.f;
               uint16_t hi, lo;
-              split16(a, C::MX, &hi, &lo);
+              split_bf16(a, &hi, &lo);
               const size_t o = static_cast<size_t>(U.q0 + c) * P.I + col;
               P.a_planes[o] = hi;
               P.a_planes[plane + o] = lo;
@@ -740,7 +551,6 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
         }
       }
     }
-    if (!range_ok) report(P.status, MOE_ERR_UNSUPPORTED);
   }
   tc_fence_before();
   __syncthreads();
@@ -776,8 +586,8 @@ moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const C
 
 }  // namespace
 
-// Both GEMV launches for bf16 blobs in the tile layout or MXFP4 blobs in the
-// stage-tiled layout.  ws holds the a planes (T*k*I*4 bytes).
+// Both GEMV launches for bf16 blobs in the tile layout.  ws holds the a
+// planes (T*k*I*4 bytes).
 moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,
                             const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
@@ -816,15 +626,10 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
     const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, 2};
     const uint64_t str[2] = {static_cast<uint64_t>(s.I) * 2, n * s.I * 2};
     const uint32_t box[3] = {64u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
-    const CUtensorMapDataType type =
-        s.fmt == MOE_W_MXFP4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const CUresult r = encode_tiled_sw128(&tm_a[i], type, 3, ws, dims, str, box);
+    const CUresult r = encode_tiled_sw128(&tm_a[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ws, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a planes failed (%d)", static_cast<int>(r));
   }
   // an expert holds at most one pair per token: with T <= 16 every chunk fits 16 rows
-  if (s.fmt == MOE_W_MXFP4)
-    return T <= 16 ? launch_both<MOE_W_MXFP4, 16>(P, tm_x, tm_a, dev, stream)
-                   : launch_both<MOE_W_MXFP4, 32>(P, tm_x, tm_a, dev, stream);
   return T <= 16 ? launch_both<MOE_W_BF16, 16>(P, tm_x, tm_a, dev, stream)
                  : launch_both<MOE_W_BF16, 32>(P, tm_x, tm_a, dev, stream);
 }

@@ -113,8 +113,8 @@ extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* w
   }
   MOE_REQUIRE(sg && su && sd, "null scale pointer for an FP4 format");
   if (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)) {
-    // stage tiles: 16-byte code chunks to their swizzled places, 8 scales per
-    // row and tile
+    // stage tiles: 16-byte code chunks to their rows, scale bytes into the
+    // tiles' scale-factor atoms
     const uint8_t* cg = static_cast<const uint8_t*>(wg);
     const uint8_t* cu = static_cast<const uint8_t*>(wu);
     const uint8_t* cd = static_cast<const uint8_t*>(wd);
@@ -124,16 +124,16 @@ extern "C" moe_status moe_pack_expert(moe_shape s, const void* wg, const void* w
         std::memcpy(b + L.wg + mx_tile_code_offset(rg, bb, s.d), cg + static_cast<size_t>(i) * (s.d / 2) + bb, 16);
         std::memcpy(b + L.wg + mx_tile_code_offset(ru, bb, s.d), cu + static_cast<size_t>(i) * (s.d / 2) + bb, 16);
       }
-      for (int j = 0; j < s.d / 32; j += 8) {
-        std::memcpy(b + L.wg + mx_tile_scale_offset(rg, j, s.d), sg + static_cast<size_t>(i) * (s.d / 32) + j, 8);
-        std::memcpy(b + L.wg + mx_tile_scale_offset(ru, j, s.d), su + static_cast<size_t>(i) * (s.d / 32) + j, 8);
+      for (int j = 0; j < s.d / 32; ++j) {
+        b[L.wg + mx_tile_scale_offset(rg, j, s.d)] = sg[static_cast<size_t>(i) * (s.d / 32) + j];
+        b[L.wg + mx_tile_scale_offset(ru, j, s.d)] = su[static_cast<size_t>(i) * (s.d / 32) + j];
       }
     }
     for (int r = 0; r < s.d; ++r) {
       for (int bb = 0; bb < s.I / 2; bb += 16)
         std::memcpy(b + L.wd + mx_tile_code_offset(r, bb, s.I), cd + static_cast<size_t>(r) * (s.I / 2) + bb, 16);
-      for (int j = 0; j < s.I / 32; j += 8)
-        std::memcpy(b + L.wd + mx_tile_scale_offset(r, j, s.I), sd + static_cast<size_t>(r) * (s.I / 32) + j, 8);
+      for (int j = 0; j < s.I / 32; ++j)
+        b[L.wd + mx_tile_scale_offset(r, j, s.I)] = sd[static_cast<size_t>(r) * (s.I / 32) + j];
     }
     return MOE_OK;
   }

@@ -312,6 +312,45 @@ moe_status moe_cache_query(const moe_cache* c, int32_t* slot_of_expert,
 moe_status moe_cache_destroy(moe_cache* c);
 
 /* ------------------------------------------------------------------------ */
+/* The host share of a split step (host only, no device call): the SwiGLU FFN
+ * of the experts the q split leaves on the host, run on the CPU cores against
+ * their blobs in the host pool, concurrently with the fills of the GPU share
+ * (explainx.ai hardware guide, "Decode: decide whether to move an expert or
+ * compute where it lives"; freetoken.wiki "FreeToken 753b model", mechanism
+ * table, "Bandwidth-adaptive execution").
+ *   host_pool: E blobs in expert order (as for moe_cache_create), any host
+ *     memory (pinned or not).
+ *   experts: n_experts ids in [0, E) (duplicates ignored; an expert no token
+ *     selected costs nothing).
+ *   x: host bf16 [T][d]; idx: host int32 [T][k]; gate: host fp32 [T][k] (the
+ *     step's routing, e.g. copied back from moe_route_topk).
+ *   out: host fp32 [T][d], overwritten with sum over pairs (t, j) whose expert
+ *     is listed of gate[t][j] * SwiGLU_{idx[t][j]}(x[t]) -- the host_partial
+ *     of moe_combine_merge.  fp32 arithmetic.
+ *   n_threads: worker threads (<= 0: one per hardware thread); the call
+ *     blocks until the sum is done.  Calls from several threads run one at a
+ *     time.
+ * Errors: MOE_ERR_INVALID_ARG for a bad shape, id or null pointer. */
+moe_status moe_host_expert_ffn(moe_shape s, const void* host_pool, const int32_t* experts, int n_experts,
+                               const void* x, const int32_t* idx, const float* gate, int T, int k, float* out,
+                               int n_threads);
+
+/* The two bandwidths the q* split balances, measured on this machine
+ * (freetoken.wiki "FreeToken 753b model", "Measure System Bandwidth"):
+ *   *h2d_gbs: pinned host -> device copy rate of whole blobs: n_blobs
+ *     cudaMemcpyAsync copies from host_pool into dev_buf (device, 256-byte
+ *     aligned, >= one blob; blobs cycle through its dev_bytes) on `stream`,
+ *     timed with CUDA events after one warm-up copy.  dev_buf NULL: skipped
+ *     (0).  The call synchronises the stream.
+ *   *host_gbs: the host expert kernel's weight bytes per second over the
+ *     first n_blobs experts of host_pool (one token each, n_threads threads,
+ *     after one warm-up expert).
+ * GB = 1e9 bytes.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_CUDA. */
+moe_status moe_profile_bandwidth(moe_shape s, const void* host_pool, int n_blobs, void* dev_buf,
+                                 size_t dev_bytes, int n_threads, cudaStream_t stream, double* h2d_gbs,
+                                 double* host_gbs);
+
+/* ------------------------------------------------------------------------ */
 /* Synchronises `stream`, reads the device status word written by kernels,
  * resets it to 0 and returns it as a moe_status (MOE_OK if it was 0). */
 moe_status moe_check_status(int32_t* dev_status, cudaStream_t stream);

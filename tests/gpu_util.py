@@ -82,3 +82,47 @@ class Built:
         out = self.layer.forward(self.logits.cuda(), self.x.cuda(), host_partial=host_partial)
         torch.cuda.synchronize()
         return out
+
+
+# ---------------------------------------------------------------- pooled oracle
+# The float64 oracle costs ~1.3 s per full-size expert (dequantisation), so
+# full-size checks split the experts into subsets, run moe_layer on each
+# subset in a spawned worker, and add the subset outputs: the layer is the sum
+# of its expert subsets (the split invariance the oracle is pinned to).  The
+# canonical weights reach the workers as .npy files mapped read-only.
+
+def _np_of(t):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    return t.numpy()
+
+
+def _oracle_subset(args):
+    wdir, keys, fmt, pos, x, logits, k, experts, act = args
+    from threadpoolctl import threadpool_limits
+    w = {key: np.load(f"{wdir}/{key}.npy", mmap_mode="r") for key in keys}
+    with threadpool_limits(1):
+        return M.moe_layer(x, logits, k, lambda e: M.dequant_expert(fmt, w, pos[e]), experts=experts,
+                           act=act)["out"]
+
+
+def pooled_oracle(x, logits, k, fmt, w_cpu, pos, experts, act="none", workers=None):
+    """moe_layer(x, logits, k, ...)["out"] over `experts`, whose canonical
+    weights sit at w_cpu[key][pos[e]], computed by a spawn pool."""
+    import multiprocessing as mp
+    import os
+    import tempfile
+    experts = sorted(int(e) for e in experts)
+    n = workers or max(1, min(16, len(os.sched_getaffinity(0))))
+    chunks = [experts[i::n] for i in range(n) if experts[i::n]]
+    x = np.asarray(x, dtype=np.float64)
+    logits = np.asarray(logits, dtype=np.float32)
+    with tempfile.TemporaryDirectory() as wdir:
+        keys = list(w_cpu.keys())
+        for key in keys:
+            np.save(f"{wdir}/{key}.npy", _np_of(w_cpu[key]))
+        args = [(wdir, keys, fmt, dict(pos), x, logits, k, c, act) for c in chunks]
+        with mp.get_context("spawn").Pool(len(chunks)) as pool:
+            outs = pool.map(_oracle_subset, args)
+    return np.sum(outs, axis=0)

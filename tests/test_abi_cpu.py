@@ -209,8 +209,9 @@ def test_pack_mxfp4_tiled_layout(moe):
     """MXFP4 blobs with d, I multiples of 256 hold W_gu (gate and up rows
     interleaved in blocks of 64) and then W_d as tiles of 128 rows x 256
     elements ordered [row / 128][k / 256], 17408 bytes each: the codes (row r
-    = a 128-byte line, 16-byte chunk c at chunk position c ^ (r % 8)), then
-    the 8 E8M0 scales of each row."""
+    = the 128 bytes at 128 r, unswizzled), then the E8M0 scales as two
+    tensor-core scale-factor atoms (32-element block j of the tile in atom
+    j // 4; row r at (r % 32) * 16 + (r // 32) * 4 + j % 4)."""
     from expert_offload_serving_b200.layer import pack_pool
     cfg = synth.LayerConfig("mxt", E=1, k=1, d=512, I=256, fmt="mxfp4")
     w = synth.make_experts(cfg, range(1), seed=6)
@@ -225,10 +226,10 @@ def test_pack_mxfp4_tiled_layout(moe):
         for r in range(R):
             rr = r % 128
             tile = (r // 128) * (K // 256) + b // 128
-            bb = b % 128
-            codes[r] = region[tile * tile_bytes + rr * 128 + (((bb // 16) ^ (rr % 8)) * 16) + bb % 16]
+            codes[r] = region[tile * tile_bytes + rr * 128 + b % 128]
             stile = (r // 128) * (K // 256) + jj // 8
-            scales[r] = region[stile * tile_bytes + 16384 + rr * 8 + jj % 8]
+            j8 = jj % 8
+            scales[r] = region[stile * tile_bytes + 16384 + (j8 // 4) * 512 + (rr % 32) * 16 + (rr // 32) * 4 + j8 % 4]
         return codes, scales
 
     gu_bytes = 2 * cfg.I * (cfg.d // 2 + cfg.d // 32)
