@@ -451,6 +451,9 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg, T)
 
+    streamed = None
+    if not args.no_prefill and not args.no_cached and world == 1:
+        streamed = run_streamed_prefill()
     prefill = None
     if not args.no_prefill:
         prefill = run_prefill(Ts=(4096,) if (args.no_sweep or world > 1) else (4096, 16384, 32768),
@@ -469,10 +472,13 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
         cmx = synth.CONFIGS["decode_mxfp4"]
         mx = {f"T{t}": decode_point(cmx, t, 8, args.warmup, min(args.steps, 1000), stream, routed_only=True)
               for t in cmx.T}
-    cached = None
+    cached = split = layered = None
     if not args.no_cached:
         hp = cached_host_pool()
         cached = [run_cached_decode(hp, T=t) for t in (1, 8)]
+        if world == 1:
+            split = run_split_sweep(hp)
+            layered = run_layered_cache(hp)
         del hp
 
     result = {
@@ -527,6 +533,12 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
             result["prefill_T_sweep"] = prefill[1:]
     if cached is not None:
         result["decode_mxfp4_cached"] = cached
+    if split is not None:
+        result["split_merge_q_sweep"] = split
+    if layered is not None:
+        result["layered_cache"] = layered
+    if streamed is not None:
+        result["prefill_streamed"] = streamed
     if sweep:
         result["decode_bf16_T_sweep"] = sweep
     if mx:
@@ -616,6 +628,67 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
     return out
 
 
+# ---------------------------------------------------------------- prefill streamed from host memory
+def run_streamed_prefill(Ts=(4096, 8192, 16384), n_layers=4, reps=2):
+    """Prefill through n_layers NVFP4 layers (E=256, k=6, d=4096, I=2048)
+    whose 3.6 GB expert pools stay in pinned host memory (every layer reads
+    the same pool here; its bytes cross PCIe once per layer either way): each
+    layer's pool is copied into one of two full-layer device buffers while
+    the GPU computes the previous layer from the other, against the same
+    layers with each copy issued only after the previous compute (the pages'
+    ablation of double buffering).  Device-timed per chunk of T tokens."""
+    import expert_offload_serving_b200 as moe
+    from expert_offload_serving_b200.layer import StreamedPrefill, pack_pool
+    cfg = synth.CONFIGS["prefill_nvfp4"]
+    w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
+    host = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, {k: v.cpu() for k, v in w.items()}, range(cfg.E), pin=True)
+    del w
+    sp = StreamedPrefill(cfg.E, cfg.d, cfg.I, cfg.k, max(Ts), [host] * n_layers)
+    B = host.numel()
+    rows = []
+    st = torch.cuda.current_stream()
+    for T in Ts:
+        inputs = []
+        for l in range(n_layers):
+            lg, x = synth.make_routing(cfg, T, 700 + l)
+            inputs.append((lg.cuda(), x.cuda()))
+        r = {"T": T}
+        for mode in (True, False):
+            sp.run(inputs, double_buffer=mode)          # warm-up
+            times = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st)
+                sp.copy.wait_event(a)
+                sp.run(inputs, double_buffer=mode)
+                st.wait_stream(sp.copy)
+                b.record(st)
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            ms = statistics.median(times)
+            r["double_buffered" if mode else "serial"] = {
+                "ms_per_chunk": round(ms, 3), "tokens_per_s": round(T / (ms / 1e3), 1),
+                "h2d_gbs": round(n_layers * B / (ms / 1e3) / 1e9, 1)}
+        # the compute alone: the layers run from a buffer already on the device
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for l in range(n_layers):
+            sp.layers[0].forward(*inputs[l])
+        b.record(st)
+        torch.cuda.synchronize()
+        r["compute_only_ms"] = round(a.elapsed_time(b), 3)
+        db, se = r["double_buffered"]["tokens_per_s"], r["serial"]["tokens_per_s"]
+        r["throughput_loss_without_double_buffering"] = round(1.0 - se / db, 4)
+        rows.append(r)
+        del inputs
+    for L_ in sp.layers:
+        moe.moe_check_status(L_.status)
+    del sp, host
+    return {"workload": f"prefill_nvfp4 x {n_layers} layers: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I}, each layer's "
+                        "3.6 GB pool streamed from pinned host memory into two full-layer buffers",
+            "timing": f"median of {reps} device-timed passes over the {n_layers} layers", "chunks": rows}
+
+
 # ---------------------------------------------------------------- decode with the expert cache
 def cached_host_pool():
     """The 256 MXFP4 experts of the cached-decode workload, packed into one
@@ -685,6 +758,193 @@ def run_cached_decode(host_pool, T=1, steps=64, warm=32):
         "fill_mb_per_step": round(misses / steps * B / 1e6, 2),
         "h2d_pinned_gbs": round(h2d_gbs, 1),
         "steps": steps,
+    }
+
+
+# ---------------------------------------------------------------- one cache shared by many layers
+def _route_on_gpu(cfg, trace, k):
+    """Routing of a trace through moe_route_topk (device), read back."""
+    import expert_offload_serving_b200 as moe
+    lg = torch.cat([l for l, _ in trace]).cuda()
+    idx = torch.empty((lg.shape[0], k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((lg.shape[0], k), dtype=torch.float32, device="cuda")
+    moe.moe_route_topk(lg, k, idx, gate)
+    return idx.cpu().numpy()
+
+
+def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, sim_steps=128,
+                      n_gpu_layers=4, gpu_slots=64, steps=48, warm=16):
+    """The pages' global LRU (one expert cache whose decisions are shared by
+    all MoE layers) against per-layer caches of equal total capacity.
+    (a) Miss rates from the cache planner alone (plan-only handles) for
+        n_sim_layers layers (43, DeepSeek-V4-Flash's depth) of E=256, k=6
+        experts, T=1 decode: per-layer routing traces with their own AR(1)
+        drifting bias and bias spreads 0.25 ... 1.5 across layers (layers with
+        sharper routing need fewer slots), each layer's routing from
+        moe_route_topk.
+    (b) On the GPU: n_gpu_layers MXFP4 layers (E=256, d=4096, I=2048) over one
+        pinned host pool, gpu_slots slots in one shared cache vs gpu_slots /
+        n_gpu_layers per layer: step time for all layers and miss rate.
+    (c) Elastic resize of the shared cache: gpu_slots -> gpu_slots/2 -> gpu_slots
+        on a full cache, device-timed (moves only, no host copy)."""
+    import expert_offload_serving_b200 as moe
+    from expert_offload_serving_b200.layer import ExpertCache, MoeLayer
+    base = synth.CONFIGS["decode_mxfp4"]
+    s = moe.shape(base.E, base.d, base.I, base.fmt)
+    # (a) planner-only miss rates
+    spreads = np.linspace(0.25, 1.5, n_sim_layers)
+    idxs = []
+    for l in range(n_sim_layers):
+        cfg_l = dataclasses.replace(base, bias_std=float(spreads[l]))
+        idxs.append(_route_on_gpu(cfg_l, synth.make_trace(cfg_l, T_sim, steps=sim_steps, seed=300 + l), base.k))
+    glob = moe.MoeCache(s, n_sim_layers * slots_per_layer, n_layers=n_sim_layers)
+    per = [moe.MoeCache(s, slots_per_layer) for _ in range(n_sim_layers)]
+    acc = {"global": [0, 0], "per_layer": [0, 0]}
+    for t in range(sim_steps):
+        for l in range(n_sim_layers):
+            U = sorted(set(idxs[l][t * T_sim:(t + 1) * T_sim].ravel().tolist()))
+            clock = t * n_sim_layers + l
+            fg = glob.fill(U, clock, protect=U, layer=l)
+            fp = per[l].fill(U, t, protect=U)
+            if t >= sim_steps // 4:                     # after the cold start
+                acc["global"][0] += len(fg)
+                acc["per_layer"][0] += len(fp)
+                acc["global"][1] += len(U)
+                acc["per_layer"][1] += len(U)
+    glob.close()
+    for c in per:
+        c.close()
+    sim = {k: round(v[0] / v[1], 4) for k, v in acc.items()}
+    # (b) GPU step time with the cache shared or split
+    res_gpu = {}
+    for mode in ("global", "per_layer"):
+        for T in (1, 8):
+            torch.cuda.synchronize()
+            if mode == "global":
+                caches = [ExpertCache(s, gpu_slots, [host_pool] * n_gpu_layers)]
+                layers = [MoeLayer(s.E, s.d, s.I, base.fmt, base.k, T, cache=caches[0], layer_id=l)
+                          for l in range(n_gpu_layers)]
+            else:
+                caches = [ExpertCache(s, gpu_slots // n_gpu_layers, host_pool) for _ in range(n_gpu_layers)]
+                layers = [MoeLayer(s.E, s.d, s.I, base.fmt, base.k, T, cache=caches[l], layer_id=0)
+                          for l in range(n_gpu_layers)]
+            traces = [synth.make_trace(dataclasses.replace(base, bias_std=float(0.25 + 1.25 * l / 3)), T,
+                                       steps=warm + steps, seed=400 + l) for l in range(n_gpu_layers)]
+            idx_h = [_route_on_gpu(base, tr, base.k) for tr in traces]
+            lgs = [[lg.cuda() for lg, _ in tr] for tr in traces]
+            xs = [[x.cuda() for _, x in tr] for tr in traces]
+            misses = looked = 0
+            st = torch.cuda.current_stream()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for t in range(warm + steps):
+                if t == warm:
+                    e0.record(st)
+                for l in range(n_gpu_layers):
+                    U = sorted(set(idx_h[l][t * T:(t + 1) * T].ravel().tolist()))
+                    clock = t * n_gpu_layers + l if mode == "global" else t
+                    f = layers[l].prepare(clock, U, protect=U)
+                    layers[l].forward(lgs[l][t], xs[l][t])
+                    if t >= warm:
+                        misses += len(f)
+                        looked += len(U)
+            e1.record(st)
+            torch.cuda.synchronize()
+            for L_ in layers:
+                moe.moe_check_status(L_.status)
+            ms = e0.elapsed_time(e1) / steps
+            res_gpu[f"{mode}_T{T}"] = {"ms_per_step_all_layers": round(ms, 4), "miss_rate": round(misses / looked, 4)}
+            # (c) resize timing on the full shared cache
+            if mode == "global" and T == 8:
+                rs = []
+                for n in (gpu_slots // 2, gpu_slots):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(st)
+                    kept = caches[0].resize(n)
+                    b.record(st)
+                    torch.cuda.synchronize()
+                    rs.append({"to_slots": n, "kept": len(kept), "ms": round(a.elapsed_time(b), 4),
+                               "moved_gb": round(len(kept) * host_pool.shape[1] / 1e9, 3)})
+                res_gpu["resize"] = rs
+            for c in caches:
+                c.close()
+            del layers, caches, lgs, xs
+    return {
+        "planner_miss_rate": {
+            "workload": f"{n_sim_layers} layers x E={base.E} k={base.k}, T={T_sim}, {sim_steps} steps (first quarter "
+                        f"excluded), AR(1) routing bias per layer, spreads 0.25..1.5; capacity "
+                        f"{n_sim_layers * slots_per_layer} slots: global vs {slots_per_layer} per layer",
+            **sim},
+        "gpu": {"workload": f"{n_gpu_layers} MXFP4 layers (E={base.E} d={base.d} I={base.I} k={base.k}) over one pinned "
+                            f"host pool; {gpu_slots} slots shared vs {gpu_slots // n_gpu_layers} per layer; "
+                            f"{steps} steps after {warm}", **res_gpu},
+    }
+
+
+# ---------------------------------------------------------------- q sweep of the miss split
+def run_split_sweep(host_pool, T=8, steps=32, warm=16, threads=0):
+    """The split/merge workload at its configured shapes (E=256, k=6, d=4096,
+    I=2048, MXFP4, 64 slots, the AR(1) trace, T=8): each step's cache misses
+    are split, a fraction q filled over PCIe on the side stream while the CPU
+    computes the rest from the pinned host pool (moe_host_expert_ffn), merged
+    by the combine.  For q = 0, 0.1, ..., 1 and for q* (from the bandwidths
+    moe_profile_bandwidth measures first): step wall time (host sync to
+    host sync), host-kernel and fill times, and the merge's deviation from the
+    all-GPU layer on the same step."""
+    import expert_offload_serving_b200 as moe
+    from expert_offload_serving_b200.layer import MoeLayer
+    cfg = synth.CONFIGS["split_merge"]
+    s = moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt)
+    B = host_pool.shape[1]
+    dev_buf = torch.empty((4, B), dtype=torch.uint8, device="cuda")
+    bw = moe.moe_profile_bandwidth(s, host_pool, 16, dev_buf.view(-1), n_threads=threads)
+    del dev_buf
+    full = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=host_pool.cuda())   # all-GPU reference
+    trace = synth.make_trace(cfg, T, steps=warm + steps, seed=0)
+    lgs = [lg.cuda() for lg, _ in trace]
+    xs = [x.cuda() for _, x in trace]
+    rows = []
+    for q in [i / 10 for i in range(11)] + [None]:
+        layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, host_pool=host_pool, n_slots=cfg.n_slots)
+        step_ms, host_ms, n_fill, n_host, n_miss = [], [], 0, 0, 0
+        dev_max = dev_mean = 0.0
+        for t in range(warm + steps):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            res = layer.split_step(t, lgs[t], xs[t], q=q, bw=bw, threads=threads)
+            torch.cuda.synchronize()
+            dt = (time.perf_counter() - t0) * 1e3
+            if t < warm:
+                continue
+            step_ms.append(dt)
+            host_ms.append(res["host_ms"])
+            n_fill += len(res["fills"])
+            n_host += len(res["host"])
+            n_miss += len(res["filled"]) + len(res["host"])
+            if t == warm + steps - 1:
+                out = layer.out[:T].clone()
+                ref = full.forward(lgs[t], xs[t]).clone()
+                err = (out - ref).abs()
+                dev_max = float(err.max() / ref.abs().max())
+                dev_mean = float(err.mean() / ref.abs().mean())
+        moe.moe_check_status(layer.status)
+        layer.cache.close()
+        rows.append({"q": "q*" if q is None else q, "step_ms": round(statistics.median(step_ms), 3),
+                     "tokens_per_s": round(T / (statistics.median(step_ms) / 1e3), 1),
+                     "host_ms": round(statistics.median(host_ms), 3),
+                     "misses_per_step": round(n_miss / steps, 2), "fills_per_step": round(n_fill / steps, 2),
+                     "host_experts_per_step": round(n_host / steps, 2),
+                     "merge_vs_all_gpu": {"max_rel": float(f"{dev_max:.3e}"), "mean_rel": float(f"{dev_mean:.3e}")}})
+    del full
+    best = min(r["step_ms"] for r in rows if r["q"] != "q*")
+    qs = next(r for r in rows if r["q"] == "q*")
+    return {
+        "workload": f"split_merge: E={cfg.E} k={cfg.k} d={cfg.d} I={cfg.I} T={T}, {cfg.n_slots} slots, AR(1) "
+                    f"trace; misses split by q, host share on the CPU ({threads or 'all'} threads) concurrently "
+                    "with the fills",
+        "bandwidth_profile": {"h2d_pinned_gbs": round(bw[0], 1), "host_kernel_gbs": round(bw[1], 1)},
+        "steps": steps, "warmup_steps": warm, "timing": "median step wall time, host sync to host sync",
+        "sweep": rows,
+        "q_star_step_ms_over_best": round(qs["step_ms"] / best, 3),
     }
 
 

@@ -60,6 +60,9 @@ _SIGS = {
                                    ctypes.POINTER(ctypes.c_double)]),
     "moe_cache_create": (_I, [moe_shape, _I, _P, _P, _P, ctypes.POINTER(_P)]),
     "moe_cache_fill": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "moe_cache_create_layers": (_I, [moe_shape, _I, _I, _P, _P, _P, ctypes.POINTER(_P)]),
+    "moe_cache_fill_layer": (_I, [_P, _I, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "moe_cache_resize": (_I, [_P, _I, _P, _P, _P, _P, _P]),
     "moe_cache_query": (_I, [_P, _P, _P, _P]),
     "moe_cache_destroy": (_I, [_P]),
     "moe_check_status": (_I, [_P, _P]),
@@ -312,28 +315,52 @@ def moe_check_status(dev_status, stream=None):
 
 
 class MoeCache:
-    """Handle of the host-side LRU bookkeeping (moe_cache_*)."""
+    """Handle of the host-side LRU bookkeeping (moe_cache_*).  n_layers > 1:
+    one cache shared by several layers (host_pool and slot_of_expert_dev are
+    then lists with one entry per layer)."""
 
-    def __init__(self, s: moe_shape, n_slots: int, slot_pool=None, host_pool=None, slot_of_expert_dev=None):
+    def __init__(self, s: moe_shape, n_slots: int, slot_pool=None, host_pool=None, slot_of_expert_dev=None,
+                 n_layers: int = 1):
         h = ctypes.c_void_p()
-        _check(lib().moe_cache_create(s, n_slots, _ptr(slot_pool), _ptr(host_pool),
-                                      _ptr(slot_of_expert_dev), ctypes.byref(h)))
+        if n_layers == 1 and not isinstance(host_pool, (list, tuple)):
+            _check(lib().moe_cache_create(s, n_slots, _ptr(slot_pool), _ptr(host_pool),
+                                          _ptr(slot_of_expert_dev), ctypes.byref(h)))
+        else:
+            if slot_pool is None:
+                hp = tb = None
+            else:
+                if len(host_pool) != n_layers or len(slot_of_expert_dev) != n_layers:
+                    raise ValueError(f"{n_layers} layers need {n_layers} host pools and slot tables")
+                hp = (ctypes.c_void_p * n_layers)(*[_ptr(p) for p in host_pool])
+                tb = (ctypes.c_void_p * n_layers)(*[_ptr(t) for t in slot_of_expert_dev])
+            _check(lib().moe_cache_create_layers(s, n_layers, n_slots, _ptr(slot_pool), hp, tb, ctypes.byref(h)))
         self.h = h
-        self.E, self.n_slots = s.E, n_slots
+        self.E, self.n_slots, self.n_layers = s.E, n_slots, n_layers
 
-    def fill(self, experts, step: int, protect=(), side=None, reads_done=None, fill_done=None):
-        """moe_cache_fill; returns the list of (expert, slot, evicted) fills."""
+    def fill(self, experts, step: int, protect=(), side=None, reads_done=None, fill_done=None, layer: int = 0):
+        """moe_cache_fill_layer; returns the list of (expert, slot, evicted key) fills."""
         ex = (ctypes.c_int32 * max(1, len(experts)))(*[int(e) for e in experts])
         pr = (ctypes.c_int32 * max(1, len(protect)))(*[int(e) for e in protect])
         fills = (ctypes.c_int32 * (3 * max(1, len(experts))))()
         nf = ctypes.c_int32(0)
         side_h = None if side is None else _stream(side)
-        _check(lib().moe_cache_fill(self.h, ex, len(experts), step, pr, len(protect), side_h,
-                                    _event(reads_done), _event(fill_done), fills, ctypes.byref(nf)))
+        _check(lib().moe_cache_fill_layer(self.h, int(layer), ex, len(experts), step, pr, len(protect), side_h,
+                                          _event(reads_done), _event(fill_done), fills, ctypes.byref(nf)))
         return [(fills[3 * i], fills[3 * i + 1], fills[3 * i + 2]) for i in range(nf.value)]
 
+    def resize(self, new_n_slots: int, new_slot_pool=None, stream=None, reads_done=None):
+        """moe_cache_resize; returns [(key, old slot)] of the kept residents in
+        their new slot order."""
+        kept = (ctypes.c_int32 * (2 * max(1, min(self.n_slots, new_n_slots))))()
+        nk = ctypes.c_int32(0)
+        st = None if new_slot_pool is None else _stream(stream)
+        _check(lib().moe_cache_resize(self.h, int(new_n_slots), _ptr(new_slot_pool), st, _event(reads_done), kept,
+                                      ctypes.byref(nk)))
+        self.n_slots = new_n_slots
+        return [(kept[2 * i], kept[2 * i + 1]) for i in range(nk.value)]
+
     def query(self):
-        soe = (ctypes.c_int32 * self.E)()
+        soe = (ctypes.c_int32 * (self.E * self.n_layers))()
         eos = (ctypes.c_int32 * self.n_slots)()
         lu = (ctypes.c_int32 * self.n_slots)()
         _check(lib().moe_cache_query(self.h, soe, eos, lu))

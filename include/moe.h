@@ -305,10 +305,58 @@ moe_status moe_cache_fill(moe_cache* c, const int32_t* experts, int n, int step,
                           const int32_t* protect, int n_protect,
                           cudaStream_t side, cudaEvent_t reads_done, cudaEvent_t fill_done,
                           int32_t* fills, int32_t* n_fills);
-/* Copies of the host bookkeeping: slot_of_expert [E], expert_of_slot [S],
- * last_used [S] (any may be NULL). */
+/* Copies of the host bookkeeping (any pointer may be NULL): slot_of_expert
+ * [L*E] (entry l*E + e: the slot of expert e of layer l, or -1),
+ * expert_of_slot [S] (the key l*E + e each slot holds, or -1), last_used [S].
+ * With one layer these are slot_of_expert [E] and expert ids. */
 moe_status moe_cache_query(const moe_cache* c, int32_t* slot_of_expert,
                            int32_t* expert_of_slot, int32_t* last_used);
+
+/* One cache shared by n_layers MoE layers of the same shape: the global LRU
+ * of the pages (freetoken.wiki "FreeToken 753b model", mechanism table,
+ * "Global LRU expert cache": cache decisions are shared across MoE layers).
+ * Residency is kept over keys (layer, expert) = l*E + e in one slot pool of
+ * n_slots blobs; every layer has its own host pool (host_pools[l], E blobs in
+ * expert order, pinned) and its own device slot table (slot_tables_dev[l],
+ * int32 [E], set to -1 by the caller before the first fill), which that
+ * layer's moe_expert_ffn and moe_combine_merge read.  All pointers NULL:
+ * a plan-only handle (no CUDA call).  moe_cache_create is this call with one
+ * layer.  Errors: MOE_ERR_INVALID_ARG. */
+moe_status moe_cache_create_layers(moe_shape s, int n_layers, int n_slots, void* slot_pool,
+                                   const void* const* host_pools, int32_t* const* slot_tables_dev,
+                                   moe_cache** out);
+
+/* moe_cache_fill for layer `layer` of a shared cache: the experts of this
+ * layer's step become resident; a victim may belong to any layer (least
+ * recent last_used over the whole pool, ties to the lowest slot, never a key
+ * of this layer in `experts` or `protect`).  `step` is the caller's clock,
+ * increasing across layers and steps (e.g. token step * n_layers + layer);
+ * `reads_done` must follow the last kernel of any layer that read the pool or
+ * a slot table.  fills: (expert of this layer, slot, evicted key or -1).
+ * moe_cache_fill is this call with layer 0. */
+moe_status moe_cache_fill_layer(moe_cache* c, int layer, const int32_t* experts, int n, int step,
+                                const int32_t* protect, int n_protect, cudaStream_t side,
+                                cudaEvent_t reads_done, cudaEvent_t fill_done, int32_t* fills,
+                                int32_t* n_fills);
+
+/* Elastic resize at a safe point (futuresignalnews.com, mechanism 3 "Elastic
+ * Memory Management": the GPU expert cache is rebuilt under a new VRAM budget
+ * at a safe scheduler point, without reloading the host pool): the cache gets
+ * new_n_slots slots in new_slot_pool (device, 256-byte aligned,
+ * new_n_slots blobs; it may be the current pool when new_n_slots does not
+ * exceed the current count).  The min(residents, new_n_slots) residents with
+ * the latest last_used (ties: lower slot first) are kept, keep their
+ * last_used, and move to slots 0, 1, ... in their old slot order; the others
+ * are evicted.  On `stream`, after a wait on `reads_done` (the last kernel
+ * that read the pool or a slot table): device-to-device copies of the kept
+ * blobs that move, then the slot-table updates of every layer.  No host-pool
+ * copy is made.  The old pool may be freed once the stream has passed this
+ * point.  kept: host int32 [min(S, new_n_slots)][2] or NULL, receives (key,
+ * old slot) per new slot; *n_kept their count.  Plan-only handles: no CUDA
+ * call, new_slot_pool ignored.  Errors: MOE_ERR_INVALID_ARG (growing in
+ * place, bad pool), MOE_ERR_CUDA (the handle then refuses further calls). */
+moe_status moe_cache_resize(moe_cache* c, int new_n_slots, void* new_slot_pool, cudaStream_t stream,
+                            cudaEvent_t reads_done, int32_t* kept, int32_t* n_kept);
 moe_status moe_cache_destroy(moe_cache* c);
 
 /* ------------------------------------------------------------------------ */

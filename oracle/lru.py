@@ -15,11 +15,21 @@ Readings (the pages give no eviction details):
   * the split: of the step's misses, the round(q * m) with the most routed
     tokens are filled (ties to the lower id), the rest are host-computed;
   * the q* policy balances fill time and host time:
-    q* = m * bw_pcie / (bw_pcie + bw_host), rounded, clamped to [0, m].
+    q* = m * bw_pcie / (bw_pcie + bw_host), rounded, clamped to [0, m];
+  * one cache shared by L layers (the pages' global LRU: cache decisions are
+    shared across MoE layers, freetoken.wiki mechanism table) is this same
+    cache over keys l*E + e, with a clock that advances per layer and step;
+  * a resize to n slots at a safe point (futuresignalnews.com, mechanism 3:
+    the cache is rebuilt under a new VRAM budget without reloading the host
+    pool) keeps the min(residents, n) residents with the latest last use
+    (ties: lower slot first), in their old slot order in slots 0, 1, ...,
+    with their last-use times; the rest are evicted.
 
-Pins (tests/test_oracle_lru.py): a hand-worked trace; invariants (hits +
+Pins (tests/test_oracle_lru.py): hand-worked traces (one layer; two layers
+sharing three slots; shrinking and growing resizes); invariants (hits +
 misses = sum |U_t|, residency <= slots, with slots >= E the misses equal the
-distinct experts seen); the pages' bandwidths for q*.
+distinct experts seen, a resize keeps exactly the most recent residents); the
+pages' bandwidths for q*.
 """
 from __future__ import annotations
 
@@ -69,6 +79,22 @@ class LRUCache:
             self.last_used[s] = t
             fills.append((e, s, old))
         return hits, fills
+
+
+    def resize(self, n: int):
+        """Rebuild the cache with n slots (see the module header).  Returns
+        [(key, old slot)] of the kept residents in their new slot order."""
+        res = [s for s in range(self.n_slots) if self.expert_of_slot[s] >= 0]
+        res.sort(key=lambda s: (-self.last_used[s], s))
+        keep = sorted(res[:n])
+        for s in res[n:]:
+            self.slot_of_expert[self.expert_of_slot[s]] = -1
+        eos, lu = [-1] * n, [-1] * n
+        for j, s in enumerate(keep):
+            eos[j], lu[j] = self.expert_of_slot[s], self.last_used[s]
+            self.slot_of_expert[eos[j]] = j
+        self.n_slots, self.expert_of_slot, self.last_used = n, eos, lu
+        return [(eos[j], s) for j, s in enumerate(keep)]
 
 
 def split_misses(misses, tokens_per_expert, q: float):

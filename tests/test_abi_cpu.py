@@ -312,6 +312,32 @@ def test_cache_planner_matches_oracle_lru(moe):
     assert total_fills > cfg.n_slots            # the trace evicts
 
 
+def test_layered_cache_planner_and_resize_match_oracle(moe):
+    """A plan-only cache shared by 4 layers makes the oracle's decisions over
+    keys l*E + e (clock = step * L + layer), and resizes (shrink, grow,
+    shrink) keep the same residents in the same slots as the oracle's."""
+    from oracle import moe as M
+    cfg = synth.CONFIGS["decode_mxfp4"]
+    Lyr, S = 4, 48
+    s = moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt)
+    c = moe.MoeCache(s, S, n_layers=Lyr)
+    ref = L.LRUCache(S, Lyr * cfg.E)
+    traces = [synth.make_trace(cfg, 4, steps=40, seed=10 + l) for l in range(Lyr)]
+    sizes = {12: 24, 22: 60, 31: 30}
+    for t in range(40):
+        if t in sizes:
+            assert c.resize(sizes[t]) == ref.resize(sizes[t])
+        for l in range(Lyr):
+            idx, _ = M.route_topk(traces[l][t][0].numpy(), cfg.k)
+            U = sorted(set(idx.ravel().tolist()))
+            clock = t * Lyr + l
+            got = c.fill(U, clock, protect=U, layer=l)
+            hits, fills = ref.step(clock, [l * cfg.E + e for e in U])
+            assert got == [(key - l * cfg.E, slot, old) for key, slot, old in fills]
+        soe, eos, lu = c.query()
+        assert soe == ref.slot_of_expert and eos == ref.expert_of_slot and lu == ref.last_used
+
+
 def test_cache_capacity_error_leaves_state(moe):
     s = moe.shape(16, 64, 64, "bf16")
     c = moe.MoeCache(s, 2)

@@ -49,26 +49,6 @@ def test_prefill_host_partial_merge(moe):
     check_tol(out, full, 1e-3, 1e-4)
 
 
-def test_prefill_full_size_sampled(moe):
-    """The prefill workload itself (E=256, k=6, d=4096, I=2048, T=4096):
-    indices and permutation bit-exact; sampled tokens' outputs vs the oracle."""
-    from oracle import moe as M
-    cfg = synth.CONFIGS["prefill_nvfp4"]
-    T = 4096
-    b = Built(cfg, T, seed=0, act="nvfp4")
-    out = b.run().cpu().numpy()
-    moe.moe_check_status(b.layer.status)
-    idx, _ = M.route_topk(b.logits.numpy(), cfg.k)
-    off, perm, _ = M.permute(idx, cfg.E)
-    assert np.array_equal(b.layer.idx.cpu().numpy(), idx)
-    assert np.array_equal(b.layer.offsets.cpu().numpy(), off)
-    assert np.array_equal(b.layer.perm[: T * cfg.k].cpu().numpy(), perm)
-    assert np.isfinite(out).all()
-    toks = [0, 1, 2047, 4095]
-    ref = b.oracle(tokens=toks)["out"]
-    check_tol(out[toks], ref[toks])
-
-
 def test_activation_codes_bit_exact(moe):
     """The NVFP4 quantisation of x (first stage of the tensor-core path) takes
     its decisions in fp32 exactly as the oracle does: every per-token scale
@@ -90,3 +70,34 @@ def test_activation_codes_bit_exact(moe):
     assert np.array_equal(got_s, s_ref)
     got = F.e2m1_decode(F.unpack_nibbles(codes)) * np.repeat(got_s, 16, axis=1)
     assert np.array_equal(got, deq_ref)
+
+
+@pytest.mark.parametrize("double_buffer", [True, False])
+def test_streamed_prefill_matches_resident_layers(moe, double_buffer):
+    """Three NVFP4 layers whose pools stay in pinned host memory, streamed
+    into two full-layer buffers (one copying while the other computes): each
+    layer's output equals the same layer run from a resident pool up to the
+    order of the fused combine's atomic adds, and the oracle within the bar."""
+    from expert_offload_serving_b200.layer import MoeLayer, StreamedPrefill, pack_pool
+    from oracle import moe as M
+    cfg = _cfg("stream", 16, 4, 512, 256)
+    T, n_layers = 128, 3
+    pools, inputs, w_cpu = [], [], []
+    for l in range(n_layers):
+        w = synth.make_experts(cfg, range(cfg.E), seed=50 + l, device="cuda")
+        w_cpu.append({k: v.cpu() for k, v in w.items()})
+        pools.append(pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w_cpu[l], range(cfg.E), pin=True))
+        logits, x = synth.make_routing(cfg, T, 60 + l)
+        inputs.append((logits, x))
+    sp = StreamedPrefill(cfg.E, cfg.d, cfg.I, cfg.k, T, pools)
+    outs = sp.run([(lg.cuda(), x.cuda()) for lg, x in inputs], double_buffer=double_buffer, keep_outputs=True)
+    torch.cuda.synchronize()
+    for l in range(n_layers):
+        res = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, device_pool=pools[l].cuda(), act="nvfp4")
+        ref_gpu = res.forward(inputs[l][0].cuda(), inputs[l][1].cuda())
+        check_tol(outs[l].cpu().numpy(), ref_gpu.cpu().numpy(), 1e-5, 1e-6)
+        ref = M.moe_layer(inputs[l][1].double().numpy(), inputs[l][0].numpy(), cfg.k,
+                          lambda e: M.dequant_expert(cfg.fmt, w_cpu[l], e), act="nvfp4")["out"]
+        check_tol(outs[l].cpu().numpy(), ref)
+    for L_ in sp.layers:
+        moe.moe_check_status(L_.status)

@@ -97,3 +97,48 @@ def test_q_sweep(moe):
         with open(os.path.join(out_dir, "split_sweep.json"), "w") as f:
             json.dump({"config": "E=256 k=6 d=1024 I=512 MXFP4 T=8, 64 slots, 16-step AR(1) trace; "
                                  "host share computed by the float64 oracle", "sweep": report}, f, indent=1)
+
+
+@pytest.mark.parametrize("q", [0.0, 0.5, 1.0, None])
+def test_split_step_host_kernel_concurrent(moe, q):
+    """MoeLayer.split_step: the step's misses split by q (None: q* from given
+    bandwidths), the GPU share filled on the side stream while the host share
+    runs in moe_host_expert_ffn on CPU threads, merged by the combine.  Every
+    step's split and fills equal the oracle's, and its output the oracle
+    layer's."""
+    from expert_offload_serving_b200.layer import MoeLayer, pack_pool
+    cfg = synth.LayerConfig("split_step", E=64, k=6, d=512, I=256, fmt="mxfp4", bias_std=0.5, n_slots=16,
+                            rho=0.9)
+    T = 4
+    bw = (50.0, 120.0)
+    w = synth.make_experts(cfg, range(cfg.E), 0, device="cuda")
+    w_cpu = {k: v.cpu() for k, v in w.items()}
+    host_pool = pack_pool(cfg.E, cfg.d, cfg.I, cfg.fmt, w_cpu, range(cfg.E), pin=True)
+    layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, T, host_pool=host_pool, n_slots=cfg.n_slots)
+    lru = L.LRUCache(cfg.n_slots, cfg.E)
+    deq = {}
+
+    def weights(e):
+        if e not in deq:
+            deq[e] = M.dequant_expert(cfg.fmt, w_cpu, e)
+        return deq[e]
+    n_host = 0
+    for t, (logits, x) in enumerate(synth.make_trace(cfg, T, steps=20, seed=9)):
+        res = layer.split_step(t, logits.cuda(), x.cuda(), q=q, bw=bw, threads=4)
+        idx, _ = M.route_topk(logits.numpy(), cfg.k)
+        U = sorted(set(idx.ravel().tolist()))
+        tok = np.bincount(idx.ravel(), minlength=cfg.E)
+        misses = [e for e in U if not lru.resident(e)]
+        qq = q if q is not None else (L.q_star(len(misses), *bw) / len(misses) if misses else 0.0)
+        filled, host = L.split_misses(misses, tok, qq)
+        assert (res["filled"], res["host"]) == (filled, host), f"step {t}"
+        gpu_set = sorted(set(U) - set(host))
+        assert res["fills"] == lru.step(t, gpu_set, protect=U)[1], f"step {t}"
+        out = layer.out[:T].cpu().numpy()
+        ref = M.moe_layer(x.double().numpy(), logits.numpy(), cfg.k, weights)["out"]
+        check_tol(out, ref, 1e-4, 1e-5)
+        n_host += len(host)
+    moe.moe_check_status(layer.status)
+    assert layer.slot.cpu().tolist() == lru.slot_of_expert
+    if q != 1.0:
+        assert n_host > 0

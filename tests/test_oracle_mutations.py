@@ -164,3 +164,15 @@ def test_nvfp4_tensor_scales_reversed_is_caught(monkeypatch):
     monkeypatch.setattr(F, "dequant_nvfp4", bad)
     assert _fails(PL.test_nvfp4_dequant_expert_tensor_scale_order)
     assert len(calls) == 3
+
+
+def test_resize_keeping_the_oldest_is_caught(monkeypatch):
+    orig = L.LRUCache.resize
+
+    def bad(self, n):
+        self.last_used = [-v for v in self.last_used]      # ranks the oldest first
+        r = orig(self, n)
+        self.last_used = [-v for v in self.last_used]
+        return r
+    monkeypatch.setattr(L.LRUCache, "resize", bad)
+    assert _fails(PR.test_resize_hand_worked)
