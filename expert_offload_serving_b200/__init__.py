@@ -42,6 +42,8 @@ _SZ = ctypes.c_size_t
 _SIGS = {
     "moe_abi_version": (_I, []),
     "moe_last_error": (ctypes.c_char_p, []),
+    "moe_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+    "moe_set_test_stall": (_I, [_I]),
     "moe_expert_blob_bytes": (_SZ, [moe_shape]),
     "moe_pack_expert": (_I, [moe_shape, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_topk": (_I, [_P, _I, _I, _I, _P, _P, _P]),
@@ -143,6 +145,18 @@ def shape(E: int, d: int, I: int, fmt) -> moe_shape:
 # ------------------------------------------------------------------ the ABI
 def moe_abi_version() -> int:
     return lib().moe_abi_version()
+
+
+def moe_set_wait_limit_ns(ns: int) -> int:
+    """Limit of the tensor-core kernels' bounded waits for later launches (0:
+    the default 2 s); returns the previous limit.  A testing aid."""
+    return int(lib().moe_set_wait_limit_ns(int(ns)))
+
+
+def moe_set_test_stall(on: bool) -> bool:
+    """Testing aid: while on, CTA 0 of each tensor-core kernel waits on a
+    barrier nothing arrives on, so the bounded-wait abort path runs."""
+    return bool(lib().moe_set_test_stall(1 if on else 0))
 
 
 def moe_expert_blob_bytes(s: moe_shape) -> int:

@@ -56,6 +56,11 @@ moe_status current_device(DeviceInfo* out);
 
 moe_status check_shape(moe_shape s);
 
+// Limit of the tensor-core kernels' bounded waits, in ns (moe_set_wait_limit_ns),
+// and the testing aid of moe_set_test_stall.
+uint64_t wait_limit_ns();
+int test_stall();
+
 // ---------------------------------------------------------------- device helpers
 constexpr unsigned kFull = 0xffffffffu;
 

@@ -373,7 +373,7 @@ __device__ void run_unit(const FfnParams& P, const int16_t* act, const int32_t* 
   for (int sl = 0; sl < pp.slices; ++sl, ++j) {
     if (pp.next_issue < pp.n_items) issue_item<FMT, PHASE>(P, act, ustart, n_act, pp, row_bytes, lane);
     const int st = static_cast<int>(j % kStages);
-    if (!mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1), nullptr)) {
+    if (!__all_sync(kFull, mbar_wait(&pp.bar[st], static_cast<uint32_t>((j / kStages) & 1), nullptr))) {
       pp.ok = false;
       return;
     }

@@ -68,6 +68,8 @@ constexpr int THREADS = 7 * 32;
 constexpr int BPROD_WARP = 6;
 
 struct MxParams {
+  uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
+  int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
   int a_box_rows[3];       // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
   const int32_t* offsets;
@@ -99,7 +101,7 @@ struct Cfg {
   static constexpr int SA = SA_FIT > 8 ? 8 : SA_FIT;
   static constexpr int A_RING = SA * A_SMEM;
   static constexpr int B_RING = SB * B_STAGE;
-  static constexpr int N_BARS = 2 * SA + 2 * SB + 5;
+  static constexpr int N_BARS = 2 * SA + 2 * SB + 6;
   static_assert(TN == 16 || TN == 32, "chunk width");
   static_assert(A_SMEM % 1024 == 0 && B_STAGE % 1024 == 0 && B_ATOM % 1024 == 0, "1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
@@ -391,6 +393,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* drain = tfull + 4;                  // [1]
   uint64_t* bfull = tfull + 5;                  // [SB] token-row terms landed
   uint64_t* bempty = bfull + C::SB;             // [SB] token-row terms free
+  uint64_t* stall = bempty + C::SB;             // [1] never arrived on (testing aid)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
@@ -413,6 +416,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(stall, 1);
     for (int s = 0; s < C::SB; ++s) {
       mbar_init(&bfull[s], 1);
       mbar_init(&bempty[s], 1);
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int sl = __ldg(P.slot + U.e);
       const uint8_t* abase = tile_base<PHASE>(P, U);
       for (int ks = 0; ks < KS; ++ks) {
-        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -530,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Unit U = unit_of<TN>(P, ustart, u);
       const int tok = token_of<PHASE>(P, U, lane, n_pairs);
       for (int ks = 0; ks < KS; ++ks) {
-        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -559,14 +563,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Unit U = unit_of<TN>(P, ustart, u);
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const int acc = it & 1;
-      if (!mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+      if (!__all_sync(0xffffffffu, mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
       for (int ks = 0; ks < KS; ++ks) {
-        if (!(mbar_wait<true>(&bfull[sb], pb, abort_flag) && mbar_wait<true>(&full[sa], pa, abort_flag))) {
+        // one verdict for the warp: its lanes then take the same path to elect.sync
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bfull[sb], pb, abort_flag, P.wait_ns) &&
+                                         mbar_wait<true>(&full[sa], pa, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -622,10 +628,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     int it = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+    // testing aid (moe_set_test_stall): CTA 0's epilogue first waits on a
+    // barrier that nothing arrives on, so the bounded wait runs out and the
+    // abort path (record, stop issuing, drain, free TMEM) runs for real
+    const bool stalled = P.stall && blockIdx.x == 0 && !mbar_wait<true>(stall, 0, abort_flag, P.wait_ns);
+    if (stalled) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
       const Unit U = unit_of<TN>(P, ustart, u);
       const int acc = it & 1;
-      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
+      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
       named_sync(1, 128);
       if (*epi_fail) {
         report(P.status, MOE_ERR_TIMEOUT);
@@ -766,6 +780,8 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   const MxWorkspace W = mx_workspace(s, T, k);
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   MxParams P{};
+  P.wait_ns = wait_limit_ns();
+  P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
   P.I = s.I;

@@ -39,6 +39,8 @@
 namespace moe {
 
 struct TcDecodeParams {
+  uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
+  int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
   int a_box_rows[3];         // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
   const int32_t* offsets;
@@ -92,7 +94,7 @@ struct Cfg {
   static constexpr int BPROD_WARP = EPI_WARP0 + 4;               // the token-row producer
   static constexpr int THREADS = (EPI_WARP0 + 5) * 32;
   static constexpr int TMEM_COLS = 64;
-  static constexpr int N_BARS = 2 * SA + 2 * SB + 5;
+  static constexpr int N_BARS = 2 * SA + 2 * SB + 6;
   static_assert(TN == 16 || TN == 32, "chunk width");
   static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
@@ -266,6 +268,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   uint64_t* drain = tfull + 4;                  // [1]
   uint64_t* bfull = tfull + 5;                  // [SB] token rows landed
   uint64_t* bempty = bfull + C::SB;             // [SB] token rows free
+  uint64_t* stall = bempty + C::SB;             // [1] never arrived on (testing aid)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
@@ -288,6 +291,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(stall, 1);
     for (int s = 0; s < C::SB; ++s) {
       mbar_init(&bfull[s], 1);
       mbar_init(&bempty[s], 1);
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
       for (int ks = 0; ks < KS; ++ks) {
         // one verdict for the warp: its lanes take the same path
-        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       const Unit U = unit_of<TN>(P, ustart, MT, u);
       const int tok = token_of<PHASE>(P, U, lane, n_pairs);
       for (int ks = 0; ks < KS; ++ks) {
-        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const uint32_t idesc = idesc_bf16(TM, n_mma);
       const int acc = it & 1;
-      if (!mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+      if (!__all_sync(0xffffffffu, mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
         ok = false;
         break;
       }
@@ -445,8 +449,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
       for (int ks = 0; ks < KS; ++ks) {
         // the token rows and the weight stage have landed
-        const bool got = mbar_wait<true>(&bfull[stage], phase, abort_flag) &&
-                         mbar_wait<true>(&full[sa], pa, abort_flag);
+        // one verdict for the warp: its lanes then take the same path to elect.sync
+        const bool got = __all_sync(0xffffffffu, mbar_wait<true>(&bfull[stage], phase, abort_flag, P.wait_ns) &&
+                                                     mbar_wait<true>(&full[sa], pa, abort_flag, P.wait_ns));
         if (!got) {
           ok = false;
           break;
@@ -493,11 +498,19 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     // ------------------------------------------------------------ epilogue (last four warps)
     const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
     int it = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+    // testing aid (moe_set_test_stall): CTA 0's epilogue first waits on a
+    // barrier that nothing arrives on, so the bounded wait runs out and the
+    // abort path (record, stop issuing, drain, free TMEM) runs for real
+    const bool stalled = P.stall && blockIdx.x == 0 && !mbar_wait<true>(stall, 0, abort_flag, P.wait_ns);
+    if (stalled) {
+      report(P.status, MOE_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
       const Unit U = unit_of<TN>(P, ustart, MT, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
-      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag)) *epi_fail = 1;
+      if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
       named_sync(1, 128);
       if (*epi_fail) {
         report(P.status, MOE_ERR_TIMEOUT);
@@ -592,6 +605,8 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
                             const int32_t* slot, const void* pool, int n_slots, const float* gate, float* y_perm,
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
   TcDecodeParams P{};
+  P.wait_ns = wait_limit_ns();
+  P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
   P.I = s.I;

@@ -60,6 +60,8 @@ constexpr int SFA_COL = 256, SFB_COL = 272;
 constexpr int THREADS = 64 + EPI_THREADS;   // producer, MMA, epilogue groups
 
 struct GemmParams {
+  uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
+  int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots, max_chunks;
   const int32_t* offsets;
   const int32_t* perm;
@@ -304,8 +306,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   uint64_t* tfull = bars + 2 * STAGES;     // [2]
   uint64_t* tempty = bars + 2 * STAGES + 2;// [2]
   uint64_t* drain = bars + 2 * STAGES + 4; // [1]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint64_t* stall = bars + 2 * STAGES + 5; // [1] never arrived on (testing aid)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
   int32_t* chunk_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E+1]
   __shared__ int ws[36];
 
@@ -325,7 +329,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       mbar_init(&tempty[a], EPI_THREADS);
     }
     mbar_init(drain, 1);
+    mbar_init(stall, 1);
     *abort_flag = 0;
+    *epi_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       // expert's further chunks read again is kept
       const uint64_t pol_a = (chunk_start[e + 1] - chunk_start[e] > 1) ? pol_keep : pol_stream;
       for (int ks = 0; ks < KS; ++ks) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+        if (!__all_sync(kFull, mbar_wait(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -414,14 +420,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       const int nmma = (nvalid + 15) & ~15;
       const uint32_t idesc = idesc_fp4(nmma);
       const int acc = it & 1;
-      if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) {
+      if (!__all_sync(kFull, mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * ACC_COLS;
       for (int ks = 0; ks < KS; ++ks) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) {
+        if (!__all_sync(kFull, mbar_wait(&full[stage], phase, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -472,7 +478,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     const int bar_grp = 1 + grp, bar_all = 3;
     const float* ts = nullptr;
     int it = 0;
-    bool ok = true;
+    // testing aid (moe_set_test_stall): CTA 0's epilogue first waits on a
+    // barrier that nothing arrives on, so the bounded wait runs out and the
+    // abort path (record, stop issuing, drain, free TMEM) runs for real
+    bool ok = !(P.stall && blockIdx.x == 0 && !mbar_wait(stall, 0, abort_flag, P.wait_ns));
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       int c, m;
       unit_coords(u, MT, &c, &m);
@@ -493,13 +502,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           col_g[eall] = good ? P.gate[p] : 0.f;
         }
       }
-      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag)) {
+      // the eight epilogue warps agree before any leaves: a warp alone at a
+      // named barrier would wait for good (this barrier also publishes the
+      // column info written above)
+      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
+      named_sync(bar_all, EPI_THREADS);
+      if (*epi_fail) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS;
-      if (PHASE == 2) named_sync(bar_all, EPI_THREADS);
       const float g_mat = (PHASE == 1) ? 0.f : __ldg(ts + 2);
       const float g_gate = (PHASE == 1) ? __ldg(ts + 0) : 0.f, g_up = (PHASE == 1) ? __ldg(ts + 1) : 0.f;
       for (int cc = 16 * grp; cc < nvalid; cc += 16 * EPI_GROUPS) {
@@ -613,7 +626,7 @@ PrefillWs prefill_ws(moe_shape s, int T, int k) {
 }
 
 constexpr size_t kGemmSmem = STAGES * STAGE_BYTES + EPI_BYTES + 256 + 1025 * 4 + 1024;
-static_assert((2 * STAGES + 5) * 8 + 16 <= 256, "barrier area");
+static_assert((2 * STAGES + 6) * 8 + 16 <= 256, "barrier area");
 
 }  // namespace
 
@@ -689,6 +702,8 @@ moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const in
     MOE_LAUNCH_CHECK("gather_x_kernel");
   }
   GemmParams P{};
+  P.wait_ns = wait_limit_ns();
+  P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
   P.I = s.I;

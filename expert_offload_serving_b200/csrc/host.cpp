@@ -1,5 +1,6 @@
 // Host-only parts of libmoe: error strings, shape checks, device attributes,
 // and moe_pack_expert (canonical tensors -> device-final expert blob).
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -20,6 +21,14 @@ moe_status fail(moe_status st, const char* fmt, ...) {
 }
 
 void clear_error() { g_err[0] = '\0'; }
+
+namespace {
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+std::atomic<int> g_stall{0};
+}
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+int test_stall() { return g_stall.load(std::memory_order_relaxed); }
 
 moe_status check_shape(moe_shape s) {
   MOE_REQUIRE(s.E >= 1 && s.E <= 1024, "E=%d outside [1, 1024]", s.E);
@@ -69,6 +78,14 @@ moe_status current_device(DeviceInfo* out) {
 using namespace moe;
 
 extern "C" int moe_abi_version(void) { return 1; }
+
+extern "C" int moe_set_test_stall(int on) { return g_stall.exchange(on ? 1 : 0); }
+
+extern "C" uint64_t moe_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t prev = g_wait_ns.load();
+  g_wait_ns.store(ns == 0 ? 2000000000ull : ns);
+  return prev;
+}
 
 extern "C" const char* moe_last_error(void) { return g_err; }
 

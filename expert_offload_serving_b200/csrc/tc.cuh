@@ -12,7 +12,7 @@
 namespace moe {
 namespace tc {
 
-constexpr uint64_t kWaitNs = 2000000000ull;   // every wait gives up after 2 s
+constexpr uint64_t kWaitNs = 2000000000ull;   // every wait gives up after 2 s (default limit)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -60,19 +60,21 @@ __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: false when 2 s pass (or another role gave up first; no
-// abort flag: abort_flag == nullptr).
+// Bounded wait: false when limit_ns pass (2 s unless the launch was given a
+// shorter limit, which only tests of this path do), or another role gave up
+// first (no abort flag: abort_flag == nullptr).
 // SLEEP: suspend between tries (measured better for the decode GEMVs, whose
 // waiting warps share issue slots with the converter warps; the prefill
 // GEMM's short stages keep the spinning form).
 template <bool SLEEP = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitNs) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 0;; ++i) {
     if (SLEEP ? mbar_try_sleep(bar, parity) : mbar_try(bar, parity)) return true;
     if ((i & 255u) == 255u) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (now_ns() - t0 > kWaitNs) return false;
+      if (now_ns() - t0 > limit_ns) return false;
     }
   }
 }

@@ -77,6 +77,24 @@ enum {
 /* Version of this ABI (bumped on any signature change). */
 int moe_abi_version(void);
 
+/* Testing aid, no counterpart in the pages: every wait of the tensor-core
+ * kernels (a pipeline stage, a token-row stage, an accumulator) is bounded;
+ * when the limit passes, the CTA records MOE_ERR_TIMEOUT in the status word,
+ * stops issuing, drains the copies and MMAs it issued (those drains keep the
+ * 2 s bound), frees its tensor memory and returns, so the context stays
+ * usable.  This sets the limit for kernels launched afterwards by any thread
+ * (ns; 0 restores the default 2 s) and returns the previous one; tests use a
+ * few ns to make that path run. */
+uint64_t moe_set_wait_limit_ns(uint64_t ns);
+
+/* Testing aid, no counterpart in the pages: while on (nonzero), the
+ * tensor-core kernels launched afterwards make CTA 0's epilogue first wait on
+ * a barrier that nothing arrives on, so that wait runs out after the limit
+ * above and the abort path runs: the call's status word then holds
+ * MOE_ERR_TIMEOUT and its outputs are incomplete.  Returns the previous
+ * setting.  Nothing faults or hangs: the wait is bounded like every other. */
+int moe_set_test_stall(int on);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char* moe_last_error(void);
 
