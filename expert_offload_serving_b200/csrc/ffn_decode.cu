@@ -596,7 +596,9 @@ size_t decode_workspace_bytes(moe_shape s, int T, int k) {
   // otherwise a: fp32 (CUDA-core path) or the two 16-bit planes of the bf16
   // tensor-core path
   if (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)) return decode_mx_workspace_bytes(s, T, k);
-  return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256);
+  // bf16 tile layout: + one gate/up completion counter per expert (one-launch schedule)
+  const size_t extra = (s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I)) ? round_up(static_cast<size_t>(s.E) * 4, 256) : 0;
+  return round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256) + extra;
 }
 
 moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int32_t* offsets, const int32_t* perm,

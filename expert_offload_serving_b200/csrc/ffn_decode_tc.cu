@@ -30,6 +30,8 @@
 // keep enough bytes in flight to run near the HBM rate.  Every wait is
 // bounded: on expiry the CTA records MOE_ERR_TIMEOUT, stops issuing, drains
 // what it issued and frees its TMEM.
+#include <cstdlib>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -51,6 +53,7 @@ struct TcDecodeParams {
   size_t blob_bytes;
   BlobLayout L;
   uint16_t* a_planes;        // [2][T*k][I] bf16: hi, lo
+  int32_t* done1;            // fused launch: per expert, gemv<1> units finished (zeroed before the launch)
   float* y_perm;             // [T*k][d] or null (then out)
   float* out;                // [T][d] (fused combine)
   int32_t* status;
@@ -82,8 +85,8 @@ struct Cfg {
   static constexpr int ATOMS = KSTAGE / 64;                      // B atoms per plane
   static constexpr int B_ATOM = TN * 128;                        // one 64-element atom of TN token rows
   static constexpr int A_STAGE = 2 * TM * 128;                   // weight bytes per stage
-  static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;
-  static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;  // up-row exchange
+  static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;   // PHASE 3: both GEMVs
+  static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;  // up-row exchange
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
   static constexpr int SB = B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3;   // token-row stages
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_STAGE;
@@ -110,23 +113,36 @@ constexpr size_t smem_bytes(int E) {
 }
 
 struct Unit {
-  int e, m, q0, nvalid;
+  int e, m, q0, nvalid, ph;   // ph: 1 = gate/up GEMV, 2 = down GEMV
 };
 
-// unit u -> (expert, tile, chunk of TN pairs); ustart[e] = first unit of expert e
-template <int TN>
-__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int MT, int u) {
-  int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
+// unit u -> (phase, expert, tile, chunk of TN pairs).  ustart[e] = first unit
+// of expert e in the table built with tiles1 tiles per chunk.  A fused launch
+// (PHASE 3) runs the n1 = ustart[E] gate/up units first and then the down
+// units, whose table is ustart scaled by tiles2 / tiles1 (both phases count
+// tiles x chunks(e) per expert).
+template <int PHASE, int TN>
+__device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* ustart, int tiles1, int tiles2,
+                                        int u) {
+  int ph = PHASE == 3 ? 1 : PHASE, num = 1, den = 1;
+  if (PHASE == 3 && u >= ustart[P.E]) {
+    ph = 2;
+    u -= ustart[P.E];
+    num = tiles2;
+    den = tiles1;
+  }
+  int lo = 0, hi = P.E;   // start(lo) <= u < start(hi)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (ustart[mid] <= u) lo = mid;
+    if (ustart[mid] / den * num <= u) lo = mid;
     else hi = mid;
   }
   Unit U;
   U.e = lo;
+  U.ph = ph;
   const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
   const int chunks = (ne + TN - 1) / TN;
-  const int local = u - ustart[lo];
+  const int local = u - ustart[lo] / den * num;
   U.m = local / chunks;
   const int c = local % chunks;
   U.q0 = q_begin + c * TN;
@@ -135,12 +151,12 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
 }
 
 // First byte of unit U's weight tile (its K stages follow at A_STAGE).
-template <int FMT, int PHASE>
+template <int FMT>
 __device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, const Unit& U) {
-  using C = Cfg<FMT, PHASE, 32>;   // the weight stages do not depend on TN
-  const int K = (PHASE == 1) ? P.d : P.I;
+  using C = Cfg<FMT, 1, 32>;   // the weight stages depend on neither phase nor TN
+  const int K = (U.ph == 1) ? P.d : P.I;
   const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-  return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / C::KSTAGE) * C::A_STAGE;
+  return blob + (U.ph == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / C::KSTAGE) * C::A_STAGE;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -186,10 +202,9 @@ __device__ __forceinline__ void split_bf16(float a, uint16_t* hi, uint16_t* lo) 
 }
 
 // gemv<1>: the token of each of the unit's pairs (lane q: pair q0 + q).
-template <int PHASE>
 __device__ __forceinline__ int token_of(const TcDecodeParams& P, const Unit& U, int lane, int n_pairs) {
   int tok = 0;
-  if (PHASE == 1 && lane < U.nvalid) {
+  if (U.ph == 1 && lane < U.nvalid) {
     const int p = __ldg(P.perm + U.q0 + lane);
     if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
     else tok = p / P.k;
@@ -206,10 +221,10 @@ __device__ __forceinline__ int a_box(const TcDecodeParams& P, int nvalid) {
 }
 
 // Bytes that land in a token-row stage of unit U.
-template <class C, int PHASE, int TN>
+template <class C, int TN>
 __device__ __forceinline__ uint32_t b_bytes(const TcDecodeParams& P, const Unit& U) {
   const uint32_t rows =
-      PHASE == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
+      U.ph == 1 ? static_cast<uint32_t>(U.nvalid) : 2u * static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
   return rows * C::ATOMS * 128u;
 }
 
@@ -217,14 +232,14 @@ __device__ __forceinline__ uint32_t b_bytes(const TcDecodeParams& P, const Unit&
 // expected bytes lane 0 has posted): gemv<1> one row TMA of x per pair and
 // atom, lane q loading pair q0 + q; gemv<2> both planes of the a box, rows
 // past the unit's pairs never read back.  Called by all lanes of one warp.
-template <class C, int PHASE, int TN>
+template <class C, int TN>
 __device__ __forceinline__ void load_b(const TcDecodeParams& P, const Unit& U, int ks, int tok, uint8_t* sB,
-                                       uint64_t* bar, const CUtensorMap* tm_b, const CUtensorMap* tm_b16,
-                                       const CUtensorMap* tm_b8, uint64_t pol, int lane) {
-  if (PHASE == 2) {
+                                       uint64_t* bar, const CUtensorMap* tm_x, const CUtensorMap* tm_a,
+                                       const CUtensorMap* tm_a16, const CUtensorMap* tm_a8, uint64_t pol, int lane) {
+  if (U.ph == 2) {
     if (lane == 0) {
       const int bi = a_box<TN>(P, U.nvalid);
-      const CUtensorMap* tm = bi == 0 ? tm_b8 : (bi == 1 ? tm_b16 : tm_b);
+      const CUtensorMap* tm = bi == 0 ? tm_a8 : (bi == 1 ? tm_a16 : tm_a);
 #pragma unroll
       for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
@@ -234,8 +249,31 @@ __device__ __forceinline__ void load_b(const TcDecodeParams& P, const Unit& U, i
   } else if (lane < U.nvalid) {
 #pragma unroll
     for (int a = 0; a < C::ATOMS; ++a)
-      tma_load_2d(sB + a * C::B_ATOM + lane * 128, tm_b, bar, ks * C::KSTAGE + 64 * a, tok, pol);
+      tma_load_2d(sB + a * C::B_ATOM + lane * 128, tm_x, bar, ks * C::KSTAGE + 64 * a, tok, pol);
   }
+}
+
+// Fused launch: lane 0 waits (bounded, like every wait) until all `target`
+// gate/up units of expert e have published their a rows, then orders the
+// TMA loads that follow after what it observed.  One verdict for the warp.
+__device__ __forceinline__ bool wait_expert_ready(const TcDecodeParams& P, int e, int target,
+                                                  volatile int* abort_flag, int lane) {
+  bool ok = true;
+  if (lane == 0) {
+    const uint64_t t0 = now_ns();
+    for (;;) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+      if (v >= target) break;
+      if (*abort_flag || now_ns() - t0 > P.wait_ns) {
+        ok = false;
+        break;
+      }
+      __nanosleep(256);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Waits for the copies of the last min(issued, n) stages of a ring to land.
@@ -252,8 +290,9 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, in
 
 template <int FMT, int PHASE, int TN>
 __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
-    gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b16,
-                   const __grid_constant__ CUtensorMap tm_b8, TcDecodeParams P) {
+    gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                   const __grid_constant__ CUtensorMap tm_a16, const __grid_constant__ CUtensorMap tm_a8,
+                   TcDecodeParams P) {
   using C = Cfg<FMT, PHASE, TN>;
   constexpr int THREADS = C::THREADS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -276,9 +315,9 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = (PHASE == 1) ? P.d : P.I;
-  const int KS = K / C::KSTAGE;
-  const int MT = (PHASE == 1) ? P.I / 64 : P.d / TM;
+  const int MT1 = P.I / 64, MT2 = P.d / TM;     // tiles per chunk: gate/up, down
+  const int MT = PHASE == 2 ? MT2 : MT1;          // ... of the unit table built below
+  auto ks_of = [&](const Unit& U) { return (U.ph == 1 ? P.d : P.I) / C::KSTAGE; };
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
@@ -342,7 +381,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int n_units = total;
+  const int n_units = PHASE == 3 ? total + total / MT1 * MT2 : total;
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight producer
@@ -352,12 +391,17 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     int issued = 0;
     bool ok = true;
     // L2 prefetch cursor over this CTA's (unit, stage) items
-    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
+    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0, pf_KS = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of<TN>(P, ustart, MT, pf_u));
+    if (pf_u < n_units) {
+      const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
+      pf_base = tile_base<FMT>(P, V);
+      pf_KS = ks_of(V);
+    }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of<TN>(P, ustart, MT, u);
-      const uint8_t* abase = tile_base<FMT, PHASE>(P, U);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
+      const uint8_t* abase = tile_base<FMT>(P, U);
+      const int KS = ks_of(U);
       for (int ks = 0; ks < KS; ++ks) {
         // one verdict for the warp: its lanes take the same path
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
@@ -374,10 +418,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
           while (pf_u < n_units && pf_ahead < PF_ITEMS) {
             prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
             ++pf_ahead;
-            if (++pf_ks == KS) {
+            if (++pf_ks == pf_KS) {
               pf_ks = 0;
               pf_u += gridDim.x;
-              if (pf_u < n_units) pf_base = tile_base<FMT, PHASE>(P, unit_of<TN>(P, ustart, MT, pf_u));
+              if (pf_u < n_units) {
+                const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
+                pf_base = tile_base<FMT>(P, V);
+                pf_KS = ks_of(V);
+              }
             }
           }
           --pf_ahead;
@@ -406,17 +454,26 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     int issued = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of<TN>(P, ustart, MT, u);
-      const int tok = token_of<PHASE>(P, U, lane, n_pairs);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
+      const int tok = token_of(P, U, lane, n_pairs);
+      const int KS = ks_of(U);
+      if (PHASE == 3 && U.ph == 2) {
+        // the a rows of this expert's pairs come from every gate/up unit of the expert
+        const int target = ustart[U.e + 1] - ustart[U.e];
+        if (!wait_expert_ready(P, U.e, target, abort_flag, lane)) {
+          ok = false;
+          break;
+        }
+      }
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
         uint8_t* sB = ring_b + stage * C::B_STAGE;
-        if (lane == 0) mbar_expect_tx(&bfull[stage], b_bytes<C, PHASE, TN>(P, U));
+        if (lane == 0) mbar_expect_tx(&bfull[stage], b_bytes<C, TN>(P, U));
         __syncwarp();
-        load_b<C, PHASE, TN>(P, U, ks, tok, sB, &bfull[stage], &tm_b, &tm_b16, &tm_b8, pol_keep, lane);
+        load_b<C, TN>(P, U, ks, tok, sB, &bfull[stage], &tm_x, &tm_a, &tm_a16, &tm_a8, pol_keep, lane);
         __syncwarp();
         ++issued;
         if (++stage == C::SB) {
@@ -437,7 +494,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = unit_of<TN>(P, ustart, MT, u);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
+      const int KS = ks_of(U);
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const uint32_t idesc = idesc_bf16(TM, n_mma);
       const int acc = it & 1;
@@ -468,7 +526,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
             const uint32_t first = (ks > 0 || kk > 0) ? 1u : 0u;
             const uint64_t da = desc_sw128(smem_u32(sA + a * TM * 128)) + 2 * (kk & 3);
             tc_mma_bf16(d_tmem, da, dh, idesc, first);
-            if (PHASE == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
+            if (U.ph == 2) tc_mma_bf16(d_tmem, da, dl, idesc, 1u);
           }
           tc_commit(&empty[sa]);
           tc_commit(&bempty[stage]);
@@ -507,7 +565,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       *abort_flag = 1;
     }
     for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
-      const Unit U = unit_of<TN>(P, ustart, MT, u);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int acc = it & 1;
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
@@ -522,7 +580,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (PHASE == 1) {
+      if (U.ph == 1) {
         // rows 0..63 of the tile are gate rows, 64..127 the matching up rows
         if (quad >= 2) {
           const int i = 32 * (quad - 2) + lane;
@@ -545,8 +603,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
               P.a_planes[plane + o] = lo;
             }
           }
+          // fused launch: the a rows are published to other CTAs (read there by TMA)
+          if (PHASE == 3) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+          }
         }
         named_sync(1, 128);
+        if (PHASE == 3 && warp == C::EPI_WARP0 && lane == 0) atomicAdd(P.done1 + U.e, 1);
       } else {
         const int row = TM * U.m + 32 * quad + lane;
 #pragma unroll
@@ -574,8 +638,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
 }
 
 template <int FMT, int PHASE, int TN>
-moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const CUtensorMap& tm16,
-                        const CUtensorMap& tm8, const DeviceInfo& dev, cudaStream_t s) {
+moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tx, const CUtensorMap& ta, const CUtensorMap& ta16,
+                        const CUtensorMap& ta8, const DeviceInfo& dev, cudaStream_t s) {
   const size_t smem = smem_bytes<FMT, PHASE, TN>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
@@ -584,17 +648,41 @@ moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tm, const CU
                                       static_cast<int>(smem)));
     attr[dev.id] = smem;
   }
-  gemv_tc_kernel<FMT, PHASE, TN><<<dev.sm_count, Cfg<FMT, PHASE, TN>::THREADS, smem, s>>>(tm, tm16, tm8, P);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(dev.sm_count);
+  cfg.blockDim = dim3(Cfg<FMT, PHASE, TN>::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  // the fused launch's CTAs wait on each other's gate/up units: all of them
+  // must be resident at once, which a cooperative launch guarantees
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = PHASE == 3 ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_tc_kernel<FMT, PHASE, TN>, tx, ta, ta16, ta8, P));
   MOE_LAUNCH_CHECK("gemv_tc_kernel");
   return MOE_OK;
+}
+
+// Both GEMVs in one cooperative launch unless MOE_DECODE_TWO_LAUNCHES is set
+// in the environment (read once; the two-launch schedule is kept for
+// comparison).
+bool fused_decode() {
+  static const bool fused = std::getenv("MOE_DECODE_TWO_LAUNCHES") == nullptr;
+  return fused;
 }
 
 template <int FMT, int TN>
 moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap (&tm_a)[3],
                        const DeviceInfo& dev, cudaStream_t stream) {
-  moe_status st = launch_phase<FMT, 1, TN>(P, tm_x, tm_x, tm_x, dev, stream);
+  if (fused_decode()) {
+    MOE_CUDA_TRY(cudaMemsetAsync(P.done1, 0, static_cast<size_t>(P.E) * sizeof(int32_t), stream));
+    return launch_phase<FMT, 3, TN>(P, tm_x, tm_a[2], tm_a[1], tm_a[0], dev, stream);
+  }
+  moe_status st = launch_phase<FMT, 1, TN>(P, tm_x, tm_a[2], tm_a[1], tm_a[0], dev, stream);
   if (st != MOE_OK) return st;
-  return launch_phase<FMT, 2, TN>(P, tm_a[2], tm_a[1], tm_a[0], dev, stream);
+  return launch_phase<FMT, 2, TN>(P, tm_x, tm_a[2], tm_a[1], tm_a[0], dev, stream);
 }
 
 }  // namespace
@@ -621,6 +709,8 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
   P.L = blob_layout(s.fmt, s.d, s.I);
   P.blob_bytes = P.L.bytes;
   P.a_planes = static_cast<uint16_t*>(ws);
+  P.done1 = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
+                                       round_up(static_cast<size_t>(T) * k * s.I * sizeof(float), 256));
   P.y_perm = y_perm;
   P.out = out;
   P.status = status;
