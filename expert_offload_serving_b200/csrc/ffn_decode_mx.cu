@@ -37,6 +37,8 @@
 // double-buffered accumulators, warp 6 loads the token-row terms and their
 // scale atoms.  Every wait is bounded: on expiry the CTA records
 // MOE_ERR_TIMEOUT, stops issuing, drains what it issued and frees its TMEM.
+#include <cstdlib>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -53,7 +55,9 @@ constexpr int TM = 128;                    // weight rows per tile
 constexpr int KSTAGE = 256;                // K elements per stage (one blob tile)
 constexpr int A_BOX = 128 * 128;           // one TMA box: 128 rows x 128 padded codes
 constexpr int A_SMEM = 2 * A_BOX + 1024;   // codes (expanded) + 2 scale atoms
-constexpr uint32_t A_TX = 2 * A_BOX + 1024;
+// bytes a weight stage's barrier expects: the 16U4_ALIGN16B loads count the
+// packed codes they read (8 KB per box), not the expanded 16 KB they write
+constexpr uint32_t A_TX = 2 * (A_BOX / 2) + 1024;
 constexpr int ACC_COLS = 32;
 constexpr int SFA_COL = 64;                // TMEM: 2 accumulators, then scale factors
 constexpr int SFB_COL = 72;
@@ -82,6 +86,7 @@ struct MxParams {
   const uint8_t* xs;       // [NX][T][d/32] E8M0 scales of the x terms
   uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
   uint8_t* as;             // [NA][T*k][I/32] their E8M0 scales
+  int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
   float* y_perm;
   float* out;
   int32_t* status;
@@ -89,14 +94,14 @@ struct MxParams {
 
 template <int PHASE, int TN>
 struct Cfg {
-  static constexpr int NT = PHASE == 1 ? NX : NA;                // terms of the B operand
+  static constexpr int NT = PHASE == 1 ? NX : NA;                // terms of the B operand (PHASE 3: both GEMVs)
   static constexpr int B_ATOM = TN * 128;                        // TN rows x 128 E4M3 values
   static constexpr int B_CODES = NT * 2 * B_ATOM;                // 2 atoms (256 K) per term
   static constexpr int B_STAGE = B_CODES + NT * 1024;            // + 2 scale atoms per term
-  static constexpr int UP_BYTES = PHASE == 1 ? 64 * 33 * 4 : 0;
+  static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
   // token-row stages: gemv<2>'s come from the a terms gemv<1> just wrote (L2)
-  static constexpr int SB = PHASE == 2 ? 2 : (B_STAGE <= 12 * 1024 ? 4 : 3);
+  static constexpr int SB = PHASE != 1 ? 2 : (B_STAGE <= 12 * 1024 ? 4 : 3);
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_SMEM;
   static constexpr int SA = SA_FIT > 8 ? 8 : SA_FIT;
   static constexpr int A_RING = SA * A_SMEM;
@@ -118,22 +123,34 @@ constexpr size_t smem_bytes(int E) {
 }
 
 struct Unit {
-  int e, m, q0, nvalid;
+  int e, m, q0, nvalid, ph;   // ph: 1 = gate/up GEMV, 2 = down GEMV
 };
 
-template <int TN>
-__device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart, int u) {
-  int lo = 0, hi = P.E;   // ustart[lo] <= u < ustart[hi]
+// unit u -> (phase, expert, tile, chunk of TN pairs).  ustart[e] = first unit
+// of expert e in the table built with tiles1 tiles per chunk.  The one-launch
+// schedule (PHASE 3) runs the n1 = ustart[E] gate/up units, then the down
+// units, whose table is ustart scaled by tiles2 / tiles1.
+template <int PHASE, int TN>
+__device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart, int tiles1, int tiles2, int u) {
+  int ph = PHASE == 3 ? 1 : PHASE, num = 1, den = 1;
+  if (PHASE == 3 && u >= ustart[P.E]) {
+    ph = 2;
+    u -= ustart[P.E];
+    num = tiles2;
+    den = tiles1;
+  }
+  int lo = 0, hi = P.E;   // start(lo) <= u < start(hi)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (ustart[mid] <= u) lo = mid;
+    if (ustart[mid] / den * num <= u) lo = mid;
     else hi = mid;
   }
   Unit U;
   U.e = lo;
+  U.ph = ph;
   const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
   const int chunks = (ne + TN - 1) / TN;
-  const int local = u - ustart[lo];
+  const int local = u - ustart[lo] / den * num;
   U.m = local / chunks;
   const int c = local % chunks;
   U.q0 = q_begin + c * TN;
@@ -141,12 +158,11 @@ __device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart
   return U;
 }
 
-// First byte of the blob tile (expert U.e, row tile U.m, k tile 0) of a phase.
-template <int PHASE>
+// First byte of the blob tile (expert U.e, row tile U.m, k tile 0) of the unit's phase.
 __device__ __forceinline__ const uint8_t* tile_base(const MxParams& P, const Unit& U) {
-  const int K = (PHASE == 1) ? P.d : P.I;
+  const int K = (U.ph == 1) ? P.d : P.I;
   const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
-  return blob + (PHASE == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / KSTAGE) * kMxTileBytes;
+  return blob + (U.ph == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / KSTAGE) * kMxTileBytes;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -261,10 +277,9 @@ __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restr
 }
 
 // ------------------------------------------------------------------ the GEMVs
-template <int PHASE>
 __device__ __forceinline__ int token_of(const MxParams& P, const Unit& U, int lane, int n_pairs) {
   int tok = 0;
-  if (PHASE == 1 && lane < U.nvalid) {
+  if (U.ph == 1 && lane < U.nvalid) {
     const int p = __ldg(P.perm + U.q0 + lane);
     if (p < 0 || p >= n_pairs) report(P.status, MOE_ERR_DEVICE);
     else tok = p / P.k;
@@ -285,21 +300,24 @@ __device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
 // unit's pairs get 2^0, their MMA columns are never read); they are made
 // visible to the tensor core's async proxy before lane 0 arrives.  Called by
 // all lanes of one warp.
-template <class C, int PHASE, int TN>
+template <class C, int TN>
 __device__ __forceinline__ void load_b(const MxParams& P, const Unit& U, int ks, int tok, uint8_t* sB,
-                                       uint64_t* bar, const CUtensorMap* tm_b, const CUtensorMap* tm_b16,
-                                       const CUtensorMap* tm_b8, uint64_t pol, int lane, int n_pairs) {
+                                       uint64_t* bar, const CUtensorMap* tm_x, const CUtensorMap* tm_a,
+                                       const CUtensorMap* tm_a16, const CUtensorMap* tm_a8, uint64_t pol, int lane,
+                                       int n_pairs) {
   uint8_t* sf = sB + C::B_CODES;
+  const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
   if (lane < TN) {
-    const int K = PHASE == 1 ? P.d : P.I;
+    const int K = U.ph == 1 ? P.d : P.I;
     const int nb = K / 32;
 #pragma unroll
     for (int j = 0; j < C::NT; ++j) {
+      if (j >= nt) break;
       uint2 v = make_uint2(0x7f7f7f7fu, 0x7f7f7f7fu);
       if (lane < U.nvalid) {
-        const size_t row = PHASE == 1 ? static_cast<size_t>(j) * P.T + tok
-                                      : static_cast<size_t>(j) * n_pairs + U.q0 + lane;
-        const uint8_t* src = (PHASE == 1 ? P.xs : P.as) + row * nb + 8 * ks;
+        const size_t row = U.ph == 1 ? static_cast<size_t>(j) * P.T + tok
+                                     : static_cast<size_t>(j) * n_pairs + U.q0 + lane;
+        const uint8_t* src = (U.ph == 1 ? P.xs : P.as) + row * nb + 8 * ks;
         v = *reinterpret_cast<const uint2*>(src);
       }
       *reinterpret_cast<uint32_t*>(sf + (2 * j) * 512 + lane * 16) = v.x;
@@ -308,27 +326,51 @@ __device__ __forceinline__ void load_b(const MxParams& P, const Unit& U, int ks,
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
-  const uint32_t rows = PHASE == 1 ? static_cast<uint32_t>(U.nvalid)
-                                   : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
-  if (lane == 0) mbar_expect_tx(bar, rows * C::NT * 2 * 128u);
+  const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid)
+                                  : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
+  if (lane == 0) mbar_expect_tx(bar, rows * static_cast<uint32_t>(nt) * 2 * 128u);
   __syncwarp();
-  if (PHASE == 2) {
+  if (U.ph == 2) {
     if (lane == 0) {
       const int bi = a_box<TN>(P, U.nvalid);
-      const CUtensorMap* tm = bi == 0 ? tm_b8 : (bi == 1 ? tm_b16 : tm_b);
+      const CUtensorMap* tm = bi == 0 ? tm_a8 : (bi == 1 ? tm_a16 : tm_a);
 #pragma unroll
-      for (int j = 0; j < C::NT; ++j)
+      for (int j = 0; j < NA; ++j)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
           tma_load_3d(sB + (2 * j + h) * C::B_ATOM, tm, bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
     }
   } else if (lane < U.nvalid) {
 #pragma unroll
-    for (int j = 0; j < C::NT; ++j)
+    for (int j = 0; j < NX; ++j)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, tm_b, bar, ks * KSTAGE + 128 * h, tok, j, pol);
+        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, tm_x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
   }
+}
+
+// One-launch schedule: lane 0 waits (bounded, like every wait) until all
+// `target` gate/up units of expert e have published their a terms, then
+// orders the TMA loads that follow after what it observed.  One verdict for
+// the warp.
+__device__ __forceinline__ bool wait_expert_ready(const MxParams& P, int e, int target, volatile int* abort_flag,
+                                                  int lane) {
+  bool ok = true;
+  if (lane == 0) {
+    const uint64_t t0 = now_ns();
+    for (;;) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+      if (v >= target) break;
+      if (*abort_flag || now_ns() - t0 > P.wait_ns) {
+        ok = false;
+        break;
+      }
+      __nanosleep(256);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, int stage, uint32_t phase) {
@@ -377,8 +419,9 @@ __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
 template <int PHASE, int TN>
 __global__ void __launch_bounds__(THREADS, 1)
-    gemv_mx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
-                   const __grid_constant__ CUtensorMap tm_b16, const __grid_constant__ CUtensorMap tm_b8,
+    gemv_mx_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
+                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
+                   const __grid_constant__ CUtensorMap tm_a16, const __grid_constant__ CUtensorMap tm_a8,
                    MxParams P) {
   using C = Cfg<PHASE, TN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -401,9 +444,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int K = (PHASE == 1) ? P.d : P.I;
-  const int KS = K / KSTAGE;
-  const int MT = (PHASE == 1) ? P.I / 64 : P.d / TM;
+  const int MT1 = P.I / 64, MT2 = P.d / TM;     // tiles per chunk: gate/up, down
+  const int MT = PHASE == 2 ? MT2 : MT1;          // ... of the unit table built below
+  auto ks_of = [&](const Unit& U) { return (U.ph == 1 ? P.d : P.I) / KSTAGE; };
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
@@ -467,7 +510,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int n_units = total;
+  const int n_units = PHASE == 3 ? total + total / MT1 * MT2 : total;
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight producer
@@ -476,13 +519,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0;
+    int pf_u = blockIdx.x, pf_ks = 0, pf_ahead = 0, pf_KS = 0;
     const uint8_t* pf_base = nullptr;
-    if (pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of<TN>(P, ustart, pf_u));
+    if (pf_u < n_units) {
+      const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
+      pf_base = tile_base(P, V);
+      pf_KS = ks_of(V);
+    }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of<TN>(P, ustart, u);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int sl = __ldg(P.slot + U.e);
-      const uint8_t* abase = tile_base<PHASE>(P, U);
+      const uint8_t* abase = tile_base(P, U);
+      const CUtensorMap* tm_w = U.ph == 1 ? &tm_w1 : &tm_w2;
+      const int KS = ks_of(U);
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
@@ -493,17 +542,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_expect_tx(&full[stage], A_TX);
           // codes: two boxes of 128 rows x 128 codes, expanded by the TMA into
           // 16-byte slots; coordinates (k in tile, row, k tile, row tile, slot)
-          tma_load_5d(sA, &tm_w, &full[stage], 0, 0, ks, U.m, sl, pol_stream);
-          tma_load_5d(sA + A_BOX, &tm_w, &full[stage], 128, 0, ks, U.m, sl, pol_stream);
+          tma_load_5d(sA, tm_w, &full[stage], 0, 0, ks, U.m, sl, pol_stream);
+          tma_load_5d(sA + A_BOX, tm_w, &full[stage], 128, 0, ks, U.m, sl, pol_stream);
           bulk_load(sA + 2 * A_BOX, abase + static_cast<size_t>(ks) * kMxTileBytes + 16384, 1024, &full[stage],
                     pol_stream);
           while (pf_u < n_units && pf_ahead < PF_ITEMS) {
             prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * kMxTileBytes, kMxTileBytes);
             ++pf_ahead;
-            if (++pf_ks == KS) {
+            if (++pf_ks == pf_KS) {
               pf_ks = 0;
               pf_u += gridDim.x;
-              if (pf_u < n_units) pf_base = tile_base<PHASE>(P, unit_of<TN>(P, ustart, pf_u));
+              if (pf_u < n_units) {
+                const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
+                pf_base = tile_base(P, V);
+                pf_KS = ks_of(V);
+              }
             }
           }
           --pf_ahead;
@@ -531,14 +584,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     int issued = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const Unit U = unit_of<TN>(P, ustart, u);
-      const int tok = token_of<PHASE>(P, U, lane, n_pairs);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
+      const int tok = token_of(P, U, lane, n_pairs);
+      const int KS = ks_of(U);
+      if (PHASE == 3 && U.ph == 2) {
+        // the a terms of this expert's pairs come from every gate/up unit of the expert
+        if (!wait_expert_ready(P, U.e, ustart[U.e + 1] - ustart[U.e], abort_flag, lane)) {
+          ok = false;
+          break;
+        }
+      }
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
-        load_b<C, PHASE, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &bfull[stage], &tm_b, &tm_b16, &tm_b8,
+        load_b<C, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &bfull[stage], &tm_x, &tm_a, &tm_a16, &tm_a8,
                              pol_keep, lane, n_pairs);
         __syncwarp();
         ++issued;
@@ -560,7 +621,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      const Unit U = unit_of<TN>(P, ustart, u);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
+      const int KS = ks_of(U);
+      const int nt = U.ph == 1 ? NX : NA;       // terms of the unit's B operand
       const int n_mma = U.nvalid <= 16 ? 16 : 32;
       const int acc = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
@@ -585,6 +648,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_cp_sf(tmem + SFA_COL + 4, desc_sf(smem_u32(sA + 2 * A_BOX + 512)));
 #pragma unroll
           for (int j = 0; j < C::NT; ++j) {
+            if (j >= nt) break;
             tc_cp_sf(tmem + SFB_COL + 8 * j, desc_sf(smem_u32(sB + C::B_CODES + (2 * j) * 512)));
             tc_cp_sf(tmem + SFB_COL + 8 * j + 4, desc_sf(smem_u32(sB + C::B_CODES + (2 * j + 1) * 512)));
           }
@@ -595,6 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t idesc = idesc_mx(n_mma, static_cast<uint32_t>(sub));
 #pragma unroll
             for (int j = 0; j < C::NT; ++j) {
+              if (j >= nt) break;
               const uint64_t db = desc_sw128(smem_u32(sB + (2 * j + h) * C::B_ATOM)) + 2 * sub;
               const uint32_t first = (ks > 0 || kk > 0 || j > 0) ? 1u : 0u;
               tc_mma_mx(d_tmem, da, db, idesc, tmem + SFA_COL + 4 * h, tmem + SFB_COL + 8 * j + 4 * h, first);
@@ -637,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       *abort_flag = 1;
     }
     for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
-      const Unit U = unit_of<TN>(P, ustart, u);
+      const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int acc = it & 1;
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
       named_sync(1, 128);
@@ -651,7 +716,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (PHASE == 1) {
+      if (U.ph == 1) {
         // rows 0..63 of the tile are gate rows, 64..127 the matching up rows
         if (quad >= 2) {
           const int i = 32 * (quad - 2) + lane;
@@ -682,8 +747,14 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
             }
           }
+          // one-launch schedule: the a terms are published to other CTAs (read there by TMA)
+          if (PHASE == 3) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+          }
         }
         named_sync(1, 128);
+        if (PHASE == 3 && warp == 2 && lane == 0) atomicAdd(P.done1 + U.e, 1);
       } else {
         const int row = TM * U.m + 32 * quad + lane;
 #pragma unroll
@@ -711,8 +782,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 template <int PHASE, int TN>
-moe_status launch_phase(const MxParams& P, const CUtensorMap& tw, const CUtensorMap& tb, const CUtensorMap& tb16,
-                        const CUtensorMap& tb8, const DeviceInfo& dev, cudaStream_t s) {
+moe_status launch_phase(const MxParams& P, const CUtensorMap& tw1, const CUtensorMap& tw2, const CUtensorMap& tx,
+                        const CUtensorMap& ta, const CUtensorMap& ta16, const CUtensorMap& ta8, const DeviceInfo& dev,
+                        cudaStream_t s) {
   const size_t smem = smem_bytes<PHASE, TN>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "MXFP4 decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
@@ -721,7 +793,19 @@ moe_status launch_phase(const MxParams& P, const CUtensorMap& tw, const CUtensor
                                       static_cast<int>(smem)));
     attr[dev.id] = smem;
   }
-  gemv_mx_kernel<PHASE, TN><<<dev.sm_count, THREADS, smem, s>>>(tw, tb, tb16, tb8, P);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(dev.sm_count);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  // the one-launch schedule's CTAs wait on each other's gate/up units: all of
+  // them must be resident at once, which a cooperative launch guarantees
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = PHASE == 3 ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_mx_kernel<PHASE, TN>, tw1, tw2, tx, ta, ta16, ta8, P));
   MOE_LAUNCH_CHECK("gemv_mx_kernel");
   return MOE_OK;
 }
@@ -746,7 +830,7 @@ CUresult encode_weight_map(CUtensorMap* map, const uint8_t* region0, int K, int 
 }
 
 struct MxWorkspace {
-  size_t xq, xs, aq, as, bytes;
+  size_t xq, xs, aq, as, done1, bytes;
 };
 
 MxWorkspace mx_workspace(moe_shape s, int T, int k) {
@@ -757,16 +841,29 @@ MxWorkspace mx_workspace(moe_shape s, int T, int k) {
   W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 32), 256);
   W.aq = o; o = round_up(o + static_cast<size_t>(NA) * n * s.I, 256);
   W.as = o; o = round_up(o + static_cast<size_t>(NA) * n * (s.I / 32), 256);
+  W.done1 = o; o = round_up(o + static_cast<size_t>(s.E) * sizeof(int32_t), 256);
   W.bytes = o;
   return W;
+}
+
+// Both GEMVs in one cooperative launch unless MOE_DECODE_TWO_LAUNCHES is set
+// in the environment (read once; the two-launch schedule is kept for
+// comparison).
+bool fused_decode() {
+  static const bool fused = std::getenv("MOE_DECODE_TWO_LAUNCHES") == nullptr;
+  return fused;
 }
 
 template <int TN>
 moe_status launch_both(const MxParams& P, const CUtensorMap& tw1, const CUtensorMap& tw2, const CUtensorMap& tx,
                        const CUtensorMap (&ta)[3], const DeviceInfo& dev, cudaStream_t stream) {
-  moe_status st = launch_phase<1, TN>(P, tw1, tx, tx, tx, dev, stream);
+  if (fused_decode()) {
+    MOE_CUDA_TRY(cudaMemsetAsync(P.done1, 0, static_cast<size_t>(P.E) * sizeof(int32_t), stream));
+    return launch_phase<3, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
+  }
+  moe_status st = launch_phase<1, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
   if (st != MOE_OK) return st;
-  return launch_phase<2, TN>(P, tw2, ta[2], ta[1], ta[0], dev, stream);
+  return launch_phase<2, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
 }
 
 }  // namespace
@@ -798,6 +895,7 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   P.xs = w8 + W.xs;
   P.aq = w8 + W.aq;
   P.as = w8 + W.as;
+  P.done1 = reinterpret_cast<int32_t*>(w8 + W.done1);
   P.y_perm = y_perm;
   P.out = out;
   P.status = status;
