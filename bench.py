@@ -473,12 +473,11 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
         mx = {f"T{t}": decode_point(cmx, t, 8, args.warmup, min(args.steps, 1000), stream, routed_only=True)
               for t in cmx.T}
     cached = split = layered = None
-    if not args.no_cached:
+    if not args.no_cached and world == 1:
         hp = cached_host_pool()
         cached = [run_cached_decode(hp, T=t) for t in (1, 8)]
-        if world == 1:
-            split = run_split_sweep(hp)
-            layered = run_layered_cache(hp)
+        split = run_split_sweep(hp)
+        layered = run_layered_cache(hp)
         del hp
 
     result = {
