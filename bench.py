@@ -321,7 +321,11 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
         print(f"warning: replicas stream only {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
               "between reuses", file=sys.stderr)
     stream = torch.cuda.Stream(device=dev)
-    launches_per_step = 5   # route, permute, ffn gate/up, ffn down, combine
+    # kernels per step: route, permute, the FFN (one cooperative launch, or
+    # gate/up + down with MOE_DECODE_TWO_LAUNCHES), combine; MXFP4 adds the
+    # split of x into E4M3 terms (the counter reset is a memset node)
+    two = os.environ.get("MOE_DECODE_TWO_LAUNCHES") is not None
+    launches_per_step = 4 + (1 if two else 0) + (1 if cfg.fmt == "mxfp4" else 0)
 
     def step_fn(r):
         L = r["layer"]
@@ -505,7 +509,8 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
             "cuda_graph": f"{G} steps per graph, cycling the replicas",
         },
         "roofline": {
-            "kernel": "moe_expert_ffn (gemv_tc_kernel gate/up + down)",
+            "kernel": "moe_expert_ffn: " + ("gemv_mx_kernel" if cfg.fmt == "mxfp4" else "gemv_tc_kernel")
+                      + (" gate/up + down (two launches)" if two else " (both GEMVs, one launch)"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
