@@ -777,7 +777,7 @@ def _route_on_gpu(cfg, trace, k):
 
 
 def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, sim_steps=128,
-                      n_gpu_layers=4, gpu_slots=64, steps=48, warm=16):
+                      n_gpu_layers=4, gpu_slots_per_layer=None, steps=48, warm=16):
     """The pages' global LRU (one expert cache whose decisions are shared by
     all MoE layers) against per-layer caches of equal total capacity.
     (a) Miss rates from the cache planner alone (plan-only handles) for
@@ -787,10 +787,11 @@ def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, s
         sharper routing need fewer slots), each layer's routing from
         moe_route_topk.
     (b) On the GPU: n_gpu_layers MXFP4 layers (E=256, d=4096, I=2048) over one
-        pinned host pool, gpu_slots slots in one shared cache vs gpu_slots /
-        n_gpu_layers per layer: step time for all layers and miss rate.
-    (c) Elastic resize of the shared cache: gpu_slots -> gpu_slots/2 -> gpu_slots
-        on a full cache, device-timed (moves only, no host copy)."""
+        pinned host pool, one shared cache of n_gpu_layers * S slots vs S per
+        layer (S = 16 at T=1, 64 at T=8, where a step can route to 48
+        experts): step time for all layers and miss rate.
+    (c) Elastic resize of the shared T=8 cache to half and back, on a full
+        cache, device-timed (moves only, no host copy)."""
     import expert_offload_serving_b200 as moe
     from expert_offload_serving_b200.layer import ExpertCache, MoeLayer
     base = synth.CONFIGS["decode_mxfp4"]
@@ -823,6 +824,8 @@ def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, s
     res_gpu = {}
     for mode in ("global", "per_layer"):
         for T in (1, 8):
+            per_layer_slots = gpu_slots_per_layer or (16 if T == 1 else 64)
+            gpu_slots = per_layer_slots * n_gpu_layers
             torch.cuda.synchronize()
             if mode == "global":
                 caches = [ExpertCache(s, gpu_slots, [host_pool] * n_gpu_layers)]
@@ -879,7 +882,7 @@ def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, s
                         f"{n_sim_layers * slots_per_layer} slots: global vs {slots_per_layer} per layer",
             **sim},
         "gpu": {"workload": f"{n_gpu_layers} MXFP4 layers (E={base.E} d={base.d} I={base.I} k={base.k}) over one pinned "
-                            f"host pool; {gpu_slots} slots shared vs {gpu_slots // n_gpu_layers} per layer; "
+                            f"host pool; {n_gpu_layers} x S slots shared vs S per layer (S = 16 at T=1, 64 at T=8); "
                             f"{steps} steps after {warm}", **res_gpu},
     }
 

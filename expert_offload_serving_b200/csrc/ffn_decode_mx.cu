@@ -83,13 +83,18 @@ struct MxParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  const uint8_t* xs;       // [NX][T][d/32] E8M0 scales of the x terms
   uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
-  uint8_t* as;             // [NA][T*k][I/32] their E8M0 scales
+  uint8_t* as;             // [NA][T*k][I/128][16] their E8M0 scales, 4 per 16-byte atom row
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
   float* y_perm;
   float* out;
   int32_t* status;
+};
+
+// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms and
+// their scale rows, the a terms and their scale rows (boxes of 8, 16, 32 rows).
+struct MxMaps {
+  CUtensorMap w1, w2, x, xs, a[3], as[3];
 };
 
 template <int PHASE, int TN>
@@ -271,7 +276,9 @@ __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restr
       uint4* dst = reinterpret_cast<uint4*>(xq + (static_cast<size_t>(term) * T + t) * d + 32 * b);
       dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-      xs[(static_cast<size_t>(term) * T + t) * nb + b] = static_cast<uint8_t>(sb);
+      // scale of block b in byte b % 4 of the 16-byte row of atom b / 4 (the
+      // tcgen05 scale-factor atom's row pitch, so one TMA box lands in place)
+      xs[((static_cast<size_t>(term) * T + t) * (nb / 4) + b / 4) * 16 + (b & 3)] = static_cast<uint8_t>(sb);
     }
   }
 }
@@ -300,52 +307,42 @@ __device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
 // unit's pairs get 2^0, their MMA columns are never read); they are made
 // visible to the tensor core's async proxy before lane 0 arrives.  Called by
 // all lanes of one warp.
+// Token-row terms of K stage ks of unit U into the B stage at sB, and their
+// E8M0 scale atoms after them, all by TMA (complete_tx on bar, whose expected
+// bytes lane 0 posts first): gemv<1> one-row loads of the x planes and of
+// their scale rows (lane q loads pair q0 + q), gemv<2> one box of a-plane
+// rows and of their scale rows per term.  The scales are stored with the
+// 16-byte row pitch of a scale-factor atom, so each box lands in place; rows
+// past the unit's pairs hold stale bytes, and their MMA columns are never
+// read.  Called by all lanes of one warp.
 template <class C, int TN>
-__device__ __forceinline__ void load_b(const MxParams& P, const Unit& U, int ks, int tok, uint8_t* sB,
-                                       uint64_t* bar, const CUtensorMap* tm_x, const CUtensorMap* tm_a,
-                                       const CUtensorMap* tm_a16, const CUtensorMap* tm_a8, uint64_t pol, int lane,
-                                       int n_pairs) {
+__device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const Unit& U, int ks, int tok,
+                                       uint8_t* sB, uint64_t* bar, uint64_t pol, int lane) {
   uint8_t* sf = sB + C::B_CODES;
   const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
-  if (lane < TN) {
-    const int K = U.ph == 1 ? P.d : P.I;
-    const int nb = K / 32;
-#pragma unroll
-    for (int j = 0; j < C::NT; ++j) {
-      if (j >= nt) break;
-      uint2 v = make_uint2(0x7f7f7f7fu, 0x7f7f7f7fu);
-      if (lane < U.nvalid) {
-        const size_t row = U.ph == 1 ? static_cast<size_t>(j) * P.T + tok
-                                     : static_cast<size_t>(j) * n_pairs + U.q0 + lane;
-        const uint8_t* src = (U.ph == 1 ? P.xs : P.as) + row * nb + 8 * ks;
-        v = *reinterpret_cast<const uint2*>(src);
-      }
-      *reinterpret_cast<uint32_t*>(sf + (2 * j) * 512 + lane * 16) = v.x;
-      *reinterpret_cast<uint32_t*>(sf + (2 * j + 1) * 512 + lane * 16) = v.y;
-    }
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncwarp();
   const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid)
                                   : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
-  if (lane == 0) mbar_expect_tx(bar, rows * static_cast<uint32_t>(nt) * 2 * 128u);
+  if (lane == 0) mbar_expect_tx(bar, rows * static_cast<uint32_t>(nt) * 2 * (128u + 16u));
   __syncwarp();
   if (U.ph == 2) {
     if (lane == 0) {
       const int bi = a_box<TN>(P, U.nvalid);
-      const CUtensorMap* tm = bi == 0 ? tm_a8 : (bi == 1 ? tm_a16 : tm_a);
 #pragma unroll
       for (int j = 0; j < NA; ++j)
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tma_load_3d(sB + (2 * j + h) * C::B_ATOM, tm, bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(sB + (2 * j + h) * C::B_ATOM, &M.a[bi], bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
+          tma_load_4d(sf + (2 * j + h) * 512, &M.as[bi], bar, 0, 2 * ks + h, U.q0, j, pol);
+        }
     }
   } else if (lane < U.nvalid) {
 #pragma unroll
     for (int j = 0; j < NX; ++j)
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, tm_x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, &M.x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
+        tma_load_4d(sf + (2 * j + h) * 512 + lane * 16, &M.xs, bar, 0, 2 * ks + h, tok, j, pol);
+      }
   }
 }
 
@@ -419,10 +416,7 @@ __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
 template <int PHASE, int TN>
 __global__ void __launch_bounds__(THREADS, 1)
-    gemv_mx_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
-                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_a,
-                   const __grid_constant__ CUtensorMap tm_a16, const __grid_constant__ CUtensorMap tm_a8,
-                   MxParams P) {
+    gemv_mx_kernel(const __grid_constant__ MxMaps M, const MxParams P) {
   using C = Cfg<PHASE, TN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -530,7 +524,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int sl = __ldg(P.slot + U.e);
       const uint8_t* abase = tile_base(P, U);
-      const CUtensorMap* tm_w = U.ph == 1 ? &tm_w1 : &tm_w2;
+      const CUtensorMap* tm_w = U.ph == 1 ? &M.w1 : &M.w2;
       const int KS = ks_of(U);
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
@@ -599,8 +593,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = false;
           break;
         }
-        load_b<C, TN>(P, U, ks, tok, ring_b + stage * C::B_STAGE, &bfull[stage], &tm_x, &tm_a, &tm_a16, &tm_a8,
-                             pol_keep, lane, n_pairs);
+        load_b<C, TN>(P, M, U, ks, tok, ring_b + stage * C::B_STAGE, &bfull[stage], pol_keep, lane);
         __syncwarp();
         ++issued;
         if (++stage == C::SB) {
@@ -743,7 +736,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 r -= times_pow2(e4m3_to_f32(t), sb);
                 const size_t plane = static_cast<size_t>(j) * n_pairs;
                 P.aq[(plane + q) * P.I + col] = static_cast<uint8_t>(t);
-                if (lane == 0) P.as[(plane + q) * nbi + blk] = static_cast<uint8_t>(sb);
+                if (lane == 0) P.as[((plane + q) * (nbi / 4) + blk / 4) * 16 + (blk & 3)] = static_cast<uint8_t>(sb);
               }
             }
           }
@@ -782,9 +775,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 template <int PHASE, int TN>
-moe_status launch_phase(const MxParams& P, const CUtensorMap& tw1, const CUtensorMap& tw2, const CUtensorMap& tx,
-                        const CUtensorMap& ta, const CUtensorMap& ta16, const CUtensorMap& ta8, const DeviceInfo& dev,
-                        cudaStream_t s) {
+moe_status launch_phase(const MxParams& P, const MxMaps& M, const DeviceInfo& dev, cudaStream_t s) {
   const size_t smem = smem_bytes<PHASE, TN>(P.E);
   if (smem > dev.smem_optin) return fail(MOE_ERR_UNSUPPORTED, "MXFP4 decode GEMV needs %zu bytes of shared memory", smem);
   static size_t attr[64] = {};
@@ -805,7 +796,7 @@ moe_status launch_phase(const MxParams& P, const CUtensorMap& tw1, const CUtenso
   at[0].val.cooperative = PHASE == 3 ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_mx_kernel<PHASE, TN>, tw1, tw2, tx, ta, ta16, ta8, P));
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_mx_kernel<PHASE, TN>, M, P));
   MOE_LAUNCH_CHECK("gemv_mx_kernel");
   return MOE_OK;
 }
@@ -838,9 +829,9 @@ MxWorkspace mx_workspace(moe_shape s, int T, int k) {
   const size_t n = static_cast<size_t>(T) * k;
   size_t o = 0;
   W.xq = o; o = round_up(o + static_cast<size_t>(NX) * T * s.d, 256);
-  W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 32), 256);
+  W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 128) * 16, 256);
   W.aq = o; o = round_up(o + static_cast<size_t>(NA) * n * s.I, 256);
-  W.as = o; o = round_up(o + static_cast<size_t>(NA) * n * (s.I / 32), 256);
+  W.as = o; o = round_up(o + static_cast<size_t>(NA) * n * (s.I / 128) * 16, 256);
   W.done1 = o; o = round_up(o + static_cast<size_t>(s.E) * sizeof(int32_t), 256);
   W.bytes = o;
   return W;
@@ -855,15 +846,14 @@ bool fused_decode() {
 }
 
 template <int TN>
-moe_status launch_both(const MxParams& P, const CUtensorMap& tw1, const CUtensorMap& tw2, const CUtensorMap& tx,
-                       const CUtensorMap (&ta)[3], const DeviceInfo& dev, cudaStream_t stream) {
+moe_status launch_both(const MxParams& P, const MxMaps& M, const DeviceInfo& dev, cudaStream_t stream) {
   if (fused_decode()) {
     MOE_CUDA_TRY(cudaMemsetAsync(P.done1, 0, static_cast<size_t>(P.E) * sizeof(int32_t), stream));
-    return launch_phase<3, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
+    return launch_phase<3, TN>(P, M, dev, stream);
   }
-  moe_status st = launch_phase<1, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
+  moe_status st = launch_phase<1, TN>(P, M, dev, stream);
   if (st != MOE_OK) return st;
-  return launch_phase<2, TN>(P, tw1, tw2, tx, ta[2], ta[1], ta[0], dev, stream);
+  return launch_phase<2, TN>(P, M, dev, stream);
 }
 
 }  // namespace
@@ -892,7 +882,6 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   P.pool = static_cast<const uint8_t*>(pool);
   P.L = blob_layout(s.fmt, s.d, s.I);
   P.blob_bytes = P.L.bytes;
-  P.xs = w8 + W.xs;
   P.aq = w8 + W.aq;
   P.as = w8 + W.as;
   P.done1 = reinterpret_cast<int32_t*>(w8 + W.done1);
@@ -904,22 +893,32 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint64_t r = static_cast<uint64_t>(8) << i;
     P.a_box_rows[i] = static_cast<int>(n < r ? n : r);
   }
-  CUtensorMap tw1, tw2, tx, ta[3];
-  CUresult r = encode_weight_map(&tw1, P.pool + P.L.wg, s.d, 2 * s.I, n_slots, P.blob_bytes);
-  if (r == CUDA_SUCCESS) r = encode_weight_map(&tw2, P.pool + P.L.wd, s.I, s.d, n_slots, P.blob_bytes);
+  MxMaps M;
+  CUresult r = encode_weight_map(&M.w1, P.pool + P.L.wg, s.d, 2 * s.I, n_slots, P.blob_bytes);
+  if (r == CUDA_SUCCESS) r = encode_weight_map(&M.w2, P.pool + P.L.wd, s.I, s.d, n_slots, P.blob_bytes);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the MXFP4 weights failed (%d)", static_cast<int>(r));
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T), static_cast<uint64_t>(NX)};
     const uint64_t str[2] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T) * s.d};
     const uint32_t box[3] = {128u, 1u, 1u};
-    r = encode_tiled_sw128(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
+    r = encode_tiled_sw128(&M.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
+    // scale rows of the x terms: (byte in the 16-byte atom row, atom, token, term)
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.d / 128), static_cast<uint64_t>(T), static_cast<uint64_t>(NX)};
+    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.d / 128) * 16, static_cast<uint64_t>(T) * (s.d / 128) * 16};
+    const uint32_t sbox[4] = {16u, 1u, 1u, 1u};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.xs, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
   }
   for (int i = 0; i < 3; ++i) {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, static_cast<uint64_t>(NA)};
     const uint64_t str[2] = {static_cast<uint64_t>(s.I), n * s.I};
     const uint32_t box[3] = {128u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
-    r = encode_tiled_sw128(&ta[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
+    r = encode_tiled_sw128(&M.a[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
+    // scale rows of the a terms: (byte in the atom row, atom, pair, term); a box of rows
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(NA)};
+    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, n * (s.I / 128) * 16};
+    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a terms failed (%d)", static_cast<int>(r));
   }
   {
@@ -928,7 +927,7 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     mx_split_x_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq, w8 + W.xs);
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
-  return T <= 16 ? launch_both<16>(P, tw1, tw2, tx, ta, dev, stream) : launch_both<32>(P, tw1, tw2, tx, ta, dev, stream);
+  return T <= 16 ? launch_both<16>(P, M, dev, stream) : launch_both<32>(P, M, dev, stream);
 }
 
 }  // namespace moe

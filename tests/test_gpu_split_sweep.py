@@ -107,7 +107,8 @@ def test_split_step_host_kernel_concurrent(moe, q):
     step's split and fills equal the oracle's, and its output the oracle
     layer's."""
     from expert_offload_serving_b200.layer import MoeLayer, pack_pool
-    cfg = synth.LayerConfig("split_step", E=64, k=6, d=512, I=256, fmt="mxfp4", bias_std=0.5, n_slots=16,
+    # 32 slots: a step of T = 4 tokens can need 24 (q = 1 fills every miss)
+    cfg = synth.LayerConfig("split_step", E=64, k=6, d=512, I=256, fmt="mxfp4", bias_std=0.5, n_slots=32,
                             rho=0.9)
     T = 4
     bw = (50.0, 120.0)
