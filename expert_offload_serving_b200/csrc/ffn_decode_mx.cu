@@ -347,27 +347,40 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 }
 
 // One-launch schedule: lane 0 waits (bounded, like every wait) until all
-// `target` gate/up units of expert e have published their a terms, then
-// orders the TMA loads that follow after what it observed.  One verdict for
-// the warp.
-__device__ __forceinline__ bool wait_expert_ready(const MxParams& P, int e, int target, volatile int* abort_flag,
-                                                  int lane) {
+// `target` gate/up units of expert e have published their a rows, then orders
+// the TMA loads that follow after what it observed.  `seen` is the counter
+// value lane 0 loaded ahead of time (relaxed, while the previous unit
+// streamed): when it already reaches the target, a fence gives the acquire
+// without another trip to memory.  One verdict for the warp.
+__device__ __forceinline__ bool wait_expert_ready(const MxParams& P, int e, int target, int seen,
+                                                  volatile int* abort_flag, int lane) {
   bool ok = true;
   if (lane == 0) {
-    const uint64_t t0 = now_ns();
-    for (;;) {
-      int v;
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
-      if (v >= target) break;
-      if (*abort_flag || now_ns() - t0 > P.wait_ns) {
-        ok = false;
-        break;
+    if (seen >= target) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    } else {
+      const uint64_t t0 = now_ns();
+      for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+        if (v >= target) break;
+        if (*abort_flag || now_ns() - t0 > P.wait_ns) {
+          ok = false;
+          break;
+        }
+        __nanosleep(256);
       }
-      __nanosleep(256);
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
   }
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// The counter of expert e, loaded without ordering (a prefetch for the wait above).
+__device__ __forceinline__ int peek_expert_counter(const MxParams& P, int e) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void drain_ring(uint64_t* full, int n, int issued, int stage, uint32_t phase) {
@@ -577,16 +590,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
+    int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int tok = token_of(P, U, lane, n_pairs);
       const int KS = ks_of(U);
       if (PHASE == 3 && U.ph == 2) {
         // the a terms of this expert's pairs come from every gate/up unit of the expert
-        if (!wait_expert_ready(P, U.e, ustart[U.e + 1] - ustart[U.e], abort_flag, lane)) {
+        if (!wait_expert_ready(P, U.e, ustart[U.e + 1] - ustart[U.e], seen, abort_flag, lane)) {
           ok = false;
           break;
         }
+      }
+      if (PHASE == 3 && lane == 0 && u + static_cast<int>(gridDim.x) < n_units) {
+        const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, u + gridDim.x);
+        seen = V.ph == 2 ? peek_expert_counter(P, V.e) : -1;   // consumed at the next unit
       }
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {

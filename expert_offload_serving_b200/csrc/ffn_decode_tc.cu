@@ -253,27 +253,41 @@ __device__ __forceinline__ void load_b(const TcDecodeParams& P, const Unit& U, i
   }
 }
 
-// Fused launch: lane 0 waits (bounded, like every wait) until all `target`
-// gate/up units of expert e have published their a rows, then orders the
-// TMA loads that follow after what it observed.  One verdict for the warp.
-__device__ __forceinline__ bool wait_expert_ready(const TcDecodeParams& P, int e, int target,
+// One-launch schedule: lane 0 waits (bounded, like every wait) until all
+// `target` gate/up units of expert e have published their a rows, then orders
+// the TMA loads that follow after what it observed.  `seen` is the counter
+// value lane 0 loaded ahead of time (relaxed, while the previous unit
+// streamed): when it already reaches the target, a fence gives the acquire
+// without another trip to memory.  One verdict for the warp.
+__device__ __forceinline__ bool wait_expert_ready(const TcDecodeParams& P, int e, int target, int seen,
                                                   volatile int* abort_flag, int lane) {
   bool ok = true;
   if (lane == 0) {
-    const uint64_t t0 = now_ns();
-    for (;;) {
-      int v;
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
-      if (v >= target) break;
-      if (*abort_flag || now_ns() - t0 > P.wait_ns) {
-        ok = false;
-        break;
+    if (seen >= target) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    } else {
+      const uint64_t t0 = now_ns();
+      for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+        if (v >= target) break;
+        if (*abort_flag || now_ns() - t0 > P.wait_ns) {
+          ok = false;
+          break;
+        }
+        __nanosleep(256);
       }
-      __nanosleep(256);
     }
     asm volatile("fence.proxy.async.global;" ::: "memory");
   }
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// The counter of expert e, loaded without ordering (a prefetch for the wait above).
+__device__ __forceinline__ int peek_expert_counter(const TcDecodeParams& P, int e) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(P.done1 + e) : "memory");
+  return v;
 }
 
 // Waits for the copies of the last min(issued, n) stages of a ring to land.
@@ -453,6 +467,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
+    int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int tok = token_of(P, U, lane, n_pairs);
@@ -460,10 +475,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
       if (PHASE == 3 && U.ph == 2) {
         // the a rows of this expert's pairs come from every gate/up unit of the expert
         const int target = ustart[U.e + 1] - ustart[U.e];
-        if (!wait_expert_ready(P, U.e, target, abort_flag, lane)) {
+        if (!wait_expert_ready(P, U.e, target, seen, abort_flag, lane)) {
           ok = false;
           break;
         }
+      }
+      if (PHASE == 3 && lane == 0 && u + static_cast<int>(gridDim.x) < n_units) {
+        const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, u + gridDim.x);
+        seen = V.ph == 2 ? peek_expert_counter(P, V.e) : -1;   // consumed at the next unit
       }
       for (int ks = 0; ks < KS; ++ks) {
         if (!__all_sync(0xffffffffu, mbar_wait<true>(&bempty[stage], phase ^ 1u, abort_flag, P.wait_ns))) {
