@@ -73,6 +73,7 @@ constexpr int BPROD_WARP = 6;
 
 struct MxParams {
   uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
+  int pf_items;              // L2 prefetch distance in stages
   int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
   int a_box_rows[3];       // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
@@ -83,6 +84,7 @@ struct MxParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
+  const uint8_t* xs;       // [NX][T][d/128][16] E8M0 scales of the x terms, 4 per 16-byte atom row
   uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
   uint8_t* as;             // [NA][T*k][I/128][16] their E8M0 scales, 4 per 16-byte atom row
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
@@ -91,10 +93,10 @@ struct MxParams {
   int32_t* status;
 };
 
-// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms and
-// their scale rows, the a terms and their scale rows (boxes of 8, 16, 32 rows).
+// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms, the
+// a terms and their scale rows (boxes of 8, 16, 32 rows).
 struct MxMaps {
-  CUtensorMap w1, w2, x, xs, a[3], as[3];
+  CUtensorMap w1, w2, x, a[3], as[3];
 };
 
 template <int PHASE, int TN>
@@ -239,8 +241,11 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 // One thread per 32-element block of a token row: NX E4M3 terms of the
 // bf16 values, each term with the E8M0 scale of the block's remaining maximum.
 __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int d,
-                                                         uint8_t* __restrict__ xq, uint8_t* __restrict__ xs) {
+                                                         uint8_t* __restrict__ xq, uint8_t* __restrict__ xs,
+                                                         int32_t* __restrict__ zero, int n_zero) {
   const int nb = d / 32;
+  // the one-launch GEMV's per-expert counters start at zero (this kernel runs right before it)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
   const long long n = static_cast<long long>(T) * nb;
   for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
        g += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -308,13 +313,15 @@ __device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
 // visible to the tensor core's async proxy before lane 0 arrives.  Called by
 // all lanes of one warp.
 // Token-row terms of K stage ks of unit U into the B stage at sB, and their
-// E8M0 scale atoms after them, all by TMA (complete_tx on bar, whose expected
-// bytes lane 0 posts first): gemv<1> one-row loads of the x planes and of
-// their scale rows (lane q loads pair q0 + q), gemv<2> one box of a-plane
-// rows and of their scale rows per term.  The scales are stored with the
-// 16-byte row pitch of a scale-factor atom, so each box lands in place; rows
-// past the unit's pairs hold stale bytes, and their MMA columns are never
-// read.  Called by all lanes of one warp.
+// E8M0 scale atoms after them, all asynchronous copies completing on bar
+// (whose expected bytes lane 0 posts first): gemv<1> one-row TMA loads of the
+// x planes and 16-byte bulk copies of their scale rows (lane q: pair q0 + q;
+// a tensor copy needs a 128-byte-aligned destination, an atom row is 16
+// bytes), gemv<2> one TMA box of a-plane rows and of their scale rows per
+// term (the box lands on a 512-byte atom).  The scales are stored with the
+// 16-byte row pitch of a scale-factor atom, so every copy lands in place;
+// rows past the unit's pairs hold stale bytes, and their MMA columns are
+// never read.  Called by all lanes of one warp.
 template <class C, int TN>
 __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const Unit& U, int ks, int tok,
                                        uint8_t* sB, uint64_t* bar, uint64_t pol, int lane) {
@@ -341,7 +348,8 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, &M.x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
-        tma_load_4d(sf + (2 * j + h) * 512 + lane * 16, &M.xs, bar, 0, 2 * ks + h, tok, j, pol);
+        bulk_load(sf + (2 * j + h) * 512 + lane * 16,
+                  P.xs + ((static_cast<size_t>(j) * P.T + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
       }
   }
 }
@@ -553,7 +561,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_5d(sA + A_BOX, tm_w, &full[stage], 128, 0, ks, U.m, sl, pol_stream);
           bulk_load(sA + 2 * A_BOX, abase + static_cast<size_t>(ks) * kMxTileBytes + 16384, 1024, &full[stage],
                     pol_stream);
-          while (pf_u < n_units && pf_ahead < PF_ITEMS) {
+          while (pf_u < n_units && pf_ahead < P.pf_items) {
             prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * kMxTileBytes, kMxTileBytes);
             ++pf_ahead;
             if (++pf_ks == pf_KS) {
@@ -865,10 +873,7 @@ bool fused_decode() {
 
 template <int TN>
 moe_status launch_both(const MxParams& P, const MxMaps& M, const DeviceInfo& dev, cudaStream_t stream) {
-  if (fused_decode()) {
-    MOE_CUDA_TRY(cudaMemsetAsync(P.done1, 0, static_cast<size_t>(P.E) * sizeof(int32_t), stream));
-    return launch_phase<3, TN>(P, M, dev, stream);
-  }
+  if (fused_decode()) return launch_phase<3, TN>(P, M, dev, stream);   // counters zeroed by mx_split_x_kernel
   moe_status st = launch_phase<1, TN>(P, M, dev, stream);
   if (st != MOE_OK) return st;
   return launch_phase<2, TN>(P, M, dev, stream);
@@ -886,6 +891,10 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   MxParams P{};
   P.wait_ns = wait_limit_ns();
+  {
+    static const char* pf = std::getenv("MOE_DECODE_PF");   // tuning sweep
+    P.pf_items = pf ? std::atoi(pf) : PF_ITEMS;
+  }
   P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
@@ -900,6 +909,7 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   P.pool = static_cast<const uint8_t*>(pool);
   P.L = blob_layout(s.fmt, s.d, s.I);
   P.blob_bytes = P.L.bytes;
+  P.xs = w8 + W.xs;
   P.aq = w8 + W.aq;
   P.as = w8 + W.as;
   P.done1 = reinterpret_cast<int32_t*>(w8 + W.done1);
@@ -920,11 +930,6 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint64_t str[2] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T) * s.d};
     const uint32_t box[3] = {128u, 1u, 1u};
     r = encode_tiled_sw128(&M.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
-    // scale rows of the x terms: (byte in the 16-byte atom row, atom, token, term)
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.d / 128), static_cast<uint64_t>(T), static_cast<uint64_t>(NX)};
-    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.d / 128) * 16, static_cast<uint64_t>(T) * (s.d / 128) * 16};
-    const uint32_t sbox[4] = {16u, 1u, 1u, 1u};
-    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.xs, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
   }
   for (int i = 0; i < 3; ++i) {
@@ -942,7 +947,8 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   {
     const long long blocks = static_cast<long long>(T) * (s.d / 32);
     const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
-    mx_split_x_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq, w8 + W.xs);
+    mx_split_x_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq, w8 + W.xs,
+                                                P.done1, fused_decode() ? s.E : 0);
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
   return T <= 16 ? launch_both<16>(P, M, dev, stream) : launch_both<32>(P, M, dev, stream);

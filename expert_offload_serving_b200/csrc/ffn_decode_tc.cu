@@ -42,6 +42,7 @@ namespace moe {
 
 struct TcDecodeParams {
   uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
+  int pf_items;              // L2 prefetch distance in stages
   int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
   int a_box_rows[3];         // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
           // keep the L2 prefetch cursor PF_ITEMS stages ahead of this one (the
           // bulk copies of a CTA complete in order, so prefetching whole blobs
           // up front would queue ahead of the stages the pipeline waits for)
-          while (pf_u < n_units && pf_ahead < PF_ITEMS) {
+          while (pf_u < n_units && pf_ahead < P.pf_items) {
             prefetch_l2(pf_base + static_cast<size_t>(pf_ks) * C::A_STAGE, C::A_STAGE);
             ++pf_ahead;
             if (++pf_ks == pf_KS) {
@@ -713,6 +714,10 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
   TcDecodeParams P{};
   P.wait_ns = wait_limit_ns();
+  {
+    static const char* pf = std::getenv("MOE_DECODE_PF");   // tuning sweep
+    P.pf_items = pf ? std::atoi(pf) : PF_ITEMS;
+  }
   P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
