@@ -18,15 +18,19 @@
 //                                     than ~2^18 below its block's maximum;
 //   a (fp32, the SwiGLU output)   -> 4 terms (16 significant bits), residual
 //                                     below 2^-16 of each block's maximum.
-// Each term is one MMA; the accumulator is fp32 in TMEM.
+// The terms are stacked along N: term j's TN token rows are B rows
+// j*TN .. j*TN+TN-1, so one MMA per 32-element K step reads the weight tile
+// from shared memory once for all terms (a skinny MMA costs about the same
+// whatever its N: the A operand read dominates), and the epilogue adds the
+// terms' fp32 accumulator columns.
 //
 //   split_x:  x [T][d] -> 2 E4M3 planes + 2 scale planes, once per token.
-//   gemv<1>:  D[128 x N] = W_gu tile (64 gate + 64 up rows of the same
-//             intermediate indices) x X^T over K = d, N <= TN token rows
-//             gathered by one-row TMA loads.  Epilogue: a = silu(D_gate) *
+//   gemv<1>:  D[128 x 2 TN] = W_gu tile (64 gate + 64 up rows of the same
+//             intermediate indices) x [X_0; X_1]^T over K = d, the x terms
+//             of <= TN token rows gathered by one-row TMA loads.  Epilogue: a = silu(D_gate) *
 //             D_up split into 4 E4M3 planes + scales (warp-wide maxima over
 //             the 32 lanes = one 32-element block of I).
-//   gemv<2>:  D[128 x N] = W_d tile x A^T over K = I, 4 MMAs per K step.
+//   gemv<2>:  D[128 x 4 TN] = W_d tile x [A_0; A_1; A_2; A_3]^T over K = I.
 //             Epilogue: y_perm rows, or out[t] += gate * y (fused combine).
 //
 // Work unit = (expert, 128-row tile, chunk of <= TN pairs), expert-major,
@@ -58,10 +62,10 @@ constexpr int A_SMEM = 2 * A_BOX + 1024;   // codes (expanded) + 2 scale atoms
 // bytes a weight stage's barrier expects: the 16U4_ALIGN16B loads count the
 // packed codes they read (8 KB per box), not the expanded 16 KB they write
 constexpr uint32_t A_TX = 2 * (A_BOX / 2) + 1024;
-constexpr int ACC_COLS = 32;
-constexpr int SFA_COL = 64;                // TMEM: 2 accumulators, then scale factors
-constexpr int SFB_COL = 72;
-constexpr int TMEM_COLS = 128;
+constexpr int ACC_COLS = 128;              // 4 terms x 32 token rows
+constexpr int SFA_COL = 2 * ACC_COLS;      // TMEM: 2 accumulators, then scale factors
+constexpr int SFB_COL = SFA_COL + 8;
+constexpr int TMEM_COLS = 512;
 constexpr int NX = 2;                      // E4M3 terms of x
 constexpr int NA = 4;                      // E4M3 terms of a
 constexpr int PF_ITEMS = 8;                // L2 prefetch distance (tiles)
@@ -84,9 +88,9 @@ struct MxParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  const uint8_t* xs;       // [NX][T][d/128][16] E8M0 scales of the x terms, 4 per 16-byte atom row
+  const uint8_t* xs;       // [32/TN][T][d/128][16] E8M0 scales of the x terms (sf_plane / sf_byte)
   uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
-  uint8_t* as;             // [NA][T*k][I/128][16] their E8M0 scales, 4 per 16-byte atom row
+  uint8_t* as;             // [32/TN][T*k][I/128][16] their E8M0 scales (sf_plane / sf_byte)
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
   float* y_perm;
   float* out;
@@ -99,12 +103,24 @@ struct MxMaps {
   CUtensorMap w1, w2, x, a[3], as[3];
 };
 
+// Scale rows of stacked terms.  B row r = j*TN + t (term j, token row t)
+// takes its 4 scales of a 128-element half from byte 4*(r/32) of the 16-byte
+// row r%32 of the half's scale-factor atom.  With G = 32/TN term row blocks
+// per 32 atom rows, term j sits in plane j%G (atom rows (j%G)*TN + t) at byte
+// group j/G, so the scale rows of a term plane are stored [plane][row][atom]
+// with 16 bytes per row: one copy of a plane's rows lands in place.
+template <int TN>
+__device__ __forceinline__ int sf_plane(int j) { return j % (32 / TN); }
+template <int TN>
+__device__ __forceinline__ int sf_byte(int j) { return 4 * (j / (32 / TN)); }
+
 template <int PHASE, int TN>
 struct Cfg {
   static constexpr int NT = PHASE == 1 ? NX : NA;                // terms of the B operand (PHASE 3: both GEMVs)
+  static constexpr int G = 32 / TN;                              // scale planes
   static constexpr int B_ATOM = TN * 128;                        // TN rows x 128 E4M3 values
-  static constexpr int B_CODES = NT * 2 * B_ATOM;                // 2 atoms (256 K) per term
-  static constexpr int B_STAGE = B_CODES + NT * 1024;            // + 2 scale atoms per term
+  static constexpr int B_CODES = NT * 2 * B_ATOM;                // per 128-element half: the terms' rows stacked
+  static constexpr int B_STAGE = B_CODES + 1024;                 // + one scale atom per half
   static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
   // token-row stages: gemv<2>'s come from the a terms gemv<1> just wrote (L2)
@@ -118,7 +134,7 @@ struct Cfg {
   static_assert(A_SMEM % 1024 == 0 && B_STAGE % 1024 == 0 && B_ATOM % 1024 == 0, "1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
   static_assert(FIXED + A_RING + B_RING <= kSmemBudget, "shared memory budget");
-  static_assert(SFB_COL + 8 * NT <= TMEM_COLS, "TMEM budget");
+  static_assert(SFB_COL + 8 <= TMEM_COLS && NT * TN <= ACC_COLS, "TMEM budget");
   static_assert(N_BARS * 8 + 16 <= kBarBytes, "barrier area");
 };
 
@@ -240,6 +256,8 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 // ------------------------------------------------------------------ split_x
 // One thread per 32-element block of a token row: NX E4M3 terms of the
 // bf16 values, each term with the E8M0 scale of the block's remaining maximum.
+// TN: the GEMV's token rows per term (the scale rows' plane and byte group).
+template <int TN>
 __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int d,
                                                          uint8_t* __restrict__ xq, uint8_t* __restrict__ xs,
                                                          int32_t* __restrict__ zero, int n_zero) {
@@ -281,9 +299,11 @@ __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restr
       uint4* dst = reinterpret_cast<uint4*>(xq + (static_cast<size_t>(term) * T + t) * d + 32 * b);
       dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-      // scale of block b in byte b % 4 of the 16-byte row of atom b / 4 (the
-      // tcgen05 scale-factor atom's row pitch, so one TMA box lands in place)
-      xs[((static_cast<size_t>(term) * T + t) * (nb / 4) + b / 4) * 16 + (b & 3)] = static_cast<uint8_t>(sb);
+      // scale of block b in byte b % 4 of the term's byte group of the 16-byte
+      // row of atom b / 4 (the tcgen05 scale-factor atom's row pitch, so one
+      // copy of a row lands in place)
+      xs[((static_cast<size_t>(sf_plane<TN>(term)) * T + t) * (nb / 4) + b / 4) * 16 + sf_byte<TN>(term) + (b & 3)] =
+          static_cast<uint8_t>(sb);
     }
   }
 }
@@ -306,22 +326,16 @@ __device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
 }
 
 // Token-row terms of K stage ks of unit U into the B stage at sB, and their
-// E8M0 scale atoms after them: gemv<1> one-row TMA loads of the x planes
-// (lane q loads pair q0 + q), gemv<2> one box of a-plane rows per term.
-// The scale bytes are plain loads and shared-memory stores (rows past the
-// unit's pairs get 2^0, their MMA columns are never read); they are made
-// visible to the tensor core's async proxy before lane 0 arrives.  Called by
-// all lanes of one warp.
-// Token-row terms of K stage ks of unit U into the B stage at sB, and their
 // E8M0 scale atoms after them, all asynchronous copies completing on bar
-// (whose expected bytes lane 0 posts first): gemv<1> one-row TMA loads of the
-// x planes and 16-byte bulk copies of their scale rows (lane q: pair q0 + q;
-// a tensor copy needs a 128-byte-aligned destination, an atom row is 16
-// bytes), gemv<2> one TMA box of a-plane rows and of their scale rows per
-// term (the box lands on a 512-byte atom).  The scales are stored with the
-// 16-byte row pitch of a scale-factor atom, so every copy lands in place;
-// rows past the unit's pairs hold stale bytes, and their MMA columns are
-// never read.  Called by all lanes of one warp.
+// (whose expected bytes lane 0 posts first).  Per 128-element half h the
+// terms' rows are stacked (term j at rows j*TN..) in one 128-byte-swizzled
+// tile, and one scale atom covers them all.  gemv<1>: one-row TMA loads of
+// the x planes and 16-byte bulk copies of their scale rows (lane q: pair
+// q0 + q; a tensor copy needs a 128-byte-aligned destination, an atom row is
+// 16 bytes); gemv<2>: one TMA box of a-plane rows per term and one box of
+// scale rows per scale plane (landing on a 256-byte boundary).  Rows past the
+// unit's pairs hold stale bytes; their MMA columns are never read.  Called by
+// all lanes of one warp.
 template <class C, int TN>
 __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const Unit& U, int ks, int tok,
                                        uint8_t* sB, uint64_t* bar, uint64_t pol, int lane) {
@@ -329,28 +343,32 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
   const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
   const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid)
                                   : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
-  if (lane == 0) mbar_expect_tx(bar, rows * static_cast<uint32_t>(nt) * 2 * (128u + 16u));
+  if (lane == 0) mbar_expect_tx(bar, rows * 2 * (static_cast<uint32_t>(nt) * 128u + C::G * 16u));
   __syncwarp();
   if (U.ph == 2) {
     if (lane == 0) {
       const int bi = a_box<TN>(P, U.nvalid);
 #pragma unroll
-      for (int j = 0; j < NA; ++j)
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tma_load_3d(sB + (2 * j + h) * C::B_ATOM, &M.a[bi], bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
-          tma_load_4d(sf + (2 * j + h) * 512, &M.as[bi], bar, 0, 2 * ks + h, U.q0, j, pol);
-        }
+        for (int j = 0; j < NA; ++j)
+          tma_load_3d(sB + (h * NA + j) * C::B_ATOM, &M.a[bi], bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
+#pragma unroll
+        for (int g = 0; g < C::G; ++g)
+          tma_load_4d(sf + h * 512 + g * TN * 16, &M.as[bi], bar, 0, 2 * ks + h, U.q0, g, pol);
+      }
     }
   } else if (lane < U.nvalid) {
 #pragma unroll
-    for (int j = 0; j < NX; ++j)
+    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tma_load_3d(sB + (2 * j + h) * C::B_ATOM + lane * 128, &M.x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
-        bulk_load(sf + (2 * j + h) * 512 + lane * 16,
-                  P.xs + ((static_cast<size_t>(j) * P.T + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
-      }
+      for (int j = 0; j < NX; ++j)
+        tma_load_3d(sB + (h * NX + j) * C::B_ATOM + lane * 128, &M.x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
+#pragma unroll
+      for (int g = 0; g < C::G; ++g)
+        bulk_load(sf + h * 512 + (g * TN + lane) * 16,
+                  P.xs + ((static_cast<size_t>(g) * P.T + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
+    }
   }
 }
 
@@ -434,6 +452,34 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a, uint64_t 
 }
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
+
+// Token row c's result for this warp's 32 TMEM lanes: the sum over the nt
+// stacked terms of accumulator columns j*TN + c (fp32, terms in order).
+template <int TN>
+__device__ __forceinline__ void load_terms(uint32_t taddr, int nt, float (&v)[32]) {
+  if (TN == 16) {
+    float t[16];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NA; ++j) {
+      if (j >= nt) break;
+      tmem_ld16(taddr + 16 * j, t);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) v[c] += t[c];
+    }
+  } else {
+    float t[32];
+    tmem_ld32(taddr, v);
+#pragma unroll
+    for (int j = 1; j < NA; ++j) {
+      if (j >= nt) break;
+      tmem_ld32(taddr + 32 * j, t);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] += t[c];
+    }
+  }
+}
 
 template <int PHASE, int TN>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -642,8 +688,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int KS = ks_of(U);
-      const int nt = U.ph == 1 ? NX : NA;       // terms of the unit's B operand
-      const int n_mma = U.nvalid <= 16 ? 16 : 32;
+      const int nt = U.ph == 1 ? NX : NA;       // terms of the unit's B operand, stacked along N
+      const uint32_t n_mma = static_cast<uint32_t>(nt * TN);
       const int acc = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait<true>(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
         ok = false;
@@ -662,27 +708,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (elect_one()) {
           const uint8_t* sA = smem + sa * A_SMEM;
           const uint8_t* sB = ring_b + sb * C::B_STAGE;
-          // scale atoms -> TMEM: weights (2 atoms = 8 blocks of 32), then each term's
+          // scale atoms -> TMEM: weights and token-row terms, one atom per
+          // 128-element half (4 blocks of 32)
           tc_cp_sf(tmem + SFA_COL, desc_sf(smem_u32(sA + 2 * A_BOX)));
           tc_cp_sf(tmem + SFA_COL + 4, desc_sf(smem_u32(sA + 2 * A_BOX + 512)));
-#pragma unroll
-          for (int j = 0; j < C::NT; ++j) {
-            if (j >= nt) break;
-            tc_cp_sf(tmem + SFB_COL + 8 * j, desc_sf(smem_u32(sB + C::B_CODES + (2 * j) * 512)));
-            tc_cp_sf(tmem + SFB_COL + 8 * j + 4, desc_sf(smem_u32(sB + C::B_CODES + (2 * j + 1) * 512)));
-          }
+          tc_cp_sf(tmem + SFB_COL, desc_sf(smem_u32(sB + C::B_CODES)));
+          tc_cp_sf(tmem + SFB_COL + 4, desc_sf(smem_u32(sB + C::B_CODES + 512)));
 #pragma unroll
           for (int kk = 0; kk < KSTAGE / 32; ++kk) {   // K = 32 per MMA: +32 bytes of the expanded rows
             const int h = kk >> 2, sub = kk & 3;
             const uint64_t da = desc_sw128(smem_u32(sA + h * A_BOX)) + 2 * sub;
-            const uint32_t idesc = idesc_mx(n_mma, static_cast<uint32_t>(sub));
-#pragma unroll
-            for (int j = 0; j < C::NT; ++j) {
-              if (j >= nt) break;
-              const uint64_t db = desc_sw128(smem_u32(sB + (2 * j + h) * C::B_ATOM)) + 2 * sub;
-              const uint32_t first = (ks > 0 || kk > 0 || j > 0) ? 1u : 0u;
-              tc_mma_mx(d_tmem, da, db, idesc, tmem + SFA_COL + 4 * h, tmem + SFB_COL + 8 * j + 4 * h, first);
-            }
+            const uint64_t db = desc_sw128(smem_u32(sB + h * nt * C::B_ATOM)) + 2 * sub;
+            const uint32_t idesc = idesc_mx(static_cast<int>(n_mma), static_cast<uint32_t>(sub));
+            tc_mma_mx(d_tmem, da, db, idesc, tmem + SFA_COL + 4 * h, tmem + SFB_COL + 4 * h,
+                      (ks > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&empty[sa]);
           tc_commit(&bempty[sb]);
@@ -732,7 +771,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
       float v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, v);
+      load_terms<TN>(tmem + (static_cast<uint32_t>(32 * quad) << 16) + acc * ACC_COLS, U.ph == 1 ? NX : NA, v);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       if (U.ph == 1) {
@@ -762,7 +801,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 r -= times_pow2(e4m3_to_f32(t), sb);
                 const size_t plane = static_cast<size_t>(j) * n_pairs;
                 P.aq[(plane + q) * P.I + col] = static_cast<uint8_t>(t);
-                if (lane == 0) P.as[((plane + q) * (nbi / 4) + blk / 4) * 16 + (blk & 3)] = static_cast<uint8_t>(sb);
+                if (lane == 0)
+                  P.as[((static_cast<size_t>(sf_plane<TN>(j)) * n_pairs + q) * (nbi / 4) + blk / 4) * 16 +
+                       sf_byte<TN>(j) + (blk & 3)] = static_cast<uint8_t>(sb);
               }
             }
           }
@@ -938,7 +979,7 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint32_t box[3] = {128u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
     r = encode_tiled_sw128(&M.a[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
     // scale rows of the a terms: (byte in the atom row, atom, pair, term); a box of rows
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(NA)};
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(T <= 16 ? 2 : 1)};
     const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, n * (s.I / 128) * 16};
     const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
     if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
@@ -947,8 +988,12 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   {
     const long long blocks = static_cast<long long>(T) * (s.d / 32);
     const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
-    mx_split_x_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq, w8 + W.xs,
-                                                P.done1, fused_decode() ? s.E : 0);
+    if (T <= 16)
+      mx_split_x_kernel<16><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+                                                      w8 + W.xs, P.done1, fused_decode() ? s.E : 0);
+    else
+      mx_split_x_kernel<32><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+                                                      w8 + W.xs, P.done1, fused_decode() ? s.E : 0);
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
   return T <= 16 ? launch_both<16>(P, M, dev, stream) : launch_both<32>(P, M, dev, stream);

@@ -10,27 +10,42 @@
 // Launches (one stream):
 //   quant_tokens x rows -> NVFP4 (E2M1 codes, one E4M3 scale per 16, unit
 //                tensor scale), once per token;
-//   gather_x     copies them in expert order into an expert-padded layout:
-//                expert e's rows start at a multiple of 128, so every
-//                128-row B tile and its scale atoms align.
-//   gemm<1>      D[128 x N] = W_gu tile (64 gate + 64 up rows) x X^T over K = d;
-//                epilogue: a = silu(g_g * D_gate) * (g_u * D_up), requantised
-//                to NVFP4 into the padded A matrix.
-//   gemm<2>      D = W_d tile (128 rows of d) x A^T over K = I; epilogue:
-//                out[t][row] += gate * g_d * D  (red.global.add.v4 on 4
-//                consecutive rows after a shared-memory transpose: the combine).
-// gemm is a persistent kernel, one CTA per SM, warp-specialised:
-//   warp 0      TMA producer: 128x128-byte A and B tiles (SWIZZLE_128B, no
-//               multicast) plus the 2 KB scale-atom slices by bulk copy, into
-//               a 5-stage ring guarded by mbarriers;
-//   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp of the scale
-//               atoms into TMEM, then 4 tcgen05.mma kind::mxf4nvf4 block16
-//               (K = 64 each) into one of two TMEM accumulators;
+//   gather_x     copies them in expert order into a chunked layout: expert
+//                e's rows are cut into chunks of up to 224 rows, chunk c
+//                occupying rows [256 c, 256 c + 224) of the padded matrix, so
+//                every chunk's rows and scale atoms start on a 128-row atom.
+//   gemm<1>      D[256 x N] = W_gu tile pair (2 x (64 gate + 64 up rows)) x
+//                X^T over K = d; epilogue: a = silu(g_g * D_gate) *
+//                (g_u * D_up), requantised to NVFP4 into the chunked A matrix.
+//   gemm<2>      D = W_d tile pair (2 x 128 rows of d) x A^T over K = I;
+//                epilogue: out[t][row] += gate * g_d * D (red.global.add.v4 on
+//                4 consecutive rows after a shared-memory transpose: the
+//                combine).
+// gemm is a persistent kernel of CTA pairs (clusters of two, one CTA per SM):
+// each pair computes a 256 x N tile (N <= 224 token rows of one chunk) with
+// tcgen05.mma cta_group::2, so every SM moves half the token operand per
+// FLOP that a single-CTA 128 x 128 tile needs.  Per CTA:
+//   warp 0      TMA producer: its own 128 weight rows (16 KB), its half of the
+//               chunk's token rows (112 rows, 14 KB), its weight-scale atoms
+//               (2 KB) and the whole chunk's token-scale atoms (4 KB) per
+//               256-element K stage, into a 5-stage ring; every copy of
+//               both CTAs completes on the even CTA's barrier (no multicast);
+//   warp 1      TMEM: both CTAs allocate 512 columns as a pair; the even
+//               CTA's warp 1 issues, per stage, tcgen05.cp of the scale atoms
+//               and 4 tcgen05.mma kind::mxf4nvf4 block16 (K = 64 each) into
+//               one of two 224-column accumulators, then commits to both
+//               CTAs' stage and accumulator barriers;
 //   warps 2-9   epilogue, two groups of four warps (each warp reads its 32
-//               TMEM lanes; the groups take alternate 16-column slabs),
-//               overlapped with the next tile's main loop.
+//               TMEM lanes of its own CTA; the groups take alternate 16-column
+//               slabs), overlapped with the next tile's main loop; the two
+//               CTAs' epilogues each release the accumulator to the even CTA.
 // Every wait is bounded; on expiry the CTA records MOE_ERR_TIMEOUT in the
-// status word, stops issuing, drains what it issued and frees its TMEM.
+// status word, stops issuing, drains what it issued and frees its TMEM.  Both
+// CTAs of a pair pass a cluster barrier after setup and before teardown, so
+// neither touches the other's shared memory or barriers outside their
+// lifetime.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -43,21 +58,29 @@ namespace {
 
 using namespace ::moe::tc;
 
-constexpr int BM = 128;                 // weight rows per tile
-constexpr int BN = 128;                 // token rows per tile (max MMA N used)
+constexpr int BM = 128;                 // weight rows per CTA (the pair: 256)
+constexpr int CH = 224;                 // token rows per chunk = max MMA N
+constexpr int VR = 256;                 // rows of the padded matrices per chunk (2 scale atoms)
+constexpr int BH = CH / 2;              // token rows per CTA box (its half of N)
 constexpr int BKB = 128;                // bytes of K per stage (256 FP4 elements)
 constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BKB;       // 16 KB
-constexpr int B_BYTES = BN * BKB;       // 16 KB
-constexpr int SF_BYTES = 2048;          // 4 atoms of 128 rows x 4 scales
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr int B_BYTES = BH * BKB;       // 14 KB
+constexpr int SFA_BYTES = 2048;         // 4 atoms: this CTA's 128 weight rows x 4 MMA K steps
+constexpr int SFB_BYTES = 4096;         // 2 atom rows (256 chunk rows) x 4 MMA K steps
+constexpr int OFF_B = A_BYTES, OFF_SFA = OFF_B + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int STAGE_BYTES = OFF_SFB + SFB_BYTES;      // 36 KB; every box lands whole (fill out of range)
 constexpr int EPI_GROUPS = 2;           // epilogue warp groups (each covers the 4 TMEM lane quadrants)
 constexpr int EPI_THREADS = 128 * EPI_GROUPS;
-constexpr int EPI_BYTES = EPI_GROUPS * 16 * 128 * 4 + 2 * 128 * 4;   // a transposed 16-column slab per group + column info
+constexpr int EPI_BYTES = EPI_GROUPS * 16 * 128 * 4 + 2 * VR * 4;   // a transposed 16-column slab per group + column info
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_COLS = 128;           // per accumulator buffer
-constexpr int SFA_COL = 256, SFB_COL = 272;
+constexpr int ACC_COLS = CH;            // per accumulator buffer (two)
+constexpr int SFA_COL = 2 * ACC_COLS;   // 4 MMA K steps x 4 columns
+constexpr int SFB_COL = SFA_COL + 16;   // 4 MMA K steps x 8 columns (rows 0-127, 128-255)
 constexpr int THREADS = 64 + EPI_THREADS;   // producer, MMA, epilogue groups
+static_assert(SFB_COL + 32 <= TMEM_COLS, "TMEM budget");
+static_assert(OFF_B % 1024 == 0 && OFF_SFA % 128 == 0 && OFF_SFB % 128 == 0 && STAGE_BYTES % 1024 == 0,
+              "stage alignment");
 
 struct GemmParams {
   uint64_t wait_ns;          // limit of every bounded wait (default 2 s)
@@ -70,34 +93,46 @@ struct GemmParams {
   const uint8_t* pool;       // slot pool
   size_t blob_bytes;
   BlobLayout L;
-  const uint8_t* act_sf;     // scale atoms of the B operand
-  uint8_t* aq;               // gemm<1> output codes  [rows][I/2]
+  uint8_t* aq;               // gemm<1> output codes  [chunk rows][I/2]
   uint8_t* aq_sf;            // gemm<1> output scale atoms
   float* out;                // gemm<2> output [T][d]
   int32_t* status;
 };
 
-// ------------------------------------------------------------------ FP4 MMA wrappers
+// The four operand maps of one GEMM (TMA, no swizzle for the scale atoms).
+struct GemmMaps {
+  CUtensorMap w;             // weight codes [slot][rows][K/2]: 128 x 128-byte box, 128-byte swizzle
+  CUtensorMap act;           // token codes [chunk rows][K/2]: 112 x 128-byte box, 128-byte swizzle
+  CUtensorMap sfa;           // weight scale atoms [slot][256-byte lines]: 8 lines (2 KB)
+  CUtensorMap sfb;           // token scale atoms [atom row][256-byte lines]: 8 lines x 2 atom rows (4 KB)
+};
+
+// ------------------------------------------------------------------ FP4 MMA wrappers (CTA pair)
 // Instruction descriptor: kind::mxf4nvf4, A and B E2M1 (packed), K-major,
-// UE4M3 scales, M = 128, N = n.
+// UE4M3 scales, M = 256 (the pair), N = n.
 __device__ __forceinline__ uint32_t idesc_fp4(int n) {
-  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>((2 * BM) >> 4) << 24);
 }
 
+// One scale atom (512 B at the same shared address in both CTAs) into the
+// same TMEM columns of both CTAs.
 __device__ __forceinline__ void tc_cp_sf(uint32_t tmem, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(sdesc) : "memory");
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(sdesc) : "memory");
 }
 
+// D (both CTAs' TMEM: rows 0-127 here, 128-255 in the odd CTA) (+)= A (each
+// CTA's 128 rows) x B^T (N rows: the first N/2 in this CTA, the rest in the
+// odd CTA), block-scaled by 16-element E4M3 scales.
 __device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                            uint32_t sfa, uint32_t sfb, uint32_t acc) {
   asm volatile(
       "{ .reg .pred p; setp.ne.b32 p, %6, 0; "
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p; }" ::"r"(
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p; }" ::"r"(
           d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
       : "memory");
 }
-
 
 // ------------------------------------------------------------------ NVFP4 quantisation
 // 16 values -> E4M3 scale byte s = e4m3_rn_satfinite(amax / 6) and 8 code
@@ -128,9 +163,9 @@ __device__ __forceinline__ uint32_t pack8(const float (&q)[8]) {
 }
 
 // ------------------------------------------------------------------ shared prologue
-// Chunks: 128-row pieces of each evaluated expert's group (tokens > 0,
-// slot >= 0).  chunk_start[e] = exclusive prefix of the chunk counts; chunk c
-// occupies padded rows [128 c, 128 c + 128).
+// Chunks: pieces of up to CH rows of each evaluated expert's group (tokens >
+// 0, slot >= 0).  chunk_start[e] = exclusive prefix of the chunk counts;
+// chunk c occupies padded rows [VR c, VR c + CH).
 __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* __restrict__ slot, int E,
                             int n_pairs, int n_slots, int32_t* chunk_start, int* ws, int32_t* status) {
   const int per = (E + blockDim.x - 1) / blockDim.x;
@@ -147,7 +182,7 @@ __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* 
       } else {
         const int s = slot[e];
         if (s >= n_slots) report(status, MOE_ERR_DEVICE);
-        else if (s >= 0) c = (b - a + BN - 1) / BN;
+        else if (s >= 0) c = (b - a + CH - 1) / CH;
       }
     }
     cnt += c;
@@ -183,7 +218,7 @@ __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* 
     const int a = offsets[e], b = offsets[e + 1];
     if (b > a && a >= 0 && b <= n_pairs) {
       const int s = slot[e];
-      if (s >= 0 && s < n_slots) run += (b - a + BN - 1) / BN;
+      if (s >= 0 && s < n_slots) run += (b - a + CH - 1) / CH;
     }
   }
   const int total = ws[32];
@@ -192,14 +227,15 @@ __device__ int build_chunks(const int32_t* __restrict__ offsets, const int32_t* 
   return total;
 }
 
-// Unit u -> (chunk, M tile), chunk-major for both GEMMs: the CTAs working at
-// the same time share one activation tile, and the M tiles of an expert with
-// several chunks are re-read while still in L2.  (Measured against M-tile-major
-// order for GEMM2, which keeps one 128-column slab of out hot for the fused
-// combine: equal at T = 4096, 8-9 % slower at T >= 16384.)
-__device__ __forceinline__ void unit_coords(int u, int MT, int* c, int* m) {
-  *c = u / MT;
-  *m = u % MT;
+// Unit u -> (chunk, pair of M tiles), chunk-major for both GEMMs: the pairs
+// working at the same time share one activation chunk, and the M tiles of an
+// expert with several chunks are re-read while still in L2.  (Measured, with
+// single-CTA tiles, against M-tile-major order for GEMM2, which keeps one
+// 128-column slab of out hot for the fused combine: equal at T = 4096, 8-9 %
+// slower at T >= 16384.)
+__device__ __forceinline__ void unit_coords(int u, int MP, int* c, int* mp) {
+  *c = u / MP;
+  *mp = u % MP;
 }
 
 // expert of chunk c: the last e with chunk_start[e] <= c
@@ -251,27 +287,32 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(const uint16_t* __res
 }
 
 // Gather: every real row of every chunk copies its token's codes into
-// xq[128 c + r][d/2] and its scale bytes, 4 blocks (one atom row) at a
-// time, into the atom layout of the padded matrix.  One warp per row.
+// xq[VR c + r][d/2] and its scale bytes, 4 blocks (one atom row) at a time,
+// into the atom layout of the padded matrix.  One warp per row.
 __global__ void __launch_bounds__(256) gather_x_kernel(const uint8_t* __restrict__ xt,
                                                       const uint8_t* __restrict__ xts, int d, int T, int k, int E,
                                                       int n_slots, const int32_t* __restrict__ offsets,
                                                       const int32_t* __restrict__ perm,
                                                       const int32_t* __restrict__ slot, uint8_t* __restrict__ xq,
-                                                      uint8_t* __restrict__ xsf, int32_t* status) {
+                                                      uint8_t* __restrict__ xsf, int max_chunks, int32_t* status) {
   __shared__ int32_t chunk_start[1025];
   __shared__ int ws[36];
   const int n_pairs = T * k;
-  const int n_chunks = build_chunks(offsets, slot, E, n_pairs, n_slots, chunk_start, ws, status);
+  int n_chunks = build_chunks(offsets, slot, E, n_pairs, n_slots, chunk_start, ws, status);
+  if (n_chunks > max_chunks) {          // offsets inconsistent with T * k: stay inside the workspace
+    if (threadIdx.x == 0) report(status, MOE_ERR_DEVICE);
+    n_chunks = max_chunks;
+  }
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
-  const long long rows = static_cast<long long>(n_chunks) * BN;
+  const long long rows = static_cast<long long>(n_chunks) * VR;
   const int row_bytes = d / 2, nb = d / 16;
   for (long long w = static_cast<long long>(blockIdx.x) * warps + (threadIdx.x >> 5); w < rows;
        w += static_cast<long long>(gridDim.x) * warps) {
-    const int c = static_cast<int>(w / BN), r = static_cast<int>(w % BN);
+    const int c = static_cast<int>(w / VR), r = static_cast<int>(w % VR);
+    if (r >= CH) continue;                                  // the chunk's last 32 padded rows: never read
     const int e = chunk_expert(chunk_start, E, c);
-    const int q = offsets[e] + (c - chunk_start[e]) * BN + r;
+    const int q = offsets[e] + (c - chunk_start[e]) * CH + r;
     if (q >= offsets[e + 1]) continue;                      // padding row: never read back
     int p = perm[q];
     if (p < 0 || p >= n_pairs) {
@@ -279,7 +320,7 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint8_t* __restrict
       p = 0;
     }
     const int t = p / k;
-    const int prow = c * BN + r;
+    const int prow = c * VR + r;
     const uint4* src = reinterpret_cast<const uint4*>(xt + static_cast<size_t>(t) * row_bytes);
     uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(prow) * row_bytes);
     for (int i = lane; i < row_bytes / 16; i += 32) dst[i] = __ldg(src + i);
@@ -291,20 +332,18 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint8_t* __restrict
 
 // ------------------------------------------------------------------ the GEMMs
 template <int PHASE>
-__global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_constant__ CUtensorMap tm_w,
-                                                              const __grid_constant__ CUtensorMap tm_act,
-                                                              GemmParams P) {
+__global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_constant__ GemmMaps M, GemmParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* epi_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
   int32_t* col_t = reinterpret_cast<int32_t*>(epi_all + EPI_GROUPS * 16 * 128);
-  float* col_g = reinterpret_cast<float*>(col_t + 128);
+  float* col_g = reinterpret_cast<float*>(col_t + VR);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
-  uint64_t* full = bars;                   // [STAGES]
-  uint64_t* empty = bars + STAGES;         // [STAGES]
-  uint64_t* tfull = bars + 2 * STAGES;     // [2]
-  uint64_t* tempty = bars + 2 * STAGES + 2;// [2]
+  uint64_t* full = bars;                   // [STAGES] even CTA: both CTAs' copies of a stage
+  uint64_t* empty = bars + STAGES;         // [STAGES] the pair's MMAs are done with a stage
+  uint64_t* tfull = bars + 2 * STAGES;     // [2] accumulator ready
+  uint64_t* tempty = bars + 2 * STAGES + 2;// [2] even CTA: both epilogues released the accumulator
   uint64_t* drain = bars + 2 * STAGES + 4; // [1]
   uint64_t* stall = bars + 2 * STAGES + 5; // [1] never arrived on (testing aid)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
@@ -314,9 +353,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();         // 0: issues the pair's MMAs
   const int K = (PHASE == 1) ? P.d : P.I;
   const int KS = K / (2 * BKB);                 // stages of 256 elements
-  const int MT = (PHASE == 1) ? (2 * P.I) / BM : P.d / BM;
+  const int MP = ((PHASE == 1) ? (2 * P.I) / BM : P.d / BM) / 2;   // pairs of M tiles
   const int n_pairs = P.T * P.k;
 
   if (threadIdx.x == 0) {
@@ -326,7 +366,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], EPI_THREADS);
+      mbar_init(&tempty[a], 2);
     }
     mbar_init(drain, 1);
     mbar_init(stall, 1);
@@ -335,33 +375,37 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
                  "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   const int n_chunks = build_chunks(P.offsets, P.slot, P.E, n_pairs, P.n_slots, chunk_start, ws, P.status);
   tc_fence_before();
   __syncthreads();
+  cluster_sync();                               // the peer's barriers exist before any copy or commit names them
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int n_chunks_used = min(n_chunks, P.max_chunks);
-  const int n_units = n_chunks_used * MT;
+  const int n_units = n_chunks_used * MP;
+  const int pair = blockIdx.x >> 1, n_pair_ctas = gridDim.x >> 1;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------- TMA producer (both CTAs)
     const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      int c, m;
-      unit_coords(u, MT, &c, &m);
+    for (int u = pair; u < n_units && ok; u += n_pair_ctas) {
+      int c, mp;
+      unit_coords(u, MP, &c, &mp);
+      const int m = 2 * mp + static_cast<int>(rank);
       const int e = chunk_expert(chunk_start, P.E, c);
       const int sl = P.slot[e];
-      const uint8_t* sfa_src = P.pool + static_cast<size_t>(sl) * P.blob_bytes +
-                               (PHASE == 1 ? P.L.sg : P.L.sd) + static_cast<size_t>(m) * (K / 64) * 512;
-      const uint8_t* sfb_src = P.act_sf + static_cast<size_t>(c) * (K / 64) * 512;
+      const int row0 = P.offsets[e] + (c - chunk_start[e]) * CH;
+      const int nmma = (min(CH, P.offsets[e + 1] - row0) + 15) & ~15;
+      const int brow = c * VR + static_cast<int>(rank) * (nmma / 2);   // this CTA's half of the chunk
+      const int sfa_line = m * (K / 64) * 2;                            // 256-byte lines of the tile's atoms
       // a weight tile read by one chunk streams through L2; one that the
       // expert's further chunks read again is kept
       const uint64_t pol_a = (chunk_start[e + 1] - chunk_start[e] > 1) ? pol_keep : pol_stream;
@@ -371,15 +415,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           break;
         }
         if (elect_one()) {
-          uint8_t* sA = stage_base + stage * STAGE_BYTES;
-          uint8_t* sB = sA + A_BYTES;
-          uint8_t* sSFA = sB + B_BYTES;
-          uint8_t* sSFB = sSFA + SF_BYTES;
-          mbar_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_3d(sA, &tm_w, &full[stage], ks * BKB, m * BM, sl, pol_a);
-          tma_load_2d(sB, &tm_act, &full[stage], ks * BKB, c * BN, pol_keep);
-          bulk_load(sSFA, sfa_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_a);
-          bulk_load(sSFB, sfb_src + ks * SF_BYTES, SF_BYTES, &full[stage], pol_keep);
+          uint8_t* st = stage_base + stage * STAGE_BYTES;
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          const uint32_t bar = cluster_addr(&full[stage], 0);
+          tma_load_3d_pair(st, &M.w, bar, ks * BKB, m * BM, sl, pol_a);
+          tma_load_2d_pair(st + OFF_B, &M.act, bar, ks * BKB, brow, pol_keep);
+          tma_load_3d_pair(st + OFF_SFA, &M.sfa, bar, 0, sfa_line + ks * 8, sl, pol_a);
+          tma_load_3d_pair(st + OFF_SFB, &M.sfb, bar, 0, ks * 8, 2 * c, pol_keep);
         }
         __syncwarp();
         ++issued;
@@ -393,101 +435,108 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       report(P.status, MOE_ERR_TIMEOUT);
       *abort_flag = 1;
     }
-    // drain: wait (bounded) until the copies last issued into the ring have
-    // landed, so none is in flight when the CTA exits
-    const int outstanding = issued < STAGES ? issued : STAGES;
-    int s = stage;
-    uint32_t ph = phase;
-    for (int i = 0; i < outstanding; ++i) {
-      if (--s < 0) {
-        s = STAGES - 1;
-        ph ^= 1u;
+    // drain: the even CTA waits (bounded) until the copies last issued into
+    // the ring by both CTAs have landed, so none is in flight at teardown
+    if (rank == 0) {
+      const int outstanding = issued < STAGES ? issued : STAGES;
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < outstanding; ++i) {
+        if (--s < 0) {
+          s = STAGES - 1;
+          ph ^= 1u;
+        }
+        mbar_drain(&full[s], ph);
       }
-      mbar_drain(&full[s], ph);
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      int c, m_unused;
-      unit_coords(u, MT, &c, &m_unused);
-      const int e = chunk_expert(chunk_start, P.E, c);
-      const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
-      const int nvalid = min(BN, P.offsets[e + 1] - row0);
-      const int nmma = (nvalid + 15) & ~15;
-      const uint32_t idesc = idesc_fp4(nmma);
-      const int acc = it & 1;
-      if (!__all_sync(kFull, mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem + acc * ACC_COLS;
-      for (int ks = 0; ks < KS; ++ks) {
-        if (!__all_sync(kFull, mbar_wait(&full[stage], phase, abort_flag, P.wait_ns))) {
+    // ---------------------------------------------------------- MMA issuer (even CTA)
+    if (rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < n_units && ok; u += n_pair_ctas, ++it) {
+        int c, mp_unused;
+        unit_coords(u, MP, &c, &mp_unused);
+        const int e = chunk_expert(chunk_start, P.E, c);
+        const int row0 = P.offsets[e] + (c - chunk_start[e]) * CH;
+        const int nmma = (min(CH, P.offsets[e + 1] - row0) + 15) & ~15;
+        const uint32_t idesc = idesc_fp4(nmma);
+        const int acc = it & 1;
+        if (!__all_sync(kFull, mbar_wait_cluster(&tempty[acc], ((it >> 1) & 1) ^ 1u, abort_flag, P.wait_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (elect_one()) {
-          uint8_t* sA = stage_base + stage * STAGE_BYTES;
-          uint8_t* sB = sA + A_BYTES;
-          uint8_t* sSFA = sB + B_BYTES;
-          uint8_t* sSFB = sSFA + SF_BYTES;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tc_cp_sf(tmem + SFA_COL + 4 * j, desc_sf(smem_u32(sSFA + 512 * j)));
-            tc_cp_sf(tmem + SFB_COL + 4 * j, desc_sf(smem_u32(sSFB + 512 * j)));
+        const uint32_t d_tmem = tmem + acc * ACC_COLS;
+        for (int ks = 0; ks < KS; ++ks) {
+          if (!__all_sync(kFull, mbar_wait(&full[stage], phase, abort_flag, P.wait_ns))) {
+            ok = false;
+            break;
           }
-          const uint64_t da = desc_sw128(smem_u32(sA));
-          const uint64_t db = desc_sw128(smem_u32(sB));
+          tc_fence_after();
+          if (elect_one()) {
+            uint8_t* st = stage_base + stage * STAGE_BYTES;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tc_mma_fp4(d_tmem, da + 2 * j, db + 2 * j, idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 4 * j,
-                       (ks > 0 || j > 0) ? 1u : 0u);
-          tc_commit(&empty[stage]);
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_sf(tmem + SFA_COL + 4 * j, desc_sf(smem_u32(st + OFF_SFA + 512 * j)));
+              tc_cp_sf(tmem + SFB_COL + 8 * j, desc_sf(smem_u32(st + OFF_SFB + 512 * j)));
+              tc_cp_sf(tmem + SFB_COL + 8 * j + 4, desc_sf(smem_u32(st + OFF_SFB + 2048 + 512 * j)));
+            }
+            const uint64_t da = desc_sw128(smem_u32(st));
+            const uint64_t db = desc_sw128(smem_u32(st + OFF_B));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma_fp4(d_tmem, da + 2 * j, db + 2 * j, idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 8 * j,
+                         (ks > 0 || j > 0) ? 1u : 0u);
+            tc_commit_pair(cluster_addr(&empty[stage], 0));
+            tc_commit_pair(cluster_addr(&empty[stage], 1));
+          }
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (elect_one()) {
+          tc_commit_pair(cluster_addr(&tfull[acc], 0));
+          tc_commit_pair(cluster_addr(&tfull[acc], 1));
         }
         __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
-      if (!ok) break;
-      if (elect_one()) tc_commit(&tfull[acc]);
+      if (!ok) {
+        report(P.status, MOE_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      if (elect_one()) tc_commit_pair(cluster_addr(drain, 0));
       __syncwarp();
+      mbar_drain(drain, 0);
     }
-    if (!ok) {
-      report(P.status, MOE_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    // every MMA this thread issued has completed before TMEM is released
-    if (elect_one()) tc_commit(drain);
-    __syncwarp();
-    mbar_drain(drain, 0);
   } else {
-    // ---------------------------------------------------------- epilogue (warps 2..9)
+    // ---------------------------------------------------------- epilogue (warps 2..9, both CTAs)
     const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
     const int grp = (warp - 2) >> 2;            // column group: slabs grp, grp+2, ...
     const int et = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
     const int eall = (warp - 2) * 32 + lane;       // 0..255 over both groups
     float* epi = epi_all + grp * 16 * 128;
     const int bar_grp = 1 + grp, bar_all = 3;
+    const uint32_t release = cluster_addr(&tempty[0], 0);   // + 8 * acc
     const float* ts = nullptr;
     int it = 0;
     // testing aid (moe_set_test_stall): CTA 0's epilogue first waits on a
     // barrier that nothing arrives on, so the bounded wait runs out and the
     // abort path (record, stop issuing, drain, free TMEM) runs for real
     bool ok = !(P.stall && blockIdx.x == 0 && !mbar_wait(stall, 0, abort_flag, P.wait_ns));
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-      int c, m;
-      unit_coords(u, MT, &c, &m);
+    for (int u = pair; u < n_units && ok; u += n_pair_ctas, ++it) {
+      int c, mp;
+      unit_coords(u, MP, &c, &mp);
+      const int m = 2 * mp + static_cast<int>(rank);
       const int e = chunk_expert(chunk_start, P.E, c);
-      const int row0 = P.offsets[e] + (c - chunk_start[e]) * BN;
-      const int nvalid = min(BN, P.offsets[e + 1] - row0);
+      const int row0 = P.offsets[e] + (c - chunk_start[e]) * CH;
+      const int nvalid = min(CH, P.offsets[e + 1] - row0);
       const uint8_t* blob = P.pool + static_cast<size_t>(P.slot[e]) * P.blob_bytes;
       ts = reinterpret_cast<const float*>(blob + P.L.ts);
       const int acc = it & 1;
@@ -569,7 +618,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           for (int j = 0; j < 8; ++j) q[j] = (s > 0.f) ? __fdiv_rn(a[j], s) : 0.f;
           const uint32_t codes = pack8(q);
           if (col < nvalid) {
-            const int prow = c * BN + col;
+            const int prow = c * VR + col;
             const int i0 = m * 64;                       // first intermediate index of the tile
             *reinterpret_cast<uint32_t*>(P.aq + static_cast<size_t>(prow) * (P.I / 2) + (i0 + 16 * b + 8 * h) / 2) =
                 codes;
@@ -578,8 +627,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           named_sync(bar_grp, 128);
         }
       }
+      // both CTAs' epilogues release the accumulator to the even CTA's MMA
+      // issuer, once all eight warps' TMEM reads are complete
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      named_sync(bar_all, EPI_THREADS);
+      if (eall == 0) mbar_arrive_cluster(release + 8u * acc);
     }
     if (!ok) {
       report(P.status, MOE_ERR_TIMEOUT);
@@ -588,24 +640,38 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();                               // the pair is done with each other's memory and TMEM
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
 }
 
 // ------------------------------------------------------------------ host side
-// Byte-element tensor map, box 128 (bytes of K) x 128 rows, 128-byte swizzle.
-moe_status make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides) {
-  const uint32_t box[3] = {static_cast<uint32_t>(BKB), 128u, 1u};
-  const CUresult r = encode_tiled_sw128(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box);
+// Byte-element tensor maps: operand codes with a 128-byte swizzle, scale
+// atoms as 256-byte lines without one.
+moe_status map_status(CUresult r) {
   if (r == CUDA_ERROR_NOT_FOUND) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return MOE_OK;
 }
 
+moe_status make_code_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                         const uint64_t* strides, uint32_t box_rows) {
+  const uint32_t box[3] = {static_cast<uint32_t>(BKB), box_rows, 1u};
+  return map_status(encode_tiled_sw128(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box));
+}
+
+moe_status make_atom_map(CUtensorMap* map, const void* base, uint64_t lines, uint64_t planes, uint64_t plane_bytes,
+                         uint32_t box_planes) {
+  const uint64_t dims[3] = {256, lines, planes};
+  const uint64_t strides[2] = {256, plane_bytes};
+  const uint32_t box[3] = {256u, 8u, box_planes};
+  return map_status(encode_tiled_plain(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box));
+}
+
 struct PrefillWs {
-  size_t rows;            // padded row capacity (multiple of 128)
+  size_t chunks;          // chunk capacity; the padded matrices have VR rows per chunk
   size_t xt, xts, xq, xsf, aq, asf, bytes;
 };
 
@@ -613,20 +679,42 @@ PrefillWs prefill_ws(moe_shape s, int T, int k) {
   PrefillWs w{};
   const size_t n = static_cast<size_t>(T) * k;
   const size_t act = n < static_cast<size_t>(s.E) ? n : static_cast<size_t>(s.E);
-  w.rows = round_up(n + act * (BN - 1), BN);
+  // sum over experts of ceil(g_e / CH) <= (n + act (CH - 1)) / CH
+  w.chunks = (n + act * (CH - 1)) / CH;
+  if (w.chunks == 0) w.chunks = 1;
+  const size_t rows = w.chunks * VR;
   size_t o = 0;
   w.xt = o; o = round_up(o + static_cast<size_t>(T) * (s.d / 2), 1024);
   w.xts = o; o = round_up(o + static_cast<size_t>(T) * (s.d / 16), 1024);
-  w.xq = o; o = round_up(o + w.rows * (s.d / 2), 1024);
-  w.xsf = o; o = round_up(o + w.rows * (s.d / 16), 1024);
-  w.aq = o; o = round_up(o + w.rows * (s.I / 2), 1024);
-  w.asf = o; o = round_up(o + w.rows * (s.I / 16), 1024);
+  w.xq = o; o = round_up(o + rows * (s.d / 2), 1024);
+  w.xsf = o; o = round_up(o + rows * (s.d / 16), 1024);
+  w.aq = o; o = round_up(o + rows * (s.I / 2), 1024);
+  w.asf = o; o = round_up(o + rows * (s.I / 16), 1024);
   w.bytes = o;
   return w;
 }
 
 constexpr size_t kGemmSmem = STAGES * STAGE_BYTES + EPI_BYTES + 256 + 1025 * 4 + 1024;
 static_assert((2 * STAGES + 6) * 8 + 16 <= 256, "barrier area");
+static_assert(kGemmSmem <= 227 * 1024, "shared memory per CTA");
+
+template <int PHASE>
+moe_status launch_gemm(const GemmMaps& maps, const GemmParams& P, int grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<PHASE>, maps, P));
+  return MOE_OK;
+}
 
 }  // namespace
 
@@ -646,50 +734,75 @@ moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const in
   uint8_t* aq = base + w.aq;
   uint8_t* asf = base + w.asf;
   const BlobLayout L = blob_layout(s.fmt, s.d, s.I);
-  const int max_chunks = static_cast<int>(w.rows / BN);
+  const int max_chunks = static_cast<int>(w.chunks);
+  const size_t rows = w.chunks * VR;
 
-  static bool attr_done[64] = {};
-  if (!attr_done[dev.id]) {
+  // grid: as many CTA pairs as can be resident at once (one CTA per SM; an
+  // SM left without a partner in its GPC stays idle rather than running a
+  // second wave)
+  static int pair_grid[64] = {};
+  if (pair_grid[dev.id] == 0) {
     MOE_CUDA_TRY(cudaFuncSetAttribute(gemm_fp4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(kGemmSmem)));
     MOE_CUDA_TRY(cudaFuncSetAttribute(gemm_fp4_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(kGemmSmem)));
-    attr_done[dev.id] = true;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>((dev.sm_count / 2) * 2));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = kGemmSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    MOE_CUDA_TRY(cudaOccupancyMaxActiveClusters(&clusters, gemm_fp4_kernel<1>, &cfg));
+    if (clusters <= 0) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the FP4 GEMM fits on this device");
+    pair_grid[dev.id] = 2 * std::min(clusters, dev.sm_count / 2);
   }
 
-  // tensor maps: weights [slot][rows][K bytes], activations [rows][K bytes]
-  CUtensorMap tm_gu, tm_d, tm_x, tm_a;
+  // tensor maps: weights [slot][rows][K bytes] and their scale atoms in the
+  // blob, activations [chunk rows][K bytes] and their scale atoms
+  GemmMaps m1{}, m2{};
   const uint8_t* pool8 = static_cast<const uint8_t*>(pool);
+  const uint64_t slots = static_cast<uint64_t>(n_slots);
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.d / 2), static_cast<uint64_t>(2 * s.I),
-                              static_cast<uint64_t>(n_slots)};
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.d / 2), static_cast<uint64_t>(2 * s.I), slots};
     const uint64_t str[2] = {static_cast<uint64_t>(s.d / 2), L.bytes};
-    moe_status st = make_map(&tm_gu, pool8 + L.wg, 3, dims, str);
+    moe_status st = make_code_map(&m1.w, pool8 + L.wg, 3, dims, str, BM);
+    if (st == MOE_OK) st = make_atom_map(&m1.sfa, pool8 + L.sg, static_cast<uint64_t>(2 * s.I) * s.d / 16 / 256, slots,
+                                         L.bytes, 1);
     if (st != MOE_OK) return st;
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.I / 2), static_cast<uint64_t>(s.d),
-                              static_cast<uint64_t>(n_slots)};
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.I / 2), static_cast<uint64_t>(s.d), slots};
     const uint64_t str[2] = {static_cast<uint64_t>(s.I / 2), L.bytes};
-    moe_status st = make_map(&tm_d, pool8 + L.wd, 3, dims, str);
+    moe_status st = make_code_map(&m2.w, pool8 + L.wd, 3, dims, str, BM);
+    if (st == MOE_OK) st = make_atom_map(&m2.sfa, pool8 + L.sd, static_cast<uint64_t>(s.d) * s.I / 16 / 256, slots,
+                                         L.bytes, 1);
     if (st != MOE_OK) return st;
   }
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(s.d / 2), w.rows};
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.d / 2), rows};
     const uint64_t str[1] = {static_cast<uint64_t>(s.d / 2)};
-    moe_status st = make_map(&tm_x, xq, 2, dims, str);
+    moe_status st = make_code_map(&m1.act, xq, 2, dims, str, BH);
+    if (st == MOE_OK) st = make_atom_map(&m1.sfb, xsf, static_cast<uint64_t>(s.d / 32), rows / 128,
+                                         static_cast<uint64_t>(s.d) * 8, 2);
     if (st != MOE_OK) return st;
   }
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(s.I / 2), w.rows};
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.I / 2), rows};
     const uint64_t str[1] = {static_cast<uint64_t>(s.I / 2)};
-    moe_status st = make_map(&tm_a, aq, 2, dims, str);
+    moe_status st = make_code_map(&m2.act, aq, 2, dims, str, BH);
+    if (st == MOE_OK) st = make_atom_map(&m2.sfb, asf, static_cast<uint64_t>(s.I / 32), rows / 128,
+                                         static_cast<uint64_t>(s.I) * 8, 2);
     if (st != MOE_OK) return st;
   }
 
   {
-    const long long rows = static_cast<long long>(w.rows);
-    long long blocks = (rows + 7) / 8;
+    long long blocks = (static_cast<long long>(rows) + 7) / 8;
     const long long cap = static_cast<long long>(dev.sm_count) * 8;
     if (blocks > cap) blocks = cap;
     long long tb = (static_cast<long long>(T) + 7) / 8;
@@ -698,7 +811,7 @@ moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const in
                                                                  base + w.xt, base + w.xts);
     MOE_LAUNCH_CHECK("quant_tokens_kernel");
     gather_x_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(base + w.xt, base + w.xts, s.d, T, k, s.E,
-                                                                  n_slots, offsets, perm, slot, xq, xsf, status);
+                                                                  n_slots, offsets, perm, slot, xq, xsf, max_chunks, status);
     MOE_LAUNCH_CHECK("gather_x_kernel");
   }
   GemmParams P{};
@@ -720,16 +833,12 @@ moe_status launch_ffn_prefill(moe_shape s, const void* x, int T, int k, const in
   P.L = L;
   P.status = status;
   P.out = out;
-  const int grid = dev.sm_count;
-  P.act_sf = xsf;
   P.aq = aq;
   P.aq_sf = asf;
-  gemm_fp4_kernel<1><<<grid, THREADS, kGemmSmem, stream>>>(tm_gu, tm_x, P);
-  MOE_LAUNCH_CHECK("gemm_fp4_kernel<1>");
-  P.act_sf = asf;
-  gemm_fp4_kernel<2><<<grid, THREADS, kGemmSmem, stream>>>(tm_d, tm_a, P);
-  MOE_LAUNCH_CHECK("gemm_fp4_kernel<2>");
-  return MOE_OK;
+  const int grid = pair_grid[dev.id];
+  moe_status st = launch_gemm<1>(m1, P, grid, stream);
+  if (st == MOE_OK) st = launch_gemm<2>(m2, P, grid, stream);
+  return st;
 }
 
 }  // namespace moe

@@ -1,7 +1,8 @@
 // PTX wrappers shared by the tensor-core kernels (prefill GEMMs and the
-// bf16 decode GEMV): shared-memory mbarriers with bounded waits, TMA and bulk
-// copies with L2 cache hints, tcgen05 descriptors, commits and TMEM loads.
-// No multicast form of any copy is used.
+// decode GEMVs): shared-memory mbarriers with bounded waits, TMA and bulk
+// copies with L2 cache hints, CTA-pair addressing, tcgen05 descriptors,
+// commits and TMEM loads.  No multicast form of any copy or commit is used:
+// a CTA pair signals its peer through explicit shared::cluster addresses.
 #pragma once
 
 #include <cstdint>
@@ -79,6 +80,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait on a barrier that the other CTA of a pair arrives on: the
+// acquire is at cluster scope, pairing with mbar_arrive_cluster's release.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t limit_ns) {
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 255u) {
+      if (abort_flag != nullptr && *abort_flag) return false;
+      if (now_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // Bounded wait that ignores the abort flag (teardown drains).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = now_ns();
@@ -133,6 +155,62 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "%4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// ---- CTA pairs (cluster of two, tcgen05 cta_group::2)
+// Rank of this CTA in its cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of the same shared-memory object in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (address from
+// cluster_addr), releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
+
+// All threads of both CTAs: barrier over the cluster (hardware barrier; every
+// thread of the cluster reaches it on every path).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Tiled TMA loads whose completion is signalled on an mbarrier that may sit in
+// the other CTA of the pair (cbar: a shared::cluster address).  The data land
+// in this CTA's shared memory.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t cbar, int x, int y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(cbar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t cbar, int x, int y,
+                                                 int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(cbar), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
+// Commit of the pair's MMAs (issued by the even CTA) to an mbarrier given by
+// its shared::cluster address: this CTA's or the peer's.
+__device__ __forceinline__ void tc_commit_pair(uint32_t cbar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cbar)
+               : "memory");
 }
 
 __device__ __forceinline__ bool elect_one() {

@@ -23,7 +23,9 @@ def _cfg(name, E, k, d, I):
 
 @pytest.mark.parametrize("E,k,d,I,T", [
     (8, 2, 512, 256, 64),       # one chunk per expert, partial N
-    (4, 2, 256, 256, 400),      # 200 rows per expert: two chunks (128 + 72)
+    (4, 2, 256, 256, 400),      # ~200 rows per expert: one chunk each
+    (4, 2, 256, 256, 700),      # ~350 rows per expert: two chunks (224 + ~126)
+    (2, 1, 512, 256, 500),      # ~250 rows per expert: a full chunk and a ragged ~26-row tail
     (16, 4, 1024, 512, 37),     # ragged small groups
     (8, 1, 256, 512, 1),        # a single token
 ])
