@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
     const int et = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
     const int eall = (warp - 2) * 32 + lane;       // 0..255 over both groups
     float* epi = epi_all + grp * 16 * 128;
-    const int bar_grp = 1 + grp, bar_all = 3;
+    const int bar_grp = 1 + grp, bar_all = 1 + EPI_GROUPS;   // named barriers (0: __syncthreads)
     const uint32_t release = cluster_addr(&tempty[0], 0);   // + 8 * acc
     const float* ts = nullptr;
     int it = 0;
