@@ -57,7 +57,8 @@ def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d.get("hbm_gbs", 6650.0), "measured"
+        if "hbm_gbs" in d:
+            return d["hbm_gbs"], "measured"
     return 6650.0, "fallback"
 
 
@@ -321,11 +322,12 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
         print(f"warning: replicas stream only {min(sum(per_step) - p for p in per_step) / 1e6:.0f} MB "
               "between reuses", file=sys.stderr)
     stream = torch.cuda.Stream(device=dev)
-    # kernels per step: route, permute, the FFN (one cooperative launch, or
-    # gate/up + down with MOE_DECODE_TWO_LAUNCHES), combine; MXFP4 adds the
-    # split of x into E4M3 terms (the counter reset is a memset node)
-    two = os.environ.get("MOE_DECODE_TWO_LAUNCHES") is not None
-    launches_per_step = 4 + (1 if two else 0) + (1 if cfg.fmt == "mxfp4" else 0)
+    # kernels per step: route, permute, the FFN's (the library reports them:
+    # one cooperative GEMV launch or gate/up + down, plus MXFP4's split of x
+    # into E4M3 terms; a one-launch counter reset is a memset node), combine
+    ffn_launches = moe.moe_expert_ffn_launches(moe.shape(cfg.E, cfg.d, cfg.I, cfg.fmt), T, cfg.k)
+    two = ffn_launches - (1 if cfg.fmt == "mxfp4" else 0) == 2
+    launches_per_step = 3 + ffn_launches
 
     def step_fn(r):
         L = r["layer"]
@@ -568,10 +570,12 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
                      pin=False).cuda()
     del w
     layer = MoeLayer(cfg.E, cfg.d, cfg.I, cfg.fmt, cfg.k, max(Ts), device_pool=pool, act="nvfp4")
-    d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
-        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    have_peaks = os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json"))
+    d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if have_peaks else {}
     bf16 = d.get("bf16_tflops", 1590.0)
     fp4_peak = 4.0 * bf16          # dense FP4 = 4 x dense BF16 (nominal 9 / 2.25 PFLOP/s)
+    fp4_src = ("4 x measured bf16 (MEASURED_PEAKS.json bf16_tflops)" if "bf16_tflops" in d
+               else "4 x fallback bf16 1590 TFLOP/s (no measured peaks file)")
     hbm, _ = peaks()
     out = []
     for T in Ts:
@@ -617,7 +621,7 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
             "ffn_ms": round(ffn_ms, 4),
             "tflops": round(tf, 1),
             "fp4_peak_tflops": round(fp4_peak, 1),
-            "fp4_peak_source": "4 x measured bf16 (MEASURED_PEAKS.json bf16_tflops)",
+            "fp4_peak_source": fp4_src,
             "frac_fp4_peak": round(tf / fp4_peak, 4),
             "weight_gbs": round(gbs, 1),
             "frac_hbm": round(gbs / hbm, 4),

@@ -51,6 +51,7 @@ _SIGS = {
     "moe_permute": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_expert_ffn_workspace_bytes": (_SZ, [moe_shape, _I, _I, _I]),
+    "moe_expert_ffn_launches": (_I, [moe_shape, _I, _I, _I]),
     "moe_expert_ffn": (_I, [moe_shape, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P, _SZ, _P, _P]),
     "moe_combine_merge": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "moe_layer_forward": (_I, [moe_shape, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P, _P, _I, _P, _I, _P,
@@ -210,6 +211,11 @@ def moe_permute_noalloc(idx, E: int, offsets, perm, inv_perm, dev_status=None, s
 
 def moe_expert_ffn_workspace_bytes(s: moe_shape, T: int, k: int, flags: int = 0) -> int:
     return lib().moe_expert_ffn_workspace_bytes(s, T, k, flags)
+
+
+def moe_expert_ffn_launches(s: moe_shape, T: int, k: int, flags: int = 0) -> int:
+    """Kernels one moe_expert_ffn call launches (no device work)."""
+    return lib().moe_expert_ffn_launches(s, T, k, flags)
 
 
 def moe_expert_ffn(s: moe_shape, x, k: int, offsets, perm, slot_of_expert, slot_pool, n_slots: int,

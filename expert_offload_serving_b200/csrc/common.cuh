@@ -61,6 +61,10 @@ moe_status check_shape(moe_shape s);
 uint64_t wait_limit_ns();
 int test_stall();
 
+// Schedule of the tcgen05 decode GEMVs: gate/up and down in one cooperative
+// launch (true) or in two launches.
+bool decode_one_launch(int fmt, int T);
+
 // ---------------------------------------------------------------- device helpers
 constexpr unsigned kFull = 0xffffffffu;
 

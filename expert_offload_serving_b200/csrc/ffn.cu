@@ -24,6 +24,15 @@ extern "C" size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int 
   return decode_workspace_bytes(s, T, k);
 }
 
+extern "C" int moe_expert_ffn_launches(moe_shape s, int T, int k, int flags) {
+  if (check_shape(s) != MOE_OK || T <= 0 || k < 1 || k > 32) return 0;
+  if (flags & MOE_FFN_ACT_NVFP4) return 4;                 // quantise x, gather, GEMM1, GEMM2
+  const int gemvs = decode_one_launch(s.fmt, T) ? 1 : 2;
+  if (s.fmt == MOE_W_MXFP4 && mx_tiled(s.d, s.I)) return 1 + gemvs;   // + the split of x into E4M3 terms
+  if (s.fmt == MOE_W_BF16 && bf16_blocked(s.d, s.I)) return gemvs;
+  return 2;                                                // CUDA-core gate/up, down
+}
+
 moe_status moe::check_ffn_args(moe_shape s, const void* x, int T, int k, const int32_t* offsets,
                                const int32_t* perm, const int32_t* slot_of_expert, const void* slot_pool,
                                int n_slots, const float* gate, const float* y_perm, const float* out, int flags,

@@ -29,6 +29,8 @@
 // layout (d, I multiples of 256) go to the tcgen05 GEMVs in ffn_decode_tc.cu.
 #include <cuda_fp16.h>
 
+#include <cstdlib>
+#include <cstring>
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -590,6 +592,24 @@ moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t
 }  // namespace
 
 size_t decode_mx_workspace_bytes(moe_shape s, int T, int k);
+
+// One cooperative launch saves the second launch and its pipeline fill, but
+// its down units wait on their expert's gate/up units while the two-launch
+// schedule streams them back to back.  Measured on B200 (fraction of HBM
+// bandwidth, one-launch vs two-launch): bf16 T = 1 0.395 / 0.414, T = 16
+// 0.856 / 0.862, T = 64 0.753 / 0.817; MXFP4 T = 1 0.294 / 0.264, T = 8
+// 0.429 / 0.489.  So one launch only for MXFP4 single-token steps.
+bool decode_one_launch(int fmt, int T) {
+  static const int forced = [] {
+    const char* e = std::getenv("MOE_DECODE_SCHEDULE");
+    if (e == nullptr) return 0;
+    if (std::strcmp(e, "one") == 0) return 1;
+    if (std::strcmp(e, "two") == 0) return 2;
+    return 0;
+  }();
+  if (forced != 0) return forced == 1;
+  return fmt == MOE_W_MXFP4 && T <= 1;
+}
 
 size_t decode_workspace_bytes(moe_shape s, int T, int k) {
   // MXFP4 tensor-core path: the E4M3 terms of x and a with their scales;

@@ -41,6 +41,7 @@
 // double-buffered accumulators, warp 6 loads the token-row terms and their
 // scale atoms.  Every wait is bounded: on expiry the CTA records
 // MOE_ERR_TIMEOUT, stops issuing, drains what it issued and frees its TMEM.
+#include <algorithm>
 #include <cstdlib>
 
 #include <cuda_bf16.h>
@@ -68,7 +69,7 @@ constexpr int SFB_COL = SFA_COL + 8;
 constexpr int TMEM_COLS = 512;
 constexpr int NX = 2;                      // E4M3 terms of x
 constexpr int NA = 4;                      // E4M3 terms of a
-constexpr int PF_ITEMS = 8;                // L2 prefetch distance (tiles)
+constexpr int PF_ITEMS = 2;                // L2 prefetch distance (tiles; measured best of 0, 2, 4, 8, 12)
 constexpr int kSmemBudget = 226 * 1024;
 constexpr int kMaxE = 1024;
 constexpr int kBarBytes = 512;
@@ -117,20 +118,22 @@ __device__ __forceinline__ int sf_byte(int j) { return 4 * (j / (32 / TN)); }
 template <int PHASE, int TN>
 struct Cfg {
   static constexpr int NT = PHASE == 1 ? NX : NA;                // terms of the B operand (PHASE 3: both GEMVs)
-  static constexpr int G = 32 / TN;                              // scale planes
+  static constexpr int G = 32 / TN;                              // term planes per 32 scale-atom rows
   static constexpr int B_ATOM = TN * 128;                        // TN rows x 128 E4M3 values
   static constexpr int B_CODES = NT * 2 * B_ATOM;                // per 128-element half: the terms' rows stacked
   static constexpr int B_STAGE = B_CODES + 1024;                 // + one scale atom per half
   static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;
   static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
-  // token-row stages: gemv<2>'s come from the a terms gemv<1> just wrote (L2)
-  static constexpr int SB = PHASE != 1 ? 2 : (B_STAGE <= 12 * 1024 ? 4 : 3);
+  // token-row stages: the rows come from L2 (x, or the a terms gemv<1> just
+  // wrote), and the ring must cover an L2 round trip at the weight stream's
+  // pace (~0.4 us per stage): 4 where they fit beside 4+ weight stages
+  static constexpr int SB = B_STAGE <= 12 * 1024 ? 4 : (PHASE == 1 ? 3 : 2);
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_SMEM;
   static constexpr int SA = SA_FIT > 8 ? 8 : SA_FIT;
   static constexpr int A_RING = SA * A_SMEM;
   static constexpr int B_RING = SB * B_STAGE;
   static constexpr int N_BARS = 2 * SA + 2 * SB + 6;
-  static_assert(TN == 16 || TN == 32, "chunk width");
+  static_assert(TN == 8 || TN == 16 || TN == 32, "chunk width");
   static_assert(A_SMEM % 1024 == 0 && B_STAGE % 1024 == 0 && B_ATOM % 1024 == 0, "1024-byte alignment");
   static_assert(SA >= 3, "weight ring");
   static_assert(FIXED + A_RING + B_RING <= kSmemBudget, "shared memory budget");
@@ -343,7 +346,8 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
   const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
   const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid)
                                   : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
-  if (lane == 0) mbar_expect_tx(bar, rows * 2 * (static_cast<uint32_t>(nt) * 128u + C::G * 16u));
+  const int planes = nt < C::G ? nt : C::G;   // scale planes of this unit's terms
+  if (lane == 0) mbar_expect_tx(bar, rows * 2 * static_cast<uint32_t>(nt * 128 + planes * 16));
   __syncwarp();
   if (U.ph == 2) {
     if (lane == 0) {
@@ -354,7 +358,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
         for (int j = 0; j < NA; ++j)
           tma_load_3d(sB + (h * NA + j) * C::B_ATOM, &M.a[bi], bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
 #pragma unroll
-        for (int g = 0; g < C::G; ++g)
+        for (int g = 0; g < (NA < C::G ? NA : C::G); ++g)
           tma_load_4d(sf + h * 512 + g * TN * 16, &M.as[bi], bar, 0, 2 * ks + h, U.q0, g, pol);
       }
     }
@@ -365,7 +369,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
       for (int j = 0; j < NX; ++j)
         tma_load_3d(sB + (h * NX + j) * C::B_ATOM + lane * 128, &M.x, bar, ks * KSTAGE + 128 * h, tok, j, pol);
 #pragma unroll
-      for (int g = 0; g < C::G; ++g)
+      for (int g = 0; g < (NX < C::G ? NX : C::G); ++g)
         bulk_load(sf + h * 512 + (g * TN + lane) * 16,
                   P.xs + ((static_cast<size_t>(g) * P.T + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
     }
@@ -457,7 +461,18 @@ __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 // stacked terms of accumulator columns j*TN + c (fp32, terms in order).
 template <int TN>
 __device__ __forceinline__ void load_terms(uint32_t taddr, int nt, float (&v)[32]) {
-  if (TN == 16) {
+  if (TN == 8) {
+    float t[8];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NA; ++j) {
+      if (j >= nt) break;
+      tmem_ld8(taddr + 8 * j, t);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[c] += t[c];
+    }
+  } else if (TN == 16) {
     float t[16];
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = 0.f;
@@ -904,17 +919,9 @@ MxWorkspace mx_workspace(moe_shape s, int T, int k) {
   return W;
 }
 
-// Both GEMVs in one cooperative launch unless MOE_DECODE_TWO_LAUNCHES is set
-// in the environment (read once; the two-launch schedule is kept for
-// comparison).
-bool fused_decode() {
-  static const bool fused = std::getenv("MOE_DECODE_TWO_LAUNCHES") == nullptr;
-  return fused;
-}
-
 template <int TN>
 moe_status launch_both(const MxParams& P, const MxMaps& M, const DeviceInfo& dev, cudaStream_t stream) {
-  if (fused_decode()) return launch_phase<3, TN>(P, M, dev, stream);   // counters zeroed by mx_split_x_kernel
+  if (decode_one_launch(MOE_W_MXFP4, P.T)) return launch_phase<3, TN>(P, M, dev, stream);   // counters zeroed by mx_split_x_kernel
   moe_status st = launch_phase<1, TN>(P, M, dev, stream);
   if (st != MOE_OK) return st;
   return launch_phase<2, TN>(P, M, dev, stream);
@@ -932,10 +939,7 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   MxParams P{};
   P.wait_ns = wait_limit_ns();
-  {
-    static const char* pf = std::getenv("MOE_DECODE_PF");   // tuning sweep
-    P.pf_items = pf ? std::atoi(pf) : PF_ITEMS;
-  }
+  P.pf_items = PF_ITEMS;
   P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;
@@ -979,7 +983,8 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint32_t box[3] = {128u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
     r = encode_tiled_sw128(&M.a[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
     // scale rows of the a terms: (byte in the atom row, atom, pair, term); a box of rows
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(T <= 16 ? 2 : 1)};
+    const int tn = T <= 8 ? 8 : (T <= 16 ? 16 : 32);
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(std::min(32 / tn, NA))};
     const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, n * (s.I / 128) * 16};
     const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
     if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
@@ -988,14 +993,18 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   {
     const long long blocks = static_cast<long long>(T) * (s.d / 32);
     const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
-    if (T <= 16)
+    if (T <= 8)
+      mx_split_x_kernel<8><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+                                                     w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
+    else if (T <= 16)
       mx_split_x_kernel<16><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
-                                                      w8 + W.xs, P.done1, fused_decode() ? s.E : 0);
+                                                      w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
     else
       mx_split_x_kernel<32><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
-                                                      w8 + W.xs, P.done1, fused_decode() ? s.E : 0);
+                                                      w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
+  if (T <= 8) return launch_both<8>(P, M, dev, stream);
   return T <= 16 ? launch_both<16>(P, M, dev, stream) : launch_both<32>(P, M, dev, stream);
 }
 

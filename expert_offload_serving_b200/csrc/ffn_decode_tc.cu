@@ -23,7 +23,7 @@
 // Work unit = (expert, 128-row tile, chunk of <= TN pairs; TN = 16 when T <=
 // 16, else 32), expert-major, chunks fastest, dealt round-robin to one
 // persistent CTA per SM.  Warp 0 produces the weight stages (bulk copy, L2
-// prefetch four stages ahead), warp 1 owns TMEM and issues the MMAs, four
+// prefetch two stages ahead), warp 1 owns TMEM and issues the MMAs, four
 // warps run the epilogue on double-buffered TMEM accumulators, and the last
 // warp loads the token rows into a ring of their own.  The weight ring takes
 // the shared memory the rest leaves (5 stages of 32 KB), so that the GEMVs
@@ -66,7 +66,7 @@ using namespace ::moe::tc;
 
 constexpr int TM = 128;                  // weight rows per tile
 constexpr int ACC_COLS = 32;             // TMEM columns per accumulator
-constexpr int PF_ITEMS = 4;              // L2 prefetch distance (stages)
+constexpr int PF_ITEMS = 2;              // L2 prefetch distance (stages; measured best of 0, 2, 4, 8, 12)
 constexpr int kSmemBudget = 226 * 1024;  // opt-in shared memory of one CTA (227 KB) less the static 1 KB
 constexpr int kMaxE = 1024;              // experts the unit table is sized for
 constexpr int kBarBytes = 512;           // mbarriers, the TMEM address and two flags
@@ -685,18 +685,10 @@ moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tx, const CU
   return MOE_OK;
 }
 
-// Both GEMVs in one cooperative launch unless MOE_DECODE_TWO_LAUNCHES is set
-// in the environment (read once; the two-launch schedule is kept for
-// comparison).
-bool fused_decode() {
-  static const bool fused = std::getenv("MOE_DECODE_TWO_LAUNCHES") == nullptr;
-  return fused;
-}
-
 template <int FMT, int TN>
 moe_status launch_both(const TcDecodeParams& P, const CUtensorMap& tm_x, const CUtensorMap (&tm_a)[3],
                        const DeviceInfo& dev, cudaStream_t stream) {
-  if (fused_decode()) {
+  if (decode_one_launch(FMT, P.T)) {
     MOE_CUDA_TRY(cudaMemsetAsync(P.done1, 0, static_cast<size_t>(P.E) * sizeof(int32_t), stream));
     return launch_phase<FMT, 3, TN>(P, tm_x, tm_a[2], tm_a[1], tm_a[0], dev, stream);
   }
@@ -714,10 +706,7 @@ moe_status launch_decode_tc(moe_shape s, const void* x, int T, int k, const int3
                             float* out, void* ws, int32_t* status, const DeviceInfo& dev, cudaStream_t stream) {
   TcDecodeParams P{};
   P.wait_ns = wait_limit_ns();
-  {
-    static const char* pf = std::getenv("MOE_DECODE_PF");   // tuning sweep
-    P.pf_items = pf ? std::atoi(pf) : PF_ITEMS;
-  }
+  P.pf_items = PF_ITEMS;
   P.stall = test_stall();
   P.E = s.E;
   P.d = s.d;

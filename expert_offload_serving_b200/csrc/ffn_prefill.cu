@@ -35,7 +35,7 @@
 //               and 4 tcgen05.mma kind::mxf4nvf4 block16 (K = 64 each) into
 //               one of two 224-column accumulators, then commits to both
 //               CTAs' stage and accumulator barriers;
-//   warps 2-9   epilogue, two groups of four warps (each warp reads its 32
+//   warps 2-17  epilogue, four groups of four warps (each warp reads its 32
 //               TMEM lanes of its own CTA; the groups take alternate 16-column
 //               slabs), overlapped with the next tile's main loop; the two
 //               CTAs' epilogues each release the accumulator to the even CTA.
@@ -70,9 +70,16 @@ constexpr int SFA_BYTES = 2048;         // 4 atoms: this CTA's 128 weight rows x
 constexpr int SFB_BYTES = 4096;         // 2 atom rows (256 chunk rows) x 4 MMA K steps
 constexpr int OFF_B = A_BYTES, OFF_SFA = OFF_B + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
 constexpr int STAGE_BYTES = OFF_SFB + SFB_BYTES;      // 36 KB; every box lands whole (fill out of range)
-constexpr int EPI_GROUPS = 2;           // epilogue warp groups (each covers the 4 TMEM lane quadrants)
+// Epilogue: four warp groups, each covering the 4 TMEM lane quadrants (with
+// two, the epilogue rather than the tensor core bounded the GEMMs at large T).
+// Each group transposes 16-column slabs through shared memory: rows of
+// EPI_PITCH floats, 129 for GEMM1 (its threads read 8 consecutive
+// intermediate values of one column: a pitch of 128 put 8 of them on one
+// bank) and 128 for GEMM2 (16-byte vector reads of 4 output rows).
+constexpr int EPI_GROUPS = 4;
 constexpr int EPI_THREADS = 128 * EPI_GROUPS;
-constexpr int EPI_BYTES = EPI_GROUPS * 16 * 128 * 4 + 2 * VR * 4;   // a transposed 16-column slab per group + column info
+constexpr int EPI_SLAB = 16 * 132;                  // floats per group's slab (pitch <= 132)
+constexpr int EPI_BYTES = EPI_GROUPS * EPI_SLAB * 4 + 2 * VR * 4;   // slabs + column info
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = CH;            // per accumulator buffer (two)
 constexpr int SFA_COL = 2 * ACC_COLS;   // 4 MMA K steps x 4 columns
@@ -136,8 +143,8 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t
 
 // ------------------------------------------------------------------ NVFP4 quantisation
 // 16 values -> E4M3 scale byte s = e4m3_rn_satfinite(amax / 6) and 8 code
-// bytes q_i = e2m1_rn_satfinite(v_i / s) (IEEE fp32 division; all zero when s
-// is 0).  Element 2i goes to the low nibble.
+// bytes q_i = e2m1_rn_satfinite(v_i / s) (of the IEEE fp32 quotient; all zero
+// when s is 0).  Element 2i goes to the low nibble.
 __device__ __forceinline__ uint32_t e4m3_byte(float x) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
@@ -156,10 +163,27 @@ __device__ __forceinline__ uint32_t e2m1x2_byte(float lo, float hi) {
   return r;
 }
 
-// codes of 8 values (already divided by the scale) -> 4 bytes
-__device__ __forceinline__ uint32_t pack8(const float (&q)[8]) {
-  return e2m1x2_byte(q[0], q[1]) | (e2m1x2_byte(q[2], q[3]) << 8) | (e2m1x2_byte(q[4], q[5]) << 16) |
-         (e2m1x2_byte(q[6], q[7]) << 24);
+// Codes of the pair (lo / s, hi / s), s > 0: the byte that the E2M1
+// conversion gives for the correctly rounded fp32 quotients.  The quotients
+// are first taken approximately (__fdividef: within 2 ulp for these
+// divisors); the conversion is monotonic, so when the approximations scaled
+// by 1 - 2^-20 and by 1 + 2^-20 (8 ulp either way, bracketing the rounded
+// quotients) convert to the same byte, that byte is the answer; otherwise
+// (a quotient within a few ulp of a rounding boundary) the IEEE divisions
+// decide.
+__device__ __forceinline__ uint32_t e2m1x2_div(float lo, float hi, float s) {
+  const float a = __fdividef(lo, s), b = __fdividef(hi, s);
+  const float up = 1.0f + 0x1p-20f, dn = 1.0f - 0x1p-20f;
+  const uint32_t c = e2m1x2_byte(a, b);
+  if (e2m1x2_byte(a * up, b * up) == c && e2m1x2_byte(a * dn, b * dn) == c) return c;
+  return e2m1x2_byte(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
+}
+
+// codes of v[0..7] / s -> 4 bytes (all zero when s is 0)
+__device__ __forceinline__ uint32_t pack8_div(const float* v, float s) {
+  if (!(s > 0.f)) return 0u;
+  return e2m1x2_div(v[0], v[1], s) | (e2m1x2_div(v[2], v[3], s) << 8) | (e2m1x2_div(v[4], v[5], s) << 16) |
+         (e2m1x2_div(v[6], v[7], s) << 24);
 }
 
 // ------------------------------------------------------------------ shared prologue
@@ -274,13 +298,8 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(const uint16_t* __res
       for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
       const uint32_t sb = e4m3_byte(__fdiv_rn(amax, 6.0f));
       const float s = e4m3_value(sb);
-      float q0[8], q1[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        q0[j] = (s > 0.f) ? __fdiv_rn(v[j], s) : 0.f;
-        q1[j] = (s > 0.f) ? __fdiv_rn(v[8 + j], s) : 0.f;
-      }
-      *reinterpret_cast<uint2*>(xt + static_cast<size_t>(t) * (d / 2) + 8 * b) = make_uint2(pack8(q0), pack8(q1));
+      *reinterpret_cast<uint2*>(xt + static_cast<size_t>(t) * (d / 2) + 8 * b) =
+          make_uint2(pack8_div(v, s), pack8_div(v + 8, s));
       xts[static_cast<size_t>(t) * nb + b] = static_cast<uint8_t>(sb);
     }
   }
@@ -337,7 +356,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* epi_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
-  int32_t* col_t = reinterpret_cast<int32_t*>(epi_all + EPI_GROUPS * 16 * 128);
+  int32_t* col_t = reinterpret_cast<int32_t*>(epi_all + EPI_GROUPS * EPI_SLAB);
   float* col_g = reinterpret_cast<float*>(col_t + VR);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
   uint64_t* full = bars;                   // [STAGES] even CTA: both CTAs' copies of a stage
@@ -516,12 +535,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
       mbar_drain(drain, 0);
     }
   } else {
-    // ---------------------------------------------------------- epilogue (warps 2..9, both CTAs)
+    // ---------------------------------------------------------- epilogue (warps 2..17, both CTAs)
     const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
     const int grp = (warp - 2) >> 2;            // column group: slabs grp, grp+2, ...
     const int et = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
     const int eall = (warp - 2) * 32 + lane;       // 0..255 over both groups
-    float* epi = epi_all + grp * 16 * 128;
+    float* epi = epi_all + grp * EPI_SLAB;
+    constexpr int PITCH = PHASE == 1 ? 129 : 128;
     const int bar_grp = 1 + grp, bar_all = 1 + EPI_GROUPS;   // named barriers (0: __syncthreads)
     const uint32_t release = cluster_addr(&tempty[0], 0);   // + 8 * acc
     const float* ts = nullptr;
@@ -551,7 +571,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           col_g[eall] = good ? P.gate[p] : 0.f;
         }
       }
-      // the eight epilogue warps agree before any leaves: a warp alone at a
+      // the epilogue warps agree before any leaves: a warp alone at a
       // named barrier would wait for good (this barrier also publishes the
       // column info written above)
       if (!mbar_wait(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
@@ -572,7 +592,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
           // thread adds 4 consecutive output rows of one column with one
           // vector reduction: out[t][row .. row+3] += gate * g_d * y
 #pragma unroll
-          for (int j = 0; j < 16; ++j) epi[j * 128 + 32 * quad + lane] = v[j];
+          for (int j = 0; j < 16; ++j) epi[j * PITCH + 32 * quad + lane] = v[j];
           named_sync(bar_grp, 128);
 #pragma unroll
           for (int it2 = 0; it2 < 4; ++it2) {
@@ -583,7 +603,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
               const int t = col_t[col];
               if (t >= 0) {
                 const float gm = col_g[col] * g_mat;
-                const float4 y = *reinterpret_cast<const float4*>(epi + cl * 128 + 4 * rq);
+                const float4 y = *reinterpret_cast<const float4*>(epi + cl * PITCH + 4 * rq);
                 float* dst = P.out + static_cast<size_t>(t) * P.d + m * BM + 4 * rq;
                 asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(gm * y.x),
                              "f"(gm * y.y), "f"(gm * y.z), "f"(gm * y.w)
@@ -595,7 +615,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
         } else {
           // transpose the 16-column slab through shared memory: epi[col][row]
 #pragma unroll
-          for (int j = 0; j < 16; ++j) epi[j * 128 + 32 * quad + lane] = v[j];
+          for (int j = 0; j < 16; ++j) epi[j * PITCH + 32 * quad + lane] = v[j];
           named_sync(bar_grp, 128);
           // item: column cl, 16-block b of the 64 intermediate indices, half h
           const int cl = et >> 3, b = (et >> 1) & 3, h = et & 1;
@@ -605,18 +625,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_fp4_kernel(const __grid_const
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int il = 16 * b + 8 * h + j;
-            const float hg = epi[cl * 128 + il] * g_gate;
-            const float hu = epi[cl * 128 + 64 + il] * g_up;
+            const float hg = epi[cl * PITCH + il] * g_gate;
+            const float hu = epi[cl * PITCH + 64 + il] * g_up;
             a[j] = __fdividef(hg, 1.0f + __expf(-hg)) * hu;
             amax = fmaxf(amax, fabsf(a[j]));
           }
           amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
           const uint32_t sb = e4m3_byte(__fdiv_rn(amax, 6.0f));
-          const float s = e4m3_value(sb);
-          float q[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) q[j] = (s > 0.f) ? __fdiv_rn(a[j], s) : 0.f;
-          const uint32_t codes = pack8(q);
+          const uint32_t codes = pack8_div(a, e4m3_value(sb));
           if (col < nvalid) {
             const int prow = c * VR + col;
             const int i0 = m * 64;                       // first intermediate index of the tile

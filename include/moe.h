@@ -202,18 +202,27 @@ moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E,
  *   dev_status: device int32 word or NULL.  Kernels record the first error
  *              there (read it with moe_check_status after the stream):
  *              MOE_ERR_DEVICE   a slot or expert index out of range;
- *              MOE_ERR_TIMEOUT  a bounded wait on the copy pipeline ran out;
- *              MOE_ERR_UNSUPPORTED  (MXFP4 on the tensor-core path, which
- *                               multiplies in f16 exactly) an E8M0 scale
- *                               above 2^13, or below 2^-23 on a block with
- *                               nonzero codes, or |x| or |a| above 65504.
+ *              MOE_ERR_TIMEOUT  a bounded wait on the copy pipeline ran out.
+ *              (The MXFP4 tensor-core path applies the E8M0 scales in the
+ *              tensor core and takes the activations as E4M3 terms under E8M0
+ *              scales of their own: no range limit beyond fp32's.)
  * Paths (chosen from the shape, the same results up to rounding order):
  *   BF16 with d, I multiples of 256 and MXFP4 with d, I multiples of 256: the
- *   tcgen05 decode GEMVs over the tile layouts of moe_pack_expert; other
- *   BF16/MXFP4 shapes and NVFP4 without MOE_FFN_ACT_NVFP4: CUDA cores;
- *   MOE_FFN_ACT_NVFP4: the tcgen05 FP4 GEMMs (d, I multiples of 256).
+ *   tcgen05 decode GEMVs over the tile layouts of moe_pack_expert (gate/up
+ *   and down in one cooperative launch or in two launches: see
+ *   moe_expert_ffn_launches); other BF16/MXFP4 shapes and NVFP4 without
+ *   MOE_FFN_ACT_NVFP4: CUDA cores; MOE_FFN_ACT_NVFP4: the tcgen05 FP4 GEMMs
+ *   (d, I multiples of 256).
  * Limits: T*k <= 1<<24. */
 size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int flags);
+
+/* Number of kernels one moe_expert_ffn call with these arguments launches on
+ * its stream (for launch accounting; no device work).  The tcgen05 decode
+ * GEMVs run gate/up and down in one cooperative launch or in two launches:
+ * the default is chosen per weight format and T from measurements, and the
+ * environment variable MOE_DECODE_SCHEDULE=one|two, read once per process,
+ * fixes it.  Returns 0 for invalid arguments or T == 0. */
+int moe_expert_ffn_launches(moe_shape s, int T, int k, int flags);
 moe_status moe_expert_ffn(moe_shape s, const void* x, int T, int k,
                           const int32_t* offsets, const int32_t* perm,
                           const int32_t* slot_of_expert, const void* slot_pool, int n_slots,

@@ -158,11 +158,12 @@ def test_many_tokens_per_expert(moe, fmt):
 
 
 @pytest.mark.parametrize("fmt", ["bf16", "mxfp4"])
-@pytest.mark.parametrize("T", [16, 17])
+@pytest.mark.parametrize("T", [8, 9, 16, 17])
 def test_chunk_width_boundary(moe, fmt, T):
-    """T = 16 runs 16-pair chunks, T = 17 32-pair chunks; E = 4, k = 4 puts
-    every token on every expert, so the groups fill the chunk exactly (16) or
-    spill one pair past it (17)."""
+    """The MXFP4 path runs 8-pair chunks up to T = 8, 16-pair chunks up to
+    T = 16 and 32-pair chunks above; bf16 16-pair chunks up to T = 16.  E = 4,
+    k = 4 puts every token on every expert, so the groups fill a chunk
+    exactly (8, 16) or spill one pair past it (9, 17)."""
     cfg = synth.LayerConfig("full", E=4, k=4, d=512, I=256, fmt=fmt)
     b = Built(cfg, T, seed=7)
     check_tol(b.run().cpu().numpy(), b.oracle()["out"], 1e-4, 1e-5)
