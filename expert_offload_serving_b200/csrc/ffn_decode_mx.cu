@@ -123,7 +123,7 @@ struct Cfg {
   static constexpr int B_CODES = NT * 2 * B_ATOM;                // per 128-element half: the terms' rows stacked
   static constexpr int B_STAGE = B_CODES + 1024;                 // + one scale atom per half
   static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;
-  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
+  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + 3 * (kMaxE + 1) * 4;   // + the unit table
   // token-row stages: the rows come from L2 (x, or the a terms gemv<1> just
   // wrote), and the ring must cover an L2 round trip at the weight stream's
   // pace (~0.4 us per stage): 4 where they fit beside 4+ weight stages
@@ -145,7 +145,7 @@ template <int PHASE, int TN>
 constexpr size_t smem_bytes(int E) {
   using C = Cfg<PHASE, TN>;
   return 1024 + static_cast<size_t>(C::A_RING) + C::B_RING + C::UP_BYTES + kBarBytes +
-         static_cast<size_t>(E + 1) * 4;
+         3 * static_cast<size_t>(E + 1) * 4;
 }
 
 struct Unit {
@@ -174,7 +174,8 @@ __device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart
   Unit U;
   U.e = lo;
   U.ph = ph;
-  const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+  const int32_t* eoff = ustart + P.E + 1;   // the unit table's copy of offsets
+  const int q_begin = eoff[lo], ne = eoff[lo + 1] - q_begin;
   const int chunks = (ne + TN - 1) / TN;
   const int local = u - ustart[lo] / den * num;
   U.m = local / chunks;
@@ -185,9 +186,9 @@ __device__ __forceinline__ Unit unit_of(const MxParams& P, const int32_t* ustart
 }
 
 // First byte of the blob tile (expert U.e, row tile U.m, k tile 0) of the unit's phase.
-__device__ __forceinline__ const uint8_t* tile_base(const MxParams& P, const Unit& U) {
+__device__ __forceinline__ const uint8_t* tile_base(const MxParams& P, const Unit& U, const int32_t* eslot) {
   const int K = (U.ph == 1) ? P.d : P.I;
-  const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
+  const uint8_t* blob = P.pool + static_cast<size_t>(eslot[U.e]) * P.blob_bytes;
   return blob + (U.ph == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / KSTAGE) * kMxTileBytes;
 }
 
@@ -210,10 +211,10 @@ __device__ void prefetch_down_units(const MxParams& P, const int32_t* ustart1, i
       if (ustart1[mid] / per1 * per2 <= u) lo = mid;
       else hi = mid;
     }
-    const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+    const int q_begin = ustart1[P.E + 1 + lo], ne = ustart1[P.E + 2 + lo] - q_begin;
     const int chunks = (ne + TN - 1) / TN;
     const int m = (u - ustart1[lo] / per1 * per2) / chunks;
-    const uint8_t* base = P.pool + static_cast<size_t>(__ldg(P.slot + lo)) * P.blob_bytes + P.L.wd +
+    const uint8_t* base = P.pool + static_cast<size_t>(ustart1[2 * (P.E + 1) + lo]) * P.blob_bytes + P.L.wd +
                           static_cast<size_t>(m) * KS2 * kMxTileBytes;
     for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
       prefetch_l2(base + static_cast<size_t>(ks) * kMxTileBytes, kMxTileBytes);
@@ -517,6 +518,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
   int32_t* ustart = reinterpret_cast<int32_t*>(ring_b + C::B_RING + C::UP_BYTES + kBarBytes);
+  int32_t* eoff = ustart + (P.E + 1);          // offsets[0..E] and slot[0..E-1], read once
+  int32_t* eslot = eoff + (P.E + 1);
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -579,9 +582,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     ustart[e] = run;
     const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
     const int s = __ldg(P.slot + e);
+    eoff[e] = a;                 // copies for the unit lookups (no global load on a producer's path)
+    eslot[e] = s;
     if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * ((b - a + TN - 1) / TN);
   }
-  if (threadIdx.x == 0) ustart[P.E] = total;
+  if (threadIdx.x == 0) {
+    ustart[P.E] = total;
+    eoff[P.E] = __ldg(P.offsets + P.E);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -599,13 +607,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint8_t* pf_base = nullptr;
     if (pf_u < n_units) {
       const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
-      pf_base = tile_base(P, V);
+      pf_base = tile_base(P, V, eslot);
       pf_KS = ks_of(V);
     }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
-      const int sl = __ldg(P.slot + U.e);
-      const uint8_t* abase = tile_base(P, U);
+      const int sl = eslot[U.e];
+      const uint8_t* abase = tile_base(P, U, eslot);
       const CUtensorMap* tm_w = U.ph == 1 ? &M.w1 : &M.w2;
       const int KS = ks_of(U);
       for (int ks = 0; ks < KS; ++ks) {
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               pf_u += gridDim.x;
               if (pf_u < n_units) {
                 const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
-                pf_base = tile_base(P, V);
+                pf_base = tile_base(P, V, eslot);
                 pf_KS = ks_of(V);
               }
             }

@@ -88,7 +88,7 @@ struct Cfg {
   static constexpr int A_STAGE = 2 * TM * 128;                   // weight bytes per stage
   static constexpr int B_STAGE = (PHASE == 1 ? 1 : 2) * ATOMS * B_ATOM;   // PHASE 3: both GEMVs
   static constexpr int UP_BYTES = PHASE != 2 ? 64 * 33 * 4 : 0;  // up-row exchange
-  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + (kMaxE + 1) * 4;
+  static constexpr int FIXED = 1024 + UP_BYTES + kBarBytes + 3 * (kMaxE + 1) * 4;   // + the unit table
   static constexpr int SB = B_STAGE <= 8192 ? (PHASE == 1 && TN == 32 ? 4 : 5) : 3;   // token-row stages
   static constexpr int SA_FIT = (kSmemBudget - FIXED - SB * B_STAGE) / A_STAGE;
   static constexpr int SA = (TN == 16 && PHASE == 1) ? 5 : (SA_FIT > 12 ? 12 : SA_FIT);   // weight stages
@@ -110,7 +110,7 @@ template <int FMT, int PHASE, int TN>
 constexpr size_t smem_bytes(int E) {
   using C = Cfg<FMT, PHASE, TN>;
   return 1024 + static_cast<size_t>(C::A_RING) + C::B_RING + C::UP_BYTES + kBarBytes +
-         static_cast<size_t>(E + 1) * 4;
+         3 * static_cast<size_t>(E + 1) * 4;
 }
 
 struct Unit {
@@ -141,7 +141,8 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
   Unit U;
   U.e = lo;
   U.ph = ph;
-  const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+  const int32_t* eoff = ustart + P.E + 1;   // the unit table's copy of offsets
+  const int q_begin = eoff[lo], ne = eoff[lo + 1] - q_begin;
   const int chunks = (ne + TN - 1) / TN;
   const int local = u - ustart[lo] / den * num;
   U.m = local / chunks;
@@ -153,10 +154,10 @@ __device__ __forceinline__ Unit unit_of(const TcDecodeParams& P, const int32_t* 
 
 // First byte of unit U's weight tile (its K stages follow at A_STAGE).
 template <int FMT>
-__device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, const Unit& U) {
+__device__ __forceinline__ const uint8_t* tile_base(const TcDecodeParams& P, const Unit& U, const int32_t* eslot) {
   using C = Cfg<FMT, 1, 32>;   // the weight stages depend on neither phase nor TN
   const int K = (U.ph == 1) ? P.d : P.I;
-  const uint8_t* blob = P.pool + static_cast<size_t>(__ldg(P.slot + U.e)) * P.blob_bytes;
+  const uint8_t* blob = P.pool + static_cast<size_t>(eslot[U.e]) * P.blob_bytes;
   return blob + (U.ph == 1 ? P.L.wg : P.L.wd) + static_cast<size_t>(U.m) * (K / C::KSTAGE) * C::A_STAGE;
 }
 
@@ -181,10 +182,10 @@ __device__ void prefetch_down_units(const TcDecodeParams& P, const int32_t* usta
       if (ustart1[mid] / per1 * per2 <= u) lo = mid;
       else hi = mid;
     }
-    const int q_begin = __ldg(P.offsets + lo), ne = __ldg(P.offsets + lo + 1) - q_begin;
+    const int q_begin = ustart1[P.E + 1 + lo], ne = ustart1[P.E + 2 + lo] - q_begin;
     const int chunks = (ne + TN - 1) / TN;
     const int m = (u - ustart1[lo] / per1 * per2) / chunks;
-    const uint8_t* base = P.pool + static_cast<size_t>(__ldg(P.slot + lo)) * P.blob_bytes + P.L.wd +
+    const uint8_t* base = P.pool + static_cast<size_t>(ustart1[2 * (P.E + 1) + lo]) * P.blob_bytes + P.L.wd +
                           static_cast<size_t>(m) * KS2 * C::A_STAGE;
     for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
       prefetch_l2(base + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE);
@@ -327,6 +328,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
   int32_t* ustart = reinterpret_cast<int32_t*>(ring_b + C::B_RING + C::UP_BYTES + kBarBytes);
+  int32_t* eoff = ustart + (P.E + 1);          // offsets[0..E] and slot[0..E-1], read once
+  int32_t* eslot = eoff + (P.E + 1);
   __shared__ int ws[36];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -389,9 +392,14 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     ustart[e] = run;
     const int a = __ldg(P.offsets + e), b = __ldg(P.offsets + e + 1);
     const int s = __ldg(P.slot + e);
+    eoff[e] = a;                 // copies for the unit lookups (no global load on a producer's path)
+    eslot[e] = s;
     if (b > a && a >= 0 && b <= n_pairs && s >= 0 && s < P.n_slots) run += MT * ((b - a + TN - 1) / TN);
   }
-  if (threadIdx.x == 0) ustart[P.E] = total;
+  if (threadIdx.x == 0) {
+    ustart[P.E] = total;
+    eoff[P.E] = __ldg(P.offsets + P.E);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -410,12 +418,12 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     const uint8_t* pf_base = nullptr;
     if (pf_u < n_units) {
       const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
-      pf_base = tile_base<FMT>(P, V);
+      pf_base = tile_base<FMT>(P, V, eslot);
       pf_KS = ks_of(V);
     }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
-      const uint8_t* abase = tile_base<FMT>(P, U);
+      const uint8_t* abase = tile_base<FMT>(P, U, eslot);
       const int KS = ks_of(U);
       for (int ks = 0; ks < KS; ++ks) {
         // one verdict for the warp: its lanes take the same path
@@ -438,7 +446,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
               pf_u += gridDim.x;
               if (pf_u < n_units) {
                 const Unit V = unit_of<PHASE, TN>(P, ustart, MT, MT2, pf_u);
-                pf_base = tile_base<FMT>(P, V);
+                pf_base = tile_base<FMT>(P, V, eslot);
                 pf_KS = ks_of(V);
               }
             }
