@@ -81,7 +81,7 @@ struct MxParams {
   int pf_items;              // L2 prefetch distance in stages
   int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
-  int a_box_rows[3];       // rows of the a-plane TMA boxes: min(8 | 16 | 32, T*k)
+  int a_rows;              // rows of each a-term plane: max(T*k, 32), so a TN-row box always fits
   const int32_t* offsets;
   const int32_t* perm;
   const int32_t* slot;
@@ -90,18 +90,20 @@ struct MxParams {
   size_t blob_bytes;
   BlobLayout L;
   const uint8_t* xs;       // [32/TN][T][d/128][16] E8M0 scales of the x terms (sf_plane / sf_byte)
-  uint8_t* aq;             // [NA][T*k][I] E4M3 terms of a (rows = sorted pairs)
-  uint8_t* as;             // [32/TN][T*k][I/128][16] their E8M0 scales (sf_plane / sf_byte)
+  uint8_t* aq;             // [NA][a_rows][I] E4M3 terms of a (rows = sorted pairs)
+  uint8_t* as;             // [32/TN][a_rows][I/128][16] their E8M0 scales (sf_plane / sf_byte)
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
   float* y_perm;
   float* out;
   int32_t* status;
 };
 
-// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms, the
-// a terms and their scale rows (boxes of 8, 16, 32 rows).
+// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms
+// (one-row boxes), and the a terms and their scale rows (boxes of TN rows of
+// every term, resp. every scale plane: the stacked B operand of one
+// 128-element half in one copy each).
 struct MxMaps {
-  CUtensorMap w1, w2, x, a[3], as[3];
+  CUtensorMap w1, w2, x, a, as;
 };
 
 // Scale rows of stacked terms.  B row r = j*TN + t (term j, token row t)
@@ -323,12 +325,6 @@ __device__ __forceinline__ int token_of(const MxParams& P, const Unit& U, int la
   return tok;
 }
 
-template <int TN>
-__device__ __forceinline__ int a_box(const MxParams& P, int nvalid) {
-  if (nvalid <= P.a_box_rows[0]) return 0;
-  return (TN == 16 || nvalid <= P.a_box_rows[1]) ? 1 : 2;
-}
-
 // Token-row terms of K stage ks of unit U into the B stage at sB, and their
 // E8M0 scale atoms after them, all asynchronous copies completing on bar
 // (whose expected bytes lane 0 posts first).  Per 128-element half h the
@@ -345,22 +341,16 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
                                        uint8_t* sB, uint64_t* bar, uint64_t pol, int lane) {
   uint8_t* sf = sB + C::B_CODES;
   const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
-  const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid)
-                                  : static_cast<uint32_t>(P.a_box_rows[a_box<TN>(P, U.nvalid)]);
+  const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid) : static_cast<uint32_t>(TN);
   const int planes = nt < C::G ? nt : C::G;   // scale planes of this unit's terms
   if (lane == 0) mbar_expect_tx(bar, rows * 2 * static_cast<uint32_t>(nt * 128 + planes * 16));
   __syncwarp();
   if (U.ph == 2) {
     if (lane == 0) {
-      const int bi = a_box<TN>(P, U.nvalid);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int j = 0; j < NA; ++j)
-          tma_load_3d(sB + (h * NA + j) * C::B_ATOM, &M.a[bi], bar, ks * KSTAGE + 128 * h, U.q0, j, pol);
-#pragma unroll
-        for (int g = 0; g < (NA < C::G ? NA : C::G); ++g)
-          tma_load_4d(sf + h * 512 + g * TN * 16, &M.as[bi], bar, 0, 2 * ks + h, U.q0, g, pol);
+        tma_load_3d(sB + h * NA * C::B_ATOM, &M.a, bar, ks * KSTAGE + 128 * h, U.q0, 0, pol);
+        tma_load_4d(sf + h * 512, &M.as, bar, 0, 2 * ks + h, U.q0, 0, pol);
       }
     }
   } else if (lane < U.nvalid) {
@@ -521,6 +511,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   int32_t* eoff = ustart + (P.E + 1);          // offsets[0..E] and slot[0..E-1], read once
   int32_t* eslot = eoff + (P.E + 1);
   __shared__ int ws[36];
+  __shared__ int s_ctok[2][32];        // down units: each column's token and gate (two units in flight)
+  __shared__ float s_cgate[2][32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT1 = P.I / 64, MT2 = P.d / TM;     // tiles per chunk: gate/up, down
@@ -785,6 +777,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int acc = it & 1;
+      if (U.ph == 2 && P.y_perm == nullptr && quad == 0 && lane < U.nvalid) {
+        // the unit's column info, fetched while its accumulator is computed
+        // (the barrier after the wait publishes it; the other buffer may still
+        // be read by warps finishing the previous unit)
+        const int p = __ldg(P.perm + U.q0 + lane);
+        const bool good = p >= 0 && p < n_pairs;
+        s_ctok[acc][lane] = good ? p / P.k : -1;
+        s_cgate[acc][lane] = good ? __ldg(P.gate + p) : 0.f;
+      }
+      // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
       named_sync(1, 128);
       if (*epi_fail) {
@@ -822,10 +824,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sb = e8m0_for(__uint_as_float(amax));
                 const uint32_t t = e4m3_rn(r * inv_pow2(sb));
                 r -= times_pow2(e4m3_to_f32(t), sb);
-                const size_t plane = static_cast<size_t>(j) * n_pairs;
+                const size_t plane = static_cast<size_t>(j) * P.a_rows;
                 P.aq[(plane + q) * P.I + col] = static_cast<uint8_t>(t);
                 if (lane == 0)
-                  P.as[((static_cast<size_t>(sf_plane<TN>(j)) * n_pairs + q) * (nbi / 4) + blk / 4) * 16 +
+                  P.as[((static_cast<size_t>(sf_plane<TN>(j)) * P.a_rows + q) * (nbi / 4) + blk / 4) * 16 +
                        sf_byte<TN>(j) + (blk & 3)] = static_cast<uint8_t>(sb);
               }
             }
@@ -847,9 +849,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (P.y_perm != nullptr) {
               P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
             } else {
-              const int p = __ldg(P.perm + q);
-              if (p >= 0 && p < n_pairs)
-                atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * v[c]);
+              const int t = s_ctok[acc][c];
+              if (t >= 0) atomicAdd(P.out + static_cast<size_t>(t) * P.d + row, s_cgate[acc][c] * v[c]);
             }
           }
         }
@@ -920,8 +921,9 @@ MxWorkspace mx_workspace(moe_shape s, int T, int k) {
   size_t o = 0;
   W.xq = o; o = round_up(o + static_cast<size_t>(NX) * T * s.d, 256);
   W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 128) * 16, 256);
-  W.aq = o; o = round_up(o + static_cast<size_t>(NA) * n * s.I, 256);
-  W.as = o; o = round_up(o + static_cast<size_t>(NA) * n * (s.I / 128) * 16, 256);
+  const size_t na = n > 32 ? n : 32;       // rows of an a-term plane (MxParams::a_rows)
+  W.aq = o; o = round_up(o + static_cast<size_t>(NA) * na * s.I, 256);
+  W.as = o; o = round_up(o + static_cast<size_t>(NA) * na * (s.I / 128) * 16, 256);
   W.done1 = o; o = round_up(o + static_cast<size_t>(s.E) * sizeof(int32_t), 256);
   W.bytes = o;
   return W;
@@ -970,10 +972,9 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   P.out = out;
   P.status = status;
   const uint64_t n = static_cast<uint64_t>(T) * k;
-  for (int i = 0; i < 3; ++i) {
-    const uint64_t r = static_cast<uint64_t>(8) << i;
-    P.a_box_rows[i] = static_cast<int>(n < r ? n : r);
-  }
+  const uint64_t na = n > 32 ? n : 32;
+  P.a_rows = static_cast<int>(na);
+  const int tn = T <= 8 ? 8 : (T <= 16 ? 16 : 32);   // token rows per term (the GEMV's TN)
   MxMaps M;
   CUresult r = encode_weight_map(&M.w1, P.pool + P.L.wg, s.d, 2 * s.I, n_slots, P.blob_bytes);
   if (r == CUDA_SUCCESS) r = encode_weight_map(&M.w2, P.pool + P.L.wd, s.I, s.d, n_slots, P.blob_bytes);
@@ -985,17 +986,19 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     r = encode_tiled_sw128(&M.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
   }
-  for (int i = 0; i < 3; ++i) {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.I), n, static_cast<uint64_t>(NA)};
-    const uint64_t str[2] = {static_cast<uint64_t>(s.I), n * s.I};
-    const uint32_t box[3] = {128u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
-    r = encode_tiled_sw128(&M.a[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
-    // scale rows of the a terms: (byte in the atom row, atom, pair, term); a box of rows
-    const int tn = T <= 8 ? 8 : (T <= 16 ? 16 : 32);
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), n, static_cast<uint64_t>(std::min(32 / tn, NA))};
-    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, n * (s.I / 128) * 16};
-    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(P.a_box_rows[i]), 1u};
-    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
+  {
+    // the a terms: (code, pair, term), a box of TN pairs of all NA terms; rows
+    // past the planes' end read as zeros
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.I), na, static_cast<uint64_t>(NA)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.I), na * s.I};
+    const uint32_t box[3] = {128u, static_cast<uint32_t>(tn), static_cast<uint32_t>(NA)};
+    r = encode_tiled_sw128(&M.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
+    // their scale rows: (byte in the atom row, atom, pair, plane), a box of TN pairs of every plane
+    const uint32_t planes = static_cast<uint32_t>(std::min(32 / tn, NA));
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), na, planes};
+    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, na * (s.I / 128) * 16};
+    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(tn), planes};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a terms failed (%d)", static_cast<int>(r));
   }
   {

@@ -331,6 +331,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   int32_t* eoff = ustart + (P.E + 1);          // offsets[0..E] and slot[0..E-1], read once
   int32_t* eslot = eoff + (P.E + 1);
   __shared__ int ws[36];
+  __shared__ int s_ctok[2][32];        // down units: each column's token and gate (two units in flight)
+  __shared__ float s_cgate[2][32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT1 = P.I / 64, MT2 = P.d / TM;     // tiles per chunk: gate/up, down
@@ -595,6 +597,15 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int acc = it & 1;
+      if (U.ph == 2 && P.y_perm == nullptr && quad == 0 && lane < U.nvalid) {
+        // the unit's column info, fetched while its accumulator is computed
+        // (the barrier after the wait publishes it; the other buffer may still
+        // be read by warps finishing the previous unit)
+        const int p = __ldg(P.perm + U.q0 + lane);
+        const bool good = p >= 0 && p < n_pairs;
+        s_ctok[acc][lane] = good ? p / P.k : -1;
+        s_cgate[acc][lane] = good ? __ldg(P.gate + p) : 0.f;
+      }
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
       named_sync(1, 128);
@@ -648,9 +659,8 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
             if (P.y_perm != nullptr) {
               P.y_perm[static_cast<size_t>(q) * P.d + row] = v[c];
             } else {
-              const int p = __ldg(P.perm + q);
-              if (p >= 0 && p < n_pairs)
-                atomicAdd(P.out + static_cast<size_t>(p / P.k) * P.d + row, __ldg(P.gate + p) * v[c]);
+              const int t = s_ctok[acc][c];
+              if (t >= 0) atomicAdd(P.out + static_cast<size_t>(t) * P.d + row, s_cgate[acc][c] * v[c]);
             }
           }
         }
