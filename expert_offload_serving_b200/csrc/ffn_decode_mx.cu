@@ -82,6 +82,7 @@ struct MxParams {
   int stall;                 // testing aid: CTA 0's epilogue waits on a barrier nothing arrives on
   int E, d, I, T, k, n_slots;
   int a_rows;              // rows of each a-term plane: max(T*k, 32), so a TN-row box always fits
+  int x_rows;              // rows of each x-term plane: max(T, 32)
   const int32_t* offsets;
   const int32_t* perm;
   const int32_t* slot;
@@ -89,7 +90,7 @@ struct MxParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  const uint8_t* xs;       // [32/TN][T][d/128][16] E8M0 scales of the x terms (sf_plane / sf_byte)
+  const uint8_t* xs;       // [32/TN][x_rows][d/128][16] E8M0 scales of the x terms (sf_plane / sf_byte)
   uint8_t* aq;             // [NA][a_rows][I] E4M3 terms of a (rows = sorted pairs)
   uint8_t* as;             // [32/TN][a_rows][I/128][16] their E8M0 scales (sf_plane / sf_byte)
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
@@ -98,12 +99,14 @@ struct MxParams {
   int32_t* status;
 };
 
-// Tensor maps of one launch: the weight tiles of both GEMVs, the x terms
-// (one-row boxes), and the a terms and their scale rows (boxes of TN rows of
-// every term, resp. every scale plane: the stacked B operand of one
-// 128-element half in one copy each).
+// Tensor maps of one launch: the weight tiles of both GEMVs; the x terms as
+// one-row boxes (TN = 32: the rows of a unit's pairs, gathered) and as boxes
+// of TN rows of both terms with their scale rows (TN <= 16: every token of
+// the step); the a terms and their scale rows (boxes of TN rows of every
+// term, resp. every scale plane).  A TN-row box is the stacked B operand of
+// one 128-element half in one copy.
 struct MxMaps {
-  CUtensorMap w1, w2, x, a, as;
+  CUtensorMap w1, w2, x, xall, xs, a, as;
 };
 
 // Scale rows of stacked terms.  B row r = j*TN + t (term j, token row t)
@@ -264,7 +267,7 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
 // bf16 values, each term with the E8M0 scale of the block's remaining maximum.
 // TN: the GEMV's token rows per term (the scale rows' plane and byte group).
 template <int TN>
-__global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int d,
+__global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int x_rows, int d,
                                                          uint8_t* __restrict__ xq, uint8_t* __restrict__ xs,
                                                          int32_t* __restrict__ zero, int n_zero) {
   const int nb = d / 32;
@@ -302,13 +305,13 @@ __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restr
         packed[i >> 2] |= q << (8 * (i & 3));
         r[i] -= times_pow2(e4m3_to_f32(q), sb);
       }
-      uint4* dst = reinterpret_cast<uint4*>(xq + (static_cast<size_t>(term) * T + t) * d + 32 * b);
+      uint4* dst = reinterpret_cast<uint4*>(xq + (static_cast<size_t>(term) * x_rows + t) * d + 32 * b);
       dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
       // scale of block b in byte b % 4 of the term's byte group of the 16-byte
       // row of atom b / 4 (the tcgen05 scale-factor atom's row pitch, so one
       // copy of a row lands in place)
-      xs[((static_cast<size_t>(sf_plane<TN>(term)) * T + t) * (nb / 4) + b / 4) * 16 + sf_byte<TN>(term) + (b & 3)] =
+      xs[((static_cast<size_t>(sf_plane<TN>(term)) * x_rows + t) * (nb / 4) + b / 4) * 16 + sf_byte<TN>(term) + (b & 3)] =
           static_cast<uint8_t>(sb);
     }
   }
@@ -341,7 +344,8 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
                                        uint8_t* sB, uint64_t* bar, uint64_t pol, int lane) {
   uint8_t* sf = sB + C::B_CODES;
   const int nt = U.ph == 1 ? NX : NA;       // terms of this unit's B operand
-  const uint32_t rows = U.ph == 1 ? static_cast<uint32_t>(U.nvalid) : static_cast<uint32_t>(TN);
+  // gemv<1> with TN <= 16 (T <= TN) loads every token's rows, else the unit's pairs' rows
+  const uint32_t rows = (U.ph == 1 && TN == 32) ? static_cast<uint32_t>(U.nvalid) : static_cast<uint32_t>(TN);
   const int planes = nt < C::G ? nt : C::G;   // scale planes of this unit's terms
   if (lane == 0) mbar_expect_tx(bar, rows * 2 * static_cast<uint32_t>(nt * 128 + planes * 16));
   __syncwarp();
@@ -353,6 +357,14 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
         tma_load_4d(sf + h * 512, &M.as, bar, 0, 2 * ks + h, U.q0, 0, pol);
       }
     }
+  } else if (TN <= 16) {
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tma_load_3d(sB + h * NX * C::B_ATOM, &M.xall, bar, ks * KSTAGE + 128 * h, 0, 0, pol);
+        tma_load_4d(sf + h * 512, &M.xs, bar, 0, 2 * ks + h, 0, 0, pol);
+      }
+    }
   } else if (lane < U.nvalid) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -362,7 +374,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 #pragma unroll
       for (int g = 0; g < (NX < C::G ? NX : C::G); ++g)
         bulk_load(sf + h * 512 + (g * TN + lane) * 16,
-                  P.xs + ((static_cast<size_t>(g) * P.T + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
+                  P.xs + ((static_cast<size_t>(g) * P.x_rows + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
     }
   }
 }
@@ -447,6 +459,16 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a, uint64_t 
 }
 
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
+
+// v[t] for a t < TN known only at run time, without indexing registers
+// dynamically (which would move v to local memory).
+template <int TN>
+__device__ __forceinline__ float pick(const float (&v)[32], int t) {
+  float g = v[0];
+#pragma unroll
+  for (int j = 1; j < TN; ++j) g = (t == j) ? v[j] : g;
+  return g;
+}
 
 // Token row c's result for this warp's 32 TMEM lanes: the sum over the nt
 // stacked terms of accumulator columns j*TN + c (fp32, terms in order).
@@ -662,7 +684,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
-      const int tok = token_of(P, U, lane, n_pairs);
+      const int tok = TN == 32 ? token_of(P, U, lane, n_pairs) : 0;
       const int KS = ks_of(U);
       if (PHASE == 3 && U.ph == 2) {
         // the a terms of this expert's pairs come from every gate/up unit of the expert
@@ -777,14 +799,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int u = blockIdx.x; u < n_units && !stalled; u += gridDim.x, ++it) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int acc = it & 1;
-      if (U.ph == 2 && P.y_perm == nullptr && quad == 0 && lane < U.nvalid) {
-        // the unit's column info, fetched while its accumulator is computed
-        // (the barrier after the wait publishes it; the other buffer may still
-        // be read by warps finishing the previous unit)
+      if (((U.ph == 2 && P.y_perm == nullptr) || (U.ph == 1 && TN <= 16)) && quad == 0 && lane < U.nvalid) {
+        // the unit's column info (its pairs' tokens; for the down GEMV's
+        // combine also their gates), fetched while its accumulator is
+        // computed (the barrier after the wait publishes it; the other buffer
+        // may still be read by warps finishing the previous unit)
         const int p = __ldg(P.perm + U.q0 + lane);
         const bool good = p >= 0 && p < n_pairs;
-        s_ctok[acc][lane] = good ? p / P.k : -1;
-        s_cgate[acc][lane] = good ? __ldg(P.gate + p) : 0.f;
+        if (!good) report(P.status, MOE_ERR_DEVICE);
+        s_ctok[acc][lane] = good ? p / P.k : (U.ph == 1 ? 0 : -1);
+        s_cgate[acc][lane] = good && U.ph == 2 ? __ldg(P.gate + p) : 0.f;
       }
       // the four warps leave together: a warp alone at a named barrier would wait for good
       if (!mbar_wait<true>(&tfull[acc], (it >> 1) & 1, abort_flag, P.wait_ns)) *epi_fail = 1;
@@ -816,7 +840,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             if (c < U.nvalid) {
-              float r = silu(v[c]) * up_buf[i * 33 + c];
+              // B column of pair c: its token (TN <= 16: every token's rows), else c
+              const int bc = TN <= 16 ? s_ctok[acc][c] : c;
+              float r = silu(TN <= 16 ? pick<TN>(v, bc) : v[c]) * up_buf[i * 33 + bc];
               const size_t q = static_cast<size_t>(U.q0 + c);
 #pragma unroll
               for (int j = 0; j < NA; ++j) {
@@ -919,8 +945,9 @@ MxWorkspace mx_workspace(moe_shape s, int T, int k) {
   MxWorkspace W{};
   const size_t n = static_cast<size_t>(T) * k;
   size_t o = 0;
-  W.xq = o; o = round_up(o + static_cast<size_t>(NX) * T * s.d, 256);
-  W.xs = o; o = round_up(o + static_cast<size_t>(NX) * T * (s.d / 128) * 16, 256);
+  const size_t tx = T > 32 ? T : 32;       // rows of an x-term plane (MxParams::x_rows)
+  W.xq = o; o = round_up(o + static_cast<size_t>(NX) * tx * s.d, 256);
+  W.xs = o; o = round_up(o + static_cast<size_t>(NX) * tx * (s.d / 128) * 16, 256);
   const size_t na = n > 32 ? n : 32;       // rows of an a-term plane (MxParams::a_rows)
   W.aq = o; o = round_up(o + static_cast<size_t>(NA) * na * s.I, 256);
   W.as = o; o = round_up(o + static_cast<size_t>(NA) * na * (s.I / 128) * 16, 256);
@@ -974,16 +1001,27 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   const uint64_t n = static_cast<uint64_t>(T) * k;
   const uint64_t na = n > 32 ? n : 32;
   P.a_rows = static_cast<int>(na);
+  const uint64_t tx = T > 32 ? T : 32;
+  P.x_rows = static_cast<int>(tx);
   const int tn = T <= 8 ? 8 : (T <= 16 ? 16 : 32);   // token rows per term (the GEMV's TN)
   MxMaps M;
   CUresult r = encode_weight_map(&M.w1, P.pool + P.L.wg, s.d, 2 * s.I, n_slots, P.blob_bytes);
   if (r == CUDA_SUCCESS) r = encode_weight_map(&M.w2, P.pool + P.L.wd, s.I, s.d, n_slots, P.blob_bytes);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the MXFP4 weights failed (%d)", static_cast<int>(r));
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T), static_cast<uint64_t>(NX)};
-    const uint64_t str[2] = {static_cast<uint64_t>(s.d), static_cast<uint64_t>(T) * s.d};
+    // the x terms: (code, token, term); one-row boxes, and boxes of TN rows of
+    // both terms with their scale rows (byte in the atom row, atom, token, plane)
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.d), tx, static_cast<uint64_t>(NX)};
+    const uint64_t str[2] = {static_cast<uint64_t>(s.d), tx * s.d};
     const uint32_t box[3] = {128u, 1u, 1u};
     r = encode_tiled_sw128(&M.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, box);
+    const uint32_t boxall[3] = {128u, static_cast<uint32_t>(tn), static_cast<uint32_t>(NX)};
+    if (r == CUDA_SUCCESS) r = encode_tiled_sw128(&M.xall, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, boxall);
+    const uint32_t planes = static_cast<uint32_t>(std::min(32 / tn, NX));
+    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.d / 128), tx, planes};
+    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.d / 128) * 16, tx * (s.d / 128) * 16};
+    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(tn), planes};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.xs, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
   }
   {
@@ -1005,13 +1043,13 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const long long blocks = static_cast<long long>(T) * (s.d / 32);
     const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
     if (T <= 8)
-      mx_split_x_kernel<8><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+      mx_split_x_kernel<8><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
                                                      w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
     else if (T <= 16)
-      mx_split_x_kernel<16><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+      mx_split_x_kernel<16><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
                                                       w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
     else
-      mx_split_x_kernel<32><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, s.d, w8 + W.xq,
+      mx_split_x_kernel<32><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
                                                       w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
