@@ -90,9 +90,9 @@ struct MxParams {
   const uint8_t* pool;
   size_t blob_bytes;
   BlobLayout L;
-  const uint8_t* xs;       // [32/TN][x_rows][d/128][16] E8M0 scales of the x terms (sf_plane / sf_byte)
+  const uint8_t* xs;       // [32/TN][d/128][x_rows][16] E8M0 scales of the x terms (sf_plane / sf_byte)
   uint8_t* aq;             // [NA][a_rows][I] E4M3 terms of a (rows = sorted pairs)
-  uint8_t* as;             // [32/TN][a_rows][I/128][16] their E8M0 scales (sf_plane / sf_byte)
+  uint8_t* as;             // [32/TN][I/128][a_rows][16] their E8M0 scales (sf_plane / sf_byte)
   int32_t* done1;          // one-launch schedule: per expert, gate/up units finished (zeroed before)
   float* y_perm;
   float* out;
@@ -113,8 +113,9 @@ struct MxMaps {
 // takes its 4 scales of a 128-element half from byte 4*(r/32) of the 16-byte
 // row r%32 of the half's scale-factor atom.  With G = 32/TN term row blocks
 // per 32 atom rows, term j sits in plane j%G (atom rows (j%G)*TN + t) at byte
-// group j/G, so the scale rows of a term plane are stored [plane][row][atom]
-// with 16 bytes per row: one copy of a plane's rows lands in place.
+// group j/G, so the scale rows are stored [plane][atom][row] with 16 bytes
+// per row: a copy of TN consecutive rows of one atom of each plane (one
+// contiguous run per plane) lands in place.
 template <int TN>
 __device__ __forceinline__ int sf_plane(int j) { return j % (32 / TN); }
 template <int TN>
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restr
       // scale of block b in byte b % 4 of the term's byte group of the 16-byte
       // row of atom b / 4 (the tcgen05 scale-factor atom's row pitch, so one
       // copy of a row lands in place)
-      xs[((static_cast<size_t>(sf_plane<TN>(term)) * x_rows + t) * (nb / 4) + b / 4) * 16 + sf_byte<TN>(term) + (b & 3)] =
+      xs[((static_cast<size_t>(sf_plane<TN>(term)) * (nb / 4) + b / 4) * x_rows + t) * 16 + sf_byte<TN>(term) + (b & 3)] =
           static_cast<uint8_t>(sb);
     }
   }
@@ -354,7 +355,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         tma_load_3d(sB + h * NA * C::B_ATOM, &M.a, bar, ks * KSTAGE + 128 * h, U.q0, 0, pol);
-        tma_load_4d(sf + h * 512, &M.as, bar, 0, 2 * ks + h, U.q0, 0, pol);
+        tma_load_3d(sf + h * 512, &M.as, bar, 4 * U.q0, 2 * ks + h, 0, pol);
       }
     }
   } else if (TN <= 16) {
@@ -362,7 +363,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         tma_load_3d(sB + h * NX * C::B_ATOM, &M.xall, bar, ks * KSTAGE + 128 * h, 0, 0, pol);
-        tma_load_4d(sf + h * 512, &M.xs, bar, 0, 2 * ks + h, 0, 0, pol);
+        tma_load_3d(sf + h * 512, &M.xs, bar, 0, 2 * ks + h, 0, pol);
       }
     }
   } else if (lane < U.nvalid) {
@@ -374,7 +375,7 @@ __device__ __forceinline__ void load_b(const MxParams& P, const MxMaps& M, const
 #pragma unroll
       for (int g = 0; g < (NX < C::G ? NX : C::G); ++g)
         bulk_load(sf + h * 512 + (g * TN + lane) * 16,
-                  P.xs + ((static_cast<size_t>(g) * P.x_rows + tok) * (P.d / 128) + 2 * ks + h) * 16, 16, bar, pol);
+                  P.xs + ((static_cast<size_t>(g) * (P.d / 128) + 2 * ks + h) * P.x_rows + tok) * 16, 16, bar, pol);
     }
   }
 }
@@ -853,7 +854,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const size_t plane = static_cast<size_t>(j) * P.a_rows;
                 P.aq[(plane + q) * P.I + col] = static_cast<uint8_t>(t);
                 if (lane == 0)
-                  P.as[((static_cast<size_t>(sf_plane<TN>(j)) * P.a_rows + q) * (nbi / 4) + blk / 4) * 16 +
+                  P.as[((static_cast<size_t>(sf_plane<TN>(j)) * (nbi / 4) + blk / 4) * P.a_rows + q) * 16 +
                        sf_byte<TN>(j) + (blk & 3)] = static_cast<uint8_t>(sb);
               }
             }
@@ -1018,10 +1019,12 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint32_t boxall[3] = {128u, static_cast<uint32_t>(tn), static_cast<uint32_t>(NX)};
     if (r == CUDA_SUCCESS) r = encode_tiled_sw128(&M.xall, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.xq, dims, str, boxall);
     const uint32_t planes = static_cast<uint32_t>(std::min(32 / tn, NX));
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.d / 128), tx, planes};
-    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.d / 128) * 16, tx * (s.d / 128) * 16};
-    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(tn), planes};
-    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.xs, sdims, sstr, sbox);
+    // scale rows [plane][atom][token][16 bytes] as 32-bit words: a box of TN
+    // consecutive rows of one atom per plane is one contiguous run
+    const uint64_t sdims[3] = {tx * 4, static_cast<uint64_t>(s.d / 128), planes};
+    const uint64_t sstr[2] = {tx * 16, static_cast<uint64_t>(s.d / 128) * tx * 16};
+    const uint32_t sbox[3] = {static_cast<uint32_t>(4 * tn), 1u, planes};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.xs, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, w8 + W.xs, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the x terms failed (%d)", static_cast<int>(r));
   }
   {
@@ -1031,12 +1034,13 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
     const uint64_t str[2] = {static_cast<uint64_t>(s.I), na * s.I};
     const uint32_t box[3] = {128u, static_cast<uint32_t>(tn), static_cast<uint32_t>(NA)};
     r = encode_tiled_sw128(&M.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w8 + W.aq, dims, str, box);
-    // their scale rows: (byte in the atom row, atom, pair, plane), a box of TN pairs of every plane
+    // their scale rows [plane][atom][pair][16 bytes] as 32-bit words, a box of
+    // TN consecutive pairs of one atom per plane
     const uint32_t planes = static_cast<uint32_t>(std::min(32 / tn, NA));
-    const uint64_t sdims[4] = {16, static_cast<uint64_t>(s.I / 128), na, planes};
-    const uint64_t sstr[3] = {16, static_cast<uint64_t>(s.I / 128) * 16, na * (s.I / 128) * 16};
-    const uint32_t sbox[4] = {16u, 1u, static_cast<uint32_t>(tn), planes};
-    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, w8 + W.as, sdims, sstr, sbox);
+    const uint64_t sdims[3] = {na * 4, static_cast<uint64_t>(s.I / 128), planes};
+    const uint64_t sstr[2] = {na * 16, static_cast<uint64_t>(s.I / 128) * na * 16};
+    const uint32_t sbox[3] = {static_cast<uint32_t>(4 * tn), 1u, planes};
+    if (r == CUDA_SUCCESS) r = encode_tiled_plain(&M.as, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, w8 + W.as, sdims, sstr, sbox);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map of the a terms failed (%d)", static_cast<int>(r));
   }
   {
