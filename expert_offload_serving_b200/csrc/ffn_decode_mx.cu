@@ -610,6 +610,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int n_units = PHASE == 3 ? total + total / MT1 * MT2 : total;
+  // two-launch schedule: the down GEMV (launched as a programmatic dependent)
+  // may take each SM as soon as this CTA leaves it; it streams its weights
+  // at once and waits for this grid only before reading the a terms
+  if (PHASE == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight producer
@@ -683,6 +687,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     int issued = 0;
     bool ok = true;
     int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
+    // the down GEMV of the two-launch schedule: the gate/up grid is complete
+    // and its a terms are visible before the first of them is read
+    if (PHASE == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int tok = TN == 32 ? token_of(P, U, lane, n_pairs) : 0;
@@ -909,11 +916,15 @@ moe_status launch_phase(const MxParams& P, const MxMaps& M, const DeviceInfo& de
   cfg.stream = s;
   // the one-launch schedule's CTAs wait on each other's gate/up units: all of
   // them must be resident at once, which a cooperative launch guarantees
-  cudaLaunchAttribute at[1];
+  // the two-launch schedule's down GEMV is a programmatic dependent of the
+  // gate/up GEMV (it waits for it in-kernel, before reading the a terms)
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = PHASE == 3 ? 1 : 0;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = PHASE == 2 ? 1 : 0;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_mx_kernel<PHASE, TN>, M, P));
   MOE_LAUNCH_CHECK("gemv_mx_kernel");
   return MOE_OK;
