@@ -41,7 +41,6 @@ using namespace ::moe::tc;
 
 constexpr int kWarps = 16;                 // warps per CTA (each its own pipeline)
 constexpr int kRW = 4;                      // weight rows per warp tile
-constexpr int kNTMaxCap = 8;               // token rows per pass, upper bound
 constexpr int kSlice = 1024;               // bytes of one row per stage
 constexpr int kStages = 3;                 // ring depth per warp
 constexpr int kStageBytes = kRW * kSlice;  // 4 KB
