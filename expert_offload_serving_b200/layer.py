@@ -71,14 +71,19 @@ class ExpertCache:
         return self.handle.fill(experts, step, protect, side=self.side, reads_done=self.reads_done,
                                 fill_done=self.fill_done, layer=layer)
 
-    def resize(self, new_n_slots: int, stream=None):
+    def resize(self, new_n_slots: int, stream=None, new_pool=None):
         """Elastic resize at a safe point: a new pool of new_n_slots blobs
-        receives the most recently used residents (device-to-device copies on
-        `stream`, after the last recorded reader); the old pool's memory goes
-        back to torch's allocator once the stream has passed the copies.
-        Returns [(key, old slot)] per kept resident."""
+        (allocated here, or the caller's uint8 [new_n_slots, blob bytes]
+        device tensor) receives the most recently used residents
+        (device-to-device copies on `stream`, after the last recorded reader);
+        the old pool's memory goes back to torch's allocator once the stream
+        has passed the copies.  Returns [(key, old slot)] per kept resident."""
         s = torch.cuda.current_stream() if stream is None else stream
-        new_pool = torch.empty((new_n_slots, self.B), dtype=torch.uint8, device=self.dev)
+        if new_pool is None:
+            new_pool = torch.empty((new_n_slots, self.B), dtype=torch.uint8, device=self.dev)
+        elif (new_pool.dtype != torch.uint8 or tuple(new_pool.shape) != (new_n_slots, self.B)
+              or new_pool.device != self.dev or not new_pool.is_contiguous()):
+            raise ValueError(f"new_pool must be a contiguous uint8 [{new_n_slots}, {self.B}] tensor on {self.dev}")
         kept = self.handle.resize(new_n_slots, new_pool, stream=s, reads_done=self.reads_done)
         self.pool.record_stream(s)
         self.pool = new_pool

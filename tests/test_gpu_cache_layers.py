@@ -47,7 +47,10 @@ def test_shared_cache_layers_with_resize(moe):
     outs = []
     for t in range(steps):
         if t in resizes:
-            assert cache.resize(resizes[t]) == ref.resize(resizes[t])
+            # the grow moves into a pool the caller allocated
+            pool = torch.empty((resizes[t], cache.B),
+                               dtype=torch.uint8, device="cuda") if t == 20 else None
+            assert cache.resize(resizes[t], new_pool=pool) == ref.resize(resizes[t])
             for l in range(n_layers):        # the tables were rewritten on the stream
                 assert layers[l].slot.cpu().tolist() == ref.slot_of_expert[l * cfg.E:(l + 1) * cfg.E]
         for l in range(n_layers):
