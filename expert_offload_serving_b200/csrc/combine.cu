@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const int32_t* __restrict__ slot,
                                                       const float* host_partial, int T, int k, int d,
                                                       int E_bound, int nq, float* out) {
+  pdl_wait();     // y_perm comes from the FFN launched before
+  pdl_trigger();
   const int t = blockIdx.y;
   const int c4 = blockIdx.x * blockDim.x + threadIdx.x;   // index of a float4 in the row
   if (t >= T || c4 * 4 >= d) return;
@@ -101,8 +103,8 @@ extern "C" moe_status moe_combine_merge(const float* y_perm, const int32_t* idx,
   if (st != MOE_OK) return st;
   const int threads = 256;
   dim3 grid((d / 4 + threads - 1) / threads, T);
-  combine_kernel<<<grid, threads, 0, stream>>>(y_perm, idx, gate, inv_perm, slot_of_expert,
-                                               host_partial, T, k, d, E, T * k, out);
+  MOE_CUDA_TRY(launch_pdl(combine_kernel, grid, dim3(threads), 0, stream, y_perm, idx, gate, inv_perm,
+                          slot_of_expert, host_partial, T, k, d, E, T * k, out));
   MOE_LAUNCH_CHECK("combine_kernel");
   return MOE_OK;
 }

@@ -68,6 +68,32 @@ bool decode_one_launch(int fmt, int T);
 // ---------------------------------------------------------------- device helpers
 constexpr unsigned kFull = 0xffffffffu;
 
+// Programmatic dependent launch.  The decode step's kernels are launched with
+// launch_pdl, so each may start (and run its prologue) while the kernel before
+// it on the stream finishes.  Each executes pdl_wait() before its first access
+// to memory that earlier work writes or reads -- it returns once the previous
+// grid has completed and its writes are visible -- and pdl_trigger() after it,
+// letting the next kernel be scheduled.  Without a programmatic launch both
+// are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }

@@ -271,6 +271,8 @@ template <int TN>
 __global__ void __launch_bounds__(256) mx_split_x_kernel(const uint16_t* __restrict__ x, int T, int x_rows, int d,
                                                          uint8_t* __restrict__ xq, uint8_t* __restrict__ xs,
                                                          int32_t* __restrict__ zero, int n_zero) {
+  pdl_wait();     // the terms and counters may still be read by the previous step's GEMVs
+  pdl_trigger();
   const int nb = d / 32;
   // the one-launch GEMV's per-expert counters start at zero (this kernel runs right before it)
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
@@ -568,6 +570,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
 
+  // the routing tables come from the kernels launched before (programmatic
+  // dependents start early: barriers and TMEM above, before the wait); the
+  // down GEMV instead waits in its token-row producer, so that its weights
+  // stream during the gate/up tail
+  if (PHASE != 2) pdl_wait();
   // ---- units per expert (evaluated experts only) and their exclusive prefix
   const int per = (P.E + THREADS - 1) / THREADS;
   const int e0 = threadIdx.x * per;
@@ -613,7 +620,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // two-launch schedule: the down GEMV (launched as a programmatic dependent)
   // may take each SM as soon as this CTA leaves it; it streams its weights
   // at once and waits for this grid only before reading the a terms
-  if (PHASE == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (PHASE == 1) pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight producer
@@ -689,7 +696,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
     // the down GEMV of the two-launch schedule: the gate/up grid is complete
     // and its a terms are visible before the first of them is read
-    if (PHASE == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (PHASE == 2) {
+      pdl_wait();
+      pdl_trigger();             // the combine after this GEMV may be scheduled
+    }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int tok = TN == 32 ? token_of(P, U, lane, n_pairs) : 0;
@@ -916,13 +926,14 @@ moe_status launch_phase(const MxParams& P, const MxMaps& M, const DeviceInfo& de
   cfg.stream = s;
   // the one-launch schedule's CTAs wait on each other's gate/up units: all of
   // them must be resident at once, which a cooperative launch guarantees
-  // the two-launch schedule's down GEMV is a programmatic dependent of the
-  // gate/up GEMV (it waits for it in-kernel, before reading the a terms)
+  // the two-launch schedule's GEMVs are programmatic dependents of the kernel
+  // before each (gate/up: the routing tables; down: the a terms), waiting for
+  // it in-kernel; the cooperative one-launch schedule is a plain launch
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = PHASE == 3 ? 1 : 0;
   at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = PHASE == 2 ? 1 : 0;
+  at[1].val.programmaticStreamSerializationAllowed = PHASE != 3 ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 2;
   MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_mx_kernel<PHASE, TN>, M, P));
@@ -1057,15 +1068,9 @@ moe_status launch_decode_mx(moe_shape s, const void* x, int T, int k, const int3
   {
     const long long blocks = static_cast<long long>(T) * (s.d / 32);
     const int grid = static_cast<int>((blocks + 255) / 256 < dev.sm_count * 4 ? (blocks + 255) / 256 : dev.sm_count * 4);
-    if (T <= 8)
-      mx_split_x_kernel<8><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
-                                                     w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
-    else if (T <= 16)
-      mx_split_x_kernel<16><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
-                                                      w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
-    else
-      mx_split_x_kernel<32><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), T, P.x_rows, s.d, w8 + W.xq,
-                                                      w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0);
+    auto split = T <= 8 ? mx_split_x_kernel<8> : (T <= 16 ? mx_split_x_kernel<16> : mx_split_x_kernel<32>);
+    MOE_CUDA_TRY(launch_pdl(split, dim3(grid), dim3(256), 0, stream, static_cast<const uint16_t*>(x), T, P.x_rows,
+                            s.d, w8 + W.xq, w8 + W.xs, P.done1, decode_one_launch(MOE_W_MXFP4, T) ? s.E : 0));
     MOE_LAUNCH_CHECK("mx_split_x_kernel");
   }
   if (T <= 8) return launch_both<8>(P, M, dev, stream);

@@ -365,6 +365,11 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
 
+  // the routing tables come from the kernels launched before (programmatic
+  // dependents start early: barriers and TMEM above, before the wait); the
+  // down GEMV instead waits in its token-row producer, so that its weights
+  // stream during the gate/up tail
+  if (PHASE != 2) pdl_wait();
   // ---- units per expert (evaluated experts only) and their exclusive prefix
   const int per = (P.E + THREADS - 1) / THREADS;
   const int e0 = threadIdx.x * per;
@@ -410,7 +415,7 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
   // two-launch schedule: the down GEMV (launched as a programmatic dependent)
   // may take each SM as soon as this CTA leaves it; it streams its weights
   // at once and waits for this grid only before reading the a terms
-  if (PHASE == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (PHASE == 1) pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ weight producer
@@ -485,7 +490,10 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
     int seen = -1;                       // lane 0: this unit's expert counter, loaded ahead
     // the down GEMV of the two-launch schedule: the gate/up grid is complete
     // and its a terms are visible before the first of them is read
-    if (PHASE == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (PHASE == 2) {
+      pdl_wait();
+      pdl_trigger();             // the combine after this GEMV may be scheduled
+    }
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit U = unit_of<PHASE, TN>(P, ustart, MT, MT2, u);
       const int tok = token_of(P, U, lane, n_pairs);
@@ -700,13 +708,14 @@ moe_status launch_phase(const TcDecodeParams& P, const CUtensorMap& tx, const CU
   cfg.stream = s;
   // the fused launch's CTAs wait on each other's gate/up units: all of them
   // must be resident at once, which a cooperative launch guarantees
-  // the two-launch schedule's down GEMV is a programmatic dependent of the
-  // gate/up GEMV (it waits for it in-kernel, before reading the a terms)
+  // the two-launch schedule's GEMVs are programmatic dependents of the kernel
+  // before each (gate/up: the routing tables; down: the a terms), waiting for
+  // it in-kernel; the cooperative one-launch schedule is a plain launch
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeCooperative;
   at[0].val.cooperative = PHASE == 3 ? 1 : 0;
   at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = PHASE == 2 ? 1 : 0;
+  at[1].val.programmaticStreamSerializationAllowed = PHASE != 3 ? 1 : 0;
   cfg.attrs = at;
   cfg.numAttrs = 2;
   MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemv_tc_kernel<FMT, PHASE, TN>, tx, ta, ta16, ta8, P));

@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(kTile) permute_fused_kernel(const int32_t* __r
                                                               int32_t* __restrict__ perm,
                                                               int32_t* __restrict__ inv_perm,
                                                               int32_t* status) {
+  pdl_wait();   // its inputs come from the previous kernel; its outputs may still be read
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem[];
   int* tile_cnt = reinterpret_cast<int*>(smem);            // [E]
   int* ws = tile_cnt + E;                                  // [33]
@@ -131,6 +133,8 @@ __global__ void __launch_bounds__(kTile) permute_fused_kernel(const int32_t* __r
 // Multi-tile, launch 1: histogram of each tile -> counts[tile][E].
 __global__ void __launch_bounds__(kTile) permute_count_kernel(const int32_t* __restrict__ idx, int n,
                                                               int E, int32_t* __restrict__ counts) {
+  pdl_wait();   // its inputs come from the previous kernel; its outputs may still be read
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem[];
   int* hist = reinterpret_cast<int*>(smem);
   for (int x = threadIdx.x; x < E; x += blockDim.x) hist[x] = 0;
@@ -150,6 +154,8 @@ __global__ void __launch_bounds__(kTile) permute_count_kernel(const int32_t* __r
 __global__ void __launch_bounds__(kTile) permute_scan_kernel(int32_t* __restrict__ counts, int ntiles,
                                                              int n, int E, int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ perm) {
+  pdl_wait();   // its inputs come from the previous kernel; its outputs may still be read
+  pdl_trigger();
   __shared__ int ws[36];
   const int e = threadIdx.x;
   int run = 0;
@@ -176,6 +182,8 @@ __global__ void __launch_bounds__(kTile) permute_scatter_kernel(const int32_t* _
                                                                 int32_t* __restrict__ perm,
                                                                 int32_t* __restrict__ inv_perm,
                                                                 int32_t* status) {
+  pdl_wait();   // its inputs come from the previous kernel; its outputs may still be read
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem[];
   int* tile_cnt = reinterpret_cast<int*>(smem);
   uint16_t* wcnt = reinterpret_cast<uint16_t*>(tile_cnt + E + 36);
@@ -260,16 +268,19 @@ extern "C" moe_status moe_permute(const int32_t* idx, int T, int k, int E, int32
   if (st != MOE_OK) return st;
   const int ntiles = (n + kTile - 1) / kTile;
   if (ntiles == 1) {
-    permute_fused_kernel<<<1, kTile, smem, stream>>>(idx, n, E, offsets, perm, inv_perm, dev_status);
+    MOE_CUDA_TRY(launch_pdl(permute_fused_kernel, dim3(1), dim3(kTile), smem, stream, idx, n, E, offsets, perm,
+                            inv_perm, dev_status));
     MOE_LAUNCH_CHECK("permute_fused_kernel");
     return MOE_OK;
   }
   int32_t* counts = static_cast<int32_t*>(scratch);
-  permute_count_kernel<<<ntiles, kTile, E * sizeof(int), stream>>>(idx, n, E, counts);
+  MOE_CUDA_TRY(launch_pdl(permute_count_kernel, dim3(ntiles), dim3(kTile), E * sizeof(int), stream, idx, n, E,
+                          counts));
   MOE_LAUNCH_CHECK("permute_count_kernel");
-  permute_scan_kernel<<<1, kTile, 0, stream>>>(counts, ntiles, n, E, offsets, perm);
+  MOE_CUDA_TRY(launch_pdl(permute_scan_kernel, dim3(1), dim3(kTile), 0, stream, counts, ntiles, n, E, offsets, perm));
   MOE_LAUNCH_CHECK("permute_scan_kernel");
-  permute_scatter_kernel<<<ntiles, kTile, smem, stream>>>(idx, n, E, counts, perm, inv_perm, dev_status);
+  MOE_CUDA_TRY(launch_pdl(permute_scatter_kernel, dim3(ntiles), dim3(kTile), smem, stream, idx, n, E, counts, perm,
+                          inv_perm, dev_status));
   MOE_LAUNCH_CHECK("permute_scatter_kernel");
   return MOE_OK;
 }

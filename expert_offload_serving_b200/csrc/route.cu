@@ -22,6 +22,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E,
                                                          int k, int32_t* __restrict__ idx,
                                                          float* __restrict__ gate) {
+  pdl_wait();     // idx and gate may still be read by the previous step's combine
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -80,8 +82,9 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* idx,
                          cudaStream_t s) {
   const int threads = 256;
   const int blocks = (T * 32 + threads - 1) / threads;
-  route_topk_kernel<VPL><<<blocks, threads, 0, s>>>(logits, T, E, k, idx, gate);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(route_topk_kernel<VPL>, dim3(blocks), dim3(threads), 0, s, logits, T, E, k, idx,
+                                   gate);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -82,7 +82,9 @@ class ExpertCache:
         if new_pool is None:
             new_pool = torch.empty((new_n_slots, self.B), dtype=torch.uint8, device=self.dev)
         elif (new_pool.dtype != torch.uint8 or tuple(new_pool.shape) != (new_n_slots, self.B)
-              or new_pool.device != self.dev or not new_pool.is_contiguous()):
+              or new_pool.device.type != "cuda" or not new_pool.is_contiguous()
+              or new_pool.device.index != (self.dev.index if self.dev.index is not None
+                                           else torch.cuda.current_device())):
             raise ValueError(f"new_pool must be a contiguous uint8 [{new_n_slots}, {self.B}] tensor on {self.dev}")
         kept = self.handle.resize(new_n_slots, new_pool, stream=s, reads_done=self.reads_done)
         self.pool.record_stream(s)
