@@ -593,11 +593,12 @@ moe_status launch_decode(const FfnParams& P, const DeviceInfo& dev, cudaStream_t
 size_t decode_mx_workspace_bytes(moe_shape s, int T, int k);
 
 // One cooperative launch saves the second launch and its pipeline fill, but
-// its down units wait on their expert's gate/up units while the two-launch
-// schedule streams them back to back.  Measured on B200 (fraction of HBM
-// bandwidth, one-launch vs two-launch): bf16 T = 1 0.395 / 0.414, T = 16
-// 0.856 / 0.862, T = 64 0.753 / 0.817; MXFP4 T = 1 0.294 / 0.264, T = 8
-// 0.429 / 0.489.  So one launch only for MXFP4 single-token steps.
+// its down units wait on their expert's gate/up units, while the two-launch
+// schedule streams the down GEMV's weights during the gate/up tail (it is a
+// programmatic dependent launch).  Measured on B200 (fraction of HBM
+// bandwidth, one launch vs two): bf16 T = 1 0.40 / 0.47, T = 16 0.85 / 0.91,
+// T = 64 0.74 / 0.85; MXFP4 T = 1 0.37 / 0.35, T = 8 0.64 / 0.68.  So one
+// launch only for MXFP4 single-token steps.
 bool decode_one_launch(int fmt, int T) {
   static const int forced = [] {
     const char* e = std::getenv("MOE_DECODE_SCHEDULE");
