@@ -165,6 +165,26 @@ def test_workspace_and_scratch_sizes(moe):
     assert moe.moe_permute_scratch_bytes(4096, 6, 256) == 24 * 256 * 4
 
 
+def test_ffn_launch_count(moe):
+    """moe_expert_ffn_launches reports the kernels an FFN call launches: the
+    decode schedule (one cooperative GEMV launch only for single-token MXFP4
+    steps, unless MOE_DECODE_SCHEDULE fixes it), the MXFP4 split of x, the
+    CUDA-core pair, the four prefill kernels; 0 for invalid arguments."""
+    import os
+    if os.environ.get("MOE_DECODE_SCHEDULE"):
+        pytest.skip("the schedule is fixed by the environment")
+    bf16 = moe.shape(128, 2048, 768, "bf16")
+    mx = moe.shape(256, 4096, 2048, "mxfp4")
+    assert moe.moe_expert_ffn_launches(bf16, 64, 8) == 2           # gate/up + down
+    assert moe.moe_expert_ffn_launches(bf16, 1, 8) == 2
+    assert moe.moe_expert_ffn_launches(mx, 8, 6) == 3              # split of x + gate/up + down
+    assert moe.moe_expert_ffn_launches(mx, 1, 6) == 2              # split of x + one cooperative launch
+    assert moe.moe_expert_ffn_launches(moe.shape(12, 264, 136, "bf16"), 9, 3) == 2   # CUDA cores
+    assert moe.moe_expert_ffn_launches(moe.shape(256, 4096, 2048, "nvfp4"), 4096, 6, moe.MOE_FFN_ACT_NVFP4) == 4
+    assert moe.moe_expert_ffn_launches(bf16, 0, 8) == 0
+    assert moe.moe_expert_ffn_launches(bf16, 4, 0) == 0
+
+
 def _canonical(name, E=3):
     base = synth.CONFIGS[name]
     cfg = synth.LayerConfig(name, E=E, k=2, d=256, I=128, fmt=base.fmt)
