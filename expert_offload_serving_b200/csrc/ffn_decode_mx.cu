@@ -202,33 +202,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// gemv<1>'s producer, once its own tiles are all issued: L2 prefetches of the
-// first tiles of the gemv<2> units this CTA will run (same round-robin deal),
-// up to `budget` bytes.  gemv<2>'s units of expert e are tiles x chunks(e) like
-// gemv<1>'s, so ustart1 scales to the gemv<2> table.
-template <int TN>
-__device__ void prefetch_down_units(const MxParams& P, const int32_t* ustart1, int per1, size_t budget) {
-  const int per2 = P.d / TM, KS2 = P.I / KSTAGE;
-  const int n2 = ustart1[P.E] / per1 * per2;
-  for (int u = blockIdx.x; u < n2 && budget > 0; u += gridDim.x) {
-    int lo = 0, hi = P.E;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (ustart1[mid] / per1 * per2 <= u) lo = mid;
-      else hi = mid;
-    }
-    const int q_begin = ustart1[P.E + 1 + lo], ne = ustart1[P.E + 2 + lo] - q_begin;
-    const int chunks = (ne + TN - 1) / TN;
-    const int m = (u - ustart1[lo] / per1 * per2) / chunks;
-    const uint8_t* base = P.pool + static_cast<size_t>(ustart1[2 * (P.E + 1) + lo]) * P.blob_bytes + P.L.wd +
-                          static_cast<size_t>(m) * KS2 * kMxTileBytes;
-    for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
-      prefetch_l2(base + static_cast<size_t>(ks) * kMxTileBytes, kMxTileBytes);
-      budget = budget > static_cast<size_t>(kMxTileBytes) ? budget - kMxTileBytes : 0;
-    }
-  }
-}
-
 // ------------------------------------------------------------------ E4M3 / E8M0 terms
 // E8M0 byte of the smallest power of two 2^e with amax <= 448 * 2^e (448 =
 // 1.75 * 2^8 is the largest E4M3 value), so that amax / 2^e rounds to a
@@ -679,7 +652,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<TN>(P, ustart, MT, 256u << 10);
     __syncwarp();
     if (!ok) {
       report(P.status, MOE_ERR_TIMEOUT);

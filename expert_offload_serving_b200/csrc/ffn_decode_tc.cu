@@ -165,35 +165,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Issued by gemv<1>'s producer once its own stages are all out: L2 prefetches
-// of the first weight stages of the gemv<2> units this CTA will run (same
-// round-robin deal), up to `budget` bytes, so that gemv<2> starts on warm L2.
-// gemv<2>'s units of expert e are proportional to gemv<1>'s: both are
-// tiles x chunks(e), so ustart1 scales to the gemv<2> table.
-template <int FMT, int TN>
-__device__ void prefetch_down_units(const TcDecodeParams& P, const int32_t* ustart1, int per1, size_t budget) {
-  using C = Cfg<FMT, 2, TN>;
-  const int MT2 = P.d / TM, KS2 = P.I / C::KSTAGE, per2 = MT2;
-  const int n2 = ustart1[P.E] / per1 * per2;
-  for (int u = blockIdx.x; u < n2 && budget > 0; u += gridDim.x) {
-    int lo = 0, hi = P.E;   // last e with ustart1[e] / per1 * per2 <= u
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (ustart1[mid] / per1 * per2 <= u) lo = mid;
-      else hi = mid;
-    }
-    const int q_begin = ustart1[P.E + 1 + lo], ne = ustart1[P.E + 2 + lo] - q_begin;
-    const int chunks = (ne + TN - 1) / TN;
-    const int m = (u - ustart1[lo] / per1 * per2) / chunks;
-    const uint8_t* base = P.pool + static_cast<size_t>(ustart1[2 * (P.E + 1) + lo]) * P.blob_bytes + P.L.wd +
-                          static_cast<size_t>(m) * KS2 * C::A_STAGE;
-    for (int ks = 0; ks < KS2 && budget > 0; ++ks) {
-      prefetch_l2(base + static_cast<size_t>(ks) * C::A_STAGE, C::A_STAGE);
-      budget = budget > static_cast<size_t>(C::A_STAGE) ? budget - C::A_STAGE : 0;
-    }
-  }
-}
-
 __device__ __forceinline__ float silu(float h) { return h / (1.0f + expf(-h)); }
 
 __device__ __forceinline__ void split_bf16(float a, uint16_t* hi, uint16_t* lo) {
@@ -472,7 +443,6 @@ __global__ void __launch_bounds__(Cfg<FMT, PHASE, TN>::THREADS, 1)
         }
       }
     }
-    if (PHASE == 1 && ok && lane == 0) prefetch_down_units<FMT, TN>(P, ustart, MT, 256u << 10);
     __syncwarp();
     if (!ok) {
       report(P.status, MOE_ERR_TIMEOUT);
