@@ -848,14 +848,18 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
             }
           }
-          // one-launch schedule: the a terms are published to other CTAs (read there by TMA)
-          if (PHASE == 3) {
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __threadfence();
-          }
+          // one-launch schedule: the a terms are published to other CTAs (read
+          // there by TMA): each writer orders its stores before the async
+          // proxy, the barrier below orders them before one thread's gpu-scope
+          // fence, and that fence before the counter increment (one fence per
+          // unit instead of one per thread)
+          if (PHASE == 3) asm volatile("fence.proxy.async.global;" ::: "memory");
         }
         named_sync(1, 128);
-        if (PHASE == 3 && warp == 2 && lane == 0) atomicAdd(P.done1 + U.e, 1);
+        if (PHASE == 3 && warp == 2 && lane == 0) {
+          __threadfence();
+          atomicAdd(P.done1 + U.e, 1);
+        }
       } else {
         const int row = TM * U.m + 32 * quad + lane;
 #pragma unroll
