@@ -553,6 +553,17 @@ def _run_gpu(args, rank, world, local, clk, timed_windows):
 
 
 # ---------------------------------------------------------------- prefill (FP4 tensor cores)
+def prefill_kernels(cfg, T):
+    """The kernels the library runs for an FP4 prefill step of T tokens: single
+    CTAs with at most 128 token rows per expert on average, else CTA pairs
+    (or what MOE_PREFILL_TILES forces)."""
+    forced = os.environ.get("MOE_PREFILL_TILES")
+    single = forced == "cta" if forced in ("cta", "pair") else T * cfg.k <= 128 * cfg.E
+    if single:
+        return "quant_tokens_cta_kernel, gather_x128_kernel, gemm_fp4_cta_kernel<1>, gemm_fp4_cta_kernel<2> (single CTAs)"
+    return "quant_tokens_kernel, gather_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2> (CTA pairs)"
+
+
 def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
     """The NVFP4 prefill layer (E=256, k=6, d=4096, I=2048, NVFP4 activations
     on tcgen05) at each token count in Ts: whole-layer time and the expert-FFN
@@ -630,7 +641,7 @@ def run_prefill(iters=20, warmup=5, Ts=(4096,), E=None, windows=None):
             "experts_touched": U,
             "timed_iters": n,
             "timing": f"median of {n} individually timed calls (FFN min/max {ffn_all[0]:.4f} / {ffn_all[-1]:.4f} ms)",
-            "kernels": "quant_tokens_kernel, gather_x_kernel, gemm_fp4_kernel<1>, gemm_fp4_kernel<2>",
+            "kernels": prefill_kernels(cfg, T),
         })
         del lg, xx
     return out

@@ -212,7 +212,10 @@ moe_status moe_permute_noalloc(const int32_t* idx, int T, int k, int E,
  *   and down in one cooperative launch or in two launches: see
  *   moe_expert_ffn_launches); other BF16/MXFP4 shapes and NVFP4 without
  *   MOE_FFN_ACT_NVFP4: CUDA cores; MOE_FFN_ACT_NVFP4: the tcgen05 FP4 GEMMs
- *   (d, I multiples of 256).
+ *   (d, I multiples of 256), on single CTAs (128 x 128 tiles) when
+ *   T*k <= 128*E, else on CTA pairs (256 x 224 tiles); the environment
+ *   variable MOE_PREFILL_TILES=cta|pair, read at every call, forces one.  The
+ *   workspace size covers both.
  * Limits: T*k <= 1<<24. */
 size_t moe_expert_ffn_workspace_bytes(moe_shape s, int T, int k, int flags);
 

@@ -32,12 +32,18 @@ def moe():
     return load_moe()
 
 
-def test_prefill_full_size_every_row(moe):
+def test_prefill_full_size_every_row(moe, monkeypatch):
+    """Every row at T = 4096, from the tiles the library picks there (single
+    CTAs: 96 rows per expert on average) and from CTA pairs forced."""
     cfg = synth.CONFIGS["prefill_nvfp4"]
     T = 4096
     b = Built(cfg, T, seed=0, act="nvfp4")
     out = b.run().cpu().numpy()
     moe.moe_check_status(b.layer.status)
+    monkeypatch.setenv("MOE_PREFILL_TILES", "pair")
+    out_pair = b.run().cpu().numpy()
+    moe.moe_check_status(b.layer.status)
+    monkeypatch.delenv("MOE_PREFILL_TILES")
     idx, _ = M.route_topk(b.logits.numpy(), cfg.k)
     off, perm, _ = M.permute(idx, cfg.E)
     assert np.array_equal(b.layer.idx.cpu().numpy(), idx)
@@ -46,11 +52,12 @@ def test_prefill_full_size_every_row(moe):
     assert len(b.used) == cfg.E                      # every expert's groups are exercised
     ref = pooled_oracle(b.x.double().numpy(), b.logits.numpy(), cfg.k, cfg.fmt, b.w_cpu, b.pos, b.used,
                         act="nvfp4")
-    m, r = check_tol(out, ref)
-    # no row is far off even if the layer as a whole is within tolerance
-    row_err = np.abs(out - ref).max(axis=1) / np.abs(ref).max()
-    assert row_err.max() <= 2e-2
-    print(f"prefill full size, all rows: max {m:.2e} mean-rel {r:.2e}")
+    for name, o in (("picked", out), ("pair", out_pair)):
+        m, r = check_tol(o, ref)
+        # no row is far off even if the layer as a whole is within tolerance
+        row_err = np.abs(o - ref).max(axis=1) / np.abs(ref).max()
+        assert row_err.max() <= 2e-2
+        print(f"prefill full size, all rows ({name} tiles): max {m:.2e} mean-rel {r:.2e}")
 
 
 @pytest.mark.parametrize("T", [1, 8])

@@ -21,21 +21,26 @@ def _cfg(name, E, k, d, I):
     return synth.LayerConfig(name, E=E, k=k, d=d, I=I, fmt="nvfp4", act="nvfp4")
 
 
+@pytest.mark.parametrize("tiles", ["auto", "cta", "pair"])
 @pytest.mark.parametrize("E,k,d,I,T", [
     (8, 2, 512, 256, 64),       # one chunk per expert, partial N
-    (4, 2, 256, 256, 400),      # ~200 rows per expert: one chunk each
-    (4, 2, 256, 256, 700),      # ~350 rows per expert: two chunks (224 + ~126)
-    (2, 1, 512, 256, 500),      # ~250 rows per expert: a full chunk and a ragged ~26-row tail
+    (4, 2, 256, 256, 400),      # ~200 rows per expert: one pair chunk each, two 128-row tiles
+    (4, 2, 256, 256, 700),      # ~350 rows per expert: two pair chunks (224 + ~126), three tiles
+    (2, 1, 512, 256, 500),      # ~250 rows per expert: a full pair chunk and a ragged ~26-row tail
     (16, 4, 1024, 512, 37),     # ragged small groups
     (8, 1, 256, 512, 1),        # a single token
 ])
-def test_prefill_small(moe, E, k, d, I, T):
+def test_prefill_small(moe, monkeypatch, E, k, d, I, T, tiles):
+    """Both tile families (CTA pairs over 224-row chunks, single CTAs over
+    128-row groups; "auto" takes the library's choice by rows per expert)."""
+    if tiles != "auto":
+        monkeypatch.setenv("MOE_PREFILL_TILES", tiles)
     b = Built(_cfg("pf", E, k, d, I), T, seed=E + T, act="nvfp4")
     out = b.run().cpu().numpy()
     moe.moe_check_status(b.layer.status)
     ref = b.oracle()
     m, r = check_tol(out, ref["out"])
-    print(f"prefill E={E} d={d} I={I} T={T}: max {m:.2e} mean-rel {r:.2e}")
+    print(f"prefill E={E} d={d} I={I} T={T} tiles={tiles}: max {m:.2e} mean-rel {r:.2e}")
 
 
 def test_prefill_host_partial_merge(moe):

@@ -21,8 +21,11 @@ def moe():
     return load_moe()
 
 
-@pytest.mark.parametrize("fmt", ["bf16", "mxfp4", "nvfp4"])
-def test_wait_expiry_is_reported_and_the_context_recovers(moe, fmt):
+@pytest.mark.parametrize("fmt", ["bf16", "mxfp4", "nvfp4", "nvfp4_pair"])
+def test_wait_expiry_is_reported_and_the_context_recovers(moe, monkeypatch, fmt):
+    if fmt == "nvfp4_pair":                  # the CTA-pair FP4 GEMMs (the default here is single CTAs)
+        monkeypatch.setenv("MOE_PREFILL_TILES", "pair")
+        fmt = "nvfp4"
     act = "nvfp4" if fmt == "nvfp4" else "none"
     cfg = synth.LayerConfig("stall", E=8, k=2, d=512, I=256, fmt=fmt, act=act)
     b = Built(cfg, 16, seed=1, act=act)
