@@ -165,6 +165,22 @@ def test_workspace_and_scratch_sizes(moe):
     assert moe.moe_permute_scratch_bytes(4096, 6, 256) == 24 * 256 * 4
 
 
+def test_workspace_never_shrinks_with_T(moe):
+    """A layer sizes its FFN workspace once, for its largest step, and runs
+    smaller steps on it; so the size must not decrease with T for any path,
+    including across the FP4 prefill's switch from single-CTA tiles to CTA
+    pairs at T*k = 128*E (where the tile family, and its layout, changes)."""
+    cases = [(moe.shape(128, 2048, 768, "bf16"), 8, 0), (moe.shape(256, 4096, 2048, "mxfp4"), 6, 0),
+             (moe.shape(256, 4096, 2048, "nvfp4"), 6, 0), (moe.shape(256, 4096, 2048, "nvfp4"), 6, 1),
+             (moe.shape(16, 1024, 512, "nvfp4"), 4, 1)]
+    for s, k, flags in cases:
+        switch = 128 * s.E // k
+        Ts = sorted(set(list(range(1, 70)) + list(range(switch - 40, switch + 40)) + list(range(1, 40000, 331))))
+        sizes = [moe.moe_expert_ffn_workspace_bytes(s, T, k, flags) for T in Ts]
+        assert all(a <= b for a, b in zip(sizes, sizes[1:])), (s.fmt, flags)
+        assert sizes[0] > 0
+
+
 def test_ffn_launch_count(moe):
     """moe_expert_ffn_launches reports the kernels an FFN call launches: the
     decode schedule (one cooperative GEMV launch only for single-token MXFP4
